@@ -1,0 +1,179 @@
+/*
+ * la2_oracle.c -- fp64 CPU oracle for decayed causal linear attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file: only the tests, the package's smoke check and the CPU
+ * baseline leg of the benchmark use it.  It shares no code, header, table or
+ * helper with the CUDA library.
+ *
+ * What it computes (per batch b and head h, rows t = 0..L-1):
+ *
+ *   o_t = sum_{j <= t} lambda^(t-j) (q_t . k_j) v_j  (+ lambda^(t+1) q_t kv0)
+ *
+ * i.e. O = (Q K^T (.) M) V with M_tj = lambda^(t-j) for j <= t, 0 above the
+ * diagonal.  lambda = 1 is plain causal linear attention.
+ *
+ * It is written as the token-by-token recurrence over a fixed-size d x e state
+ * -- the "recurrent form" that the Lightning Attention glossary page
+ * (jisaku.com, section "主な特徴・仕組み": recurrent and parallel forms, a
+ * constant-size state for inference) names, and the running "cumulative
+ * summation" of k^T v that the Lightning Attention-2 notes page
+ * (phantomic12.github.io, opening paragraph) says the causal case needs:
+ *
+ *   kv_t = lambda * kv_{t-1} + k_t^T v_t      (kv_{-1} = kv0, or 0)
+ *   o_t  = q_t kv_t                            (the state already holds token t)
+ *
+ * No blocking, no reordering: one token at a time, fp64 accumulation.
+ * The pages give no decay, feature map, normalisation or scaling; inputs are
+ * taken as already mapped, and no denominator is applied.
+ *
+ * Layout: q,k [B,H,L,d], v [B,H,L,e] contiguous row-major (float, which holds
+ * bf16 and fp32 inputs exactly); lambda [H] double; states [B,H,d,e] double;
+ * outputs double.  Every (b,h) problem is independent; OpenMP only spreads
+ * those independent problems over host cores.
+ */
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Forward: o (and optionally the final state kv_out) from the recurrence. */
+void oracle_forward(int B, int H, long L, int d, int e,
+                    const float *q, const float *k, const float *v,
+                    const double *lambda, const double *kv0,
+                    double *o, double *kv_out)
+{
+    long BH = (long)B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; bh++) {
+        int h = (int)(bh % H);
+        double lam = lambda[h];
+        double *kv = (double *)malloc(sizeof(double) * d * e);
+        if (kv0) memcpy(kv, kv0 + bh * d * e, sizeof(double) * d * e);
+        else memset(kv, 0, sizeof(double) * d * e);
+        const float *qb = q + bh * L * d, *kb = k + bh * L * d, *vb = v + bh * L * e;
+        double *ob = o + bh * L * e;
+        for (long t = 0; t < L; t++) {
+            const float *qt = qb + t * d, *kt = kb + t * d, *vt = vb + t * e;
+            /* state update: decay the old state, add the outer product k_t^T v_t */
+            for (int i = 0; i < d; i++)
+                for (int j = 0; j < e; j++)
+                    kv[i * e + j] = lam * kv[i * e + j] + (double)kt[i] * (double)vt[j];
+            /* read-out: o_t = q_t kv_t */
+            for (int j = 0; j < e; j++) {
+                double acc = 0.0;
+                for (int i = 0; i < d; i++) acc += (double)qt[i] * kv[i * e + j];
+                ob[t * e + j] = acc;
+            }
+        }
+        if (kv_out) memcpy(kv_out + bh * d * e, kv, sizeof(double) * d * e);
+        free(kv);
+    }
+}
+
+/*
+ * Backward of the same recurrence for an upstream gradient dO (the gradient
+ * of a scalar loss with respect to o).  Applying the chain rule to the two
+ * lines of the recurrence:
+ *
+ *   dq_t = dO_t kv_t^T                               (forward state kv_t)
+ *   G_t  = q_t^T dO_t + lambda * G_{t+1},  G_L = 0    (adjoint of kv_t)
+ *   dk_t = v_t G_t^T,   dv_t = k_t G_t
+ *   dkv0 = lambda * G_0                               (gradient w.r.t. kv0)
+ *
+ * The "tiling in both forward and backward" of the Lightning Attention-2 notes
+ * page ("Tiling." paragraph) is a faster schedule of exactly these sums.
+ */
+void oracle_backward(int B, int H, long L, int d, int e,
+                     const float *q, const float *k, const float *v,
+                     const double *lambda, const double *kv0, const float *dO,
+                     double *dq, double *dk, double *dv, double *dkv0)
+{
+    long BH = (long)B * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; bh++) {
+        int h = (int)(bh % H);
+        double lam = lambda[h];
+        double *st = (double *)malloc(sizeof(double) * d * e);
+        const float *qb = q + bh * L * d, *kb = k + bh * L * d, *vb = v + bh * L * e;
+        const float *gb = dO + bh * L * e;
+
+        /* forward sweep: rebuild kv_t, dq_t = dO_t kv_t^T */
+        if (kv0) memcpy(st, kv0 + bh * d * e, sizeof(double) * d * e);
+        else memset(st, 0, sizeof(double) * d * e);
+        for (long t = 0; t < L; t++) {
+            const float *kt = kb + t * d, *vt = vb + t * e, *gt = gb + t * e;
+            for (int i = 0; i < d; i++)
+                for (int j = 0; j < e; j++)
+                    st[i * e + j] = lam * st[i * e + j] + (double)kt[i] * (double)vt[j];
+            for (int i = 0; i < d; i++) {
+                double acc = 0.0;
+                for (int j = 0; j < e; j++) acc += (double)gt[j] * st[i * e + j];
+                dq[(bh * L + t) * d + i] = acc;
+            }
+        }
+
+        /* reverse sweep: G_t = q_t^T dO_t + lambda G_{t+1} */
+        memset(st, 0, sizeof(double) * d * e);
+        for (long t = L - 1; t >= 0; t--) {
+            const float *qt = qb + t * d, *kt = kb + t * d, *vt = vb + t * e, *gt = gb + t * e;
+            for (int i = 0; i < d; i++)
+                for (int j = 0; j < e; j++)
+                    st[i * e + j] = lam * st[i * e + j] + (double)qt[i] * (double)gt[j];
+            for (int i = 0; i < d; i++) {          /* dk_t = v_t G_t^T */
+                double acc = 0.0;
+                for (int j = 0; j < e; j++) acc += (double)vt[j] * st[i * e + j];
+                dk[(bh * L + t) * d + i] = acc;
+            }
+            for (int j = 0; j < e; j++) {          /* dv_t = k_t G_t */
+                double acc = 0.0;
+                for (int i = 0; i < d; i++) acc += (double)kt[i] * st[i * e + j];
+                dv[(bh * L + t) * e + j] = acc;
+            }
+        }
+        if (dkv0)
+            for (int i = 0; i < d * e; i++) dkv0[bh * d * e + i] = lam * st[i];
+        free(st);
+    }
+}
+
+/*
+ * One decode step: the recurrence above applied to a single new token per
+ * (b,h), with the fixed-size state kept by the caller between calls (the
+ * constant-size inference state of the glossary page, "主な特徴・仕組み").
+ *   kv <- lambda kv + k^T v;  o = q kv.
+ * q,k [B,H,d], v [B,H,e] float; kv [B,H,d,e] double, updated in place;
+ * o [B,H,e] double.
+ */
+void oracle_decode_step(int B, int H, int d, int e,
+                        const float *q, const float *k, const float *v,
+                        const double *lambda, double *kv, double *o)
+{
+    long BH = (long)B * H;
+#pragma omp parallel for schedule(static)
+    for (long bh = 0; bh < BH; bh++) {
+        int h = (int)(bh % H);
+        double lam = lambda[h];
+        double *s = kv + bh * d * e;
+        const float *qt = q + bh * d, *kt = k + bh * d, *vt = v + bh * e;
+        for (int i = 0; i < d; i++)
+            for (int j = 0; j < e; j++)
+                s[i * e + j] = lam * s[i * e + j] + (double)kt[i] * (double)vt[j];
+        for (int j = 0; j < e; j++) {
+            double acc = 0.0;
+            for (int i = 0; i < d; i++) acc += (double)qt[i] * s[i * e + j];
+            o[bh * e + j] = acc;
+        }
+    }
+}

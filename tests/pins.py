@@ -1,0 +1,262 @@
+"""Independent pins for the fp64 oracle.
+
+Each ``pin_*`` function takes a loaded oracle (``oracle.Oracle``) and raises
+AssertionError when the oracle disagrees with something that is fixed
+independently of it: a brute-force quadratic formula, a textbook routine
+(``numpy.cumsum``), a closed form, central finite differences, an identity
+the mathematics forces, or a hand-derived golden example.  The pins are run
+against the real oracle (``test_oracle_pins.py``) and against deliberately
+broken copies of it (``test_oracle_mutants.py``) to show they bite.
+
+None of this code is used by the CUDA path.
+"""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+# ----------------------------------------------------------------- helpers
+def bf16_exact(shape, seed, scale=1.0):
+    """Random normals rounded to bf16, returned as float32 (exact values)."""
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(shape, generator=g, dtype=torch.float32) * scale
+    return x.to(torch.bfloat16).to(torch.float32).numpy()
+
+
+def small_case(B=2, H=3, L=23, d=5, e=4, seed=1, lams=(1.0, 0.9, 0.37), kv0=True):
+    q = bf16_exact((B, H, L, d), seed, 0.5)
+    k = bf16_exact((B, H, L, d), seed + 1, 0.5)
+    v = bf16_exact((B, H, L, e), seed + 2)
+    dO = bf16_exact((B, H, L, e), seed + 3)
+    lam = np.array(lams[:H], np.float64)
+    s0 = bf16_exact((B, H, d, e), seed + 4, 0.3).astype(np.float64) if kv0 else None
+    return q, k, v, dO, lam, s0
+
+
+def decay_mask(L, lam):
+    """M[t, j] = lam^(t-j) for j <= t, else 0 (0^0 = 1)."""
+    t = np.arange(L)[:, None]
+    j = np.arange(L)[None, :]
+    n = t - j
+    with np.errstate(divide="ignore", invalid="ignore"):
+        m = np.where(n >= 0, np.power(float(lam), np.maximum(n, 0)), 0.0)
+    return m
+
+
+def assert_close(x, ref, tol, what):
+    x = np.asarray(x, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert x.shape == ref.shape, (what, x.shape, ref.shape)
+    scale = max(1.0, float(np.max(np.abs(ref))) if ref.size else 1.0)
+    err = float(np.max(np.abs(x - ref))) if ref.size else 0.0
+    assert err <= tol * scale, f"{what}: max err {err:.3e} > {tol:.1e}*{scale:.3e}"
+
+
+# ------------------------------------------- brute-force quadratic attention
+def quadratic_forward(q, k, v, lam, kv0):
+    """O = (Q K^T (.) M) V + diag(lam^(t+1)) Q kv0, per (b,h), fp64."""
+    B, H, L, d = q.shape
+    o = np.zeros(v.shape[:3] + (v.shape[-1],), np.float64)
+    for b in range(B):
+        for h in range(H):
+            Q, K, V = (a[b, h].astype(np.float64) for a in (q, k, v))
+            M = decay_mask(L, lam[h])
+            o[b, h] = ((Q @ K.T) * M) @ V
+            if kv0 is not None:
+                a = np.power(float(lam[h]), np.arange(1, L + 1))
+                o[b, h] += a[:, None] * (Q @ kv0[b, h])
+    return o
+
+
+def quadratic_state(k, v, lam, kv0):
+    """kv_L = lam^L kv0 + sum_j lam^(L-1-j) k_j^T v_j."""
+    B, H, L, d = k.shape
+    out = np.zeros((B, H, d, v.shape[-1]))
+    for b in range(B):
+        for h in range(H):
+            w = np.power(float(lam[h]), np.arange(L - 1, -1, -1))
+            out[b, h] = (k[b, h].astype(np.float64) * w[:, None]).T @ v[b, h]
+            if kv0 is not None:
+                out[b, h] += float(lam[h]) ** L * kv0[b, h]
+    return out
+
+
+def pin_bruteforce(orc):
+    for kv0 in (False, True):
+        q, k, v, dO, lam, s0 = small_case(kv0=kv0)
+        o, st = orc.forward(q, k, v, lam, s0, want_state=True)
+        assert_close(o, quadratic_forward(q, k, v, lam, s0), 1e-12, "o vs quadratic")
+        assert_close(st, quadratic_state(k, v, lam, s0), 1e-12, "state vs quadratic")
+
+
+def pin_prefix_sum(orc):
+    """lambda = 1: o_t = q_t . cumsum_j (k_j^T v_j) -- the running sum of the
+    causal case, built with numpy's cumsum."""
+    q, k, v, dO, _, _ = small_case(H=2, lams=(1.0, 1.0), kv0=False)
+    lam = np.ones(2)
+    outer = k[..., :, None].astype(np.float64) * v[..., None, :]
+    cum = np.cumsum(outer, axis=2)
+    ref = np.einsum("bhti,bhtij->bhtj", q.astype(np.float64), cum)
+    o, st = orc.forward(q, k, v, lam, want_state=True)
+    assert_close(o, ref, 1e-12, "o vs cumsum")
+    assert_close(st, cum[:, :, -1], 1e-12, "state vs cumsum")
+
+
+def pin_lambda_zero(orc):
+    """lambda = 0 keeps only the diagonal: o_t = (q_t . k_t) v_t."""
+    q, k, v, dO, _, s0 = small_case(H=1, lams=(0.0,), kv0=True)
+    lam = np.zeros(1)
+    ref = np.sum(q.astype(np.float64) * k, -1, keepdims=True) * v
+    o, st = orc.forward(q, k, v, lam, s0, want_state=True)
+    assert_close(o, ref, 1e-13, "o, lambda=0")
+    last = k[:, :, -1, :, None].astype(np.float64) * v[:, :, -1, None, :]
+    assert_close(st, last, 1e-13, "state, lambda=0")
+    dq, dk, dv, dkv0 = orc.backward(q, k, v, lam, dO, s0)
+    g = np.sum(dO.astype(np.float64) * v, -1, keepdims=True)
+    assert_close(dq, g * k, 1e-13, "dq, lambda=0")
+    assert_close(dk, g * q, 1e-13, "dk, lambda=0")
+    assert_close(dv, np.sum(q.astype(np.float64) * k, -1, keepdims=True) * dO,
+                 1e-13, "dv, lambda=0")
+    assert_close(dkv0, np.zeros_like(dkv0), 0, "dkv0, lambda=0")
+
+
+def pin_length_one(orc):
+    """L = 1: o_0 = q_0 (lambda kv0 + k_0^T v_0)."""
+    q, k, v, dO, lam, s0 = small_case(L=1, kv0=True)
+    o = orc.forward(q, k, v, lam, s0)
+    for b in range(q.shape[0]):
+        for h in range(q.shape[1]):
+            S = float(lam[h]) * s0[b, h] + np.outer(k[b, h, 0], v[b, h, 0])
+            assert_close(o[b, h, 0], q[b, h, 0].astype(np.float64) @ S, 1e-13, "L=1")
+
+
+# ------------------------------------------------------- backward closed forms
+def quadratic_backward(q, k, v, lam, dO, kv0):
+    """dQ = (dO V^T (.) M) K + diag(lam^(t+1)) dO kv0^T,
+    dK = (dO V^T (.) M)^T Q,  dV = (Q K^T (.) M)^T dO,
+    dkv0 = sum_t lam^(t+1) q_t^T dO_t."""
+    B, H, L, d = q.shape
+    e = v.shape[-1]
+    dq = np.zeros((B, H, L, d)); dk = np.zeros((B, H, L, d))
+    dv = np.zeros((B, H, L, e)); dkv0 = np.zeros((B, H, d, e))
+    for b in range(B):
+        for h in range(H):
+            Q, K, V, G = (a[b, h].astype(np.float64) for a in (q, k, v, dO))
+            M = decay_mask(L, lam[h])
+            dP = (G @ V.T) * M
+            P = (Q @ K.T) * M
+            dq[b, h] = dP @ K
+            dk[b, h] = dP.T @ Q
+            dv[b, h] = P.T @ G
+            a = np.power(float(lam[h]), np.arange(1, L + 1))
+            if kv0 is not None:
+                dq[b, h] += a[:, None] * (G @ kv0[b, h].T)
+            dkv0[b, h] = (Q * a[:, None]).T @ G
+    return dq, dk, dv, dkv0
+
+
+def pin_backward_closed_form(orc):
+    for kv0 in (False, True):
+        q, k, v, dO, lam, s0 = small_case(kv0=kv0)
+        got = orc.backward(q, k, v, lam, dO, s0)
+        ref = quadratic_backward(q, k, v, lam, dO, s0)
+        for name, x, r in zip(("dq", "dk", "dv", "dkv0"), got, ref):
+            assert_close(x, r, 1e-12, f"{name} vs closed form (kv0={kv0})")
+
+
+def pin_finite_difference(orc):
+    """loss = sum(o * dO) is linear in each input, so a central difference
+    with a step that keeps the perturbed inputs exact in fp32 reproduces the
+    gradient up to fp64 rounding."""
+    q, k, v, dO, lam, s0 = small_case(B=1, H=2, L=9, d=3, e=4, lams=(0.8, 1.0))
+    dq, dk, dv, dkv0 = orc.backward(q, k, v, lam, dO, s0)
+
+    def loss(qq, kk, vv, ss):
+        return float(np.sum(orc.forward(qq, kk, vv, lam, ss) * dO))
+
+    h = 2.0 ** -6
+    rng = np.random.default_rng(0)
+    for name, arr, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv), ("kv0", s0, dkv0)):
+        for _ in range(6):
+            idx = tuple(int(rng.integers(0, n)) for n in arr.shape)
+            plus, minus = arr.copy(), arr.copy()
+            plus[idx] += h
+            minus[idx] -= h
+            args = {"q": q, "k": k, "v": v, "kv0": s0}
+            args[name] = plus
+            lp = loss(args["q"], args["k"], args["v"], args["kv0"])
+            args[name] = minus
+            lm = loss(args["q"], args["k"], args["v"], args["kv0"])
+            fd = (lp - lm) / (2 * h)
+            assert abs(fd - grad[idx]) <= 1e-9 * max(1.0, abs(fd)), \
+                f"finite difference d{name}{idx}: {fd} vs {grad[idx]}"
+
+
+def pin_adjoint(orc):
+    """o is linear in q and bilinear in (k,v) / (q,kv0); Euler's identity for
+    homogeneous functions gives
+      sum dq*q = sum dO*o,  sum dk*k + sum dkv0*kv0 = sum dO*o,
+      sum dv*v + sum dkv0*kv0 = sum dO*o."""
+    q, k, v, dO, lam, s0 = small_case(kv0=True)
+    o = orc.forward(q, k, v, lam, s0)
+    dq, dk, dv, dkv0 = orc.backward(q, k, v, lam, dO, s0)
+    ref = float(np.sum(o * dO))
+    t0 = float(np.sum(dkv0 * s0))
+    for name, val in (("q", float(np.sum(dq * q))),
+                      ("k", float(np.sum(dk * k)) + t0),
+                      ("v", float(np.sum(dv * v)) + t0)):
+        assert abs(val - ref) <= 1e-11 * max(1.0, abs(ref)), (name, val, ref)
+
+
+# --------------------------------------------------------------- state pins
+def pin_state_handoff(orc):
+    q, k, v, dO, lam, s0 = small_case(L=30, kv0=True)
+    o, st = orc.forward(q, k, v, lam, s0, want_state=True)
+    L1 = 11
+    o1, st1 = orc.forward(q[:, :, :L1], k[:, :, :L1], v[:, :, :L1], lam, s0, want_state=True)
+    o2, st2 = orc.forward(q[:, :, L1:], k[:, :, L1:], v[:, :, L1:], lam, st1, want_state=True)
+    assert_close(np.concatenate([o1, o2], 2), o, 1e-13, "split forward")
+    assert_close(st2, st, 1e-13, "split state")
+
+
+def pin_decode_equals_forward(orc):
+    q, k, v, dO, lam, s0 = small_case(L=12, kv0=True)
+    o, st = orc.forward(q, k, v, lam, s0, want_state=True)
+    kv = np.ascontiguousarray(s0.copy())
+    for t in range(q.shape[2]):
+        ot = orc.decode_step(q[:, :, t], k[:, :, t], v[:, :, t], lam, kv)
+        assert_close(ot, o[:, :, t], 1e-13, f"decode step {t}")
+    assert_close(kv, st, 1e-13, "decode final state")
+
+
+# ------------------------------------------------------------- golden pins
+def pin_golden(orc):
+    with open(os.path.join(GOLDEN, "hand_examples.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        L, d, e = c["L"], c["d"], c["e"]
+        q = np.array(c["q"], np.float32).reshape(1, 1, L, d)
+        k = np.array(c["k"], np.float32).reshape(1, 1, L, d)
+        v = np.array(c["v"], np.float32).reshape(1, 1, L, e)
+        dO = np.array(c["dO"], np.float32).reshape(1, 1, L, e)
+        lam = np.array([c["lambda"]], np.float64)
+        s0 = None if c["kv0"] is None else np.array(c["kv0"], np.float64).reshape(1, 1, d, e)
+        o, st = orc.forward(q, k, v, lam, s0, want_state=True)
+        assert_close(o.reshape(L, e), np.array(c["o"]), 0, c["name"] + " o")
+        assert_close(st.reshape(d, e), np.array(c["kv_out"]), 0, c["name"] + " kv_out")
+        dq, dk, dv, dkv0 = orc.backward(q, k, v, lam, dO, s0)
+        assert_close(dq.reshape(L, d), np.array(c["dq"]), 0, c["name"] + " dq")
+        assert_close(dk.reshape(L, d), np.array(c["dk"]), 0, c["name"] + " dk")
+        assert_close(dv.reshape(L, e), np.array(c["dv"]), 0, c["name"] + " dv")
+        assert_close(dkv0.reshape(d, e), np.array(c["dkv0"]), 0, c["name"] + " dkv0")
+
+
+ALL_PINS = [pin_bruteforce, pin_prefix_sum, pin_lambda_zero, pin_length_one,
+            pin_backward_closed_form, pin_finite_difference, pin_adjoint,
+            pin_state_handoff, pin_decode_equals_forward, pin_golden]
