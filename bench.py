@@ -1,0 +1,432 @@
+"""Benchmark: fwd+bwd tokens/s of tiled causal linear attention over the
+length sweep (H=32, d=e=128, bf16, 65,536 tokens per batch at
+(B,L) in {(16,4K),(8,8K),(4,16K),(2,32K),(1,64K)}), on one B200 per rank.
+
+One step = forward + backward at every sweep point (5 x 65,536 tokens,
+32 heads each).  Inputs (512 MiB per tensor) are larger than L2, so no L2
+flush is needed between steps.  Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl la2|reference]
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (the only other code path this script runs).
+Multi-GPU (torchrun): every rank runs the whole sweep on its own GPU with no
+collective on the data path (weak scaling); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "fwd+bwd tokens/s vs L (H=32,d=e=128,bf16); % of bf16 tensor-core peak"
+SWEEP = [(16, 4096), (8, 8192), (4, 16384), (2, 32768), (1, 65536)]
+H, D, E = 32, 128, 128
+TOKENS = 65536
+# Algorithmic work per token per head (d = e = 128, bf16 I/O):
+#   bytes each kernel must move: forward reads q,k,v and writes o; the dQ
+#   kernel reads k,v,dO and writes dq; the dK/dV kernel reads q,k,v,dO and
+#   writes dk,dv.  The whole fwd+bwd needs at least 2,816 B.
+BYTES_PER_TH = {"tc_fwd": 1024, "simt_fwd": 1024, "tc_dq": 1024, "simt_dq": 1024,
+                "tc_dkdv": 1536, "simt_dkdv": 1536}
+FWD_BWD_MIN_BYTES = 2816
+# method flops per token-head, intra part over the causal triangle at a
+# fixed C = 64 accounting: fwd (C+1)(d+e) + 4de, bwd (C+1)(3d+2e) + 10de
+ALG_FLOPS_PER_TH = 65 * (D + E) + 4 * D * E + 65 * (3 * D + 2 * E) + 10 * D * E
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": float(j["hbm_gbs"]), "bf16_tflops": float(j["bf16_tflops"]),
+                "bf16_tflops_sustained": float(j.get("bf16_tflops_sustained", j["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"la2_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.index), "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        busy = [s for s in sm if mx and s > 0.3 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------ distributed
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------- workloads
+def make_sweep_inputs(dev):
+    from causal_linear_attention_fwd_b200 import inputs
+    x = inputs.make_inputs(1, H, TOKENS, D, E, dtype=torch.bfloat16, device=dev, seed=0)
+    lam = inputs.decay_lambdas(H, dev)
+    return x, lam
+
+
+def sweep_views(x, Bn, L):
+    return {n: t.view(Bn, H, L, t.shape[-1]) for n, t in x.items()}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "causal_linear_attention_fwd_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, units: int):
+    """dram bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; scaled to `units` token-heads."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    if j.get("source_hash") != kernel_source_hash():
+        return None
+    k = j.get("kernels", {}).get(kernel)
+    if not k:
+        return None
+    return k["dram_bytes_per_token_head"] * units
+
+
+def cpu_baseline(x, lam, budget_s=12.0):
+    """The fp64 oracle (as it stands) on host cores on a bounded sample of the
+    sweep workload: whole (b,h) problems of the L=4096 point, fwd+bwd."""
+    import oracle
+    orc = oracle.load()
+    xs = sweep_views(x, 16, 4096)
+    lam_h = lam.double().cpu().numpy()
+    threads = orc.num_threads()
+    heads_total = 16 * H
+    nh = min(heads_total, max(1, threads))
+    host = {}
+    elapsed = 0.0
+    while True:
+        flat = {n: t.view(16 * H, 4096, t.shape[-1])[:nh].float().cpu().numpy()[None]
+                for n, t in xs.items()}
+        lh = np.array([lam_h[i % H] for i in range(nh)])
+        t0 = time.perf_counter()
+        orc.forward(flat["q"], flat["k"], flat["v"], lh)
+        orc.backward(flat["q"], flat["k"], flat["v"], lh, flat["dO"])
+        elapsed = time.perf_counter() - t0
+        if elapsed >= budget_s / 4 or nh >= heads_total:
+            break
+        nh = min(heads_total, nh * max(2, int(math.ceil(budget_s / 2 / max(elapsed, 1e-3)))))
+    token_heads = nh * 4096
+    return {"value": token_heads / H / elapsed, "unit": "tokens/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"fwd+bwd of {nh} whole (b,h) sequences of the L=4096 sweep point "
+                      f"({token_heads} token-heads; tokens/s counts 32 heads per token) "
+                      f"in {elapsed:.2f} s"}
+
+
+# ------------------------------------------------------------------- main
+def run_la2(args, world, rank, local):
+    import causal_linear_attention_fwd_b200 as la2
+    dev = torch.device("cuda", local)
+    pk = peaks()
+    x, lam = make_sweep_inputs(dev)
+    outs = {n: torch.empty_like(x[src]) for n, src in
+            (("o", "v"), ("dq", "q"), ("dk", "k"), ("dv", "v"))}
+    stream = torch.cuda.current_stream()
+    ws_need = max(max(la2.workspace_size(op, Bn, H, L, D, E, torch.bfloat16)
+                      for op in (0, 1)) for Bn, L in SWEEP)
+    ws = torch.empty(max(ws_need, 16), dtype=torch.uint8, device=dev)
+
+    def one_shape(Bn, L, xin=None, oo=None):
+        xv = sweep_views(xin or x, Bn, L)
+        ov = sweep_views(oo or outs, Bn, L)
+        la2.forward(xv["q"], xv["k"], xv["v"], lam, out=ov["o"], workspace=ws)
+        la2.backward(xv["q"], xv["k"], xv["v"], lam, xv["dO"],
+                     outs=(ov["dq"], ov["dk"], ov["dv"]), workspace=ws)
+
+    for _ in range(args.warmup):
+        for Bn, L in SWEEP:
+            one_shape(Bn, L)
+    torch.cuda.synchronize()
+    assert la2.last_device_error() == 0
+
+    clocks = ClockSampler(local)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(SWEEP) + 1)]
+          for _ in range(args.steps)]
+    la2.profile_enable(True)
+    la2.profile_report()  # clear
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(args.steps):
+        ev[s][0].record(stream)
+        for i, (Bn, L) in enumerate(SWEEP):
+            one_shape(Bn, L)
+            ev[s][i + 1].record(stream)
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    prof = la2.profile_report()
+    la2.profile_enable(False)
+    assert la2.last_device_error() == 0
+    ms_local = t_start.elapsed_time(t_stop)
+    ms = max_over_ranks(ms_local, world)
+    per_shape = [sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps)) / args.steps
+                 for i in range(len(SWEEP))]
+
+    tokens_step = TOKENS * len(SWEEP)
+    value = world * tokens_step * args.steps / (ms / 1e3)
+    sweep = [{"B": Bn, "L": L, "tokens_per_s": TOKENS / (t / 1e3), "ms": t}
+             for (Bn, L), t in zip(SWEEP, per_shape)]
+    rates = [s["tokens_per_s"] for s in sweep]
+    th_per_launch = TOKENS * H
+
+    # dominant kernel and its roofline
+    launches = sum(v["launches"] for v in prof.values())
+    top = max(prof.items(), key=lambda kv: kv[1]["ms"]) if prof else None
+    roof = None
+    if top:
+        name, rec = top
+        avg_ms = rec["ms"] / rec["launches"]
+        bpt = BYTES_PER_TH.get(name)
+        if bpt:
+            alg = bpt * th_per_launch
+            ach = alg / (avg_ms / 1e3) / 1e9
+            tr = traffic_for(name, th_per_launch)
+            roof = {"kernel": name, "bound": "hbm", "achieved": round(ach, 1),
+                    "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(ach / pk["hbm_gbs"], 4),
+                    "traffic": tr, "alg_bytes_per_launch": alg, "avg_launch_ms": avg_ms,
+                    "peak_source": pk["source"] + " (hbm_gbs, STREAM-style copy)"}
+    tc_tflops = ALG_FLOPS_PER_TH * H * value / world / 1e12 if world else 0
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "length sweep fwd+bwd, H=32, d=e=128, bf16, 65,536 tokens/batch",
+                   "sweep": [[b, l] for b, l in SWEEP], "global_batch_tokens": TOKENS * world,
+                   "heads": H, "d": D, "e": E, "decay": "lambda_h = 1 - 2^-(5+8h/H)",
+                   "l2": "inputs 512 MiB per tensor, larger than L2; no flush",
+                   "parallelism": f"replicas x{world} (independent sequences per GPU)"},
+        "sweep": sweep, "sweep_spread": max(rates) / min(rates),
+        "roofline": roof,
+        "tensor": {"alg_flops_per_token_head": ALG_FLOPS_PER_TH,
+                   "achieved_tflops_per_gpu": round(tc_tflops, 2),
+                   "frac_of_bf16_peak": round(tc_tflops / pk["bf16_tflops_sustained"], 4),
+                   "peak": pk["bf16_tflops_sustained"], "peak_source": pk["source"] + " sustained"},
+        "hbm_frac_fwd_bwd_min": round(FWD_BWD_MIN_BYTES * H * value / world / 1e9 / pk["hbm_gbs"], 4),
+        "kernels": prof, "gpu_launches": launches, "clocks": clk,
+    }
+
+    # end to end through the public API with host buffers (pinned), copies timed
+    if not args.no_e2e:
+        line["e2e"] = run_e2e(args, la2, lam, ws, dev, world)
+    if rank == 0 and world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(x, lam)
+    elif rank == 0:
+        line["cpu_baseline"] = None
+    return line
+
+
+def run_e2e(args, la2, lam, ws, dev, world):
+    from causal_linear_attention_fwd_b200 import inputs
+    hx = inputs.make_inputs(1, H, TOKENS, D, E, dtype=torch.bfloat16, device="cpu", seed=0)
+    hin = {n: t.pin_memory() for n, t in hx.items()}
+    hout = {n: torch.empty(hin[s].shape, dtype=torch.bfloat16).pin_memory()
+            for n, s in (("o", "v"), ("dq", "q"), ("dk", "k"), ("dv", "v"))}
+    din = {n: torch.empty_like(t, device=dev) for n, t in hin.items()}
+    dout = {n: torch.empty_like(t, device=dev) for n, t in hout.items()}
+    stream = torch.cuda.current_stream()
+    bi = sum(t.numel() * t.element_size() for t in hin.values()) * len(SWEEP)
+    bo = sum(t.numel() * t.element_size() for t in hout.values()) * len(SWEEP)
+
+    def step():
+        for Bn, L in SWEEP:
+            for n in din:
+                din[n].copy_(hin[n], non_blocking=True)
+            xv = sweep_views(din, Bn, L)
+            ov = sweep_views(dout, Bn, L)
+            la2.forward(xv["q"], xv["k"], xv["v"], lam, out=ov["o"], workspace=ws)
+            la2.backward(xv["q"], xv["k"], xv["v"], lam, xv["dO"],
+                         outs=(ov["dq"], ov["dk"], ov["dv"]), workspace=ws)
+            for n in hout:
+                hout[n].copy_(dout[n], non_blocking=True)
+
+    for _ in range(min(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 3))
+    barrier(world)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(a.elapsed_time(b), world)
+    return {"value": round(world * TOKENS * len(SWEEP) * steps / (ms / 1e3), 1),
+            "unit": "tokens/s", "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+            "steps": steps, "note": "pinned host q,k,v,dO -> device, fwd+bwd, o,dq,dk,dv -> host"}
+
+
+def run_reference(args, world, rank):
+    """The oracle on host cores: each step is one bounded sample."""
+    if rank != 0:
+        return None
+    from causal_linear_attention_fwd_b200 import inputs
+    import oracle
+    orc = oracle.load()
+    lam = inputs.decay_lambdas(H, "cpu").double().numpy()
+    nh = max(1, orc.num_threads())
+    L = 4096
+    x = inputs.make_inputs(1, nh, L, D, E, dtype=torch.bfloat16, device="cpu", seed=0)
+    h = {n: t.float().numpy() for n, t in x.items()}
+    lh = np.array([lam[i % H] for i in range(nh)])
+
+    def step():
+        orc.forward(h["q"], h["k"], h["v"], lh)
+        orc.backward(h["q"], h["k"], h["v"], lh, h["dO"])
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    sec = time.perf_counter() - t0
+    value = nh * L * args.steps / H / sec
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": sec * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "length sweep fwd+bwd, H=32, d=e=128, bf16 inputs; "
+                                   f"each step = {nh} (b,h) sequences at L={L}",
+                       "heads": H, "d": D, "e": E},
+            "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": nh,
+                             "kind": "oracle",
+                             "sample": f"{nh} whole (b,h) sequences of L={L}, fwd+bwd, per step"},
+            "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="la2", choices=["la2", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3) if args.impl == "la2" else args.warmup
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        line = run_la2(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,19 @@
+"""B200-native tiled causal linear attention with per-head decay.
+
+O = (Q K^T (.) M) V, M_tj = lambda_h^(t-j) for j <= t (lambda_h = 1: plain
+causal linear attention), computed with the Lightning Attention-2 block
+schedule -- intra-block dense masked products plus an inter-block carried
+d x e state -- in forward and backward, plus the recurrent decode step.
+
+The computation lives in the C-ABI library libla2.so (include/la2.h); this
+package is its thin Python binding.  The library is loaded on first use and
+its absence raises an error: there is no CPU fallback.
+"""
+from ._binding import (  # noqa: F401
+    LA2Error, LA2_OP_BACKWARD, LA2_OP_FORWARD, LA2_OPT_PATH, LA2_OPT_SPLIT,
+    backward, decode_step, forward, last_device_error, library, profile_enable,
+    profile_report, set_option, status_string, version, workspace_size)
+
+__all__ = ["forward", "backward", "decode_step", "workspace_size",
+           "last_device_error", "set_option", "profile_enable", "profile_report",
+           "status_string", "version", "library", "LA2Error"]

@@ -1,0 +1,217 @@
+"""ctypes binding of libla2 (include/la2.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libla2.so.  PyTorch supplies device memory (outputs, scratch
+workspace) and the current CUDA stream.  There is no fallback: if the
+library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import json
+import os
+import threading
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libla2.so")
+
+LA2_OK, LA2_ERR_INVALID, LA2_ERR_UNSUPPORTED, LA2_ERR_CUDA, LA2_ERR_TIMEOUT = range(5)
+LA2_F32, LA2_BF16 = 0, 1
+LA2_OP_FORWARD, LA2_OP_BACKWARD = 0, 1
+LA2_OPT_SPLIT, LA2_OPT_PATH = 0, 1
+
+_lock = threading.Lock()
+_lib = None
+
+
+class LA2Error(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {status_string(code)}")
+
+
+def library():
+    """Load libla2.so (built in-tree by ``build.py``); raise if it is absent."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"libla2.so is not built ({LIB_PATH}); run "
+                "`python -c 'import __graft_entry__ as g; g.build()'` or "
+                "`python causal_linear_attention_fwd_b200/build.py`")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+        lib.la2_workspace_size.argtypes = [I, I, I, I64, I, I, I]
+        lib.la2_workspace_size.restype = SZ
+        lib.la2_forward.argtypes = [P, P, P, P, P, P, P, I, I, I64, I, I, I, P, SZ, P]
+        lib.la2_forward.restype = I
+        lib.la2_backward.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I64, I, I, I,
+                                     P, SZ, P]
+        lib.la2_backward.restype = I
+        lib.la2_decode_step.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
+        lib.la2_decode_step.restype = I
+        lib.la2_last_device_error.argtypes = [P]
+        lib.la2_last_device_error.restype = I
+        lib.la2_status_string.argtypes = [I]
+        lib.la2_status_string.restype = ctypes.c_char_p
+        lib.la2_set_option.argtypes = [I, I]
+        lib.la2_set_option.restype = I
+        lib.la2_profile_enable.argtypes = [I]
+        lib.la2_profile_enable.restype = None
+        lib.la2_profile_report.argtypes = [ctypes.c_char_p, SZ]
+        lib.la2_profile_report.restype = SZ
+        lib.la2_version.argtypes = []
+        lib.la2_version.restype = ctypes.c_char_p
+        _lib = lib
+        return lib
+
+
+def status_string(code: int) -> str:
+    try:
+        return library().la2_status_string(int(code)).decode()
+    except Exception:  # library missing: still give a name
+        return {0: "LA2_OK", 1: "LA2_ERR_INVALID", 2: "LA2_ERR_UNSUPPORTED",
+                3: "LA2_ERR_CUDA", 4: "LA2_ERR_TIMEOUT"}.get(int(code), str(code))
+
+
+def _check(code: int, what: str):
+    if code != LA2_OK:
+        raise LA2Error(code, what)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return LA2_F32
+    if t.dtype == torch.bfloat16:
+        return LA2_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dev(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def set_option(option: int, value: int) -> int:
+    return int(library().la2_set_option(int(option), int(value)))
+
+
+def version() -> str:
+    return library().la2_version().decode()
+
+
+def workspace_size(op: int, B: int, H: int, L: int, d: int, e: int, dtype) -> int:
+    dt = LA2_F32 if dtype == torch.float32 else LA2_BF16
+    return int(library().la2_workspace_size(op, B, H, L, d, e, dt))
+
+
+def _workspace(nbytes: int, device):
+    if nbytes == 0:
+        return None
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def forward(q, k, v, lam, kv0=None, *, want_state: bool = False, out=None,
+            workspace=None, stream=None):
+    """o = (Q K^T (.) M) V (+ the kv0 term); optionally the final state."""
+    lib = library()
+    for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam)):
+        _dev(t, name)
+    B, H, L, d = q.shape
+    e = v.shape[-1]
+    if k.shape != q.shape or v.shape[:3] != (B, H, L):
+        raise ValueError("shape mismatch among q, k, v")
+    if lam.dtype != torch.float32 or lam.numel() != H:
+        raise ValueError("lam must be float32 [H]")
+    if kv0 is not None:
+        _dev(kv0, "kv0")
+        if kv0.dtype != torch.float32 or kv0.shape != (B, H, d, e):
+            raise ValueError("kv0 must be float32 [B,H,d,e]")
+    o = out if out is not None else torch.empty((B, H, L, e), dtype=q.dtype, device=q.device)
+    st = torch.empty((B, H, d, e), dtype=torch.float32, device=q.device) if want_state else None
+    ws = workspace
+    if ws is None:
+        ws = _workspace(workspace_size(LA2_OP_FORWARD, B, H, L, d, e, q.dtype), q.device)
+    code = lib.la2_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(o), _ptr(st),
+                           B, H, L, d, e, _dt(q), _ptr(ws), 0 if ws is None else ws.numel(),
+                           _stream(stream))
+    _check(code, "la2_forward")
+    return (o, st) if want_state else o
+
+
+def backward(q, k, v, lam, dO, kv0=None, *, want_dkv0: bool = False, outs=None,
+             workspace=None, stream=None):
+    """Gradients (dq, dk, dv[, dkv0]) of sum(o * dO)."""
+    lib = library()
+    for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam), ("dO", dO)):
+        _dev(t, name)
+    B, H, L, d = q.shape
+    e = v.shape[-1]
+    if k.shape != q.shape or v.shape[:3] != (B, H, L) or dO.shape != v.shape:
+        raise ValueError("shape mismatch among q, k, v, dO")
+    if lam.dtype != torch.float32 or lam.numel() != H:
+        raise ValueError("lam must be float32 [H]")
+    if kv0 is not None:
+        _dev(kv0, "kv0")
+    if outs is not None:
+        dq, dk, dv = outs
+    else:
+        dq = torch.empty_like(q)
+        dk = torch.empty_like(k)
+        dv = torch.empty_like(v)
+    dkv0 = torch.empty((B, H, d, e), dtype=torch.float32, device=q.device) if want_dkv0 else None
+    ws = workspace
+    if ws is None:
+        ws = _workspace(workspace_size(LA2_OP_BACKWARD, B, H, L, d, e, q.dtype), q.device)
+    code = lib.la2_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(dO),
+                            _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dkv0), B, H, L, d, e, _dt(q),
+                            _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream))
+    _check(code, "la2_backward")
+    return (dq, dk, dv, dkv0) if want_dkv0 else (dq, dk, dv)
+
+
+def decode_step(q, k, v, lam, kv, *, out=None, stream=None):
+    """kv <- lam kv + k^T v (in place); returns o = q kv."""
+    lib = library()
+    for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam), ("kv", kv)):
+        _dev(t, name)
+    B, H, d = q.shape
+    e = v.shape[-1]
+    if kv.dtype != torch.float32 or kv.shape != (B, H, d, e):
+        raise ValueError("kv must be float32 [B,H,d,e]")
+    o = out if out is not None else torch.empty((B, H, e), dtype=q.dtype, device=q.device)
+    code = lib.la2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv), _ptr(o),
+                               B, H, d, e, _dt(q), _stream(stream))
+    _check(code, "la2_decode_step")
+    return o
+
+
+def last_device_error(stream=None) -> int:
+    return int(library().la2_last_device_error(_stream(stream)))
+
+
+def profile_enable(on: bool = True):
+    library().la2_profile_enable(1 if on else 0)
+
+
+def profile_report() -> dict:
+    # one report clears the records, so size the buffer generously up front
+    n = 1 << 16
+    buf = ctypes.create_string_buffer(n)
+    library().la2_profile_report(buf, n)
+    return json.loads(buf.value.decode() or "{}")

@@ -1,0 +1,478 @@
+// la2_api.cu -- the C ABI of libla2 (see include/la2.h): argument checks,
+// chunk planning, workspace carving, kernel dispatch, device error word and
+// per-kernel event timing.  The whole library is this one translation unit.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <initializer_list>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/la2.h"
+#include "la2_common.cuh"
+#include "la2_decode.cuh"
+#include "la2_simt.cuh"
+#include "la2_tc.cuh"
+
+namespace {
+
+using la2::Geo;
+
+std::atomic<int> g_opt_split{0};
+std::atomic<int> g_opt_path{0};
+
+// ------------------------------------------------------------ profiling
+enum KernelId {
+  K_SIMT_FWD_STATE, K_SIMT_FWD_SCAN, K_SIMT_FWD, K_SIMT_DQ, K_SIMT_REV_STATE,
+  K_SIMT_REV_SCAN, K_SIMT_DKDV, K_DECODE, K_TC_FWD_STATE, K_TC_FWD, K_TC_DQ,
+  K_TC_REV_STATE, K_TC_DKDV, K_SCAN_FWD, K_SCAN_REV, K_COUNT
+};
+const char *kKernelName[K_COUNT] = {
+    "simt_fwd_chunk_state", "simt_scan_fwd", "simt_fwd", "simt_dq",
+    "simt_rev_chunk_state", "simt_scan_rev", "simt_dkdv", "decode_step",
+    "tc_fwd_chunk_state", "tc_fwd", "tc_dq", "tc_rev_chunk_state", "tc_dkdv",
+    "scan_fwd", "scan_rev"};
+
+struct ProfRec {
+  int kid;
+  cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+std::atomic<int> g_prof_on{0};
+std::vector<ProfRec> g_prof;
+std::vector<cudaEvent_t> g_ev_pool;
+constexpr size_t kMaxProfRecs = 1 << 16;
+
+cudaEvent_t ev_get() {
+  if (!g_ev_pool.empty()) {
+    cudaEvent_t e = g_ev_pool.back();
+    g_ev_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Runs `launch` (which enqueues one kernel on `st`) and, while profiling is
+// on, brackets it with events.  Returns the launch error, if any.
+template <typename F>
+cudaError_t timed(int kid, cudaStream_t st, F &&launch) {
+  if (!g_prof_on.load(std::memory_order_relaxed)) {
+    launch();
+    return cudaGetLastError();
+  }
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  cudaEvent_t a = nullptr, b = nullptr;
+  if (g_prof.size() < kMaxProfRecs) {
+    a = ev_get();
+    b = ev_get();
+  }
+  if (a) cudaEventRecord(a, st);
+  launch();
+  cudaError_t err = cudaGetLastError();
+  if (a && b) {
+    cudaEventRecord(b, st);
+    g_prof.push_back({kid, a, b});
+  }
+  return err;
+}
+
+// ------------------------------------------------------------- helpers
+int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 148;
+  return n > 0 ? n : 148;
+}
+
+int device_cc() {
+  int dev = 0, ma = 0, mi = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  cudaDeviceGetAttribute(&ma, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&mi, cudaDevAttrComputeCapabilityMinor, dev);
+  return ma * 10 + mi;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Span {
+  const void *p;
+  size_t n;
+};
+bool overlaps(Span x, Span y) {
+  if (!x.p || !y.p || x.n == 0 || y.n == 0) return false;
+  uintptr_t a0 = reinterpret_cast<uintptr_t>(x.p), a1 = a0 + x.n;
+  uintptr_t b0 = reinterpret_cast<uintptr_t>(y.p), b1 = b0 + y.n;
+  return a0 < b1 && b0 < a1;
+}
+bool any_overlap(const std::vector<Span> &outs, const std::vector<Span> &all) {
+  for (size_t i = 0; i < outs.size(); i++)
+    for (size_t j = 0; j < all.size(); j++)
+      if (outs[i].p != all[j].p || outs[i].n != all[j].n)
+        if (overlaps(outs[i], all[j])) return true;
+  // two outputs at the same address also overlap
+  for (size_t i = 0; i < outs.size(); i++)
+    for (size_t j = i + 1; j < outs.size(); j++)
+      if (overlaps(outs[i], outs[j])) return true;
+  return false;
+}
+
+bool shape_supported(int d, int e, la2_dtype dt) {
+  return (d == 64 || d == 128) && (e == 64 || e == 128) &&
+         (dt == LA2_F32 || dt == LA2_BF16);
+}
+
+size_t esize(la2_dtype dt) { return dt == LA2_F32 ? 4 : 2; }
+
+// Which kernel family serves a call.
+enum Path { PATH_SIMT = 0, PATH_TC = 1, PATH_NONE = 2 };
+Path choose_path(int d, int e, la2_dtype dt) {
+  const int opt = g_opt_path.load();
+  const bool tc_ok = la2::tc::supports(d, e, dt == LA2_BF16) && device_cc() == 100;
+  if (opt == 1) return PATH_SIMT;
+  if (opt == 2) return tc_ok ? PATH_TC : PATH_NONE;
+  return tc_ok ? PATH_TC : PATH_SIMT;
+}
+
+// Chunk plan: split each (b,h) sequence into S chunks of Lc rows (Lc a
+// multiple of the block size `blk`) so that B*H*S CTAs fill the GPU.
+Geo plan(int B, int H, int64_t L, int blk, Path path) {
+  Geo g;
+  g.B = B;
+  g.H = H;
+  g.L = L;
+  const int64_t nblk = (L + blk - 1) / blk;
+  int64_t S = g_opt_split.load();
+  if (S <= 0) {
+    const int64_t BH = (int64_t)B * H;
+    const int sms = device_sms();
+    S = path == PATH_TC ? la2::tc::auto_split(BH, nblk, sms)
+                        : (BH >= 2 * sms ? 1 : (2 * sms + BH - 1) / BH);
+  }
+  if (S > nblk) S = nblk;
+  if (S < 1) S = 1;
+  const int64_t per = (nblk + S - 1) / S;
+  g.Lc = per * blk;
+  g.S = (int)((L + g.Lc - 1) / g.Lc);
+  if (g.S < 1) g.S = 1;
+  return g;
+}
+
+int block_rows(Path p) { return p == PATH_TC ? la2::tc::BLOCK : la2::simt::C; }
+
+size_t ws_bytes(int op, const Geo &g, int d, int e) {
+  if (g.S <= 1) return 0;
+  size_t one = (size_t)g.B * g.H * g.S * d * e * sizeof(float);
+  return op == LA2_OP_BACKWARD ? 2 * one : one;
+}
+
+// ------------------------------------------------------ SIMT dispatch
+template <typename T, int D, int E>
+cudaError_t simt_forward(const void *q, const void *k, const void *v,
+                         const float *lam, const float *kv0, void *o,
+                         float *kv_out, float *ws, const Geo &g, cudaStream_t st) {
+  using namespace la2::simt;
+  const T *Q = (const T *)q, *K = (const T *)k, *V = (const T *)v;
+  cudaError_t err = cudaSuccess;
+  const int64_t BH = (int64_t)g.B * g.H;
+  if (g.S > 1) {
+    auto kst = fwd_kernel<T, D, E, false>;
+    cudaFuncSetAttribute(kst, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fwd_smem<D, E>());
+    err = timed(K_SIMT_FWD_STATE, st, [&] {
+      kst<<<(unsigned)(BH * (g.S - 1)), NT, fwd_smem<D, E>(), st>>>(
+          Q, K, V, lam, nullptr, nullptr, nullptr, ws, g);
+    });
+    if (err) return err;
+    err = timed(K_SIMT_FWD_SCAN, st, [&] {
+      scan_fwd_kernel<D, E><<<dim3((D * E + NT - 1) / NT, (unsigned)BH), NT, 0, st>>>(ws, kv0, lam, g);
+    });
+    if (err) return err;
+  }
+  auto kf = fwd_kernel<T, D, E, true>;
+  cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fwd_smem<D, E>());
+  return timed(K_SIMT_FWD, st, [&] {
+    kf<<<(unsigned)(BH * g.S), NT, fwd_smem<D, E>(), st>>>(Q, K, V, lam, kv0, (T *)o, kv_out, ws, g);
+  });
+}
+
+template <typename T, int D, int E>
+cudaError_t simt_backward(const void *q, const void *k, const void *v,
+                          const float *lam, const float *kv0, const void *dO,
+                          void *dq, void *dk, void *dv, float *dkv0, float *ws,
+                          const Geo &g, cudaStream_t st) {
+  using namespace la2::simt;
+  const T *Q = (const T *)q, *K = (const T *)k, *V = (const T *)v, *G = (const T *)dO;
+  const int64_t BH = (int64_t)g.B * g.H;
+  float *wsf = ws;
+  float *wsr = ws ? ws + (size_t)BH * g.S * D * E : nullptr;
+  cudaError_t err = cudaSuccess;
+  if (g.S > 1) {
+    auto kst = fwd_kernel<T, D, E, false>;
+    cudaFuncSetAttribute(kst, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fwd_smem<D, E>());
+    err = timed(K_SIMT_FWD_STATE, st, [&] {
+      kst<<<(unsigned)(BH * (g.S - 1)), NT, fwd_smem<D, E>(), st>>>(
+          Q, K, V, lam, nullptr, nullptr, nullptr, wsf, g);
+    });
+    if (err) return err;
+    err = timed(K_SIMT_FWD_SCAN, st, [&] {
+      scan_fwd_kernel<D, E><<<dim3((D * E + NT - 1) / NT, (unsigned)BH), NT, 0, st>>>(wsf, kv0, lam, g);
+    });
+    if (err) return err;
+    auto krs = rev_state_kernel<T, D, E>;
+    cudaFuncSetAttribute(krs, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rev_smem<D, E>());
+    err = timed(K_SIMT_REV_STATE, st, [&] {
+      krs<<<(unsigned)(BH * (g.S - 1)), NT, rev_smem<D, E>(), st>>>(Q, G, lam, wsr, g);
+    });
+    if (err) return err;
+    err = timed(K_SIMT_REV_SCAN, st, [&] {
+      scan_rev_kernel<D, E><<<dim3((D * E + NT - 1) / NT, (unsigned)BH), NT, 0, st>>>(wsr, lam, g);
+    });
+    if (err) return err;
+  }
+  auto kq = dq_kernel<T, D, E>;
+  cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dq_smem<D, E>());
+  err = timed(K_SIMT_DQ, st, [&] {
+    kq<<<(unsigned)(BH * g.S), NT, dq_smem<D, E>(), st>>>(K, V, G, lam, kv0, (T *)dq, wsf, g);
+  });
+  if (err) return err;
+  auto kk = dkdv_kernel<T, D, E>;
+  cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dkdv_smem<D, E>());
+  return timed(K_SIMT_DKDV, st, [&] {
+    kk<<<(unsigned)(BH * g.S), NT, dkdv_smem<D, E>(), st>>>(Q, K, V, G, lam, (T *)dk, (T *)dv,
+                                                           dkv0, wsr, g);
+  });
+}
+
+template <typename T, int D, int E>
+cudaError_t decode(const void *q, const void *k, const void *v, const float *lam,
+                   float *kv, void *o, int B, int H, cudaStream_t st) {
+  return timed(K_DECODE, st, [&] {
+    la2::dec::decode_kernel<T, D, E><<<(unsigned)((int64_t)B * H), la2::dec::NT, 0, st>>>(
+        (const T *)q, (const T *)k, (const T *)v, lam, kv, (T *)o, H);
+  });
+}
+
+#define LA2_DISPATCH_DE(d, e, FN, T, ...)                                   \
+  ((d) == 64 && (e) == 64     ? FN<T, 64, 64>(__VA_ARGS__)                  \
+   : (d) == 64 && (e) == 128  ? FN<T, 64, 128>(__VA_ARGS__)                 \
+   : (d) == 128 && (e) == 64  ? FN<T, 128, 64>(__VA_ARGS__)                 \
+                              : FN<T, 128, 128>(__VA_ARGS__))
+
+la2_status to_status(cudaError_t e) { return e == cudaSuccess ? LA2_OK : LA2_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char *la2_status_string(la2_status s) {
+  switch (s) {
+    case LA2_OK: return "LA2_OK";
+    case LA2_ERR_INVALID: return "LA2_ERR_INVALID";
+    case LA2_ERR_UNSUPPORTED: return "LA2_ERR_UNSUPPORTED";
+    case LA2_ERR_CUDA: return "LA2_ERR_CUDA";
+    case LA2_ERR_TIMEOUT: return "LA2_ERR_TIMEOUT";
+  }
+  return "LA2_ERR_UNKNOWN";
+}
+
+const char *la2_version(void) { return "la2 0.1 sm_100a"; }
+
+int la2_set_option(int option, int value) {
+  if (option == LA2_OPT_SPLIT) return g_opt_split.exchange(value);
+  if (option == LA2_OPT_PATH) return g_opt_path.exchange(value);
+  return -1;
+}
+
+size_t la2_workspace_size(int op, int B, int H, int64_t L, int d, int e, la2_dtype dt) {
+  if (B <= 0 || H <= 0 || L <= 0 || !shape_supported(d, e, dt)) return 0;
+  if (op != LA2_OP_FORWARD && op != LA2_OP_BACKWARD) return 0;
+  Path p = choose_path(d, e, dt);
+  if (p == PATH_NONE) return 0;
+  Geo g = plan(B, H, L, block_rows(p), p);
+  return ws_bytes(op, g, d, e);
+}
+
+la2_status la2_forward(const void *q, const void *k, const void *v,
+                       const float *lambda, const float *kv0, void *o, float *kv_out,
+                       int B, int H, int64_t L, int d, int e, la2_dtype dt,
+                       void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (B < 0 || H < 0 || L < 0) return LA2_ERR_INVALID;
+  if (dt != LA2_F32 && dt != LA2_BF16) return LA2_ERR_UNSUPPORTED;
+  if (!shape_supported(d, e, dt)) return LA2_ERR_UNSUPPORTED;
+  const int64_t BH = (int64_t)B * H;
+  const size_t es = esize(dt);
+  const size_t nq = (size_t)BH * L * d * es, nv = (size_t)BH * L * e * es;
+  const size_t ns = (size_t)BH * d * e * sizeof(float);
+  if (BH == 0) return LA2_OK;
+  if (!lambda || (L > 0 && (!q || !k || !v || !o))) return LA2_ERR_INVALID;
+  for (const void *p : std::initializer_list<const void *>{(const void *)q, (const void *)k, (const void *)v, (const void *)lambda,
+                        (const void *)kv0, (const void *)o, (const void *)kv_out, workspace})
+    if (p && !aligned16(p)) return LA2_ERR_INVALID;
+  if (kv_out && kv_out == kv0) return LA2_ERR_INVALID;
+  std::vector<Span> ins = {{q, nq}, {k, nq}, {v, nv}, {lambda, (size_t)H * 4}, {kv0, kv0 ? ns : 0}};
+  std::vector<Span> outs = {{o, nv}, {kv_out, kv_out ? ns : 0}, {workspace, workspace_bytes}};
+  std::vector<Span> all = ins;
+  all.insert(all.end(), outs.begin(), outs.end());
+  if (any_overlap(outs, all)) return LA2_ERR_INVALID;
+
+  if (L == 0) {
+    if (!kv_out) return LA2_OK;
+    cudaError_t err = kv0 ? cudaMemcpyAsync(kv_out, kv0, ns, cudaMemcpyDeviceToDevice, stream)
+                          : cudaMemsetAsync(kv_out, 0, ns, stream);
+    return to_status(err);
+  }
+  Path p = choose_path(d, e, dt);
+  if (p == PATH_NONE) return LA2_ERR_UNSUPPORTED;
+  Geo g = plan(B, H, L, block_rows(p), p);
+  const size_t need = ws_bytes(LA2_OP_FORWARD, g, d, e);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return LA2_ERR_INVALID;
+  float *ws = (float *)workspace;
+  cudaError_t err;
+  if (p == PATH_TC) {
+    err = la2::tc::forward(q, k, v, lambda, kv0, o, kv_out, ws, g, stream,
+                           [&](int which, auto &&fn) {
+                             return timed(which == 0 ? K_TC_FWD_STATE : which == 1 ? K_SCAN_FWD : K_TC_FWD,
+                                          stream, fn);
+                           });
+  } else if (dt == LA2_F32) {
+    err = LA2_DISPATCH_DE(d, e, simt_forward, float, q, k, v, lambda, kv0, o, kv_out, ws, g, stream);
+  } else {
+    err = LA2_DISPATCH_DE(d, e, simt_forward, __nv_bfloat16, q, k, v, lambda, kv0, o, kv_out, ws, g,
+                          stream);
+  }
+  return to_status(err);
+}
+
+la2_status la2_backward(const void *q, const void *k, const void *v,
+                        const float *lambda, const float *kv0, const void *dO,
+                        void *dq, void *dk, void *dv, float *dkv0,
+                        int B, int H, int64_t L, int d, int e, la2_dtype dt,
+                        void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (B < 0 || H < 0 || L < 0) return LA2_ERR_INVALID;
+  if (dt != LA2_F32 && dt != LA2_BF16) return LA2_ERR_UNSUPPORTED;
+  if (!shape_supported(d, e, dt)) return LA2_ERR_UNSUPPORTED;
+  const int64_t BH = (int64_t)B * H;
+  const size_t es = esize(dt);
+  const size_t nq = (size_t)BH * L * d * es, nv = (size_t)BH * L * e * es;
+  const size_t ns = (size_t)BH * d * e * sizeof(float);
+  if (BH == 0) return LA2_OK;
+  if (!lambda || (L > 0 && (!q || !k || !v || !dO || !dq || !dk || !dv))) return LA2_ERR_INVALID;
+  for (const void *p : std::initializer_list<const void *>{(const void *)q, (const void *)k, (const void *)v, (const void *)lambda,
+                        (const void *)kv0, (const void *)dO, (const void *)dq, (const void *)dk,
+                        (const void *)dv, (const void *)dkv0, workspace})
+    if (p && !aligned16(p)) return LA2_ERR_INVALID;
+  std::vector<Span> ins = {{q, nq}, {k, nq}, {v, nv}, {dO, nv}, {lambda, (size_t)H * 4},
+                           {kv0, kv0 ? ns : 0}};
+  std::vector<Span> outs = {{dq, nq}, {dk, nq}, {dv, nv}, {dkv0, dkv0 ? ns : 0},
+                            {workspace, workspace_bytes}};
+  std::vector<Span> all = ins;
+  all.insert(all.end(), outs.begin(), outs.end());
+  if (any_overlap(outs, all)) return LA2_ERR_INVALID;
+
+  if (L == 0) {
+    if (!dkv0) return LA2_OK;
+    return to_status(cudaMemsetAsync(dkv0, 0, ns, stream));
+  }
+  Path p = choose_path(d, e, dt);
+  if (p == PATH_NONE) return LA2_ERR_UNSUPPORTED;
+  Geo g = plan(B, H, L, block_rows(p), p);
+  const size_t need = ws_bytes(LA2_OP_BACKWARD, g, d, e);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return LA2_ERR_INVALID;
+  float *ws = (float *)workspace;
+  cudaError_t err;
+  if (p == PATH_TC) {
+    err = la2::tc::backward(q, k, v, lambda, kv0, dO, dq, dk, dv, dkv0, ws, g, stream,
+                            [&](int which, auto &&fn) {
+                              static const int ids[] = {K_TC_FWD_STATE, K_SCAN_FWD, K_TC_DQ,
+                                                        K_TC_REV_STATE, K_SCAN_REV, K_TC_DKDV};
+                              return timed(ids[which], stream, fn);
+                            });
+  } else if (dt == LA2_F32) {
+    err = LA2_DISPATCH_DE(d, e, simt_backward, float, q, k, v, lambda, kv0, dO, dq, dk, dv, dkv0,
+                          ws, g, stream);
+  } else {
+    err = LA2_DISPATCH_DE(d, e, simt_backward, __nv_bfloat16, q, k, v, lambda, kv0, dO, dq, dk,
+                          dv, dkv0, ws, g, stream);
+  }
+  return to_status(err);
+}
+
+la2_status la2_decode_step(const void *q, const void *k, const void *v, const float *lambda,
+                           float *kv, void *o, int B, int H, int d, int e, la2_dtype dt,
+                           cudaStream_t stream) {
+  if (B < 0 || H < 0) return LA2_ERR_INVALID;
+  if (dt != LA2_F32 && dt != LA2_BF16) return LA2_ERR_UNSUPPORTED;
+  if (!shape_supported(d, e, dt)) return LA2_ERR_UNSUPPORTED;
+  const int64_t BH = (int64_t)B * H;
+  if (BH == 0) return LA2_OK;
+  if (!q || !k || !v || !lambda || !kv || !o) return LA2_ERR_INVALID;
+  for (const void *p : std::initializer_list<const void *>{(const void *)q, (const void *)k, (const void *)v, (const void *)lambda,
+                        (const void *)kv, (const void *)o})
+    if (!aligned16(p)) return LA2_ERR_INVALID;
+  const size_t es = esize(dt);
+  std::vector<Span> ins = {{q, BH * d * es}, {k, BH * d * es}, {v, BH * e * es},
+                           {lambda, (size_t)H * 4}};
+  std::vector<Span> outs = {{kv, BH * d * e * sizeof(float)}, {o, BH * e * es}};
+  std::vector<Span> all = ins;
+  all.insert(all.end(), outs.begin(), outs.end());
+  if (any_overlap(outs, all)) return LA2_ERR_INVALID;
+  cudaError_t err = dt == LA2_F32
+                        ? LA2_DISPATCH_DE(d, e, decode, float, q, k, v, lambda, kv, o, B, H, stream)
+                        : LA2_DISPATCH_DE(d, e, decode, __nv_bfloat16, q, k, v, lambda, kv, o, B, H,
+                                          stream);
+  return to_status(err);
+}
+
+la2_status la2_last_device_error(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return LA2_ERR_CUDA;
+  unsigned int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, la2::g_error_word, sizeof(word)) != cudaSuccess)
+    return LA2_ERR_CUDA;
+  if (word && cudaMemcpyToSymbol(la2::g_error_word, &zero, sizeof(zero)) != cudaSuccess)
+    return LA2_ERR_CUDA;
+  if (word & la2::ERR_TIMEOUT) return LA2_ERR_TIMEOUT;
+  if (word) return LA2_ERR_CUDA;
+  return LA2_OK;
+}
+
+void la2_profile_enable(int on) { g_prof_on.store(on ? 1 : 0); }
+
+size_t la2_profile_report(char *buf, size_t buf_bytes) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  double ms[K_COUNT] = {0};
+  long n[K_COUNT] = {0};
+  for (auto &r : g_prof) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&t, r.a, r.b) == cudaSuccess) {
+      ms[r.kid] += t;
+      n[r.kid] += 1;
+    }
+    g_ev_pool.push_back(r.a);
+    g_ev_pool.push_back(r.b);
+  }
+  g_prof.clear();
+  std::string s = "{";
+  bool first = true;
+  for (int i = 0; i < K_COUNT; i++) {
+    if (!n[i]) continue;
+    char tmp[160];
+    snprintf(tmp, sizeof(tmp), "%s\"%s\": {\"launches\": %ld, \"ms\": %.6f}", first ? "" : ", ",
+             kKernelName[i], n[i], ms[i]);
+    s += tmp;
+    first = false;
+  }
+  s += "}";
+  if (buf && buf_bytes) {
+    size_t m = s.size() < buf_bytes - 1 ? s.size() : buf_bytes - 1;
+    memcpy(buf, s.data(), m);
+    buf[m] = 0;
+  }
+  return s.size() + 1;
+}
+
+}  // extern "C"

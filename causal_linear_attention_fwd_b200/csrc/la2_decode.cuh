@@ -1,0 +1,107 @@
+// la2_decode.cuh -- one recurrent decode step, HBM-bound.
+//
+//   kv <- lambda kv + k^T v,   o = q kv        (per (b,h), kv fp32 d x e)
+//
+// The recurrent form with a fixed-size state (Lightning Attention glossary
+// page, section "主な特徴・仕組み").  Each step must read and write the whole
+// fp32 state once, so the kernel is a streaming pass over 2 * d * e * 4 bytes
+// per (b,h): one CTA per state, each warp owns d/8 rows, each lane a 16-byte
+// (e = 128) or 8-byte (e = 64) column slice, so every warp-wide load or store
+// is one contiguous 512/256-byte row.  All of a thread's row loads are issued
+// before any arithmetic so ~64 KB per CTA is in flight; loads and stores use
+// the streaming (evict-first) cache hint since the state is touched once per
+// step.  The column sums o_j = sum_i q_i kv_ij are reduced across warps in
+// shared memory.
+#pragma once
+
+#include "la2_common.cuh"
+
+namespace la2 {
+namespace dec {
+
+constexpr int NT = 256;
+constexpr int NW = NT / 32;
+
+template <int VEC> struct vec_t;
+template <> struct vec_t<4> {
+  using type = float4;
+  static __device__ __forceinline__ float4 ld(const float *p) {
+    return __ldcs(reinterpret_cast<const float4 *>(p));
+  }
+  static __device__ __forceinline__ void st(float *p, float4 x) {
+    __stcs(reinterpret_cast<float4 *>(p), x);
+  }
+  static __device__ __forceinline__ float &at(float4 &x, int i) {
+    return reinterpret_cast<float *>(&x)[i];
+  }
+};
+template <> struct vec_t<2> {
+  using type = float2;
+  static __device__ __forceinline__ float2 ld(const float *p) {
+    return __ldcs(reinterpret_cast<const float2 *>(p));
+  }
+  static __device__ __forceinline__ void st(float *p, float2 x) {
+    __stcs(reinterpret_cast<float2 *>(p), x);
+  }
+  static __device__ __forceinline__ float &at(float2 &x, int i) {
+    return reinterpret_cast<float *>(&x)[i];
+  }
+};
+
+template <typename T, int D, int E>
+__global__ void __launch_bounds__(NT)
+decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
+              const T *__restrict__ v, const float *__restrict__ lambda,
+              float *__restrict__ kv, T *__restrict__ o, int H) {
+  constexpr int ROWS = D / NW;   // rows per warp
+  constexpr int VEC = E / 32;    // columns per lane
+  using V = vec_t<VEC>;
+  __shared__ float qs[D], ks[D], vs[E];
+  __shared__ float red[NW][E];
+
+  const int64_t bh = blockIdx.x;
+  const int tid = threadIdx.x, w = tid / 32, l = tid % 32;
+  if (tid < D) {
+    qs[tid] = io<T>::ld(q + bh * D + tid);
+    ks[tid] = io<T>::ld(k + bh * D + tid);
+  }
+  if (tid < E) vs[tid] = io<T>::ld(v + bh * E + tid);
+  const float lam = lambda[bh % H];
+
+  float *base = kv + bh * (int64_t)D * E + (int64_t)(w * ROWS) * E + l * VEC;
+  typename V::type x[ROWS];
+#pragma unroll
+  for (int r = 0; r < ROWS; r++) x[r] = V::ld(base + (int64_t)r * E);
+  __syncthreads();
+
+  float vv[VEC], acc[VEC];
+#pragma unroll
+  for (int c = 0; c < VEC; c++) {
+    vv[c] = vs[l * VEC + c];
+    acc[c] = 0.f;
+  }
+#pragma unroll
+  for (int r = 0; r < ROWS; r++) {
+    const int i = w * ROWS + r;
+    const float ki = ks[i], qi = qs[i];
+#pragma unroll
+    for (int c = 0; c < VEC; c++) {
+      float s = fmaf(lam, V::at(x[r], c), ki * vv[c]);
+      V::at(x[r], c) = s;
+      acc[c] = fmaf(qi, s, acc[c]);
+    }
+    V::st(base + (int64_t)r * E, x[r]);
+  }
+#pragma unroll
+  for (int c = 0; c < VEC; c++) red[w][l * VEC + c] = acc[c];
+  __syncthreads();
+  if (tid < E) {
+    float s = 0.f;
+#pragma unroll
+    for (int ww = 0; ww < NW; ww++) s += red[ww][tid];
+    io<T>::st(o + bh * E + tid, s);
+  }
+}
+
+}  // namespace dec
+}  // namespace la2

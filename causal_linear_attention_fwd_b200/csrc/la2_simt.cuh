@@ -1,0 +1,397 @@
+// la2_simt.cuh -- portable fp32-FMA kernels for every supported shape.
+//
+// These kernels are the fp32 I/O path (fp32 FMA keeps the 1e-4 accuracy that
+// tf32 tensor-core products would miss) and the path for head sizes the
+// tensor-core kernels do not cover.  They follow the same block schedule as
+// the tensor-core kernels -- intra-block masked dense part plus inter-block
+// part through a carried d x e state (Lightning Attention-2 notes page,
+// "Tiling." paragraph) -- with a smaller block (C = 32 rows) and all tiles in
+// shared memory as fp32.
+//
+// Per (b,h) the sequence is cut into S chunks of Lc rows (Lc a multiple of the
+// block size); chunks run in parallel CTAs.  Chunk entry states come from a
+// pre-pass (the chunk's own state contribution, started from zero) and a
+// short scan over chunks:  KV_in[c] = lambda^Lc KV_in[c-1] + dKV[c-1].
+//
+// Block i covers rows [p, p+cb), local rows s, t in [0, cb):
+//   forward  O_i = (Q_i K_i^T (.) M) V_i + diag(lambda^(s+1)) Q_i KV
+//            KV <- lambda^cb KV + (diag(lambda^(cb-1-t)) K_i)^T V_i
+//   dQ       dQ_i = (dO_i V_i^T (.) M) K_i + diag(lambda^(s+1)) dO_i KV^T
+//   dK, dV   (reverse scan over D = sum_{t beyond the block} lambda^.. q_t^T dO_t)
+//            dK_i = (dO_i V_i^T (.) M)^T Q_i + diag(lambda^(cb-s)) V_i D^T
+//            dV_i = (Q_i K_i^T (.) M)^T dO_i + diag(lambda^(cb-s)) K_i D
+//            D <- lambda^cb D + (diag(lambda^s) Q_i)^T dO_i
+// with M[s,t] = lambda^(s-t) for t <= s.
+#pragma once
+
+#include "la2_common.cuh"
+
+namespace la2 {
+
+struct Geo {
+  int B, H;
+  int64_t L;
+  int S;        // chunks per (b,h)
+  int64_t Lc;   // rows per chunk (multiple of the block size); last may be short
+};
+
+namespace simt {
+
+constexpr int C = 32;         // block rows
+constexpr int NT = 256;       // threads per CTA
+
+template <typename T, int W>
+__device__ __forceinline__ void load_tile(float *dst, int ld, const T *src,
+                                          int cb) {
+  // rows >= cb are zero-filled
+  for (int idx = threadIdx.x; idx < C * W; idx += NT) {
+    int r = idx / W, c = idx % W;
+    dst[r * ld + c] = r < cb ? io<T>::ld(src + (int64_t)r * W + c) : 0.f;
+  }
+}
+
+__device__ __forceinline__ void fill_pow(float *pw, float lam) {
+  for (int n = threadIdx.x; n <= C; n += NT) pw[n] = (float)pow_int((double)lam, n);
+}
+
+// ------------------------------------------------------------- forward
+// OUT = true : full forward for chunk c (grid = B*H*S)
+// OUT = false: chunk-state pre-pass for chunks 0..S-2 (grid = B*H*(S-1));
+//              writes the chunk's state, started from zero, to ws slot c+1.
+template <typename T, int D, int E, bool OUT>
+__global__ void __launch_bounds__(NT)
+fwd_kernel(const T *__restrict__ q, const T *__restrict__ k,
+           const T *__restrict__ v, const float *__restrict__ lambda,
+           const float *__restrict__ kv0, T *__restrict__ o,
+           float *__restrict__ kv_out, float *__restrict__ ws, Geo g) {
+  constexpr int LDQ = D + 1, LDV = E, LDP = C + 1, LDS = E + 1;
+  extern __shared__ float sm[];
+  float *KV = sm;                     // D x (E+1)
+  float *Qs = KV + D * LDS;           // C x (D+1)
+  float *Ks = Qs + C * LDQ;           // C x (D+1)
+  float *Vs = Ks + C * LDQ;           // C x E
+  float *Ps = Vs + C * LDV;           // C x (C+1)
+  float *pw = Ps + C * LDP;           // C+1
+
+  const int nch = OUT ? g.S : g.S - 1;
+  const int64_t bh = blockIdx.x / nch;
+  const int c = blockIdx.x % nch;
+  const int h = (int)(bh % g.H);
+  const int64_t a = (int64_t)c * g.Lc;
+  const int64_t b = g.L < a + g.Lc ? g.L : a + g.Lc;
+
+  fill_pow(pw, lambda[h]);
+  const float *init = nullptr;
+  if (OUT) {
+    if (c == 0) init = kv0 ? kv0 + bh * D * E : nullptr;
+    else init = ws + (bh * g.S + c) * (int64_t)D * E;
+  }
+  for (int idx = threadIdx.x; idx < D * E; idx += NT)
+    KV[(idx / E) * LDS + idx % E] = init ? init[idx] : 0.f;
+  __syncthreads();
+
+  for (int64_t p = a; p < b; p += C) {
+    const int cb = (int)(b - p < C ? b - p : C);
+    if (OUT) load_tile<T, D>(Qs, LDQ, q + (bh * g.L + p) * D, cb);
+    load_tile<T, D>(Ks, LDQ, k + (bh * g.L + p) * D, cb);
+    load_tile<T, E>(Vs, LDV, v + (bh * g.L + p) * E, cb);
+    __syncthreads();
+    if (OUT) {
+      // P = (Q K^T) (.) M over the causal triangle
+      for (int idx = threadIdx.x; idx < C * C; idx += NT) {
+        int s = idx / C, t = idx % C;
+        float val = 0.f;
+        if (t <= s && s < cb) {
+          float acc = 0.f;
+#pragma unroll 8
+          for (int i = 0; i < D; i++) acc += Qs[s * LDQ + i] * Ks[t * LDQ + i];
+          val = acc * pw[s - t];
+        }
+        Ps[s * LDP + t] = val;
+      }
+      __syncthreads();
+      // O = P V + diag(lambda^(s+1)) Q KV
+      for (int idx = threadIdx.x; idx < C * E; idx += NT) {
+        int s = idx / E, j = idx % E;
+        if (s >= cb) continue;
+        float acc1 = 0.f, acc2 = 0.f;
+        for (int t = 0; t <= s; t++) acc1 += Ps[s * LDP + t] * Vs[t * LDV + j];
+#pragma unroll 8
+        for (int i = 0; i < D; i++) acc2 += Qs[s * LDQ + i] * KV[i * LDS + j];
+        io<T>::st(o + (bh * g.L + p + s) * E + j, acc1 + pw[s + 1] * acc2);
+      }
+      __syncthreads();
+    }
+    // KV <- lambda^cb KV + (diag(lambda^(cb-1-t)) K)^T V
+    for (int idx = threadIdx.x; idx < D * E; idx += NT) {
+      int i = idx / E, j = idx % E;
+      float acc = 0.f;
+      for (int t = 0; t < cb; t++)
+        acc += pw[cb - 1 - t] * Ks[t * LDQ + i] * Vs[t * LDV + j];
+      KV[i * LDS + j] = pw[cb] * KV[i * LDS + j] + acc;
+    }
+    __syncthreads();
+  }
+  float *dst = nullptr;
+  if (OUT) dst = (kv_out && c == g.S - 1) ? kv_out + bh * D * E : nullptr;
+  else dst = ws + (bh * g.S + c + 1) * (int64_t)D * E;
+  if (dst)
+    for (int idx = threadIdx.x; idx < D * E; idx += NT)
+      dst[idx] = KV[(idx / E) * LDS + idx % E];
+}
+
+// Forward chunk-entry scan, one thread per state element:
+// run = kv0 (or 0); for c = 1..S-1: run = lambda^Lc run + ws[c]; ws[c] = run.
+template <int D, int E>
+__global__ void __launch_bounds__(NT)
+scan_fwd_kernel(float *__restrict__ ws, const float *__restrict__ kv0,
+                const float *__restrict__ lambda, Geo g) {
+  const int64_t bh = blockIdx.y;
+  const int idx = blockIdx.x * NT + threadIdx.x;
+  if (idx >= D * E) return;
+  const float decay = (float)pow_int((double)lambda[bh % g.H], g.Lc);
+  float run = kv0 ? kv0[bh * D * E + idx] : 0.f;
+  for (int c = 1; c < g.S; c++) {
+    float *p = ws + (bh * g.S + c) * (int64_t)D * E + idx;
+    run = decay * run + *p;
+    *p = run;
+  }
+}
+
+// ------------------------------------------------------------- backward dQ
+template <typename T, int D, int E>
+__global__ void __launch_bounds__(NT)
+dq_kernel(const T *__restrict__ k, const T *__restrict__ v,
+          const T *__restrict__ dO, const float *__restrict__ lambda,
+          const float *__restrict__ kv0, T *__restrict__ dq,
+          const float *__restrict__ ws, Geo g) {
+  constexpr int LDS = E + 1, LDG = E + 1, LDK = D, LDP = C + 1;
+  extern __shared__ float sm[];
+  float *KV = sm;                 // D x (E+1)
+  float *Gs = KV + D * LDS;       // C x (E+1)   dO
+  float *Vs = Gs + C * LDG;       // C x (E+1)
+  float *Ks = Vs + C * LDG;       // C x D
+  float *Ps = Ks + C * LDK;       // C x (C+1)
+  float *pw = Ps + C * LDP;
+
+  const int64_t bh = blockIdx.x / g.S;
+  const int c = blockIdx.x % g.S;
+  const int h = (int)(bh % g.H);
+  const int64_t a = (int64_t)c * g.Lc;
+  const int64_t b = g.L < a + g.Lc ? g.L : a + g.Lc;
+  fill_pow(pw, lambda[h]);
+  const float *init = c == 0 ? (kv0 ? kv0 + bh * D * E : nullptr)
+                             : ws + (bh * g.S + c) * (int64_t)D * E;
+  for (int idx = threadIdx.x; idx < D * E; idx += NT)
+    KV[(idx / E) * LDS + idx % E] = init ? init[idx] : 0.f;
+  __syncthreads();
+
+  for (int64_t p = a; p < b; p += C) {
+    const int cb = (int)(b - p < C ? b - p : C);
+    load_tile<T, E>(Gs, LDG, dO + (bh * g.L + p) * E, cb);
+    load_tile<T, E>(Vs, LDG, v + (bh * g.L + p) * E, cb);
+    load_tile<T, D>(Ks, LDK, k + (bh * g.L + p) * D, cb);
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < C * C; idx += NT) {
+      int s = idx / C, t = idx % C;
+      float val = 0.f;
+      if (t <= s && s < cb) {
+        float acc = 0.f;
+#pragma unroll 8
+        for (int j = 0; j < E; j++) acc += Gs[s * LDG + j] * Vs[t * LDG + j];
+        val = acc * pw[s - t];
+      }
+      Ps[s * LDP + t] = val;
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < C * D; idx += NT) {
+      int s = idx / D, i = idx % D;
+      if (s >= cb) continue;
+      float acc1 = 0.f, acc2 = 0.f;
+      for (int t = 0; t <= s; t++) acc1 += Ps[s * LDP + t] * Ks[t * LDK + i];
+#pragma unroll 8
+      for (int j = 0; j < E; j++) acc2 += Gs[s * LDG + j] * KV[i * LDS + j];
+      io<T>::st(dq + (bh * g.L + p + s) * D + i, acc1 + pw[s + 1] * acc2);
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < D * E; idx += NT) {
+      int i = idx / E, j = idx % E;
+      float acc = 0.f;
+      for (int t = 0; t < cb; t++)
+        acc += pw[cb - 1 - t] * Ks[t * LDK + i] * Vs[t * LDG + j];
+      KV[i * LDS + j] = pw[cb] * KV[i * LDS + j] + acc;
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------ backward dK, dV
+// Reverse chunk states: for chunks c = 1..S-1 (grid B*H*(S-1)) the chunk's own
+// contribution to the reverse state at its first row,
+//   dD[c] = sum_{t in chunk c} lambda^(t - a_c) q_t^T dO_t,
+// written to ws slot c-1.
+template <typename T, int D, int E>
+__global__ void __launch_bounds__(NT)
+rev_state_kernel(const T *__restrict__ q, const T *__restrict__ dO,
+                 const float *__restrict__ lambda, float *__restrict__ ws, Geo g) {
+  constexpr int LDQ = D, LDG = E;
+  extern __shared__ float sm[];
+  float *Dst = sm;               // D x E
+  float *Qs = Dst + D * E;       // C x D
+  float *Gs = Qs + C * LDQ;      // C x E
+  float *pw = Gs + C * LDG;
+
+  const int nch = g.S - 1;
+  const int64_t bh = blockIdx.x / nch;
+  const int c = 1 + blockIdx.x % nch;
+  const int h = (int)(bh % g.H);
+  const int64_t a = (int64_t)c * g.Lc;
+  const int64_t b = g.L < a + g.Lc ? g.L : a + g.Lc;
+  fill_pow(pw, lambda[h]);
+  for (int idx = threadIdx.x; idx < D * E; idx += NT) Dst[idx] = 0.f;
+  __syncthreads();
+  const int64_t nb = (b - a + C - 1) / C;
+  for (int64_t ib = nb - 1; ib >= 0; ib--) {
+    const int64_t p = a + ib * C;
+    const int cb = (int)(b - p < C ? b - p : C);
+    load_tile<T, D>(Qs, LDQ, q + (bh * g.L + p) * D, cb);
+    load_tile<T, E>(Gs, LDG, dO + (bh * g.L + p) * E, cb);
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < D * E; idx += NT) {
+      int i = idx / E, j = idx % E;
+      float acc = 0.f;
+      for (int s = 0; s < cb; s++) acc += pw[s] * Qs[s * LDQ + i] * Gs[s * LDG + j];
+      Dst[idx] = pw[cb] * Dst[idx] + acc;
+    }
+    __syncthreads();
+  }
+  float *dst = ws + (bh * g.S + c - 1) * (int64_t)D * E;
+  for (int idx = threadIdx.x; idx < D * E; idx += NT) dst[idx] = Dst[idx];
+}
+
+// Reverse scan: run = 0; for c = S-2..0: run = lambda^len(c+1) run + ws[c];
+// ws[c] = run.  Afterwards ws[c] is the reverse state entering chunk c from
+// the right (the state at its last row + 1).
+template <int D, int E>
+__global__ void __launch_bounds__(NT)
+scan_rev_kernel(float *__restrict__ ws, const float *__restrict__ lambda, Geo g) {
+  const int64_t bh = blockIdx.y;
+  const int idx = blockIdx.x * NT + threadIdx.x;
+  if (idx >= D * E) return;
+  const double lam = (double)lambda[bh % g.H];
+  const float full = (float)pow_int(lam, g.Lc);
+  const float last = (float)pow_int(lam, g.L - (int64_t)(g.S - 1) * g.Lc);
+  float run = 0.f;
+  for (int c = g.S - 2; c >= 0; c--) {
+    float *p = ws + (bh * g.S + c) * (int64_t)D * E + idx;
+    run = (c + 1 == g.S - 1 ? last : full) * run + *p;
+    *p = run;
+  }
+}
+
+template <typename T, int D, int E>
+__global__ void __launch_bounds__(NT)
+dkdv_kernel(const T *__restrict__ q, const T *__restrict__ k,
+            const T *__restrict__ v, const T *__restrict__ dO,
+            const float *__restrict__ lambda, T *__restrict__ dk,
+            T *__restrict__ dv, float *__restrict__ dkv0,
+            const float *__restrict__ ws, Geo g) {
+  constexpr int LDQ = D + 1, LDG = E + 1, LDS = E + 1, LDP = C + 1;
+  extern __shared__ float sm[];
+  float *Dst = sm;                 // D x (E+1)
+  float *Qs = Dst + D * LDS;       // C x (D+1)
+  float *Ks = Qs + C * LDQ;        // C x (D+1)
+  float *Vs = Ks + C * LDQ;        // C x (E+1)
+  float *Gs = Vs + C * LDG;        // C x (E+1)
+  float *Pt = Gs + C * LDG;        // C x (C+1)  (Q K^T (.) M)^T
+  float *dPt = Pt + C * LDP;       // C x (C+1)  (dO V^T (.) M)^T
+  float *pw = dPt + C * LDP;
+
+  const int64_t bh = blockIdx.x / g.S;
+  const int c = blockIdx.x % g.S;
+  const int h = (int)(bh % g.H);
+  const int64_t a = (int64_t)c * g.Lc;
+  const int64_t b = g.L < a + g.Lc ? g.L : a + g.Lc;
+  fill_pow(pw, lambda[h]);
+  const float *init = c == g.S - 1 ? nullptr : ws + (bh * g.S + c) * (int64_t)D * E;
+  for (int idx = threadIdx.x; idx < D * E; idx += NT)
+    Dst[(idx / E) * LDS + idx % E] = init ? init[idx] : 0.f;
+  __syncthreads();
+
+  const int64_t nb = (b - a + C - 1) / C;
+  for (int64_t ib = nb - 1; ib >= 0; ib--) {
+    const int64_t p = a + ib * C;
+    const int cb = (int)(b - p < C ? b - p : C);
+    load_tile<T, D>(Qs, LDQ, q + (bh * g.L + p) * D, cb);
+    load_tile<T, D>(Ks, LDQ, k + (bh * g.L + p) * D, cb);
+    load_tile<T, E>(Vs, LDG, v + (bh * g.L + p) * E, cb);
+    load_tile<T, E>(Gs, LDG, dO + (bh * g.L + p) * E, cb);
+    __syncthreads();
+    // transposed masked products, [t][s] with s >= t
+    for (int idx = threadIdx.x; idx < C * C; idx += NT) {
+      int t = idx / C, s = idx % C;
+      float pv = 0.f, dpv = 0.f;
+      if (s >= t && s < cb) {
+        float a1 = 0.f, a2 = 0.f;
+#pragma unroll 8
+        for (int i = 0; i < D; i++) a1 += Qs[s * LDQ + i] * Ks[t * LDQ + i];
+#pragma unroll 8
+        for (int j = 0; j < E; j++) a2 += Gs[s * LDG + j] * Vs[t * LDG + j];
+        pv = a1 * pw[s - t];
+        dpv = a2 * pw[s - t];
+      }
+      Pt[t * LDP + s] = pv;
+      dPt[t * LDP + s] = dpv;
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < C * D; idx += NT) {
+      int t = idx / D, i = idx % D;
+      if (t >= cb) continue;
+      float acc1 = 0.f, acc2 = 0.f;
+      for (int s = t; s < cb; s++) acc1 += dPt[t * LDP + s] * Qs[s * LDQ + i];
+#pragma unroll 8
+      for (int j = 0; j < E; j++) acc2 += Vs[t * LDG + j] * Dst[i * LDS + j];
+      io<T>::st(dk + (bh * g.L + p + t) * D + i, acc1 + pw[cb - t] * acc2);
+    }
+    for (int idx = threadIdx.x; idx < C * E; idx += NT) {
+      int t = idx / E, j = idx % E;
+      if (t >= cb) continue;
+      float acc1 = 0.f, acc2 = 0.f;
+      for (int s = t; s < cb; s++) acc1 += Pt[t * LDP + s] * Gs[s * LDG + j];
+#pragma unroll 8
+      for (int i = 0; i < D; i++) acc2 += Ks[t * LDQ + i] * Dst[i * LDS + j];
+      io<T>::st(dv + (bh * g.L + p + t) * E + j, acc1 + pw[cb - t] * acc2);
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < D * E; idx += NT) {
+      int i = idx / E, j = idx % E;
+      float acc = 0.f;
+      for (int s = 0; s < cb; s++) acc += pw[s] * Qs[s * LDQ + i] * Gs[s * LDG + j];
+      Dst[i * LDS + j] = pw[cb] * Dst[i * LDS + j] + acc;
+    }
+    __syncthreads();
+  }
+  if (c == 0 && dkv0) {
+    const float lam = lambda[h];
+    for (int idx = threadIdx.x; idx < D * E; idx += NT)
+      dkv0[bh * D * E + idx] = lam * Dst[(idx / E) * LDS + idx % E];
+  }
+}
+
+// Shared-memory bytes of each kernel (must match the carve-ups above).
+template <int D, int E> constexpr size_t fwd_smem() {
+  return sizeof(float) * (D * (E + 1) + 2 * C * (D + 1) + C * E + C * (C + 1) + C + 1);
+}
+template <int D, int E> constexpr size_t dq_smem() {
+  return sizeof(float) * (D * (E + 1) + 2 * C * (E + 1) + C * D + C * (C + 1) + C + 1);
+}
+template <int D, int E> constexpr size_t rev_smem() {
+  return sizeof(float) * (D * E + C * D + C * E + C + 1);
+}
+template <int D, int E> constexpr size_t dkdv_smem() {
+  return sizeof(float) * (D * (E + 1) + 2 * C * (D + 1) + 2 * C * (E + 1) +
+                          2 * C * (C + 1) + C + 1);
+}
+
+}  // namespace simt
+}  // namespace la2

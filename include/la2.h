@@ -1,0 +1,175 @@
+/*
+ * la2.h -- C ABI of libla2: tiled causal linear attention with per-head decay
+ * (the Lightning Attention-2 schedule) for NVIDIA B200 (sm_100a).
+ *
+ * The operation, per batch b and head h (rows t, j = 0..L-1):
+ *
+ *     o_t = sum_{j <= t} lambda_h^(t-j) (q_t . k_j) v_j  +  lambda_h^(t+1) q_t kv0
+ *
+ * i.e. O = (Q K^T (.) M) V with M_tj = lambda_h^(t-j) for j <= t and 0 above
+ * the diagonal; lambda_h = 1 is plain causal linear attention.  The
+ * Lightning Attention-2 notes page (phantomic12.github.io, "Lightning
+ * Attention-2: A Free Lunch for Handling Unlimited Sequence Lengths in Large
+ * Language Models", "Tiling." paragraph) describes the schedule used here: an
+ * intra-block part done as ordinary dense masked attention and an inter-block
+ * part done through the linear-attention state, in forward and backward.  The
+ * Lightning Attention glossary page (jisaku.com, section "主な特徴・仕組み")
+ * gives the two equivalent forms -- parallel for training, recurrent with a
+ * fixed-size state for inference -- that la2_forward/la2_backward and
+ * la2_decode_step implement.  The decay lambda_h, the fp32 state and the
+ * argument conventions below are this library's definition; the pages give
+ * none of them.
+ *
+ * Conventions common to every call
+ *   - All tensor pointers are DEVICE pointers, contiguous row-major:
+ *       q, k, dq, dk      [B, H, L, d]
+ *       v, o, dO, dv      [B, H, L, e]
+ *       states            [B, H, d, e]  fp32 (kv0, kv_out, dkv0, decode kv)
+ *       lambda            [H]           fp32, one decay per head
+ *     `dt` (LA2_F32 or LA2_BF16) is the element type of q, k, v, o, dO, dq,
+ *     dk, dv.  Arithmetic is fp32 (bf16 tensor-core products with fp32
+ *     accumulation for LA2_BF16; fp32 FMA for LA2_F32).
+ *   - Supported head sizes: d, e in {64, 128}.
+ *   - Every pointer must be 16-byte aligned.
+ *   - The caller owns all memory.  The library allocates nothing on the
+ *     device: scratch memory comes from the caller as `workspace`, sized by
+ *     la2_workspace_size() for the same arguments.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and never synchronised: results are ready when the stream is.
+ *   - Arguments are validated before anything is launched.  A call that
+ *     returns an error has enqueued nothing.
+ *   - lambda values are read on the device; any finite value is accepted,
+ *     values in [0, 1] are the meaningful range (0^0 is taken as 1).
+ *   - L, B or H equal to 0 is an empty problem: nothing is computed except
+ *     that state outputs are still written (kv_out = kv0 or 0; dkv0 = 0).
+ *
+ * Errors: LA2_ERR_INVALID for bad arguments (null required pointer, negative
+ * size, unaligned pointer, an output overlapping an input, kv_out == kv0,
+ * workspace too small); LA2_ERR_UNSUPPORTED for (d, e, dt) outside the
+ * supported set; LA2_ERR_CUDA when a launch fails; device-side watchdog
+ * expiries are reported later by la2_last_device_error().
+ */
+#ifndef LA2_H
+#define LA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#ifndef __CUDA_RUNTIME_API_H__
+typedef struct CUstream_st *cudaStream_t;
+#endif
+
+typedef enum {
+    LA2_OK = 0,
+    LA2_ERR_INVALID = 1,
+    LA2_ERR_UNSUPPORTED = 2,
+    LA2_ERR_CUDA = 3,
+    LA2_ERR_TIMEOUT = 4
+} la2_status;
+
+typedef enum { LA2_F32 = 0, LA2_BF16 = 1 } la2_dtype;
+
+/* Operation codes for la2_workspace_size(). */
+enum { LA2_OP_FORWARD = 0, LA2_OP_BACKWARD = 1 };
+
+/*
+ * Bytes of device scratch that la2_forward (op = LA2_OP_FORWARD) or
+ * la2_backward (op = LA2_OP_BACKWARD) needs for these sizes on the CURRENT
+ * device.  The scratch holds the fp32 d x e states at the boundaries of the
+ * sequence chunks that run in parallel (the split of one long sequence over
+ * several CTAs); it may be 0 when the sequence is not split.  Returns 0 for
+ * unsupported arguments as well; the call then reports the error.
+ */
+size_t la2_workspace_size(int op, int B, int H, int64_t L, int d, int e,
+                          la2_dtype dt);
+
+/*
+ * Forward pass.  Writes o [B,H,L,e] and, when kv_out is not NULL, the state
+ * after the last row, kv_out = lambda^L kv0 + sum_j lambda^(L-1-j) k_j^T v_j
+ * (fp32 [B,H,d,e]), which la2_decode_step or a later la2_forward (as kv0) can
+ * continue from.  kv0 may be NULL (zero initial state).
+ * Source: Lightning Attention-2 notes page, "Tiling." paragraph (intra-block
+ * dense part + inter-block state part); glossary page, FAQ Q1 (aggregate
+ * K^T V first, then multiply by Q).
+ */
+la2_status la2_forward(const void *q, const void *k, const void *v,
+                       const float *lambda, const float *kv0,
+                       void *o, float *kv_out,
+                       int B, int H, int64_t L, int d, int e, la2_dtype dt,
+                       void *workspace, size_t workspace_bytes,
+                       cudaStream_t stream);
+
+/*
+ * Backward pass for an upstream gradient dO [B,H,L,e]: writes dq, dk [B,H,L,d],
+ * dv [B,H,L,e] -- the gradients of sum(o * dO) -- and, when dkv0 is not NULL,
+ * the gradient with respect to the initial state (fp32 [B,H,d,e]).  Inputs
+ * are those of the forward call (kv0 may be NULL).  dq is found by a forward
+ * scan that rebuilds the state; dk and dv by a reverse scan over a second
+ * d x e state.
+ * Source: Lightning Attention-2 notes page, "Tiling." paragraph (the same
+ * tiling applied in the backward pass).
+ */
+la2_status la2_backward(const void *q, const void *k, const void *v,
+                        const float *lambda, const float *kv0, const void *dO,
+                        void *dq, void *dk, void *dv, float *dkv0,
+                        int B, int H, int64_t L, int d, int e, la2_dtype dt,
+                        void *workspace, size_t workspace_bytes,
+                        cudaStream_t stream);
+
+/*
+ * One recurrent decode step for one new token per (b,h):
+ *     kv <- lambda kv + k^T v,    o = q kv
+ * q, k [B,H,d], v, o [B,H,e] of type dt; kv fp32 [B,H,d,e] updated IN PLACE
+ * (the constant-size state; it does not grow with the number of steps).  The
+ * updated state includes the current token, matching M_tt = 1.
+ * Source: glossary page, section "主な特徴・仕組み" (recurrent inference with
+ * a fixed-size state; KV cache constant regardless of length).
+ */
+la2_status la2_decode_step(const void *q, const void *k, const void *v,
+                           const float *lambda, float *kv, void *o,
+                           int B, int H, int d, int e, la2_dtype dt,
+                           cudaStream_t stream);
+
+/*
+ * Synchronises `stream`, then reports and clears the device error word that
+ * the kernels' bounded waits set when a wait gives up (LA2_ERR_TIMEOUT), or
+ * LA2_ERR_CUDA if the synchronisation itself fails.  LA2_OK otherwise.
+ */
+la2_status la2_last_device_error(cudaStream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char *la2_status_string(la2_status s);
+
+/*
+ * Process-wide tuning overrides (for tests and sweeps; not thread-safe with
+ * concurrent calls).  LA2_OPT_SPLIT: number of chunks each (b,h) sequence is
+ * split into (0 = automatic).  LA2_OPT_PATH: 0 = automatic, 1 = force the
+ * portable fp32-FMA kernels, 2 = require the tensor-core kernels (calls whose
+ * shape they do not cover return LA2_ERR_UNSUPPORTED).  Returns the previous
+ * value, or -1 for an unknown option.
+ */
+enum { LA2_OPT_SPLIT = 0, LA2_OPT_PATH = 1 };
+int la2_set_option(int option, int value);
+
+/*
+ * Per-kernel device timing.  While enabled, every kernel the library
+ * launches is bracketed by a pair of CUDA events on its stream.
+ * la2_profile_report() synchronises on those events and writes a JSON object
+ * {"<kernel>": {"launches": n, "ms": total}, ...} into buf (truncated to
+ * buf_bytes), clears the records and returns the number of bytes needed.
+ */
+void la2_profile_enable(int on);
+size_t la2_profile_report(char *buf, size_t buf_bytes);
+
+/* Library version string, e.g. "la2 0.1 sm_100a". */
+const char *la2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LA2_H */

@@ -1,0 +1,144 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/la2.h declares, and rejects bad arguments before
+touching the device.  Pointers here are fake addresses that are never
+dereferenced: every case returns during validation."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import causal_linear_attention_fwd_b200 as la2
+from causal_linear_attention_fwd_b200 import _binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(la2_\w+)\s*\(", src))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import __graft_entry__
+    __graft_entry__.build()
+    return la2.library()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert {"la2_forward", "la2_backward", "la2_decode_step",
+            "la2_workspace_size"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), f"libla2.so does not export {n}"
+
+
+def test_status_strings(lib):
+    for code, name in enumerate(["LA2_OK", "LA2_ERR_INVALID", "LA2_ERR_UNSUPPORTED",
+                                 "LA2_ERR_CUDA", "LA2_ERR_TIMEOUT"]):
+        assert la2.status_string(code) == name
+
+
+def test_set_option_roundtrip(lib):
+    old = la2.set_option(la2.LA2_OPT_SPLIT, 5)
+    assert la2.set_option(la2.LA2_OPT_SPLIT, old) == 5
+    assert la2.set_option(99, 1) == -1
+
+
+# fake, 16-byte aligned, non-overlapping device addresses
+MB = 1 << 20
+Q, K, V, O, LAM, KV0, KVO, WS, DO, DQ, DK, DV, DKV = [(i + 1) * 64 * MB for i in range(13)]
+
+
+def fwd(lib, q=Q, k=K, v=V, lam=LAM, kv0=None, o=O, kvo=None, Bn=1, H=2, L=100, d=64, e=64,
+        dt=B.LA2_BF16, ws=None, wsb=0):
+    return lib.la2_forward(q, k, v, lam, kv0, o, kvo, Bn, H, L, d, e, dt, ws, wsb, None)
+
+
+def bwd(lib, q=Q, k=K, v=V, lam=LAM, kv0=None, dO=DO, dq=DQ, dk=DK, dv=DV, dkv=None, Bn=1, H=2,
+        L=100, d=64, e=64, dt=B.LA2_BF16, ws=None, wsb=0):
+    return lib.la2_backward(q, k, v, lam, kv0, dO, dq, dk, dv, dkv, Bn, H, L, d, e, dt, ws, wsb,
+                            None)
+
+
+def test_forward_validation(lib):
+    INV, UNS = B.LA2_ERR_INVALID, B.LA2_ERR_UNSUPPORTED
+    assert fwd(lib, q=None) == INV
+    assert fwd(lib, o=None) == INV
+    assert fwd(lib, lam=None) == INV
+    assert fwd(lib, Bn=-1) == INV
+    assert fwd(lib, L=-5) == INV
+    assert fwd(lib, d=96) == UNS
+    assert fwd(lib, e=32) == UNS
+    assert fwd(lib, dt=7) == UNS
+    assert fwd(lib, q=Q + 8) == INV                 # not 16-byte aligned
+    assert fwd(lib, kv0=KV0, kvo=KV0) == INV         # kv_out == kv0
+    assert fwd(lib, o=Q + 64) == INV                 # o overlaps q
+    assert fwd(lib, kvo=V + 1024) == INV             # kv_out overlaps v
+    assert fwd(lib, Bn=0) == B.LA2_OK                # empty batch: nothing to do
+    assert fwd(lib, H=0) == B.LA2_OK
+
+
+def test_backward_validation(lib):
+    INV, UNS = B.LA2_ERR_INVALID, B.LA2_ERR_UNSUPPORTED
+    assert bwd(lib, dO=None) == INV
+    assert bwd(lib, dq=None) == INV
+    assert bwd(lib, dk=DQ) == INV                    # two outputs at one address
+    assert bwd(lib, dv=DO) == INV                    # output aliases an input
+    assert bwd(lib, dkv=DQ + 16) == INV              # dkv0 inside dq
+    assert bwd(lib, d=128, e=96) == UNS
+    assert bwd(lib, H=-1) == INV
+    assert bwd(lib, Bn=0) == B.LA2_OK
+
+
+def test_decode_validation(lib):
+    INV = B.LA2_ERR_INVALID
+    f = lib.la2_decode_step
+    assert f(None, K, V, LAM, KV0, O, 2, 2, 64, 64, B.LA2_BF16, None) == INV
+    assert f(Q, K, V, LAM, KV0, KV0 + 16, 2, 2, 64, 64, B.LA2_BF16, None) == INV
+    assert f(Q, K, V, LAM, KV0 + 4, O, 2, 2, 64, 64, B.LA2_BF16, None) == INV
+    assert f(Q, K, V, LAM, KV0, O, 2, 2, 64, 80, B.LA2_BF16, None) == B.LA2_ERR_UNSUPPORTED
+    assert f(Q, K, V, LAM, KV0, O, 0, 2, 64, 64, B.LA2_BF16, None) == B.LA2_OK
+
+
+def test_workspace_rules(lib):
+    # a long sequence with few (b,h) pairs is split, so scratch is needed ...
+    need = lib.la2_workspace_size(B.LA2_OP_FORWARD, 1, 2, 1 << 16, 64, 64, B.LA2_BF16)
+    assert need > 0 and need % (64 * 64 * 4) == 0
+    bneed = lib.la2_workspace_size(B.LA2_OP_BACKWARD, 1, 2, 1 << 16, 64, 64, B.LA2_BF16)
+    assert bneed == 2 * need
+    # ... and a call that brings too little is rejected before any launch
+    assert fwd(lib, L=1 << 16, ws=WS, wsb=need - 1) == B.LA2_ERR_INVALID
+    assert fwd(lib, L=1 << 16, ws=None, wsb=0) == B.LA2_ERR_INVALID
+    # invalid arguments size to 0
+    assert lib.la2_workspace_size(B.LA2_OP_FORWARD, 1, 2, 100, 64, 96, B.LA2_BF16) == 0
+    assert lib.la2_workspace_size(7, 1, 2, 100, 64, 64, B.LA2_BF16) == 0
+
+
+def test_forced_split_sizes_workspace(lib):
+    old = la2.set_option(la2.LA2_OPT_SPLIT, 4)
+    try:
+        n = lib.la2_workspace_size(B.LA2_OP_FORWARD, 2, 3, 1000, 64, 128, B.LA2_F32)
+        assert n == 2 * 3 * 4 * 64 * 128 * 4
+        la2.set_option(la2.LA2_OPT_SPLIT, 1)
+        assert lib.la2_workspace_size(B.LA2_OP_FORWARD, 2, 3, 1000, 64, 128, B.LA2_F32) == 0
+    finally:
+        la2.set_option(la2.LA2_OPT_SPLIT, old)
+
+
+def test_product_path_does_not_reference_oracle():
+    """The package never imports or loads the oracle."""
+    pkg = os.path.join(ROOT, "causal_linear_attention_fwd_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(dirpath, f)).read()
+                for pat in (r"^\s*import\s+oracle", r"^\s*from\s+oracle", r"la2_oracle",
+                            r"oracle\.(load|build|Oracle)"):
+                    assert not re.search(pat, src, flags=re.M), f"{f} reaches the oracle ({pat})"
