@@ -177,34 +177,41 @@ def traffic_for(kernel: str, units: int):
     return k["dram_bytes_per_token_head"] * units
 
 
-def cpu_baseline(x, lam, budget_s=12.0):
+def cpu_baseline(x, lam, target_s=30.0):
     """The fp64 oracle (as it stands) on host cores on a bounded sample of the
-    sweep workload: whole (b,h) problems of the L=4096 point, fwd+bwd."""
+    sweep workload: whole (b,h) sequences of the L=4096 sweep point, fwd+bwd
+    (all 512 of them -- the whole sweep point -- when that fits in about
+    `target_s` seconds, else as many as do)."""
     import oracle
     orc = oracle.load()
     xs = sweep_views(x, 16, 4096)
     lam_h = lam.double().cpu().numpy()
     threads = orc.num_threads()
-    heads_total = 16 * H
-    nh = min(heads_total, max(1, threads))
-    host = {}
-    elapsed = 0.0
-    while True:
-        flat = {n: t.view(16 * H, 4096, t.shape[-1])[:nh].float().cpu().numpy()[None]
+    total = 16 * H
+
+    def run(nh):
+        flat = {n: t.view(total, 4096, t.shape[-1])[:nh].float().cpu().numpy()[None]
                 for n, t in xs.items()}
         lh = np.array([lam_h[i % H] for i in range(nh)])
         t0 = time.perf_counter()
         orc.forward(flat["q"], flat["k"], flat["v"], lh)
         orc.backward(flat["q"], flat["k"], flat["v"], lh, flat["dO"])
-        elapsed = time.perf_counter() - t0
-        if elapsed >= budget_s / 4 or nh >= heads_total:
-            break
-        nh = min(heads_total, nh * max(2, int(math.ceil(budget_s / 2 / max(elapsed, 1e-3)))))
+        return time.perf_counter() - t0
+
+    nh = min(total, max(1, threads))
+    probe = run(nh)
+    per_wave = probe  # one head per thread
+    waves_fit = max(1, int(target_s / max(per_wave, 1e-6)))
+    nh2 = min(total, waves_fit * max(1, threads))
+    if nh2 > nh:
+        nh, elapsed = nh2, run(nh2)
+    else:
+        elapsed = probe
     token_heads = nh * 4096
     return {"value": token_heads / H / elapsed, "unit": "tokens/s", "cores": threads,
             "kind": "oracle",
-            "sample": f"fwd+bwd of {nh} whole (b,h) sequences of the L=4096 sweep point "
-                      f"({token_heads} token-heads; tokens/s counts 32 heads per token) "
+            "sample": f"fwd+bwd of {nh} of the 512 whole (b,h) sequences of the L=4096 sweep "
+                      f"point ({token_heads} token-heads; tokens/s counts 32 heads per token) "
                       f"in {elapsed:.2f} s"}
 
 
@@ -408,7 +415,15 @@ def main():
     ap.add_argument("--impl", default="la2", choices=["la2", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--only", default=None,
+                    help="B:L -- time a single sweep point instead of the whole sweep "
+                         "(profiling aid; not the metric)")
     args = ap.parse_args()
+    if args.only:
+        global SWEEP
+        b_, l_ = (int(x) for x in args.only.split(":"))
+        assert b_ * l_ == TOKENS, "--only must keep 65,536 tokens per batch"
+        SWEEP = [(b_, l_)]
     args.warmup = max(args.warmup, 3) if args.impl == "la2" else args.warmup
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))

@@ -389,7 +389,8 @@ la2_status la2_backward(const void *q, const void *k, const void *v,
     err = la2::tc::backward(q, k, v, lambda, kv0, dO, dq, dk, dv, dkv0, ws, g, stream,
                             [&](int which, auto &&fn) {
                               static const int ids[] = {K_TC_FWD_STATE, K_SCAN_FWD, K_TC_DQ,
-                                                        K_TC_REV_STATE, K_SCAN_REV, K_TC_DKDV};
+                                                        K_SIMT_REV_STATE, K_SIMT_REV_SCAN,
+                                                        K_SIMT_DKDV};
                               return timed(ids[which], stream, fn);
                             });
   } else if (dt == LA2_F32) {

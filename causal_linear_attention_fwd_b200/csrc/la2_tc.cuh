@@ -1,31 +1,526 @@
-// la2_tc.cuh -- tensor-core (tcgen05 / TMEM / TMA) kernels for bf16, d = e = 128.
+// la2_tc.cuh -- tensor-core kernels (tcgen05 + TMEM + TMA) for bf16, d = e = 128.
+//
+// One CTA owns one chunk of one (b,h) sequence and walks its blocks of
+// C = 128 rows in order, keeping the d x e state on chip (fp32 in TMEM) the
+// whole way -- the intra-block / inter-block split of the Lightning
+// Attention-2 notes page ("Tiling." paragraph), re-derived for sm_100a:
+//
+//   S  = A0 B1^T                 (QK^T; dQ pass: dO V^T)        -> TMEM S
+//   X  = A0 KV                   (state term; dQ pass: dO KV^T)  -> TMEM X
+//   P  = S (.) M  (bf16)         written back into TMEM over S   (CUDA cores)
+//   Y  = P B2                    (A operand read from TMEM)      -> TMEM Y
+//   B1 <- diag(lambda^(cb-1-t)) B1   in place in shared memory    (CUDA cores)
+//   KV <- lambda^cb KV + Kb^T V  (accumulated in TMEM)
+//   O  = Y + diag(lambda^(s+1)) X   -> bf16 -> shared -> TMA store
+//
+// with M[s,t] = lambda^(s-t) for t <= s.  The forward pass uses
+// (A0, B1, B2) = (Q, K, V); the dQ pass of the backward uses (dO, V, K): the
+// same schedule with K and V exchanging roles and the state transposed.  The
+// chunk-state pre-pass (MODE_STATE) runs only the state recurrence over K, V
+// from a zero state and writes the chunk's state to the workspace.
+//
+// Data path: TMA (128-byte swizzle, two 64-column boxes per 128 x 128 tile)
+// double-buffers the next block's tiles while the current one is processed;
+// every MMA is M = 128, N = 128, K = 16 steps issued by one thread;
+// completion is signalled through mbarriers, and every wait is bounded (see
+// la2_sm100.cuh).  TMEM: S [0,128), X [128,256), Y [256,384), KV [384,512).
 #pragma once
+
+#include <cuda.h>
 
 #include "la2_common.cuh"
 #include "la2_simt.cuh"
+#include "la2_sm100.cuh"
 
 namespace la2 {
 namespace tc {
 
-constexpr int BLOCK = 128;
+constexpr int BLOCK = 128;       // rows per block (MMA M)
+constexpr int NT = 256;          // 8 warps: (lane quarter) x (column half)
+constexpr uint32_t BOX = 16384;  // 128 rows x 64 bf16 (one TMA box)
+constexpr uint32_t TILE = 32768; // 128 rows x 128 bf16
 
-inline bool supports(int d, int e, bool bf16) { return false && bf16 && d == 128 && e == 128; }
+enum { MODE_FWD = 0, MODE_DQ = 1, MODE_STATE = 2 };
 
+template <int MODE> struct Layout {
+  static constexpr bool OUT = MODE != MODE_STATE;
+  static constexpr int NSTAGE = OUT ? 2 : 3;
+  static constexpr uint32_t STAGE = OUT ? 3 * TILE : 2 * TILE;
+  static constexpr uint32_t KVBF = NSTAGE * STAGE;
+  static constexpr uint32_t MISC = KVBF + (OUT ? TILE : 0);
+  static constexpr uint32_t MISC_BYTES = 8 * (NSTAGE + 1) + 16 + 4 * (BLOCK + 1);
+  static constexpr uint32_t SMEM = MISC + MISC_BYTES + 1024;  // + alignment slack
+  static constexpr uint32_t TMEM_COLS = OUT ? 512 : 128;
+  static constexpr uint32_t COL_S = 0, COL_X = 128, COL_Y = 256;
+  static constexpr uint32_t COL_KV = OUT ? 384 : 0;
+};
+
+inline bool supports(int d, int e, bool bf16) { return bf16 && d == 128 && e == 128; }
+
+// Chunks per (b,h): enough CTAs (one per SM at most, they use all of TMEM)
+// to cover every SM once when B*H alone does not.
 inline int64_t auto_split(int64_t BH, int64_t nblk, int sms) {
-  return BH >= sms ? 1 : (sms + BH - 1) / BH;
+  if (BH >= sms) return 1;
+  return (sms + BH - 1) / BH;
 }
 
-template <typename Timed>
-cudaError_t forward(const void *, const void *, const void *, const float *, const float *,
-                    void *, float *, float *, const Geo &, cudaStream_t, Timed &&) {
-  return cudaErrorNotSupported;
+using namespace la2::sm100;
+
+// Write 32 fp32 values as bf16 into row `row`, logical 16-byte chunks
+// [chunk0, chunk0+4) of a 128-byte-swizzled [rows][64] box at `box`.
+__device__ __forceinline__ void st_row_bf16_sw128(uint8_t *box, int row, int chunk0,
+                                                  const float *v) {
+#pragma unroll
+  for (int q = 0; q < 4; q++) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    const int chunk = chunk0 + q;
+    *reinterpret_cast<uint4 *>(box + row * 128 + ((chunk ^ (row & 7)) << 4)) = w;
+  }
 }
 
+// Multiply one 64-element row of a swizzled box by f, in place.
+__device__ __forceinline__ void scale_row_sw128(uint8_t *box, int row, float f) {
+#pragma unroll
+  for (int c = 0; c < 8; c++) {
+    uint4 *p = reinterpret_cast<uint4 *>(box + row * 128 + ((c ^ (row & 7)) << 4));
+    uint4 w = *p;
+    uint32_t *u = reinterpret_cast<uint32_t *>(&w);
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162 *>(&u[j]);
+      float2 f2 = __bfloat1622float2(x);
+      u[j] = pack_bf16x2(f2.x * f, f2.y * f);
+    }
+    *p = w;
+  }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(NT, 1)
+chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
+             const __grid_constant__ CUtensorMap tm2, const __grid_constant__ CUtensorMap tmo,
+             const float *__restrict__ lambda, const float *__restrict__ kv0,
+             float *__restrict__ ws, float *__restrict__ kv_out, Geo g) {
+  using LY = Layout<MODE>;
+  constexpr bool OUT = LY::OUT;
+  constexpr int NS = LY::NSTAGE;
+  constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
+  constexpr uint32_t IDESC_X = idesc_bf16(128, 128, false, MODE == MODE_FWD);
+  constexpr uint32_t IDESC_Y = idesc_bf16(128, 128, false, true);
+  constexpr uint32_t IDESC_D = idesc_bf16(128, 128, true, true);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + LY::MISC);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NS + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  float *pw = reinterpret_cast<float *>(tmem_slot + 4);
+  const uint32_t bar_full0 = smem_u32(bars);
+  const uint32_t bar_mma = smem_u32(bars + NS);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quarter = warp & 3, half = warp >> 2;
+  const int row = quarter * 32 + lane;
+  const int nch = OUT ? g.S : g.S - 1;
+  const int64_t bh = blockIdx.x / nch;
+  const int c = blockIdx.x % nch;
+  const int h = (int)(bh % g.H);
+  const int64_t a = (int64_t)c * g.Lc;
+  const int64_t b = g.L < a + g.Lc ? g.L : a + g.Lc;
+  const int nblk = (int)((b - a + BLOCK - 1) / BLOCK);
+
+  if (tid <= BLOCK) pw[tid] = (float)pow_int((double)lambda[h], tid);
+  if (tid == 0) {
+    for (int s = 0; s < NS; s++) mbar_init(bar_full0 + 8 * s, 1);
+    mbar_init(bar_mma, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    if (OUT) tma_prefetch_desc(&tm0);
+    tma_prefetch_desc(&tm1);
+    tma_prefetch_desc(&tm2);
+    if (OUT) tma_prefetch_desc(&tmo);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), LY::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);  // this warp's lane quarter
+
+  auto issue_load = [&](int j, int st) {
+    const int y = (int)(a + (int64_t)j * BLOCK), z = (int)bh;
+    const uint32_t bar = bar_full0 + 8 * st;
+    uint32_t dst = sbase + st * LY::STAGE;
+    mbar_expect_tx(bar, LY::STAGE);
+    if (OUT) {
+      tma_load_3d(dst, &tm0, bar, 0, y, z);
+      tma_load_3d(dst + BOX, &tm0, bar, 64, y, z);
+      dst += TILE;
+    }
+    tma_load_3d(dst, &tm1, bar, 0, y, z);
+    tma_load_3d(dst + BOX, &tm1, bar, 64, y, z);
+    tma_load_3d(dst + TILE, &tm2, bar, 0, y, z);
+    tma_load_3d(dst + TILE + BOX, &tm2, bar, 64, y, z);
+  };
+  int issued = 0;
+  if (tid == 0)
+    for (; issued < NS && issued < nblk; issued++) issue_load(issued, issued);
+
+  // initial state -> TMEM (fp32) and, for the output passes, a bf16 copy in
+  // shared memory (row d = this thread's row, columns e of this half)
+  {
+    const float *init = nullptr;
+    if (MODE != MODE_STATE) {
+      if (c == 0) init = kv0 ? kv0 + bh * 128 * 128 : nullptr;
+      else init = ws + (bh * g.S + c) * (int64_t)128 * 128;
+    }
+    uint8_t *kvbf = smem + LY::KVBF + half * BOX;
+#pragma unroll
+    for (int part = 0; part < 2; part++) {
+      const int col = half * 64 + part * 32;
+      uint32_t r[32];
+      float f[32];
+      if (init) {
+        const float4 *src = reinterpret_cast<const float4 *>(init + (int64_t)row * 128 + col);
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+          float4 x = src[j];
+          f[4 * j] = x.x; f[4 * j + 1] = x.y; f[4 * j + 2] = x.z; f[4 * j + 3] = x.w;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; j++) f[j] = 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 32; j++) r[j] = __float_as_uint(f[j]);
+      tmem_st32(tl + LY::COL_KV + col, r);
+      if (OUT) st_row_bf16_sw128(kvbf, row, part * 4, f);
+    }
+    tmem_wait_st();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+
+  uint32_t mma_phase = 0;
+  bool aborted = false;
+  int i = 0;
+  for (; i < nblk; i++) {
+    const int st = i % NS;
+    const int64_t p = a + (int64_t)i * BLOCK;
+    const int cb = (int)(b - p < BLOCK ? b - p : BLOCK);
+    uint8_t *stage = smem + st * LY::STAGE;
+    const uint32_t sT0 = sbase + st * LY::STAGE;
+    const uint32_t sT1 = OUT ? sT0 + TILE : sT0;
+    const uint32_t sT2 = sT1 + TILE;
+    uint8_t *T0 = stage;
+    uint8_t *T1 = OUT ? stage + TILE : stage;
+    const uint32_t sKV = sbase + LY::KVBF;
+
+    bool ok = mbar_wait(bar_full0 + 8 * st, (uint32_t)((i / NS) & 1), abort_flag);
+    if (__syncthreads_or(!ok)) { aborted = true; break; }
+    tc_fence_after();
+
+    if (OUT) {
+      // ---- phase 1: S = A0 B1^T, X = A0 KV
+      if (tid == 0) {
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+          const uint32_t koff = (k >> 2) * BOX + (k & 3) * 32;
+          mma_ss(tmem + LY::COL_S, sdesc_sw128(sT0 + koff, 16, 1024),
+                 sdesc_sw128(sT1 + koff, 16, 1024), IDESC_S, k > 0);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+          const uint32_t koff = (k >> 2) * BOX + (k & 3) * 32;
+          const uint64_t bd = MODE == MODE_FWD ? sdesc_sw128(sKV + k * 2048, BOX, 1024)
+                                               : sdesc_sw128(sKV + koff, 16, 1024);
+          mma_ss(tmem + LY::COL_X, sdesc_sw128(sT0 + koff, 16, 1024), bd, IDESC_X, k > 0);
+        }
+        mma_commit(bar_mma);
+      }
+      ok = mbar_wait(bar_mma, mma_phase, abort_flag);
+      mma_phase ^= 1;
+      if (__syncthreads_or(!ok)) { aborted = true; break; }
+      tc_fence_after();
+
+      // ---- phase 2a: P = S (.) M -> bf16, into the S columns of this half
+#pragma unroll
+      for (int part = 0; part < 2; part++) {
+        const int col0 = half * 64 + part * 32;
+        uint32_t r[32];
+        tmem_ld32(tl + LY::COL_S + col0, r);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 16; j++) {
+          const int t0 = col0 + 2 * j, t1 = t0 + 1;
+          const float f0 = t0 <= row ? __uint_as_float(r[2 * j]) * pw[row - t0] : 0.f;
+          const float f1 = t1 <= row ? __uint_as_float(r[2 * j + 1]) * pw[row - t1] : 0.f;
+          pk[j] = pack_bf16x2(f0, f1);
+        }
+        tmem_st16(tl + LY::COL_S + half * 64 + part * 16, pk);
+      }
+    }
+    // ---- phase 2b: B1 rows scaled by lambda^(cb-1-t) in place (the state's key-side decay)
+    {
+      const float f = row < cb ? pw[cb - 1 - row] : 0.f;
+      scale_row_sw128(T1 + half * BOX, row, f);
+    }
+    // ---- phase 2c: KV acc *= lambda^cb
+    {
+      const float dec = pw[cb];
+#pragma unroll
+      for (int part = 0; part < 2; part++) {
+        const uint32_t col = LY::COL_KV + half * 64 + part * 32;
+        uint32_t r[32];
+        tmem_ld32(tl + col, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; j++) r[j] = __float_as_uint(__uint_as_float(r[j]) * dec);
+        tmem_st32(tl + col, r);
+      }
+    }
+    tmem_wait_st();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // ---- phase 3: Y = P B2 (P from TMEM), KV += A^T B (state update)
+    if (tid == 0) {
+      if (OUT) {
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+          const uint32_t pa = tmem + LY::COL_S + (k >> 2) * 64 + (k & 3) * 8;
+          mma_ts(tmem + LY::COL_Y, pa, sdesc_sw128(sT2 + k * 2048, BOX, 1024), IDESC_Y, k > 0);
+        }
+      }
+      const uint32_t sA = MODE == MODE_DQ ? sT2 : sT1;
+      const uint32_t sB = MODE == MODE_DQ ? sT1 : sT2;
+#pragma unroll
+      for (int k = 0; k < 8; k++)
+        mma_ss(tmem + LY::COL_KV, sdesc_sw128(sA + k * 2048, BOX, 1024),
+               sdesc_sw128(sB + k * 2048, BOX, 1024), IDESC_D, 1);
+      mma_commit(bar_mma);
+    }
+    ok = mbar_wait(bar_mma, mma_phase, abort_flag);
+    mma_phase ^= 1;
+    if (__syncthreads_or(!ok)) { aborted = true; break; }
+    tc_fence_after();
+
+    if (OUT) {
+      // ---- phase 4: O = Y + diag(lambda^(s+1)) X -> bf16 -> staging (A0's slot);
+      //               KV -> bf16 copy for the next block's X
+      const float as = pw[row + 1];
+      uint8_t *stg = T0 + half * BOX;
+      uint8_t *kvbf = smem + LY::KVBF + half * BOX;
+#pragma unroll
+      for (int part = 0; part < 2; part++) {
+        const int col = half * 64 + part * 32;
+        uint32_t ry[32], rx[32];
+        tmem_ld32(tl + LY::COL_Y + col, ry);
+        tmem_ld32(tl + LY::COL_X + col, rx);
+        tmem_wait_ld();
+        float o[32];
+#pragma unroll
+        for (int j = 0; j < 32; j++) o[j] = __uint_as_float(ry[j]) + as * __uint_as_float(rx[j]);
+        st_row_bf16_sw128(stg, row, part * 4, o);
+        uint32_t rk[32];
+        tmem_ld32(tl + LY::COL_KV + col, rk);
+        tmem_wait_ld();
+        float f[32];
+#pragma unroll
+        for (int j = 0; j < 32; j++) f[j] = __uint_as_float(rk[j]);
+        st_row_bf16_sw128(kvbf, row, part * 4, f);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        tma_store_3d(&tmo, sT0, 0, (int)p, (int)bh);
+        tma_store_3d(&tmo, sT0 + BOX, 64, (int)p, (int)bh);
+        tma_store_commit();
+        tma_store_wait_read0();  // the slot is refilled below
+      }
+    }
+    if (tid == 0 && issued < nblk) {
+      issue_load(issued, issued % NS);
+      issued++;
+    }
+  }
+
+  if (!aborted) {
+    // final state of the chunk
+    float *dst = nullptr;
+    if (MODE == MODE_FWD) dst = (kv_out && c == g.S - 1) ? kv_out + bh * 128 * 128 : nullptr;
+    if (MODE == MODE_STATE) dst = ws + (bh * g.S + c + 1) * (int64_t)128 * 128;
+    if (dst) {
+#pragma unroll
+      for (int part = 0; part < 2; part++) {
+        const int col = half * 64 + part * 32;
+        uint32_t r[32];
+        tmem_ld32(tl + LY::COL_KV + col, r);
+        tmem_wait_ld();
+        float4 *d4 = reinterpret_cast<float4 *>(dst + (int64_t)row * 128 + col);
+#pragma unroll
+        for (int j = 0; j < 8; j++)
+          d4[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                              __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+      }
+    }
+  } else if (tid == 0) {
+    // drain the loads still in flight before the shared memory is released
+    for (int j = i; j < issued; j++) {
+      volatile int dummy = 0;
+      mbar_wait(bar_full0 + 8 * (j % NS), (uint32_t)((j / NS) & 1), &dummy);
+    }
+  }
+  if (OUT && tid == 0) tma_store_wait0();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, LY::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [BH, L, 128] bf16, boxes of 128 rows x 64 columns, 128-byte swizzle; rows
+// outside [0, L) read as zero and are not written.
+inline bool make_map(CUtensorMap *m, const void *ptr, int64_t BH, int64_t L) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {128, (cuuint64_t)L, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {128 * 2, (cuuint64_t)L * 128 * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE>
+cudaError_t launch_chunk(const CUtensorMap &m0, const CUtensorMap &m1, const CUtensorMap &m2,
+                         const CUtensorMap &mo, const float *lam, const float *kv0, float *ws,
+                         float *kv_out, const Geo &g, cudaStream_t st) {
+  using LY = Layout<MODE>;
+  auto k = chunk_kernel<MODE>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::SMEM);
+  if (e != cudaSuccess) return e;
+  const int64_t nch = LY::OUT ? g.S : g.S - 1;
+  const int64_t grid = (int64_t)g.B * g.H * nch;
+  k<<<(unsigned)grid, NT, LY::SMEM, st>>>(m0, m1, m2, mo, lam, kv0, ws, kv_out, g);
+  return cudaGetLastError();
+}
+
+inline bool geometry_ok(const Geo &g) {
+  return g.L < (int64_t(1) << 31) && (int64_t)g.B * g.H < (int64_t(1) << 31);
+}
+
+// Forward: [chunk states + scan] + main pass.
 template <typename Timed>
-cudaError_t backward(const void *, const void *, const void *, const float *, const float *,
-                     const void *, void *, void *, void *, float *, float *, const Geo &,
-                     cudaStream_t, Timed &&) {
-  return cudaErrorNotSupported;
+cudaError_t forward(const void *q, const void *k, const void *v, const float *lam,
+                    const float *kv0, void *o, float *kv_out, float *ws, const Geo &g,
+                    cudaStream_t st, Timed &&timed) {
+  if (!geometry_ok(g)) return cudaErrorInvalidValue;
+  const int64_t BH = (int64_t)g.B * g.H;
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map(&mq, q, BH, g.L) || !make_map(&mk, k, BH, g.L) || !make_map(&mv, v, BH, g.L) ||
+      !make_map(&mo, o, BH, g.L))
+    return cudaErrorInvalidValue;
+  cudaError_t err = cudaSuccess;
+  if (g.S > 1) {
+    err = timed(0, [&] { launch_chunk<MODE_STATE>(mk, mk, mv, mk, lam, nullptr, ws, nullptr, g, st); });
+    if (err) return err;
+    err = timed(1, [&] {
+      la2::simt::scan_fwd_kernel<128, 128>
+          <<<dim3(128 * 128 / la2::simt::NT, (unsigned)BH), la2::simt::NT, 0, st>>>(ws, kv0, lam, g);
+    });
+    if (err) return err;
+  }
+  return timed(2, [&] { launch_chunk<MODE_FWD>(mq, mk, mv, mo, lam, kv0, ws, kv_out, g, st); });
+}
+
+// Backward: dQ on the tensor cores (forward-state scan); dK, dV on the
+// portable kernels for now (reverse-state scan).
+template <typename Timed>
+cudaError_t backward(const void *q, const void *k, const void *v, const float *lam,
+                     const float *kv0, const void *dO, void *dq, void *dk, void *dv, float *dkv0,
+                     float *ws, const Geo &g, cudaStream_t st, Timed &&timed) {
+  if (!geometry_ok(g)) return cudaErrorInvalidValue;
+  using T = __nv_bfloat16;
+  const int64_t BH = (int64_t)g.B * g.H;
+  CUtensorMap mk, mv, mg, mdq;
+  if (!make_map(&mk, k, BH, g.L) || !make_map(&mv, v, BH, g.L) || !make_map(&mg, dO, BH, g.L) ||
+      !make_map(&mdq, dq, BH, g.L))
+    return cudaErrorInvalidValue;
+  float *wsf = ws;
+  float *wsr = ws ? ws + (size_t)BH * g.S * 128 * 128 : nullptr;
+  cudaError_t err = cudaSuccess;
+  if (g.S > 1) {
+    err = timed(0, [&] { launch_chunk<MODE_STATE>(mk, mk, mv, mk, lam, nullptr, wsf, nullptr, g, st); });
+    if (err) return err;
+    err = timed(1, [&] {
+      la2::simt::scan_fwd_kernel<128, 128>
+          <<<dim3(128 * 128 / la2::simt::NT, (unsigned)BH), la2::simt::NT, 0, st>>>(wsf, kv0, lam, g);
+    });
+    if (err) return err;
+  }
+  err = timed(2, [&] { launch_chunk<MODE_DQ>(mg, mv, mk, mdq, lam, kv0, wsf, nullptr, g, st); });
+  if (err) return err;
+  // Reverse pass on the portable kernels, with their own (finer) block size
+  // but the same chunk boundaries.
+  using namespace la2::simt;
+  if (g.S > 1) {
+    auto krs = rev_state_kernel<T, 128, 128>;
+    cudaFuncSetAttribute(krs, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rev_smem<128, 128>());
+    err = timed(3, [&] {
+      krs<<<(unsigned)(BH * (g.S - 1)), la2::simt::NT, rev_smem<128, 128>(), st>>>(
+          (const T *)q, (const T *)dO, lam, wsr, g);
+    });
+    if (err) return err;
+    err = timed(4, [&] {
+      scan_rev_kernel<128, 128><<<dim3(128 * 128 / la2::simt::NT, (unsigned)BH), la2::simt::NT, 0, st>>>(
+          wsr, lam, g);
+    });
+    if (err) return err;
+  }
+  auto kk = dkdv_kernel<T, 128, 128>;
+  cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dkdv_smem<128, 128>());
+  return timed(5, [&] {
+    kk<<<(unsigned)(BH * g.S), la2::simt::NT, dkdv_smem<128, 128>(), st>>>(
+        (const T *)q, (const T *)k, (const T *)v, (const T *)dO, lam, (T *)dk, (T *)dv, dkv0, wsr, g);
+  });
 }
 
 }  // namespace tc
