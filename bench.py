@@ -38,10 +38,11 @@ H, D, E = 32, 128, 128
 TOKENS = 65536
 # Algorithmic work per token per head (d = e = 128, bf16 I/O):
 #   bytes each kernel must move: forward reads q,k,v and writes o; the dQ
-#   kernel reads k,v,dO and writes dq; the dK/dV kernel reads q,k,v,dO and
-#   writes dk,dv.  The whole fwd+bwd needs at least 2,816 B.
+#   kernel reads k,v,dO and writes dq; the dV kernel reads k,q,dO and writes
+#   dv; the dK kernel reads v,dO,q and writes dk (the portable dK/dV kernel
+#   reads q,k,v,dO and writes dk,dv).  The whole fwd+bwd needs at least 2,816 B.
 BYTES_PER_TH = {"tc_fwd": 1024, "simt_fwd": 1024, "tc_dq": 1024, "simt_dq": 1024,
-                "tc_dkdv": 1536, "simt_dkdv": 1536}
+                "tc_dv": 1024, "tc_dk": 1024, "simt_dkdv": 1536}
 FWD_BWD_MIN_BYTES = 2816
 # method flops per token-head, intra part over the causal triangle at a
 # fixed C = 64 accounting: fwd (C+1)(d+e) + 4de, bwd (C+1)(3d+2e) + 10de
@@ -407,6 +408,134 @@ def run_reference(args, world, rank):
             "gpu_launches": 0}
 
 
+def _common(world, steps, warmup, value, unit, metric, workload_cfg, ms, extra):
+    line = {"metric": metric, "value": round(value, 1), "unit": unit, "n_gpus": world,
+            "steps": steps, "warmup": warmup, "ms_per_step": ms / steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "data": "synthetic", "config": workload_cfg}
+    line.update(extra)
+    return line
+
+
+def run_long(args, world, rank, local):
+    """B=1, H=64, L=1,048,576 forward only (secondary workload)."""
+    import causal_linear_attention_fwd_b200 as la2
+    from causal_linear_attention_fwd_b200 import inputs
+    dev = torch.device("cuda", local)
+    pk = peaks()
+    Bn, Hh, L = 1, 64, 1 << 20
+    x = inputs.make_inputs(Bn, Hh, L, D, E, dtype=torch.bfloat16, device=dev, seed=0,
+                           with_dO=False)
+    lam = inputs.decay_lambdas(Hh, dev)
+    o = torch.empty_like(x["v"])
+    ws_n = la2.workspace_size(0, Bn, Hh, L, D, E, torch.bfloat16)
+    ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        la2.forward(x["q"], x["k"], x["v"], lam, out=o, workspace=ws)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    la2.profile_enable(True)
+    la2.profile_report()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        la2.forward(x["q"], x["k"], x["v"], lam, out=o, workspace=ws)
+    b.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    prof = la2.profile_report()
+    la2.profile_enable(False)
+    assert la2.last_device_error() == 0
+    ms = max_over_ranks(a.elapsed_time(b), world)
+    value = world * L * args.steps / (ms / 1e3)
+    top = max(prof.items(), key=lambda kv: kv[1]["ms"])
+    name, rec = top
+    avg = rec["ms"] / rec["launches"]
+    roof = None
+    if name in BYTES_PER_TH:
+        alg = 1024 * Hh * L
+        ach = alg / (avg / 1e3) / 1e9
+        roof = {"kernel": name, "bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": round(ach / pk["hbm_gbs"], 4),
+                "traffic": traffic_for(name, Hh * L), "alg_bytes_per_launch": alg,
+                "avg_launch_ms": avg}
+    return _common(world, args.steps, args.warmup, value, "tokens/s",
+                   "long-context forward tokens/s (B=1,H=64,L=1M,d=e=128,bf16)",
+                   {"workload": "long-context forward, B=1, H=64, L=1,048,576, d=e=128, bf16",
+                    "l2": "inputs 16 GiB per tensor, larger than L2; no flush"}, ms,
+                   {"dtype": "bf16", "roofline": roof, "kernels": prof,
+                    "gpu_launches": sum(v["launches"] for v in prof.values()), "clocks": clk,
+                    "hbm_frac_fwd_min": round(1024 * Hh * value / world / 1e9 / pk["hbm_gbs"], 4)})
+
+
+def run_decode(args, world, rank, local):
+    """Recurrent decode, batch 256, H=64, d=e=128, fp32 state; one step of
+    this workload = `--decode-steps` consecutive decode steps replayed from a
+    CUDA graph (secondary workload)."""
+    import causal_linear_attention_fwd_b200 as la2
+    from causal_linear_attention_fwd_b200 import inputs
+    dev = torch.device("cuda", local)
+    pk = peaks()
+    Bn, Hh, n = 256, 64, args.decode_steps
+    lam = inputs.decay_lambdas(Hh, dev)
+    kv = inputs.decode_state0(Bn, Hh, D, E, device=dev, seed=0)
+    gen = inputs.DecodeStream(Bn, Hh, D, E, device=dev, seed=0)
+    toks = [gen.next() for _ in range(n)]
+    outs = torch.empty((n, Bn, Hh, E), dtype=torch.bfloat16, device=dev)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for t in range(min(n, 8)):  # eager warm-up launches
+            la2.decode_step(*toks[t], lam, kv, out=outs[t], stream=s)
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for t in range(n):
+            la2.decode_step(*toks[t], lam, kv, out=outs[t], stream=s)
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    assert la2.last_device_error() == 0
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream()
+    a.record(cur)
+    for _ in range(args.steps):
+        g.replay()
+    b.record(cur)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms = max_over_ranks(a.elapsed_time(b), world)
+    value = world * Bn * n * args.steps / (ms / 1e3)
+    per_launch_ms = ms / (n * args.steps)
+    bytes_launch = Bn * Hh * (2 * D * E * 4 + (2 * D + 2 * E) * 2)
+    ach = bytes_launch / (per_launch_ms / 1e3) / 1e9
+    roof = {"kernel": "decode_step", "bound": "hbm", "achieved": round(ach, 1),
+            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(ach / pk["hbm_gbs"], 4),
+            "traffic": traffic_for("decode_step", Bn * Hh), "alg_bytes_per_launch": bytes_launch,
+            "avg_launch_ms": per_launch_ms,
+            "note": "launch time = graph replay time / launches (1024 launches per replay)"}
+    line = _common(world, args.steps, args.warmup, value, "tokens/s",
+                   "decode tokens/s (batch 256, H=64, d=e=128, fp32 state); % of HBM bandwidth",
+                   {"workload": f"recurrent decode, batch 256, H=64, d=e=128, fp32 state "
+                                f"(1 GiB), {n} steps per graph replay",
+                    "l2": "state 1 GiB, larger than L2; no flush"}, ms,
+                   {"dtype": "f32", "roofline": roof, "gpu_launches": n * args.steps,
+                    "clocks": clk})
+    del g
+    return line
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -415,6 +544,9 @@ def main():
     ap.add_argument("--impl", default="la2", choices=["la2", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--workload", default="sweep", choices=["sweep", "long", "decode"],
+                    help="sweep (the metric; default), long (1M-token forward), decode")
+    ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--only", default=None,
                     help="B:L -- time a single sweep point instead of the whole sweep "
                          "(profiling aid; not the metric)")
@@ -434,7 +566,8 @@ def main():
         return
     world, rank, local = dist_setup(args.gpus)
     try:
-        line = run_la2(args, world, rank, local)
+        fn = {"sweep": run_la2, "long": run_long, "decode": run_decode}[args.workload]
+        line = fn(args, world, rank, local)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

@@ -23,17 +23,18 @@ using la2::Geo;
 
 std::atomic<int> g_opt_split{0};
 std::atomic<int> g_opt_path{0};
+std::atomic<int> g_opt_inject{0};
 
 // ------------------------------------------------------------ profiling
 enum KernelId {
   K_SIMT_FWD_STATE, K_SIMT_FWD_SCAN, K_SIMT_FWD, K_SIMT_DQ, K_SIMT_REV_STATE,
   K_SIMT_REV_SCAN, K_SIMT_DKDV, K_DECODE, K_TC_FWD_STATE, K_TC_FWD, K_TC_DQ,
-  K_TC_REV_STATE, K_TC_DKDV, K_SCAN_FWD, K_SCAN_REV, K_COUNT
+  K_TC_REV_STATE, K_TC_DV, K_TC_DK, K_SCAN_FWD, K_SCAN_REV, K_COUNT
 };
 const char *kKernelName[K_COUNT] = {
     "simt_fwd_chunk_state", "simt_scan_fwd", "simt_fwd", "simt_dq",
     "simt_rev_chunk_state", "simt_scan_rev", "simt_dkdv", "decode_step",
-    "tc_fwd_chunk_state", "tc_fwd", "tc_dq", "tc_rev_chunk_state", "tc_dkdv",
+    "tc_fwd_chunk_state", "tc_fwd", "tc_dq", "tc_rev_chunk_state", "tc_dv", "tc_dk",
     "scan_fwd", "scan_rev"};
 
 struct ProfRec {
@@ -143,6 +144,7 @@ Path choose_path(int d, int e, la2_dtype dt) {
 // multiple of the block size `blk`) so that B*H*S CTAs fill the GPU.
 Geo plan(int B, int H, int64_t L, int blk, Path path) {
   Geo g;
+  g.inject = 0;
   g.B = B;
   g.H = H;
   g.L = L;
@@ -285,6 +287,7 @@ const char *la2_version(void) { return "la2 0.1 sm_100a"; }
 int la2_set_option(int option, int value) {
   if (option == LA2_OPT_SPLIT) return g_opt_split.exchange(value);
   if (option == LA2_OPT_PATH) return g_opt_path.exchange(value);
+  if (option == LA2_OPT_INJECT_TIMEOUT) return g_opt_inject.exchange(value);
   return -1;
 }
 
@@ -334,6 +337,7 @@ la2_status la2_forward(const void *q, const void *k, const void *v,
   float *ws = (float *)workspace;
   cudaError_t err;
   if (p == PATH_TC) {
+    g.inject = g_opt_inject.exchange(0);
     err = la2::tc::forward(q, k, v, lambda, kv0, o, kv_out, ws, g, stream,
                            [&](int which, auto &&fn) {
                              return timed(which == 0 ? K_TC_FWD_STATE : which == 1 ? K_SCAN_FWD : K_TC_FWD,
@@ -389,8 +393,8 @@ la2_status la2_backward(const void *q, const void *k, const void *v,
     err = la2::tc::backward(q, k, v, lambda, kv0, dO, dq, dk, dv, dkv0, ws, g, stream,
                             [&](int which, auto &&fn) {
                               static const int ids[] = {K_TC_FWD_STATE, K_SCAN_FWD, K_TC_DQ,
-                                                        K_SIMT_REV_STATE, K_SIMT_REV_SCAN,
-                                                        K_SIMT_DKDV};
+                                                        K_TC_REV_STATE, K_SCAN_REV, K_TC_DV,
+                                                        K_TC_DK};
                               return timed(ids[which], stream, fn);
                             });
   } else if (dt == LA2_F32) {

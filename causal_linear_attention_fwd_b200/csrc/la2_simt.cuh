@@ -33,6 +33,8 @@ struct Geo {
   int64_t L;
   int S;        // chunks per (b,h)
   int64_t Lc;   // rows per chunk (multiple of the block size); last may be short
+  int inject;   // test hook: CTA 0 of a tensor-core pass withholds one MMA
+                // completion signal so that its bounded wait runs out
 };
 
 namespace simt {

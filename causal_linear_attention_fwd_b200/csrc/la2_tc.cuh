@@ -14,10 +14,12 @@
 //   O  = Y + diag(lambda^(s+1)) X   -> bf16 -> shared -> TMA store
 //
 // with M[s,t] = lambda^(s-t) for t <= s.  The forward pass uses
-// (A0, B1, B2) = (Q, K, V); the dQ pass of the backward uses (dO, V, K): the
-// same schedule with K and V exchanging roles and the state transposed.  The
-// chunk-state pre-pass (MODE_STATE) runs only the state recurrence over K, V
-// from a zero state and writes the chunk's state to the workspace.
+// (A0, B1, B2) = (Q, K, V); the backward runs the same schedule three more
+// times with other tiles, factors and directions (see the MODE_ list below):
+// dQ by a forward scan, dV and dK by reverse scans over the reverse state
+// D = sum_{t beyond the block} lambda^.. q_t^T dO_t.  The chunk-state
+// pre-passes run only the state recurrence from a zero state and write the
+// chunk's state to the workspace.
 //
 // Data path: TMA (128-byte swizzle, two 64-column boxes per 128 x 128 tile)
 // double-buffers the next block's tiles while the current one is processed;
@@ -40,10 +42,28 @@ constexpr int NT = 256;          // 8 warps: (lane quarter) x (column half)
 constexpr uint32_t BOX = 16384;  // 128 rows x 64 bf16 (one TMA box)
 constexpr uint32_t TILE = 32768; // 128 rows x 128 bf16
 
-enum { MODE_FWD = 0, MODE_DQ = 1, MODE_STATE = 2 };
+// Passes of the one chunk kernel.  (A0, B1, B2) are the three tiles each
+// block loads; S = A0 B1^T, Y = P B2, X = A0 (state or state^T), and the
+// state update is B1s^T B2 or B2^T B1s with B1s = B1 after its row decay.
+//   FWD    (Q,  K,  V ) forward order, O  = Y + lambda^(s+1)  X,  KV += (b K)^T V
+//   DQ     (dO, V,  K ) forward order, dQ = Y + lambda^(s+1)  X,  KV += K^T (b V)
+//   DV     (K,  Q,  dO) reverse order, dV = Y + lambda^(cb-t) X,  D  += (g Q)^T dO
+//   DK     (V,  dO, Q ) reverse order, dK = Y + lambda^(cb-t) X,  D  += Q^T (g dO)
+//   STATE  (-,  K,  V ) forward chunk state from zero
+//   RSTATE (-,  Q,  dO) reverse chunk state from zero
+// b_t = lambda^(cb-1-t) (key side, forward), g_s = lambda^s (query side, reverse).
+// The reverse passes use the transposed mask: S^T[t][s] kept for s >= t.
+enum { MODE_FWD = 0, MODE_DQ = 1, MODE_STATE = 2, MODE_DV = 3, MODE_DK = 4, MODE_RSTATE = 5 };
+
+template <int MODE> struct Traits {
+  static constexpr bool OUT = MODE != MODE_STATE && MODE != MODE_RSTATE;
+  static constexpr bool REV = MODE == MODE_DV || MODE == MODE_DK || MODE == MODE_RSTATE;
+  static constexpr bool SWAP = MODE == MODE_DQ || MODE == MODE_DK;  // state A/B from (B2, B1)
+  static constexpr bool X_MN = MODE == MODE_FWD || MODE == MODE_DV; // X's B operand MN-major
+};
 
 template <int MODE> struct Layout {
-  static constexpr bool OUT = MODE != MODE_STATE;
+  static constexpr bool OUT = Traits<MODE>::OUT;
   static constexpr int NSTAGE = OUT ? 2 : 3;
   static constexpr uint32_t STAGE = OUT ? 3 * TILE : 2 * TILE;
   static constexpr uint32_t KVBF = NSTAGE * STAGE;
@@ -106,10 +126,12 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
              const float *__restrict__ lambda, const float *__restrict__ kv0,
              float *__restrict__ ws, float *__restrict__ kv_out, Geo g) {
   using LY = Layout<MODE>;
+  using TR = Traits<MODE>;
   constexpr bool OUT = LY::OUT;
+  constexpr bool REV = TR::REV;
   constexpr int NS = LY::NSTAGE;
   constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
-  constexpr uint32_t IDESC_X = idesc_bf16(128, 128, false, MODE == MODE_FWD);
+  constexpr uint32_t IDESC_X = idesc_bf16(128, 128, false, TR::X_MN);
   constexpr uint32_t IDESC_Y = idesc_bf16(128, 128, false, true);
   constexpr uint32_t IDESC_D = idesc_bf16(128, 128, true, true);
 
@@ -129,7 +151,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
   const int row = quarter * 32 + lane;
   const int nch = OUT ? g.S : g.S - 1;
   const int64_t bh = blockIdx.x / nch;
-  const int c = blockIdx.x % nch;
+  const int c = blockIdx.x % nch + (MODE == MODE_RSTATE ? 1 : 0);
   const int h = (int)(bh % g.H);
   const int64_t a = (int64_t)c * g.Lc;
   const int64_t b = g.L < a + g.Lc ? g.L : a + g.Lc;
@@ -156,8 +178,10 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
   const uint32_t tmem = *tmem_slot;
   const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);  // this warp's lane quarter
 
+  // block visited at step j (reverse passes walk the chunk backwards)
+  auto block_of = [&](int j) { return REV ? nblk - 1 - j : j; };
   auto issue_load = [&](int j, int st) {
-    const int y = (int)(a + (int64_t)j * BLOCK), z = (int)bh;
+    const int y = (int)(a + (int64_t)block_of(j) * BLOCK), z = (int)bh;
     const uint32_t bar = bar_full0 + 8 * st;
     uint32_t dst = sbase + st * LY::STAGE;
     mbar_expect_tx(bar, LY::STAGE);
@@ -179,9 +203,11 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
   // shared memory (row d = this thread's row, columns e of this half)
   {
     const float *init = nullptr;
-    if (MODE != MODE_STATE) {
+    if (MODE == MODE_FWD || MODE == MODE_DQ) {
       if (c == 0) init = kv0 ? kv0 + bh * 128 * 128 : nullptr;
       else init = ws + (bh * g.S + c) * (int64_t)128 * 128;
+    } else if (MODE == MODE_DV || MODE == MODE_DK) {
+      if (c != g.S - 1) init = ws + (bh * g.S + c) * (int64_t)128 * 128;
     }
     uint8_t *kvbf = smem + LY::KVBF + half * BOX;
 #pragma unroll
@@ -216,7 +242,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
   int i = 0;
   for (; i < nblk; i++) {
     const int st = i % NS;
-    const int64_t p = a + (int64_t)i * BLOCK;
+    const int64_t p = a + (int64_t)block_of(i) * BLOCK;
     const int cb = (int)(b - p < BLOCK ? b - p : BLOCK);
     uint8_t *stage = smem + st * LY::STAGE;
     const uint32_t sT0 = sbase + st * LY::STAGE;
@@ -242,11 +268,12 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
 #pragma unroll
         for (int k = 0; k < 8; k++) {
           const uint32_t koff = (k >> 2) * BOX + (k & 3) * 32;
-          const uint64_t bd = MODE == MODE_FWD ? sdesc_sw128(sKV + k * 2048, BOX, 1024)
-                                               : sdesc_sw128(sKV + koff, 16, 1024);
+          const uint64_t bd = TR::X_MN ? sdesc_sw128(sKV + k * 2048, BOX, 1024)
+                                       : sdesc_sw128(sKV + koff, 16, 1024);
           mma_ss(tmem + LY::COL_X, sdesc_sw128(sT0 + koff, 16, 1024), bd, IDESC_X, k > 0);
         }
-        mma_commit(bar_mma);
+        // test hook: withhold this signal once so the waits below run out
+        if (!(g.inject && blockIdx.x == 0 && i == 0)) mma_commit(bar_mma);
       }
       ok = mbar_wait(bar_mma, mma_phase, abort_flag);
       mma_phase ^= 1;
@@ -254,6 +281,8 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
       tc_fence_after();
 
       // ---- phase 2a: P = S (.) M -> bf16, into the S columns of this half
+      //      (forward: keep col <= row, factor lambda^(row-col);
+      //       reverse, S^T: keep col >= row, factor lambda^(col-row))
 #pragma unroll
       for (int part = 0; part < 2; part++) {
         const int col0 = half * 64 + part * 32;
@@ -264,16 +293,23 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
 #pragma unroll
         for (int j = 0; j < 16; j++) {
           const int t0 = col0 + 2 * j, t1 = t0 + 1;
-          const float f0 = t0 <= row ? __uint_as_float(r[2 * j]) * pw[row - t0] : 0.f;
-          const float f1 = t1 <= row ? __uint_as_float(r[2 * j + 1]) * pw[row - t1] : 0.f;
+          float f0, f1;
+          if (REV) {
+            f0 = t0 >= row ? __uint_as_float(r[2 * j]) * pw[t0 - row] : 0.f;
+            f1 = t1 >= row ? __uint_as_float(r[2 * j + 1]) * pw[t1 - row] : 0.f;
+          } else {
+            f0 = t0 <= row ? __uint_as_float(r[2 * j]) * pw[row - t0] : 0.f;
+            f1 = t1 <= row ? __uint_as_float(r[2 * j + 1]) * pw[row - t1] : 0.f;
+          }
           pk[j] = pack_bf16x2(f0, f1);
         }
         tmem_st16(tl + LY::COL_S + half * 64 + part * 16, pk);
       }
     }
-    // ---- phase 2b: B1 rows scaled by lambda^(cb-1-t) in place (the state's key-side decay)
+    // ---- phase 2b: B1 rows decayed in place for the state update
+    //      (forward lambda^(cb-1-t), reverse lambda^s; rows past the block end: 0)
     {
-      const float f = row < cb ? pw[cb - 1 - row] : 0.f;
+      const float f = row < cb ? (REV ? pw[row] : pw[cb - 1 - row]) : 0.f;
       scale_row_sw128(T1 + half * BOX, row, f);
     }
     // ---- phase 2c: KV acc *= lambda^cb
@@ -305,8 +341,8 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
           mma_ts(tmem + LY::COL_Y, pa, sdesc_sw128(sT2 + k * 2048, BOX, 1024), IDESC_Y, k > 0);
         }
       }
-      const uint32_t sA = MODE == MODE_DQ ? sT2 : sT1;
-      const uint32_t sB = MODE == MODE_DQ ? sT1 : sT2;
+      const uint32_t sA = TR::SWAP ? sT2 : sT1;
+      const uint32_t sB = TR::SWAP ? sT1 : sT2;
 #pragma unroll
       for (int k = 0; k < 8; k++)
         mma_ss(tmem + LY::COL_KV, sdesc_sw128(sA + k * 2048, BOX, 1024),
@@ -319,9 +355,9 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
     tc_fence_after();
 
     if (OUT) {
-      // ---- phase 4: O = Y + diag(lambda^(s+1)) X -> bf16 -> staging (A0's slot);
-      //               KV -> bf16 copy for the next block's X
-      const float as = pw[row + 1];
+      // ---- phase 4: out = Y + diag(factor) X -> bf16 -> staging (A0's slot);
+      //               state -> bf16 copy for the next block's X
+      const float as = REV ? pw[cb - row < 0 ? 0 : cb - row] : pw[row + 1];
       uint8_t *stg = T0 + half * BOX;
       uint8_t *kvbf = smem + LY::KVBF + half * BOX;
 #pragma unroll
@@ -362,8 +398,14 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
   if (!aborted) {
     // final state of the chunk
     float *dst = nullptr;
+    float scale = 1.f;
     if (MODE == MODE_FWD) dst = (kv_out && c == g.S - 1) ? kv_out + bh * 128 * 128 : nullptr;
     if (MODE == MODE_STATE) dst = ws + (bh * g.S + c + 1) * (int64_t)128 * 128;
+    if (MODE == MODE_RSTATE) dst = ws + (bh * g.S + c - 1) * (int64_t)128 * 128;
+    if (MODE == MODE_DV && c == 0 && kv_out) {  // dkv0 = lambda * D(0)
+      dst = kv_out + bh * 128 * 128;
+      scale = lambda[h];
+    }
     if (dst) {
 #pragma unroll
       for (int part = 0; part < 2; part++) {
@@ -374,8 +416,8 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
         float4 *d4 = reinterpret_cast<float4 *>(dst + (int64_t)row * 128 + col);
 #pragma unroll
         for (int j = 0; j < 8; j++)
-          d4[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                              __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+          d4[j] = make_float4(scale * __uint_as_float(r[4 * j]), scale * __uint_as_float(r[4 * j + 1]),
+                              scale * __uint_as_float(r[4 * j + 2]), scale * __uint_as_float(r[4 * j + 3]));
       }
     }
   } else if (tid == 0) {
@@ -471,56 +513,45 @@ cudaError_t forward(const void *q, const void *k, const void *v, const float *la
   return timed(2, [&] { launch_chunk<MODE_FWD>(mq, mk, mv, mo, lam, kv0, ws, kv_out, g, st); });
 }
 
-// Backward: dQ on the tensor cores (forward-state scan); dK, dV on the
-// portable kernels for now (reverse-state scan).
+// Backward: dQ by a forward scan (chunk states of K, V + scan), then dV and
+// dK by reverse scans (chunk states of Q, dO + reverse scan); dkv0 comes
+// out of the dV pass's first chunk.
 template <typename Timed>
 cudaError_t backward(const void *q, const void *k, const void *v, const float *lam,
                      const float *kv0, const void *dO, void *dq, void *dk, void *dv, float *dkv0,
                      float *ws, const Geo &g, cudaStream_t st, Timed &&timed) {
   if (!geometry_ok(g)) return cudaErrorInvalidValue;
-  using T = __nv_bfloat16;
   const int64_t BH = (int64_t)g.B * g.H;
-  CUtensorMap mk, mv, mg, mdq;
-  if (!make_map(&mk, k, BH, g.L) || !make_map(&mv, v, BH, g.L) || !make_map(&mg, dO, BH, g.L) ||
-      !make_map(&mdq, dq, BH, g.L))
+  CUtensorMap mq, mk, mv, mg, mdq, mdk, mdv;
+  if (!make_map(&mq, q, BH, g.L) || !make_map(&mk, k, BH, g.L) || !make_map(&mv, v, BH, g.L) ||
+      !make_map(&mg, dO, BH, g.L) || !make_map(&mdq, dq, BH, g.L) ||
+      !make_map(&mdk, dk, BH, g.L) || !make_map(&mdv, dv, BH, g.L))
     return cudaErrorInvalidValue;
   float *wsf = ws;
   float *wsr = ws ? ws + (size_t)BH * g.S * 128 * 128 : nullptr;
+  const dim3 sgrid(128 * 128 / la2::simt::NT, (unsigned)BH);
   cudaError_t err = cudaSuccess;
   if (g.S > 1) {
     err = timed(0, [&] { launch_chunk<MODE_STATE>(mk, mk, mv, mk, lam, nullptr, wsf, nullptr, g, st); });
     if (err) return err;
     err = timed(1, [&] {
-      la2::simt::scan_fwd_kernel<128, 128>
-          <<<dim3(128 * 128 / la2::simt::NT, (unsigned)BH), la2::simt::NT, 0, st>>>(wsf, kv0, lam, g);
+      la2::simt::scan_fwd_kernel<128, 128><<<sgrid, la2::simt::NT, 0, st>>>(wsf, kv0, lam, g);
     });
     if (err) return err;
   }
   err = timed(2, [&] { launch_chunk<MODE_DQ>(mg, mv, mk, mdq, lam, kv0, wsf, nullptr, g, st); });
   if (err) return err;
-  // Reverse pass on the portable kernels, with their own (finer) block size
-  // but the same chunk boundaries.
-  using namespace la2::simt;
   if (g.S > 1) {
-    auto krs = rev_state_kernel<T, 128, 128>;
-    cudaFuncSetAttribute(krs, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rev_smem<128, 128>());
-    err = timed(3, [&] {
-      krs<<<(unsigned)(BH * (g.S - 1)), la2::simt::NT, rev_smem<128, 128>(), st>>>(
-          (const T *)q, (const T *)dO, lam, wsr, g);
-    });
+    err = timed(3, [&] { launch_chunk<MODE_RSTATE>(mq, mq, mg, mq, lam, nullptr, wsr, nullptr, g, st); });
     if (err) return err;
     err = timed(4, [&] {
-      scan_rev_kernel<128, 128><<<dim3(128 * 128 / la2::simt::NT, (unsigned)BH), la2::simt::NT, 0, st>>>(
-          wsr, lam, g);
+      la2::simt::scan_rev_kernel<128, 128><<<sgrid, la2::simt::NT, 0, st>>>(wsr, lam, g);
     });
     if (err) return err;
   }
-  auto kk = dkdv_kernel<T, 128, 128>;
-  cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dkdv_smem<128, 128>());
-  return timed(5, [&] {
-    kk<<<(unsigned)(BH * g.S), la2::simt::NT, dkdv_smem<128, 128>(), st>>>(
-        (const T *)q, (const T *)k, (const T *)v, (const T *)dO, lam, (T *)dk, (T *)dv, dkv0, wsr, g);
-  });
+  err = timed(5, [&] { launch_chunk<MODE_DV>(mk, mq, mg, mdv, lam, nullptr, wsr, dkv0, g, st); });
+  if (err) return err;
+  return timed(6, [&] { launch_chunk<MODE_DK>(mv, mg, mq, mdk, lam, nullptr, wsr, nullptr, g, st); });
 }
 
 }  // namespace tc

@@ -149,10 +149,14 @@ const char *la2_status_string(la2_status s);
  * concurrent calls).  LA2_OPT_SPLIT: number of chunks each (b,h) sequence is
  * split into (0 = automatic).  LA2_OPT_PATH: 0 = automatic, 1 = force the
  * portable fp32-FMA kernels, 2 = require the tensor-core kernels (calls whose
- * shape they do not cover return LA2_ERR_UNSUPPORTED).  Returns the previous
- * value, or -1 for an unknown option.
+ * shape they do not cover return LA2_ERR_UNSUPPORTED).
+ * LA2_OPT_INJECT_TIMEOUT (test hook): when nonzero, the next tensor-core
+ * la2_forward withholds one internal completion signal in its first CTA, so
+ * that CTA's bounded wait gives up (about 2 s) and la2_last_device_error()
+ * then reports LA2_ERR_TIMEOUT; the option resets itself.  Returns the
+ * previous value, or -1 for an unknown option.
  */
-enum { LA2_OPT_SPLIT = 0, LA2_OPT_PATH = 1 };
+enum { LA2_OPT_SPLIT = 0, LA2_OPT_PATH = 1, LA2_OPT_INJECT_TIMEOUT = 2 };
 int la2_set_option(int option, int value);
 
 /*

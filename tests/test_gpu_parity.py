@@ -275,3 +275,24 @@ def test_decode_matches_forward(orc):
     o_d = torch.stack(outs, dim=2)
     check("decode vs forward o", o_d, host(o_f), torch.float32)
     check("decode vs forward state", kv, host(st_f), torch.float32)
+
+
+# ----------------------------------------------- failure detection (no fault)
+def test_bounded_wait_reports_timeout():
+    """A tensor-core pass whose completion signal is withheld (test hook) gives
+    up after its bounded wait, reports LA2_ERR_TIMEOUT, and leaves the context
+    usable: the next call is correct."""
+    x = inputs.make_inputs(1, 1, 256, 128, 128, dtype=torch.bfloat16, device=DEV, seed=2,
+                           with_dO=False)
+    lam = inputs.decay_lambdas(1, DEV)
+    with options(path="tc"):
+        ref = la2.forward(x["q"], x["k"], x["v"], lam)
+        torch.cuda.synchronize()
+        assert la2.last_device_error() == 0
+        la2.set_option(la2.LA2_OPT_INJECT_TIMEOUT, 1)
+        la2.forward(x["q"], x["k"], x["v"], lam)
+        assert la2.last_device_error() == 4  # LA2_ERR_TIMEOUT
+        again = la2.forward(x["q"], x["k"], x["v"], lam)
+        torch.cuda.synchronize()
+        assert la2.last_device_error() == 0
+    assert torch.equal(again, ref)
