@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(HERE, "libla2.so")
 LA2_OK, LA2_ERR_INVALID, LA2_ERR_UNSUPPORTED, LA2_ERR_CUDA, LA2_ERR_TIMEOUT = range(5)
 LA2_F32, LA2_BF16 = 0, 1
 LA2_OP_FORWARD, LA2_OP_BACKWARD = 0, 1
-LA2_OPT_SPLIT, LA2_OPT_PATH, LA2_OPT_INJECT_TIMEOUT = 0, 1, 2
+LA2_OPT_SPLIT, LA2_OPT_PATH, LA2_OPT_INJECT_TIMEOUT, LA2_OPT_VARIANT = 0, 1, 2, 3
 
 _lock = threading.Lock()
 _lib = None

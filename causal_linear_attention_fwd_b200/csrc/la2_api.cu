@@ -24,6 +24,7 @@ using la2::Geo;
 std::atomic<int> g_opt_split{0};
 std::atomic<int> g_opt_path{0};
 std::atomic<int> g_opt_inject{0};
+std::atomic<int> g_opt_variant{0};
 
 // ------------------------------------------------------------ profiling
 enum KernelId {
@@ -145,6 +146,7 @@ Path choose_path(int d, int e, la2_dtype dt) {
 Geo plan(int B, int H, int64_t L, int blk, Path path) {
   Geo g;
   g.inject = 0;
+  g.variant = g_opt_variant.load();
   g.B = B;
   g.H = H;
   g.L = L;
@@ -288,6 +290,7 @@ int la2_set_option(int option, int value) {
   if (option == LA2_OPT_SPLIT) return g_opt_split.exchange(value);
   if (option == LA2_OPT_PATH) return g_opt_path.exchange(value);
   if (option == LA2_OPT_INJECT_TIMEOUT) return g_opt_inject.exchange(value);
+  if (option == LA2_OPT_VARIANT) return g_opt_variant.exchange(value);
   return -1;
 }
 

@@ -35,6 +35,7 @@ struct Geo {
   int64_t Lc;   // rows per chunk (multiple of the block size); last may be short
   int inject;   // test hook: CTA 0 of a tensor-core pass withholds one MMA
                 // completion signal so that its bounded wait runs out
+  int variant;  // tensor-core kernel form (0: warp-specialised, 1: phase-serial)
 };
 
 namespace simt {

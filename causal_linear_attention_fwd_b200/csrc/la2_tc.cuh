@@ -77,11 +77,28 @@ template <int MODE> struct Layout {
 
 inline bool supports(int d, int e, bool bf16) { return bf16 && d == 128 && e == 128; }
 
-// Chunks per (b,h): enough CTAs (one per SM at most, they use all of TMEM)
-// to cover every SM once when B*H alone does not.
+// Chunks per (b,h).  One CTA per SM at a time (each uses all of TMEM), so a
+// pass over BH*S chunks of ceil(nblk/S) blocks takes
+//   ceil(BH*S / sms) waves x (blocks per chunk + ~1 block of pipeline fill),
+// and a split (S > 1) adds the chunk-state pre-pass over S-1 chunks, which
+// moves half the bytes per block.  Pick the S with the smallest estimate.
 inline int64_t auto_split(int64_t BH, int64_t nblk, int sms) {
-  if (BH >= sms) return 1;
-  return (sms + BH - 1) / BH;
+  int64_t best_s = 1;
+  double best = 1e300;
+  const int64_t smax = nblk < 256 ? nblk : 256;
+  for (int64_t S = 1; S <= smax; S++) {
+    const int64_t per = (nblk + S - 1) / S;
+    const int64_t s_eff = (nblk + per - 1) / per;
+    if (s_eff != S) continue;  // same plan as a smaller S
+    const double blocks = (double)per + 1.0;
+    double cost = (double)((BH * S + sms - 1) / sms) * blocks;
+    if (S > 1) cost += 0.5 * (double)((BH * (S - 1) + sms - 1) / sms) * blocks;
+    if (cost < best * 0.999) {
+      best = cost;
+      best_s = S;
+    }
+  }
+  return best_s;
 }
 
 using namespace la2::sm100;
@@ -436,6 +453,397 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
   }
 }
 
+// ================================================================ v2
+// Warp-specialised form of the same schedule.  Roles (320 threads):
+//   warp 0      TMA producer (one thread): fills the stage ring
+//   warp 1      MMA issuer (one thread)
+//   warps 2-5   "mask" warpgroup: P = S (.) M into TMEM, row decays of A0, B1
+//   warps 6-9   "epilogue" warpgroup: out -> bf16 -> TMA store, state ->
+//               bf16 operand copy, state *= lambda^cb for the next block
+// The row factor of the state term is folded into A0 (A0 <- diag(f) A0 after
+// S = A0 B1^T has read it), so Y and X share one accumulator:
+//   O = P B2 + A0f * state.
+// TMEM: S double-buffered [0,128) and [128,256), O [256,384), state [384,512);
+// the MMA for S of block i+1 is issued while block i is still being masked
+// and stored, so tensor-core, CUDA-core and copy work overlap.
+constexpr int NT2 = 320;
+
+template <int MODE> struct Layout2 {
+  static constexpr bool OUT = Traits<MODE>::OUT;
+  static constexpr int NSTAGE = OUT ? 2 : 3;
+  static constexpr uint32_t STAGE = OUT ? 3 * TILE : 2 * TILE;
+  static constexpr uint32_t KVBF = NSTAGE * STAGE;
+  static constexpr uint32_t MISC = KVBF + (OUT ? TILE : 0);
+  // full[NS] empty[NS] sfull[2] pfull[NS] ofull oempty done
+  static constexpr uint32_t NBAR = 3 * NSTAGE + 5;
+  static constexpr uint32_t MISC_BYTES = 8 * NBAR + 16 + 4 * (BLOCK + 1);
+  static constexpr uint32_t SMEM = MISC + MISC_BYTES + 1024;
+  static constexpr uint32_t TMEM_COLS = OUT ? 512 : 128;
+  static constexpr uint32_t COL_O = 256;
+  static constexpr uint32_t COL_KV = OUT ? 384 : 0;
+};
+
+// OR of `v` over the `n` threads that share named barrier `id`.
+__device__ __forceinline__ bool role_any(bool v, int id, int n) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void role_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(NT2, 1)
+chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
+              const __grid_constant__ CUtensorMap tm2, const __grid_constant__ CUtensorMap tmo,
+              const float *__restrict__ lambda, const float *__restrict__ kv0,
+              float *__restrict__ ws, float *__restrict__ kv_out, Geo g) {
+  using LY = Layout2<MODE>;
+  using TR = Traits<MODE>;
+  constexpr bool OUT = LY::OUT;
+  constexpr bool REV = TR::REV;
+  constexpr int NS = LY::NSTAGE;
+  constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
+  constexpr uint32_t IDESC_X = idesc_bf16(128, 128, false, TR::X_MN);
+  constexpr uint32_t IDESC_Y = idesc_bf16(128, 128, false, true);
+  constexpr uint32_t IDESC_D = idesc_bf16(128, 128, true, true);
+  constexpr int BAR_MASK = 1, BAR_EPI = 2;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + LY::MISC);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + LY::NBAR);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  float *pw = reinterpret_cast<float *>(tmem_slot + 4);
+  const uint32_t b_full = smem_u32(bars);
+  const uint32_t b_empty = b_full + 8 * NS;
+  const uint32_t b_sfull = b_empty + 8 * NS;
+  const uint32_t b_pfull = b_sfull + 16;
+  const uint32_t b_ofull = b_pfull + 8 * NS;
+  const uint32_t b_oempty = b_ofull + 8;
+  const uint32_t b_done = b_oempty + 8;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nch = OUT ? g.S : g.S - 1;
+  const int64_t bh = blockIdx.x / nch;
+  const int c = blockIdx.x % nch + (MODE == MODE_RSTATE ? 1 : 0);
+  const int h = (int)(bh % g.H);
+  const int64_t a = (int64_t)c * g.Lc;
+  const int64_t b = g.L < a + g.Lc ? g.L : a + g.Lc;
+  const int nblk = (int)((b - a + BLOCK - 1) / BLOCK);
+  auto block_of = [&](int j) { return REV ? nblk - 1 - j : j; };
+  auto p_of = [&](int j) { return a + (int64_t)block_of(j) * BLOCK; };
+  auto cb_of = [&](int j) {
+    const int64_t r = b - p_of(j);
+    return (int)(r < BLOCK ? r : BLOCK);
+  };
+
+  if (tid <= BLOCK) pw[tid] = (float)pow_int((double)lambda[h], tid);
+  if (tid == 0) {
+    for (int s = 0; s < NS; s++) {
+      mbar_init(b_full + 8 * s, 1);
+      mbar_init(b_empty + 8 * s, 1);
+      mbar_init(b_pfull + 8 * s, 128);
+    }
+    mbar_init(b_sfull, 1);
+    mbar_init(b_sfull + 8, 1);
+    mbar_init(b_ofull, 1);
+    mbar_init(b_oempty, 128);
+    mbar_init(b_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    if (OUT) tma_prefetch_desc(&tm0);
+    tma_prefetch_desc(&tm1);
+    tma_prefetch_desc(&tm2);
+    if (OUT) tma_prefetch_desc(&tmo);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), LY::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int j = 0;
+      for (; j < nblk; j++) {
+        const int st = j % NS;
+        if (j >= NS && !mbar_wait(b_empty + 8 * st, (uint32_t)((j / NS - 1) & 1), abort_flag))
+          break;
+        const int y = (int)p_of(j), z = (int)bh;
+        const uint32_t bar = b_full + 8 * st;
+        uint32_t dst = sbase + st * LY::STAGE;
+        mbar_expect_tx(bar, LY::STAGE);
+        if (OUT) {
+          tma_load_3d(dst, &tm0, bar, 0, y, z);
+          tma_load_3d(dst + BOX, &tm0, bar, 64, y, z);
+          dst += TILE;
+        }
+        tma_load_3d(dst, &tm1, bar, 0, y, z);
+        tma_load_3d(dst + BOX, &tm1, bar, 64, y, z);
+        tma_load_3d(dst + TILE, &tm2, bar, 0, y, z);
+        tma_load_3d(dst + TILE + BOX, &tm2, bar, 64, y, z);
+      }
+      // every issued load has landed before shared memory is released
+      volatile int never = 0;
+      for (int k = j - NS < 0 ? 0 : j - NS; k < j; k++)
+        mbar_wait(b_full + 8 * (k % NS), (uint32_t)((k / NS) & 1), &never);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      auto stage_addr = [&](int j) { return sbase + (j % NS) * LY::STAGE; };
+      auto issue_S = [&](int j) {
+        const uint32_t sA0 = stage_addr(j), sB1 = sA0 + TILE;
+        const uint32_t d = tmem + 128u * (uint32_t)(j & 1);
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+          const uint32_t koff = (k >> 2) * BOX + (k & 3) * 32;
+          mma_ss(d, sdesc_sw128(sA0 + koff, 16, 1024), sdesc_sw128(sB1 + koff, 16, 1024),
+                 IDESC_S, k > 0);
+        }
+        mma_commit(b_sfull + 8 * (j & 1));
+      };
+      bool ok = true;
+      if (OUT && nblk > 0) {
+        ok = mbar_wait(b_full, 0, abort_flag);
+        if (ok) {
+          tc_fence_after();
+          issue_S(0);
+        }
+      }
+      for (int i = 0; ok && i < nblk; i++) {
+        if (OUT && i + 1 < nblk) {
+          ok = mbar_wait(b_full + 8 * ((i + 1) % NS), (uint32_t)(((i + 1) / NS) & 1), abort_flag);
+          if (ok && i >= 1) ok = mbar_wait(b_ofull, (uint32_t)((i - 1) & 1), abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          issue_S(i + 1);
+        }
+        ok = mbar_wait(b_pfull + 8 * (i % NS), (uint32_t)((i / NS) & 1), abort_flag);
+        if (ok) ok = mbar_wait(b_oempty, (uint32_t)(i & 1), abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t sA0 = stage_addr(i);
+        const uint32_t sB1 = OUT ? sA0 + TILE : sA0;
+        const uint32_t sB2 = sB1 + TILE;
+        if (OUT) {
+          const uint32_t pa = tmem + 128u * (uint32_t)(i & 1);
+          const uint32_t sKV = sbase + LY::KVBF;
+#pragma unroll
+          for (int k = 0; k < 8; k++)
+            mma_ts(tmem + LY::COL_O, pa + 8 * k, sdesc_sw128(sB2 + k * 2048, BOX, 1024), IDESC_Y,
+                   k > 0);
+#pragma unroll
+          for (int k = 0; k < 8; k++) {
+            const uint32_t koff = (k >> 2) * BOX + (k & 3) * 32;
+            const uint64_t bd = TR::X_MN ? sdesc_sw128(sKV + k * 2048, BOX, 1024)
+                                         : sdesc_sw128(sKV + koff, 16, 1024);
+            mma_ss(tmem + LY::COL_O, sdesc_sw128(sA0 + koff, 16, 1024), bd, IDESC_X, 1);
+          }
+        }
+        const uint32_t sA = TR::SWAP ? sB2 : sB1;
+        const uint32_t sB = TR::SWAP ? sB1 : sB2;
+#pragma unroll
+        for (int k = 0; k < 8; k++)
+          mma_ss(tmem + LY::COL_KV, sdesc_sw128(sA + k * 2048, BOX, 1024),
+                 sdesc_sw128(sB + k * 2048, BOX, 1024), IDESC_D, 1);
+        // test hook: CTA 0 withholds its first completion signal
+        if (!(g.inject && blockIdx.x == 0 && i == 0)) mma_commit(b_ofull);
+      }
+      // all MMAs issued by this thread have finished before TMEM is freed
+      mma_commit(b_done);
+      volatile int never = 0;
+      mbar_wait(b_done, 0, &never);
+    }
+  } else if (warp < 6) {
+    // -------------------------------------------------------- mask warps
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    for (int i = 0; i < nblk; i++) {
+      const int st = i % NS;
+      const int cb = cb_of(i);
+      bool ok = OUT ? mbar_wait(b_sfull + 8 * (i & 1), (uint32_t)((i >> 1) & 1), abort_flag)
+                    : mbar_wait(b_full + 8 * st, (uint32_t)((i / NS) & 1), abort_flag);
+      if (role_any(!ok, BAR_MASK, 128)) break;
+      tc_fence_after();
+      uint8_t *stage = smem + st * LY::STAGE;
+      uint8_t *B1 = OUT ? stage + TILE : stage;
+      if (OUT) {
+        const uint32_t sb = 128u * (uint32_t)(i & 1);
+#pragma unroll
+        for (int part = 0; part < 4; part++) {
+          uint32_t r[32];
+          tmem_ld32(tl + sb + part * 32, r);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; j++) {
+            const int t0 = part * 32 + 2 * j, t1 = t0 + 1;
+            float f0, f1;
+            if (REV) {
+              f0 = t0 >= row ? __uint_as_float(r[2 * j]) * pw[t0 - row] : 0.f;
+              f1 = t1 >= row ? __uint_as_float(r[2 * j + 1]) * pw[t1 - row] : 0.f;
+            } else {
+              f0 = t0 <= row ? __uint_as_float(r[2 * j]) * pw[row - t0] : 0.f;
+              f1 = t1 <= row ? __uint_as_float(r[2 * j + 1]) * pw[row - t1] : 0.f;
+            }
+            pk[j] = pack_bf16x2(f0, f1);
+          }
+          tmem_st16(tl + sb + part * 16, pk);
+        }
+        // A0 rows carry the state term's row factor
+        const float f = REV ? (row < cb ? pw[cb - row] : 0.f) : pw[row + 1];
+        scale_row_sw128(stage, row, f);
+        scale_row_sw128(stage + BOX, row, f);
+      }
+      // B1 rows carry the state update's decay
+      const float fb = row < cb ? (REV ? pw[row] : pw[cb - 1 - row]) : 0.f;
+      scale_row_sw128(B1, row, fb);
+      scale_row_sw128(B1 + BOX, row, fb);
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(b_pfull + 8 * st);
+    }
+  } else {
+    // ---------------------------------------------------- epilogue warps
+    const int row = (warp & 3) * 32 + lane;
+    const int wtid = tid - 6 * 32;  // 0..127
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    uint8_t *kvbf = smem + LY::KVBF;
+    // initial state: TMEM (already decayed for block 0's update), bf16 copy
+    {
+      const float *init = nullptr;
+      if (MODE == MODE_FWD || MODE == MODE_DQ) {
+        if (c == 0) init = kv0 ? kv0 + bh * 128 * 128 : nullptr;
+        else init = ws + (bh * g.S + c) * (int64_t)128 * 128;
+      } else if (MODE == MODE_DV || MODE == MODE_DK) {
+        if (c != g.S - 1) init = ws + (bh * g.S + c) * (int64_t)128 * 128;
+      }
+      const float dec = pw[nblk > 0 ? cb_of(0) : 0];
+#pragma unroll
+      for (int part = 0; part < 4; part++) {
+        float f[32];
+        if (init) {
+          const float4 *src = reinterpret_cast<const float4 *>(init + (int64_t)row * 128 + part * 32);
+#pragma unroll
+          for (int j = 0; j < 8; j++) {
+            float4 x = src[j];
+            f[4 * j] = x.x; f[4 * j + 1] = x.y; f[4 * j + 2] = x.z; f[4 * j + 3] = x.w;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; j++) f[j] = 0.f;
+        }
+        if (OUT) st_row_bf16_sw128(kvbf + (part >> 1) * BOX, row, (part & 1) * 4, f);
+        uint32_t r[32];
+#pragma unroll
+        for (int j = 0; j < 32; j++) r[j] = __float_as_uint(f[j] * dec);
+        tmem_st32(tl + LY::COL_KV + part * 32, r);
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(b_oempty);
+    }
+    float *dst = nullptr;
+    float dscale = 1.f;
+    if (MODE == MODE_FWD) dst = (kv_out && c == g.S - 1) ? kv_out + bh * 128 * 128 : nullptr;
+    if (MODE == MODE_STATE) dst = ws + (bh * g.S + c + 1) * (int64_t)128 * 128;
+    if (MODE == MODE_RSTATE) dst = ws + (bh * g.S + c - 1) * (int64_t)128 * 128;
+    if (MODE == MODE_DV && c == 0 && kv_out) {  // dkv0 = lambda * D(0)
+      dst = kv_out + bh * 128 * 128;
+      dscale = lambda[h];
+    }
+    for (int i = 0; i < nblk; i++) {
+      const int st = i % NS;
+      bool ok = mbar_wait(b_ofull, (uint32_t)(i & 1), abort_flag);
+      if (role_any(!ok, BAR_EPI, 128)) break;
+      tc_fence_after();
+      uint8_t *stg = smem + st * LY::STAGE;  // A0's slot
+      if (OUT) {
+#pragma unroll
+        for (int part = 0; part < 4; part++) {
+          uint32_t r[32];
+          tmem_ld32(tl + LY::COL_O + part * 32, r);
+          tmem_wait_ld();
+          float o[32];
+#pragma unroll
+          for (int j = 0; j < 32; j++) o[j] = __uint_as_float(r[j]);
+          st_row_bf16_sw128(stg + (part >> 1) * BOX, row, (part & 1) * 4, o);
+        }
+      }
+      const bool last = i == nblk - 1;
+      const float dec = last ? 1.f : pw[cb_of(i + 1)];
+#pragma unroll
+      for (int part = 0; part < 4; part++) {
+        uint32_t r[32];
+        tmem_ld32(tl + LY::COL_KV + part * 32, r);
+        tmem_wait_ld();
+        if (!last) {
+          if (OUT) {
+            float f[32];
+#pragma unroll
+            for (int j = 0; j < 32; j++) f[j] = __uint_as_float(r[j]);
+            st_row_bf16_sw128(kvbf + (part >> 1) * BOX, row, (part & 1) * 4, f);
+          }
+#pragma unroll
+          for (int j = 0; j < 32; j++) r[j] = __float_as_uint(__uint_as_float(r[j]) * dec);
+          tmem_st32(tl + LY::COL_KV + part * 32, r);
+        } else if (dst) {
+          float4 *d4 = reinterpret_cast<float4 *>(dst + (int64_t)row * 128 + part * 32);
+#pragma unroll
+          for (int j = 0; j < 8; j++)
+            d4[j] = make_float4(dscale * __uint_as_float(r[4 * j]), dscale * __uint_as_float(r[4 * j + 1]),
+                                dscale * __uint_as_float(r[4 * j + 2]), dscale * __uint_as_float(r[4 * j + 3]));
+        }
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(b_oempty);
+      if (OUT) role_sync(BAR_EPI, 128);  // the whole output tile is in shared memory
+      if (wtid == 0) {
+        if (OUT) {
+          const uint32_t sst = sbase + st * LY::STAGE;
+          const int y = (int)p_of(i), z = (int)bh;
+          tma_store_3d(&tmo, sst, 0, y, z);
+          tma_store_3d(&tmo, sst + BOX, 64, y, z);
+          tma_store_commit();
+          tma_store_wait_read0();
+        }
+        mbar_arrive(b_empty + 8 * st);
+      }
+    }
+    if (OUT && wtid == 0) tma_store_wait0();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, LY::TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ host
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -475,13 +883,21 @@ template <int MODE>
 cudaError_t launch_chunk(const CUtensorMap &m0, const CUtensorMap &m1, const CUtensorMap &m2,
                          const CUtensorMap &mo, const float *lam, const float *kv0, float *ws,
                          float *kv_out, const Geo &g, cudaStream_t st) {
-  using LY = Layout<MODE>;
-  auto k = chunk_kernel<MODE>;
+  const int64_t nch = Layout<MODE>::OUT ? g.S : g.S - 1;
+  const int64_t grid = (int64_t)g.B * g.H * nch;
+  if (g.variant == 1) {  // first (phase-serial) form of the kernel
+    using LY = Layout<MODE>;
+    auto k = chunk_kernel<MODE>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::SMEM);
+    if (e != cudaSuccess) return e;
+    k<<<(unsigned)grid, NT, LY::SMEM, st>>>(m0, m1, m2, mo, lam, kv0, ws, kv_out, g);
+    return cudaGetLastError();
+  }
+  using LY = Layout2<MODE>;
+  auto k = chunk_kernel2<MODE>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::SMEM);
   if (e != cudaSuccess) return e;
-  const int64_t nch = LY::OUT ? g.S : g.S - 1;
-  const int64_t grid = (int64_t)g.B * g.H * nch;
-  k<<<(unsigned)grid, NT, LY::SMEM, st>>>(m0, m1, m2, mo, lam, kv0, ws, kv_out, g);
+  k<<<(unsigned)grid, NT2, LY::SMEM, st>>>(m0, m1, m2, mo, lam, kv0, ws, kv_out, g);
   return cudaGetLastError();
 }
 

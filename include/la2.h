@@ -153,10 +153,12 @@ const char *la2_status_string(la2_status s);
  * LA2_OPT_INJECT_TIMEOUT (test hook): when nonzero, the next tensor-core
  * la2_forward withholds one internal completion signal in its first CTA, so
  * that CTA's bounded wait gives up (about 2 s) and la2_last_device_error()
- * then reports LA2_ERR_TIMEOUT; the option resets itself.  Returns the
- * previous value, or -1 for an unknown option.
+ * then reports LA2_ERR_TIMEOUT; the option resets itself.
+ * LA2_OPT_VARIANT: form of the tensor-core kernel (0 = warp-specialised,
+ * the default; 1 = the simpler phase-serial form, kept for comparison).
+ * Returns the previous value, or -1 for an unknown option.
  */
-enum { LA2_OPT_SPLIT = 0, LA2_OPT_PATH = 1, LA2_OPT_INJECT_TIMEOUT = 2 };
+enum { LA2_OPT_SPLIT = 0, LA2_OPT_PATH = 1, LA2_OPT_INJECT_TIMEOUT = 2, LA2_OPT_VARIANT = 3 };
 int la2_set_option(int option, int value);
 
 /*

@@ -21,9 +21,10 @@ PATHS = {"simt": 1, "tc": 2}
 
 
 @contextlib.contextmanager
-def options(path=None, split=None):
+def options(path=None, split=None, variant=None):
     old_p = la2.set_option(la2.LA2_OPT_PATH, PATHS[path]) if path else None
     old_s = la2.set_option(la2.LA2_OPT_SPLIT, split) if split is not None else None
+    old_v = la2.set_option(la2.LA2_OPT_VARIANT, variant) if variant is not None else None
     try:
         yield
     finally:
@@ -31,6 +32,8 @@ def options(path=None, split=None):
             la2.set_option(la2.LA2_OPT_PATH, old_p)
         if split is not None:
             la2.set_option(la2.LA2_OPT_SPLIT, old_s)
+        if variant is not None:
+            la2.set_option(la2.LA2_OPT_VARIANT, old_v)
 
 
 def run_fwd_bwd(x, lam, kv0=None):
@@ -114,6 +117,19 @@ def test_forced_split(orc, path, split):
     if got is None:
         pytest.skip(f"{path} path unavailable")
     compare(got, oracle_all(orc, x, lam, x["kv0"]), torch.bfloat16, f"{path} S={split}")
+
+
+@pytest.mark.parametrize("split", [1, 3])
+@pytest.mark.parametrize("L", [200, 1000])
+def test_tc_phase_serial_variant(orc, L, split):
+    """The simpler phase-serial form of the tensor-core kernel (kept for
+    comparison) gives the oracle's result too."""
+    x = inputs.make_inputs(2, 2, L, 128, 128, dtype=torch.bfloat16, device=DEV, seed=L,
+                           with_kv0=True)
+    lam = inputs.fixed_lambdas((0.9, 1.0), DEV)
+    with options(path="tc", split=split, variant=1):
+        got = run_fwd_bwd(x, lam, x["kv0"])
+    compare(got, oracle_all(orc, x, lam, x["kv0"]), torch.bfloat16, f"v1 L={L} S={split}")
 
 
 def test_split_invariance_gpu():
