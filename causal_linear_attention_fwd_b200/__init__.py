@@ -11,7 +11,7 @@ its absence raises an error: there is no CPU fallback.
 """
 from ._binding import (  # noqa: F401
     LA2Error, LA2_OP_BACKWARD, LA2_OP_FORWARD, LA2_OPT_INJECT_TIMEOUT, LA2_OPT_PATH,
-    LA2_OPT_SPLIT, LA2_OPT_VARIANT,
+    LA2_OPT_SPLIT, LA2_OPT_TRACE, LA2_OPT_VARIANT, trace_read,
     backward, decode_step, forward, last_device_error, library, profile_enable,
     profile_report, set_option, status_string, version, workspace_size)
 

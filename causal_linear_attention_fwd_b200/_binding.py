@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(HERE, "libla2.so")
 LA2_OK, LA2_ERR_INVALID, LA2_ERR_UNSUPPORTED, LA2_ERR_CUDA, LA2_ERR_TIMEOUT = range(5)
 LA2_F32, LA2_BF16 = 0, 1
 LA2_OP_FORWARD, LA2_OP_BACKWARD = 0, 1
-LA2_OPT_SPLIT, LA2_OPT_PATH, LA2_OPT_INJECT_TIMEOUT, LA2_OPT_VARIANT = 0, 1, 2, 3
+LA2_OPT_SPLIT, LA2_OPT_PATH, LA2_OPT_INJECT_TIMEOUT, LA2_OPT_VARIANT, LA2_OPT_TRACE = 0, 1, 2, 3, 4
 
 _lock = threading.Lock()
 _lib = None
@@ -64,6 +64,8 @@ def library():
         lib.la2_profile_enable.restype = None
         lib.la2_profile_report.argtypes = [ctypes.c_char_p, SZ]
         lib.la2_profile_report.restype = SZ
+        lib.la2_trace_read.argtypes = [P, SZ]
+        lib.la2_trace_read.restype = SZ
         lib.la2_version.argtypes = []
         lib.la2_version.restype = ctypes.c_char_p
         _lib = lib
@@ -203,6 +205,15 @@ def decode_step(q, k, v, lam, kv, *, out=None, stream=None):
 
 def last_device_error(stream=None) -> int:
     return int(library().la2_last_device_error(_stream(stream)))
+
+
+def trace_read():
+    """Trace buffer as a [16 events, 512 blocks] int64 tensor (ns; 0 = unset)."""
+    lib = library()
+    n = int(lib.la2_trace_read(None, 0))
+    buf = torch.zeros(n, dtype=torch.int64)
+    lib.la2_trace_read(ctypes.c_void_p(buf.data_ptr()), n)
+    return buf.view(16, -1)
 
 
 def profile_enable(on: bool = True):

@@ -25,6 +25,7 @@ std::atomic<int> g_opt_split{0};
 std::atomic<int> g_opt_path{0};
 std::atomic<int> g_opt_inject{0};
 std::atomic<int> g_opt_variant{0};
+std::atomic<int> g_opt_trace{0};
 
 // ------------------------------------------------------------ profiling
 enum KernelId {
@@ -147,6 +148,7 @@ Geo plan(int B, int H, int64_t L, int blk, Path path) {
   Geo g;
   g.inject = 0;
   g.variant = g_opt_variant.load();
+  g.trace = g_opt_trace.load() - 1;
   g.B = B;
   g.H = H;
   g.L = L;
@@ -291,6 +293,7 @@ int la2_set_option(int option, int value) {
   if (option == LA2_OPT_PATH) return g_opt_path.exchange(value);
   if (option == LA2_OPT_INJECT_TIMEOUT) return g_opt_inject.exchange(value);
   if (option == LA2_OPT_VARIANT) return g_opt_variant.exchange(value);
+  if (option == LA2_OPT_TRACE) return g_opt_trace.exchange(value);
   return -1;
 }
 
@@ -446,6 +449,17 @@ la2_status la2_last_device_error(cudaStream_t stream) {
   if (word & la2::ERR_TIMEOUT) return LA2_ERR_TIMEOUT;
   if (word) return LA2_ERR_CUDA;
   return LA2_OK;
+}
+
+size_t la2_trace_read(uint64_t *out, size_t n) {
+  const size_t total = (size_t)la2::kTraceEvents * la2::kTraceBlocks;
+  if (!out || n == 0) return total;
+  if (cudaDeviceSynchronize() != cudaSuccess) return 0;
+  const size_t m = n < total ? n : total;
+  if (cudaMemcpyFromSymbol(out, la2::g_trace, m * sizeof(uint64_t)) != cudaSuccess) return 0;
+  static const unsigned long long zeros[la2::kTraceEvents * la2::kTraceBlocks] = {0};
+  cudaMemcpyToSymbol(la2::g_trace, zeros, sizeof(zeros));
+  return m;
 }
 
 void la2_profile_enable(int on) { g_prof_on.store(on ? 1 : 0); }

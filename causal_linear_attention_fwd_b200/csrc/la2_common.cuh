@@ -18,6 +18,11 @@ __device__ unsigned int g_error_word = 0;
 
 enum : unsigned int { ERR_TIMEOUT = 1u, ERR_BOUNDS = 2u };
 
+// Trace buffer: when a pass is traced, CTA 0 stamps %globaltimer at fixed
+// points of each block into g_trace[event * kTraceBlocks + block].
+constexpr int kTraceEvents = 16, kTraceBlocks = 512;
+__device__ unsigned long long g_trace[kTraceEvents * kTraceBlocks];
+
 __device__ __forceinline__ void raise_error(unsigned int bits) {
   atomicOr(&g_error_word, bits);
 }

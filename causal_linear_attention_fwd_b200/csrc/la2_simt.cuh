@@ -36,6 +36,7 @@ struct Geo {
   int inject;   // test hook: CTA 0 of a tensor-core pass withholds one MMA
                 // completion signal so that its bounded wait runs out
   int variant;  // tensor-core kernel form (0: warp-specialised, 1: phase-serial)
+  int trace;    // tensor-core pass whose CTA 0 stamps the trace buffer (-1: none)
 };
 
 namespace simt {

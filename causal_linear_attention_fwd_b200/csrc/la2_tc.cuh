@@ -468,6 +468,20 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
 // and stored, so tensor-core, CUDA-core and copy work overlap.
 constexpr int NT2 = 320;
 
+// Multiply one 64-element row of a swizzled box by f with packed bf16x2
+// multiplies (f rounded once to bf16; no unpack/repack through fp32).
+__device__ __forceinline__ void scale_row_sw128_bf16(uint8_t *box, int row, __nv_bfloat162 f2) {
+#pragma unroll
+  for (int c = 0; c < 8; c++) {
+    uint4 *p = reinterpret_cast<uint4 *>(box + row * 128 + ((c ^ (row & 7)) << 4));
+    uint4 w = *p;
+    __nv_bfloat162 *u = reinterpret_cast<__nv_bfloat162 *>(&w);
+#pragma unroll
+    for (int j = 0; j < 4; j++) u[j] = __hmul2(u[j], f2);
+    *p = w;
+  }
+}
+
 template <int MODE> struct Layout2 {
   static constexpr bool OUT = Traits<MODE>::OUT;
   static constexpr int NSTAGE = OUT ? 2 : 3;
@@ -476,7 +490,8 @@ template <int MODE> struct Layout2 {
   static constexpr uint32_t MISC = KVBF + (OUT ? TILE : 0);
   // full[NS] empty[NS] sfull[2] pfull[NS] ofull oempty done
   static constexpr uint32_t NBAR = 3 * NSTAGE + 5;
-  static constexpr uint32_t MISC_BYTES = 8 * NBAR + 16 + 4 * (BLOCK + 1);
+  // decay table: 128 zeros then lambda^0..lambda^128 (see chunk_kernel2)
+  static constexpr uint32_t MISC_BYTES = 8 * NBAR + 16 + 4 * (2 * BLOCK + 1);
   static constexpr uint32_t SMEM = MISC + MISC_BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = OUT ? 512 : 128;
   static constexpr uint32_t COL_O = 256;
@@ -499,6 +514,12 @@ __device__ __forceinline__ bool role_any(bool v, int id, int n) {
 __device__ __forceinline__ void role_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
+// Trace stamp (only CTA 0 of the traced pass records; events listed where used).
+#define LA2_TRACE(ev, blk)                                                                \
+  do {                                                                                    \
+    if (tracing && (blk) < kTraceBlocks) g_trace[(ev) * kTraceBlocks + (blk)] = globaltimer(); \
+  } while (0)
+
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
@@ -527,7 +548,11 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + LY::MISC);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + LY::NBAR);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  float *pw = reinterpret_cast<float *>(tmem_slot + 4);
+  // pwz[k] = lambda^(k-128) for k >= 128, 0 below: pw = pwz + 128 holds
+  // lambda^0..lambda^128 and pw[n] for n in [-128, 0) reads as 0, which is
+  // the causal mask (a negative distance means a masked entry).
+  float *pwz = reinterpret_cast<float *>(tmem_slot + 4);
+  float *pw = pwz + 128;
   const uint32_t b_full = smem_u32(bars);
   const uint32_t b_empty = b_full + 8 * NS;
   const uint32_t b_sfull = b_empty + 8 * NS;
@@ -550,12 +575,19 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
     const int64_t r = b - p_of(j);
     return (int)(r < BLOCK ? r : BLOCK);
   };
+  // trace events: 0 load issued, 1 S issued, 2 P.B2/X/state issued, 3 mask
+  // start, 4 mask done, 5 epilogue start, 6 state handed back, 7 store read
+  // done, 8 kernel entry, 9 set-up done
+  const bool tracing = g.trace == MODE && blockIdx.x == 0;
+  if (tid == 0) LA2_TRACE(8, 0);
 
   if (tid <= BLOCK) pw[tid] = (float)pow_int((double)lambda[h], tid);
+  if (tid < BLOCK) pwz[tid] = 0.f;
   if (tid == 0) {
     for (int s = 0; s < NS; s++) {
       mbar_init(b_full + 8 * s, 1);
       mbar_init(b_empty + 8 * s, 1);
+      // P written and the A0 / B1 row decays applied (mask warps)
       mbar_init(b_pfull + 8 * s, 128);
     }
     mbar_init(b_sfull, 1);
@@ -578,6 +610,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (tid == 0) LA2_TRACE(9, 0);
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
@@ -600,6 +633,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
         tma_load_3d(dst + BOX, &tm1, bar, 64, y, z);
         tma_load_3d(dst + TILE, &tm2, bar, 0, y, z);
         tma_load_3d(dst + TILE + BOX, &tm2, bar, 64, y, z);
+        LA2_TRACE(0, j);
       }
       // every issued load has landed before shared memory is released
       volatile int never = 0;
@@ -620,27 +654,9 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
                  IDESC_S, k > 0);
         }
         mma_commit(b_sfull + 8 * (j & 1));
+        LA2_TRACE(1, j);
       };
-      bool ok = true;
-      if (OUT && nblk > 0) {
-        ok = mbar_wait(b_full, 0, abort_flag);
-        if (ok) {
-          tc_fence_after();
-          issue_S(0);
-        }
-      }
-      for (int i = 0; ok && i < nblk; i++) {
-        if (OUT && i + 1 < nblk) {
-          ok = mbar_wait(b_full + 8 * ((i + 1) % NS), (uint32_t)(((i + 1) / NS) & 1), abort_flag);
-          if (ok && i >= 1) ok = mbar_wait(b_ofull, (uint32_t)((i - 1) & 1), abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          issue_S(i + 1);
-        }
-        ok = mbar_wait(b_pfull + 8 * (i % NS), (uint32_t)((i / NS) & 1), abort_flag);
-        if (ok) ok = mbar_wait(b_oempty, (uint32_t)(i & 1), abort_flag);
-        if (!ok) break;
-        tc_fence_after();
+      auto issue_P3 = [&](int i) {
         const uint32_t sA0 = stage_addr(i);
         const uint32_t sB1 = OUT ? sA0 + TILE : sA0;
         const uint32_t sB2 = sB1 + TILE;
@@ -667,6 +683,48 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
                  sdesc_sw128(sB + k * 2048, BOX, 1024), IDESC_D, 1);
         // test hook: CTA 0 withholds its first completion signal
         if (!(g.inject && blockIdx.x == 0 && i == 0)) mma_commit(b_ofull);
+        LA2_TRACE(2, i);
+      };
+      // Two streams of work are issued as their inputs become ready, polled
+      // without blocking: S of block j (tiles loaded, its TMEM buffer free,
+      // i.e. the products of block j-2 done) and the products of block i (P
+      // and row decays ready, state handed back).  The products take
+      // priority.  nS / nP count issued S / product groups, seen counts
+      // completed product groups; at most one product group is in flight and
+      // S of block j needs products j-2 done, so no waiter can fall two
+      // phases behind a barrier.
+      int nS = 0, nP = 0, seen = 0;
+      uint64_t t_last = globaltimer();
+      while (nP < nblk) {
+        bool did = false;
+        if ((!OUT || nS > nP) && seen >= nP &&
+            mbar_test(b_pfull + 8 * (nP % NS), (uint32_t)((nP / NS) & 1)) &&
+            mbar_test(b_oempty, (uint32_t)(nP & 1))) {
+          tc_fence_after();
+          issue_P3(nP);
+          nP++;
+          did = true;
+        }
+        if (OUT && nS < nblk && seen >= nS - 1 &&
+            mbar_test(b_full + 8 * (nS % NS), (uint32_t)((nS / NS) & 1))) {
+          tc_fence_after();
+          issue_S(nS);
+          nS++;
+          did = true;
+        }
+        if (seen < nP && mbar_test(b_ofull, (uint32_t)(seen & 1))) {
+          seen++;
+          did = true;
+        }
+        if (did) {
+          t_last = globaltimer();
+        } else if (*abort_flag) {
+          break;
+        } else if (globaltimer() - t_last > kWaitTimeoutNs) {
+          *abort_flag = 1;
+          raise_error(ERR_TIMEOUT);
+          break;
+        }
       }
       // all MMAs issued by this thread have finished before TMEM is freed
       mma_commit(b_done);
@@ -684,43 +742,47 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
                     : mbar_wait(b_full + 8 * st, (uint32_t)((i / NS) & 1), abort_flag);
       if (role_any(!ok, BAR_MASK, 128)) break;
       tc_fence_after();
+      if (row == 0) LA2_TRACE(3, i);
       uint8_t *stage = smem + st * LY::STAGE;
       uint8_t *B1 = OUT ? stage + TILE : stage;
       if (OUT) {
         const uint32_t sb = 128u * (uint32_t)(i & 1);
 #pragma unroll
-        for (int part = 0; part < 4; part++) {
-          uint32_t r[32];
-          tmem_ld32(tl + sb + part * 32, r);
+        for (int pair = 0; pair < 2; pair++) {
+          uint32_t r[64];
+          tmem_ld32(tl + sb + pair * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          tmem_ld32(tl + sb + pair * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
           tmem_wait_ld();
-          uint32_t pk[16];
+          uint32_t pk[32];
 #pragma unroll
-          for (int j = 0; j < 16; j++) {
-            const int t0 = part * 32 + 2 * j, t1 = t0 + 1;
-            float f0, f1;
-            if (REV) {
-              f0 = t0 >= row ? __uint_as_float(r[2 * j]) * pw[t0 - row] : 0.f;
-              f1 = t1 >= row ? __uint_as_float(r[2 * j + 1]) * pw[t1 - row] : 0.f;
-            } else {
-              f0 = t0 <= row ? __uint_as_float(r[2 * j]) * pw[row - t0] : 0.f;
-              f1 = t1 <= row ? __uint_as_float(r[2 * j + 1]) * pw[row - t1] : 0.f;
-            }
+          for (int j = 0; j < 32; j++) {
+            const int t0 = pair * 64 + 2 * j;
+            // causal mask and decay in one lookup: distance < 0 reads 0
+            const int n0 = REV ? t0 - row : row - t0;
+            const float f0 = __uint_as_float(r[2 * j]) * pw[n0];
+            const float f1 = __uint_as_float(r[2 * j + 1]) * pw[REV ? n0 + 1 : n0 - 1];
             pk[j] = pack_bf16x2(f0, f1);
           }
-          tmem_st16(tl + sb + part * 16, pk);
+          tmem_st16(tl + sb + pair * 32, &pk[0]);
+          tmem_st16(tl + sb + pair * 32 + 16, &pk[16]);
         }
         // A0 rows carry the state term's row factor
         const float f = REV ? (row < cb ? pw[cb - row] : 0.f) : pw[row + 1];
-        scale_row_sw128(stage, row, f);
-        scale_row_sw128(stage + BOX, row, f);
+        const __nv_bfloat162 f2 = __float2bfloat162_rn(f);
+        scale_row_sw128_bf16(stage, row, f2);
+        scale_row_sw128_bf16(stage + BOX, row, f2);
       }
       // B1 rows carry the state update's decay
-      const float fb = row < cb ? (REV ? pw[row] : pw[cb - 1 - row]) : 0.f;
-      scale_row_sw128(B1, row, fb);
-      scale_row_sw128(B1 + BOX, row, fb);
+      {
+        const float fb = row < cb ? (REV ? pw[row] : pw[cb - 1 - row]) : 0.f;
+        const __nv_bfloat162 fb2 = __float2bfloat162_rn(fb);
+        scale_row_sw128_bf16(B1, row, fb2);
+        scale_row_sw128_bf16(B1 + BOX, row, fb2);
+      }
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
+      if (row == 0) LA2_TRACE(4, i);
       mbar_arrive(b_pfull + 8 * st);
     }
   } else {
@@ -778,40 +840,40 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       bool ok = mbar_wait(b_ofull, (uint32_t)(i & 1), abort_flag);
       if (role_any(!ok, BAR_EPI, 128)) break;
       tc_fence_after();
+      if (wtid == 0) LA2_TRACE(5, i);
       uint8_t *stg = smem + st * LY::STAGE;  // A0's slot
       if (OUT) {
 #pragma unroll
-        for (int part = 0; part < 4; part++) {
-          uint32_t r[32];
-          tmem_ld32(tl + LY::COL_O + part * 32, r);
+        for (int pair = 0; pair < 2; pair++) {
+          uint32_t r[64];
+          tmem_ld32(tl + LY::COL_O + pair * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          tmem_ld32(tl + LY::COL_O + pair * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
           tmem_wait_ld();
-          float o[32];
-#pragma unroll
-          for (int j = 0; j < 32; j++) o[j] = __uint_as_float(r[j]);
-          st_row_bf16_sw128(stg + (part >> 1) * BOX, row, (part & 1) * 4, o);
+          st_row_bf16_sw128(stg + pair * BOX, row, 0, reinterpret_cast<const float *>(&r[0]));
+          st_row_bf16_sw128(stg + pair * BOX, row, 4, reinterpret_cast<const float *>(&r[32]));
         }
       }
       const bool last = i == nblk - 1;
       const float dec = last ? 1.f : pw[cb_of(i + 1)];
 #pragma unroll
-      for (int part = 0; part < 4; part++) {
-        uint32_t r[32];
-        tmem_ld32(tl + LY::COL_KV + part * 32, r);
+      for (int pair = 0; pair < 2; pair++) {
+        uint32_t r[64];
+        tmem_ld32(tl + LY::COL_KV + pair * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(tl + LY::COL_KV + pair * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         tmem_wait_ld();
         if (!last) {
           if (OUT) {
-            float f[32];
-#pragma unroll
-            for (int j = 0; j < 32; j++) f[j] = __uint_as_float(r[j]);
-            st_row_bf16_sw128(kvbf + (part >> 1) * BOX, row, (part & 1) * 4, f);
+            st_row_bf16_sw128(kvbf + pair * BOX, row, 0, reinterpret_cast<const float *>(&r[0]));
+            st_row_bf16_sw128(kvbf + pair * BOX, row, 4, reinterpret_cast<const float *>(&r[32]));
           }
 #pragma unroll
-          for (int j = 0; j < 32; j++) r[j] = __float_as_uint(__uint_as_float(r[j]) * dec);
-          tmem_st32(tl + LY::COL_KV + part * 32, r);
+          for (int j = 0; j < 64; j++) r[j] = __float_as_uint(__uint_as_float(r[j]) * dec);
+          tmem_st32(tl + LY::COL_KV + pair * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          tmem_st32(tl + LY::COL_KV + pair * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         } else if (dst) {
-          float4 *d4 = reinterpret_cast<float4 *>(dst + (int64_t)row * 128 + part * 32);
+          float4 *d4 = reinterpret_cast<float4 *>(dst + (int64_t)row * 128 + pair * 64);
 #pragma unroll
-          for (int j = 0; j < 8; j++)
+          for (int j = 0; j < 16; j++)
             d4[j] = make_float4(dscale * __uint_as_float(r[4 * j]), dscale * __uint_as_float(r[4 * j + 1]),
                                 dscale * __uint_as_float(r[4 * j + 2]), dscale * __uint_as_float(r[4 * j + 3]));
         }
@@ -819,6 +881,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
+      if (wtid == 0) LA2_TRACE(6, i);
       mbar_arrive(b_oempty);
       if (OUT) role_sync(BAR_EPI, 128);  // the whole output tile is in shared memory
       if (wtid == 0) {
@@ -830,6 +893,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
           tma_store_commit();
           tma_store_wait_read0();
         }
+        LA2_TRACE(7, i);
         mbar_arrive(b_empty + 8 * st);
       }
     }

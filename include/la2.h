@@ -156,9 +156,27 @@ const char *la2_status_string(la2_status s);
  * then reports LA2_ERR_TIMEOUT; the option resets itself.
  * LA2_OPT_VARIANT: form of the tensor-core kernel (0 = warp-specialised,
  * the default; 1 = the simpler phase-serial form, kept for comparison).
- * Returns the previous value, or -1 for an unknown option.
+ * LA2_OPT_TRACE: 0 = off; p + 1 = while set, the first CTA of every launch
+ * of tensor-core pass p (0 forward, 1 dQ, 2 forward chunk state, 3 dV,
+ * 4 dK, 5 reverse chunk state) of the warp-specialised kernel stamps the
+ * device clock at fixed points of each block into the trace buffer (see
+ * la2_trace_read).  Returns the previous value, or -1 for an unknown option.
  */
-enum { LA2_OPT_SPLIT = 0, LA2_OPT_PATH = 1, LA2_OPT_INJECT_TIMEOUT = 2, LA2_OPT_VARIANT = 3 };
+enum {
+    LA2_OPT_SPLIT = 0, LA2_OPT_PATH = 1, LA2_OPT_INJECT_TIMEOUT = 2, LA2_OPT_VARIANT = 3,
+    LA2_OPT_TRACE = 4
+};
+
+/*
+ * Synchronises the device and copies the trace buffer (uint64 nanosecond
+ * stamps, laid out [event][block] with 16 events x 512 blocks; 0 = not
+ * recorded) into host memory `out` (n entries at most), then clears it.
+ * Events: 0 loads issued, 1 S = A0 B1^T issued, 2 P.B2 / state term / state
+ * update issued, 3 mask start, 4 mask done, 5 epilogue start, 6 state handed
+ * back to the MMA issuer, 7 output tile read by the store, 8 kernel entry,
+ * 9 set-up done.  With out == NULL returns the buffer's entry count.
+ */
+size_t la2_trace_read(uint64_t *out, size_t n);
 int la2_set_option(int option, int value);
 
 /*
