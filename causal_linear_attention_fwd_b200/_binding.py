@@ -49,6 +49,8 @@ def library():
         lib.la2_workspace_size.restype = SZ
         lib.la2_forward.argtypes = [P, P, P, P, P, P, P, I, I, I64, I, I, I, P, SZ, P]
         lib.la2_forward.restype = I
+        lib.la2_forward_noalloc.argtypes = [P, P, P, P, P, P, P, I, I, I64, I, I, I, P]
+        lib.la2_forward_noalloc.restype = I
         lib.la2_backward.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I64, I, I, I,
                                      P, SZ, P]
         lib.la2_backward.restype = I
@@ -153,6 +155,29 @@ def forward(q, k, v, lam, kv0=None, *, want_state: bool = False, out=None,
                            B, H, L, d, e, _dt(q), _ptr(ws), 0 if ws is None else ws.numel(),
                            _stream(stream))
     _check(code, "la2_forward")
+    return (o, st) if want_state else o
+
+
+def forward_noalloc(q, k, v, lam, kv0=None, *, want_state: bool = False, out=None,
+                    stream=None):
+    """forward() for callers that cannot allocate device scratch: the library
+    keeps the chunk-boundary states in its own fixed 32 MiB device array
+    (see la2_forward_noalloc in include/la2.h).  Outputs are still allocated
+    here unless `out` (and the caller's own state buffer) are passed."""
+    lib = library()
+    for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam)):
+        _dev(t, name)
+    B, H, L, d = q.shape
+    e = v.shape[-1]
+    if k.shape != q.shape or v.shape[:3] != (B, H, L):
+        raise ValueError("shape mismatch among q, k, v")
+    if lam.dtype != torch.float32 or lam.numel() != H:
+        raise ValueError("lam must be float32 [H]")
+    o = out if out is not None else torch.empty((B, H, L, e), dtype=q.dtype, device=q.device)
+    st = torch.empty((B, H, d, e), dtype=torch.float32, device=q.device) if want_state else None
+    code = lib.la2_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(o),
+                                   _ptr(st), B, H, L, d, e, _dt(q), _stream(stream))
+    _check(code, "la2_forward_noalloc")
     return (o, st) if want_state else o
 
 

@@ -498,3 +498,57 @@ size_t la2_profile_report(char *buf, size_t buf_bytes) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------
+// Forward pass for callers that cannot allocate device memory.
+//
+// Some callers cannot call cudaMalloc or any allocating routine: plug-ins
+// whose host framework owns every byte of device memory through its own
+// allocator, latency-critical code paths where cudaMalloc's implicit device
+// synchronisation would stall other streams, and callbacks that receive only
+// device pointers and have no allocator at hand.  For them la2_forward_noalloc
+// takes the chunk-boundary states from the fixed array below instead of a
+// caller-provided workspace.  The array is part of the library's device
+// image: every GPU that loads the library holds it until the process exits.
+namespace {
+
+constexpr size_t kNoallocScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+// Device address of the array on the current device; looked up once per
+// device (host code cannot use the array's name as a device address).
+void *noalloc_scratch_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = p;
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" la2_status la2_forward_noalloc(const void *q, const void *k, const void *v,
+                                          const float *lambda, const float *kv0, void *o,
+                                          float *kv_out, int B, int H, int64_t L, int d, int e,
+                                          la2_dtype dt, cudaStream_t stream) {
+  // Same plan as la2_forward; refuse plans whose scratch exceeds the array.
+  if (B > 0 && H > 0 && L > 0 && shape_supported(d, e, dt)) {
+    const Path p = choose_path(d, e, dt);
+    if (p != PATH_NONE) {
+      const Geo g = plan(B, H, L, block_rows(p), p);
+      if (ws_bytes(LA2_OP_FORWARD, g, d, e) > kNoallocScratchBytes) return LA2_ERR_UNSUPPORTED;
+    }
+  }
+  void *scratch = noalloc_scratch_ptr();
+  if (!scratch) return LA2_ERR_CUDA;
+  return la2_forward(q, k, v, lambda, kv0, o, kv_out, B, H, L, d, e, dt, scratch,
+                     kNoallocScratchBytes, stream);
+}

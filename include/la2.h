@@ -104,6 +104,31 @@ la2_status la2_forward(const void *q, const void *k, const void *v,
                        cudaStream_t stream);
 
 /*
+ * Forward pass that allocates nothing and takes no workspace, for callers
+ * that cannot call cudaMalloc or any allocating routine (plug-ins whose host
+ * framework owns all device memory, latency-critical paths that cannot
+ * afford cudaMalloc's device synchronisation, callbacks that only receive
+ * device pointers).  The pages have no counterpart of this entry point; it
+ * is a convenience of this library.  Arguments, results and errors are those
+ * of la2_forward; the chunk-boundary states live instead in a fixed 32 MiB
+ * device array that every GPU loading the library holds until the process
+ * exits.  Calls whose plan needs more than 32 MiB of states (B*H*S*d*e*4
+ * bytes, S = chunks per sequence) return LA2_ERR_UNSUPPORTED before
+ * launching anything.  The first call on a device looks up the array's
+ * device address (once per device) and should come before any stream
+ * capture.  All calls share the array and it keeps the last call's contents
+ * (every state it holds is written before it is read, so nothing needs
+ * clearing); calls that overlap on the same GPU -- from concurrent streams
+ * or host threads -- race on it, so serialise them.  Each GPU has its own
+ * copy of the array.
+ */
+la2_status la2_forward_noalloc(const void *q, const void *k, const void *v,
+                               const float *lambda, const float *kv0,
+                               void *o, float *kv_out,
+                               int B, int H, int64_t L, int d, int e, la2_dtype dt,
+                               cudaStream_t stream);
+
+/*
  * Backward pass for an upstream gradient dO [B,H,L,e]: writes dq, dk [B,H,L,d],
  * dv [B,H,L,e] -- the gradients of sum(o * dO) -- and, when dkv0 is not NULL,
  * the gradient with respect to the initial state (fp32 [B,H,d,e]).  Inputs
