@@ -488,8 +488,14 @@ template <int MODE> struct Layout2 {
   static constexpr uint32_t STAGE = OUT ? 3 * TILE : 2 * TILE;
   static constexpr uint32_t KVBF = NSTAGE * STAGE;
   static constexpr uint32_t MISC = KVBF + (OUT ? TILE : 0);
-  // full[NS] empty[NS] sfull[2] pfull[NS] ofull oempty done
-  static constexpr uint32_t NBAR = 3 * NSTAGE + 5;
+  // Per stage two tile groups with their own full/empty barriers: "ab" =
+  // (A0, B1), freed as soon as the block's products are done; "c" = B2,
+  // which doubles as the output staging tile and is freed after the store.
+  // full_ab[NS] full_c[NS] empty_ab[NS] empty_c[NS] sfull[2] pfull[NS]
+  // ofull oempty done
+  static constexpr uint32_t NBAR = 5 * NSTAGE + 5;
+  static constexpr uint32_t AB_BYTES = OUT ? 2 * TILE : TILE;
+  static constexpr uint32_t C_OFF = AB_BYTES;
   // decay table: 128 zeros then lambda^0..lambda^128 (see chunk_kernel2)
   static constexpr uint32_t MISC_BYTES = 8 * NBAR + 16 + 4 * (2 * BLOCK + 1);
   static constexpr uint32_t SMEM = MISC + MISC_BYTES + 1024;
@@ -553,9 +559,11 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   // the causal mask (a negative distance means a masked entry).
   float *pwz = reinterpret_cast<float *>(tmem_slot + 4);
   float *pw = pwz + 128;
-  const uint32_t b_full = smem_u32(bars);
-  const uint32_t b_empty = b_full + 8 * NS;
-  const uint32_t b_sfull = b_empty + 8 * NS;
+  const uint32_t b_fab = smem_u32(bars);
+  const uint32_t b_fc = b_fab + 8 * NS;
+  const uint32_t b_eab = b_fc + 8 * NS;
+  const uint32_t b_ec = b_eab + 8 * NS;
+  const uint32_t b_sfull = b_ec + 8 * NS;
   const uint32_t b_pfull = b_sfull + 16;
   const uint32_t b_ofull = b_pfull + 8 * NS;
   const uint32_t b_oempty = b_ofull + 8;
@@ -585,8 +593,10 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   if (tid < BLOCK) pwz[tid] = 0.f;
   if (tid == 0) {
     for (int s = 0; s < NS; s++) {
-      mbar_init(b_full + 8 * s, 1);
-      mbar_init(b_empty + 8 * s, 1);
+      mbar_init(b_fab + 8 * s, 1);
+      mbar_init(b_fc + 8 * s, 1);
+      mbar_init(b_eab + 8 * s, 1);
+      mbar_init(b_ec + 8 * s, 1);
       // P written and the A0 / B1 row decays applied (mask warps)
       mbar_init(b_pfull + 8 * s, 128);
     }
@@ -615,30 +625,38 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int j = 0;
-      for (; j < nblk; j++) {
+      int nab = 0, nc = 0;  // blocks whose (A0, B1) / B2 loads were issued
+      for (int j = 0; j < nblk; j++) {
         const int st = j % NS;
-        if (j >= NS && !mbar_wait(b_empty + 8 * st, (uint32_t)((j / NS - 1) & 1), abort_flag))
-          break;
+        const uint32_t ph = (uint32_t)((j / NS - 1) & 1);
         const int y = (int)p_of(j), z = (int)bh;
-        const uint32_t bar = b_full + 8 * st;
         uint32_t dst = sbase + st * LY::STAGE;
-        mbar_expect_tx(bar, LY::STAGE);
+        // (A0, B1): their slots free once block j-NS's products are done
+        if (j >= NS && !mbar_wait(b_eab + 8 * st, ph, abort_flag)) break;
+        mbar_expect_tx(b_fab + 8 * st, LY::AB_BYTES);
         if (OUT) {
-          tma_load_3d(dst, &tm0, bar, 0, y, z);
-          tma_load_3d(dst + BOX, &tm0, bar, 64, y, z);
+          tma_load_3d(dst, &tm0, b_fab + 8 * st, 0, y, z);
+          tma_load_3d(dst + BOX, &tm0, b_fab + 8 * st, 64, y, z);
           dst += TILE;
         }
-        tma_load_3d(dst, &tm1, bar, 0, y, z);
-        tma_load_3d(dst + BOX, &tm1, bar, 64, y, z);
-        tma_load_3d(dst + TILE, &tm2, bar, 0, y, z);
-        tma_load_3d(dst + TILE + BOX, &tm2, bar, 64, y, z);
+        tma_load_3d(dst, &tm1, b_fab + 8 * st, 0, y, z);
+        tma_load_3d(dst + BOX, &tm1, b_fab + 8 * st, 64, y, z);
+        nab++;
+        // B2: its slot free once block j-NS's output has left it
+        if (j >= NS && !mbar_wait(b_ec + 8 * st, ph, abort_flag)) break;
+        dst = sbase + st * LY::STAGE + LY::C_OFF;
+        mbar_expect_tx(b_fc + 8 * st, TILE);
+        tma_load_3d(dst, &tm2, b_fc + 8 * st, 0, y, z);
+        tma_load_3d(dst + BOX, &tm2, b_fc + 8 * st, 64, y, z);
+        nc++;
         LA2_TRACE(0, j);
       }
       // every issued load has landed before shared memory is released
       volatile int never = 0;
-      for (int k = j - NS < 0 ? 0 : j - NS; k < j; k++)
-        mbar_wait(b_full + 8 * (k % NS), (uint32_t)((k / NS) & 1), &never);
+      for (int k = nab - NS < 0 ? 0 : nab - NS; k < nab; k++)
+        mbar_wait(b_fab + 8 * (k % NS), (uint32_t)((k / NS) & 1), &never);
+      for (int k = nc - NS < 0 ? 0 : nc - NS; k < nc; k++)
+        mbar_wait(b_fc + 8 * (k % NS), (uint32_t)((k / NS) & 1), &never);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
@@ -659,7 +677,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       auto issue_P3 = [&](int i) {
         const uint32_t sA0 = stage_addr(i);
         const uint32_t sB1 = OUT ? sA0 + TILE : sA0;
-        const uint32_t sB2 = sB1 + TILE;
+        const uint32_t sB2 = sA0 + LY::C_OFF;
         if (OUT) {
           const uint32_t pa = tmem + 128u * (uint32_t)(i & 1);
           const uint32_t sKV = sbase + LY::KVBF;
@@ -683,6 +701,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
                  sdesc_sw128(sB + k * 2048, BOX, 1024), IDESC_D, 1);
         // test hook: CTA 0 withholds its first completion signal
         if (!(g.inject && blockIdx.x == 0 && i == 0)) mma_commit(b_ofull);
+        mma_commit(b_eab + 8 * (i % NS));  // A0, B1 slots reusable
         LA2_TRACE(2, i);
       };
       // Two streams of work are issued as their inputs become ready, polled
@@ -699,6 +718,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
         bool did = false;
         if ((!OUT || nS > nP) && seen >= nP &&
             mbar_test(b_pfull + 8 * (nP % NS), (uint32_t)((nP / NS) & 1)) &&
+            mbar_test(b_fc + 8 * (nP % NS), (uint32_t)((nP / NS) & 1)) &&
             mbar_test(b_oempty, (uint32_t)(nP & 1))) {
           tc_fence_after();
           issue_P3(nP);
@@ -706,7 +726,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
           did = true;
         }
         if (OUT && nS < nblk && seen >= nS - 1 &&
-            mbar_test(b_full + 8 * (nS % NS), (uint32_t)((nS / NS) & 1))) {
+            mbar_test(b_fab + 8 * (nS % NS), (uint32_t)((nS / NS) & 1))) {
           tc_fence_after();
           issue_S(nS);
           nS++;
@@ -739,7 +759,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       const int st = i % NS;
       const int cb = cb_of(i);
       bool ok = OUT ? mbar_wait(b_sfull + 8 * (i & 1), (uint32_t)((i >> 1) & 1), abort_flag)
-                    : mbar_wait(b_full + 8 * st, (uint32_t)((i / NS) & 1), abort_flag);
+                    : mbar_wait(b_fab + 8 * st, (uint32_t)((i / NS) & 1), abort_flag);
       if (role_any(!ok, BAR_MASK, 128)) break;
       tc_fence_after();
       if (row == 0) LA2_TRACE(3, i);
@@ -841,7 +861,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       if (role_any(!ok, BAR_EPI, 128)) break;
       tc_fence_after();
       if (wtid == 0) LA2_TRACE(5, i);
-      uint8_t *stg = smem + st * LY::STAGE;  // A0's slot
+      uint8_t *stg = smem + st * LY::STAGE + LY::C_OFF;  // B2's slot
       if (OUT) {
 #pragma unroll
         for (int pair = 0; pair < 2; pair++) {
@@ -886,7 +906,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       if (OUT) role_sync(BAR_EPI, 128);  // the whole output tile is in shared memory
       if (wtid == 0) {
         if (OUT) {
-          const uint32_t sst = sbase + st * LY::STAGE;
+          const uint32_t sst = sbase + st * LY::STAGE + LY::C_OFF;
           const int y = (int)p_of(i), z = (int)bh;
           tma_store_3d(&tmo, sst, 0, y, z);
           tma_store_3d(&tmo, sst + BOX, 64, y, z);
@@ -894,7 +914,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
           tma_store_wait_read0();
         }
         LA2_TRACE(7, i);
-        mbar_arrive(b_empty + 8 * st);
+        mbar_arrive(b_ec + 8 * st);  // B2 slot reusable
       }
     }
     if (OUT && wtid == 0) tma_store_wait0();
