@@ -454,19 +454,20 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
 }
 
 // ================================================================ v2
-// Warp-specialised form of the same schedule.  Roles (320 threads):
-//   warp 0      TMA producer (one thread): fills the stage ring
-//   warp 1      MMA issuer (one thread)
-//   warps 2-5   "mask" warpgroup: P = S (.) M into TMEM, row decays of A0, B1
-//   warps 6-9   "epilogue" warpgroup: out -> bf16 -> TMA store, state ->
-//               bf16 operand copy, state *= lambda^cb for the next block
+// Warp-specialised form of the same schedule.  Roles (448 threads):
+//   warp 0       TMA producer (one thread): fills the stage ring
+//   warp 1       MMA issuer (one thread)
+//   warps 2-5    "mask" warpgroup: P = S (.) M into TMEM
+//   warps 6-9    "epilogue" warpgroup: out -> bf16 -> TMA store, state ->
+//                bf16 operand copy, state *= lambda^cb for the next block
+//   warps 10-13  "decay" warpgroup: row decays of A0 and B1 in shared memory
 // The row factor of the state term is folded into A0 (A0 <- diag(f) A0 after
 // S = A0 B1^T has read it), so Y and X share one accumulator:
 //   O = P B2 + A0f * state.
 // TMEM: S double-buffered [0,128) and [128,256), O [256,384), state [384,512);
 // the MMA for S of block i+1 is issued while block i is still being masked
 // and stored, so tensor-core, CUDA-core and copy work overlap.
-constexpr int NT2 = 320;
+constexpr int NT2 = 448;
 
 // Multiply one 64-element row of a swizzled box by f with packed bf16x2
 // multiplies (f rounded once to bf16; no unpack/repack through fp32).
@@ -545,7 +546,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   constexpr uint32_t IDESC_X = idesc_bf16(128, 128, false, TR::X_MN);
   constexpr uint32_t IDESC_Y = idesc_bf16(128, 128, false, true);
   constexpr uint32_t IDESC_D = idesc_bf16(128, 128, true, true);
-  constexpr int BAR_MASK = 1, BAR_EPI = 2;
+  constexpr int BAR_MASK = 1, BAR_EPI = 2, BAR_DECAY = 3;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -597,8 +598,9 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       mbar_init(b_fc + 8 * s, 1);
       mbar_init(b_eab + 8 * s, 1);
       mbar_init(b_ec + 8 * s, 1);
-      // P written and the A0 / B1 row decays applied (mask warps)
-      mbar_init(b_pfull + 8 * s, 128);
+      // P written (mask warps, output passes) and the A0 / B1 row decays
+      // applied (decay warps)
+      mbar_init(b_pfull + 8 * s, OUT ? 256 : 128);
     }
     mbar_init(b_sfull, 1);
     mbar_init(b_sfull + 8, 1);
@@ -716,6 +718,13 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       uint64_t t_last = globaltimer();
       while (nP < nblk) {
         bool did = false;
+        if (OUT && nS < nblk && seen >= nS - 1 &&
+            mbar_test(b_fab + 8 * (nS % NS), (uint32_t)((nS / NS) & 1))) {
+          tc_fence_after();
+          issue_S(nS);
+          nS++;
+          did = true;
+        }
         if ((!OUT || nS > nP) && seen >= nP &&
             mbar_test(b_pfull + 8 * (nP % NS), (uint32_t)((nP / NS) & 1)) &&
             mbar_test(b_fc + 8 * (nP % NS), (uint32_t)((nP / NS) & 1)) &&
@@ -723,13 +732,6 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
           tc_fence_after();
           issue_P3(nP);
           nP++;
-          did = true;
-        }
-        if (OUT && nS < nblk && seen >= nS - 1 &&
-            mbar_test(b_fab + 8 * (nS % NS), (uint32_t)((nS / NS) & 1))) {
-          tc_fence_after();
-          issue_S(nS);
-          nS++;
           did = true;
         }
         if (seen < nP && mbar_test(b_ofull, (uint32_t)(seen & 1))) {
@@ -755,57 +757,36 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
     // -------------------------------------------------------- mask warps
     const int row = (warp & 3) * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    for (int i = 0; i < nblk; i++) {
+    for (int i = 0; OUT && i < nblk; i++) {
       const int st = i % NS;
-      const int cb = cb_of(i);
-      bool ok = OUT ? mbar_wait(b_sfull + 8 * (i & 1), (uint32_t)((i >> 1) & 1), abort_flag)
-                    : mbar_wait(b_fab + 8 * st, (uint32_t)((i / NS) & 1), abort_flag);
+      bool ok = mbar_wait(b_sfull + 8 * (i & 1), (uint32_t)((i >> 1) & 1), abort_flag);
       if (role_any(!ok, BAR_MASK, 128)) break;
       tc_fence_after();
       if (row == 0) LA2_TRACE(3, i);
-      uint8_t *stage = smem + st * LY::STAGE;
-      uint8_t *B1 = OUT ? stage + TILE : stage;
-      if (OUT) {
-        const uint32_t sb = 128u * (uint32_t)(i & 1);
+      const uint32_t sb = 128u * (uint32_t)(i & 1);
 #pragma unroll
-        for (int pair = 0; pair < 2; pair++) {
-          uint32_t r[64];
-          tmem_ld32(tl + sb + pair * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-          tmem_ld32(tl + sb + pair * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-          tmem_wait_ld();
-          uint32_t pk[32];
+      for (int part = 0; part < 4; part++) {
+        uint32_t r[32];
+        tmem_ld32(tl + sb + part * 32, r);
+        tmem_wait_ld();
+        uint32_t pk[16];
 #pragma unroll
-          for (int j = 0; j < 32; j++) {
-            const int t0 = pair * 64 + 2 * j;
-            // causal mask and decay in one lookup: distance < 0 reads 0
-            const int n0 = REV ? t0 - row : row - t0;
-            const float f0 = __uint_as_float(r[2 * j]) * pw[n0];
-            const float f1 = __uint_as_float(r[2 * j + 1]) * pw[REV ? n0 + 1 : n0 - 1];
-            pk[j] = pack_bf16x2(f0, f1);
-          }
-          tmem_st16(tl + sb + pair * 32, &pk[0]);
-          tmem_st16(tl + sb + pair * 32 + 16, &pk[16]);
+        for (int j = 0; j < 16; j++) {
+          const int t0 = part * 32 + 2 * j;
+          // causal mask and decay in one lookup: distance < 0 reads 0
+          const int n0 = REV ? t0 - row : row - t0;
+          const float f0 = __uint_as_float(r[2 * j]) * pw[n0];
+          const float f1 = __uint_as_float(r[2 * j + 1]) * pw[REV ? n0 + 1 : n0 - 1];
+          pk[j] = pack_bf16x2(f0, f1);
         }
-        // A0 rows carry the state term's row factor
-        const float f = REV ? (row < cb ? pw[cb - row] : 0.f) : pw[row + 1];
-        const __nv_bfloat162 f2 = __float2bfloat162_rn(f);
-        scale_row_sw128_bf16(stage, row, f2);
-        scale_row_sw128_bf16(stage + BOX, row, f2);
-      }
-      // B1 rows carry the state update's decay
-      {
-        const float fb = row < cb ? (REV ? pw[row] : pw[cb - 1 - row]) : 0.f;
-        const __nv_bfloat162 fb2 = __float2bfloat162_rn(fb);
-        scale_row_sw128_bf16(B1, row, fb2);
-        scale_row_sw128_bf16(B1 + BOX, row, fb2);
+        tmem_st16(tl + sb + part * 16, pk);
       }
       tmem_wait_st();
-      fence_proxy_async_smem();
       tc_fence_before();
       if (row == 0) LA2_TRACE(4, i);
       mbar_arrive(b_pfull + 8 * st);
     }
-  } else {
+  } else if (warp < 10) {
     // ---------------------------------------------------- epilogue warps
     const int row = (warp & 3) * 32 + lane;
     const int wtid = tid - 6 * 32;  // 0..127
@@ -918,6 +899,32 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       }
     }
     if (OUT && wtid == 0) tma_store_wait0();
+  } else {
+    // ------------------------------------------------------- decay warps
+    // Row decays, in place, once S has read the tiles: A0 rows by the state
+    // term's factor (output passes), B1 rows by the state update's decay.
+    const int row = (warp & 3) * 32 + lane;
+    for (int j = 0; j < nblk; j++) {
+      const int st = j % NS;
+      const int cbj = cb_of(j);
+      const bool ok = OUT ? mbar_wait(b_sfull + 8 * (j & 1), (uint32_t)((j >> 1) & 1), abort_flag)
+                          : mbar_wait(b_fab + 8 * st, (uint32_t)((j / NS) & 1), abort_flag);
+      if (role_any(!ok, BAR_DECAY, 128)) break;
+      uint8_t *stage = smem + st * LY::STAGE;
+      if (OUT) {
+        const float f = REV ? (row < cbj ? pw[cbj - row] : 0.f) : pw[row + 1];
+        const __nv_bfloat162 f2 = __float2bfloat162_rn(f);
+        scale_row_sw128_bf16(stage, row, f2);
+        scale_row_sw128_bf16(stage + BOX, row, f2);
+      }
+      uint8_t *B1 = OUT ? stage + TILE : stage;
+      const float fb = row < cbj ? (REV ? pw[row] : pw[cbj - 1 - row]) : 0.f;
+      const __nv_bfloat162 fb2 = __float2bfloat162_rn(fb);
+      scale_row_sw128_bf16(B1, row, fb2);
+      scale_row_sw128_bf16(B1 + BOX, row, fb2);
+      fence_proxy_async_smem();
+      mbar_arrive(b_pfull + 8 * st);
+    }
   }
 
   tc_fence_before();
