@@ -225,16 +225,18 @@ def run_la2(args, world, rank, local):
     outs = {n: torch.empty_like(x[src]) for n, src in
             (("o", "v"), ("dq", "q"), ("dk", "k"), ("dv", "v"))}
     stream = torch.cuda.current_stream()
-    ws_need = max(max(la2.workspace_size(op, Bn, H, L, D, E, torch.bfloat16)
-                      for op in (0, 1)) for Bn, L in SWEEP)
+    ws_need = max(la2.workspace_size(1, Bn, H, L, D, E, torch.bfloat16) for Bn, L in SWEEP)
     ws = torch.empty(max(ws_need, 16), dtype=torch.uint8, device=dev)
 
     def one_shape(Bn, L, xin=None, oo=None):
+        # a training step: the backward reuses the chunk states the forward
+        # left in the shared workspace
         xv = sweep_views(xin or x, Bn, L)
         ov = sweep_views(oo or outs, Bn, L)
         la2.forward(xv["q"], xv["k"], xv["v"], lam, out=ov["o"], workspace=ws)
         la2.backward(xv["q"], xv["k"], xv["v"], lam, xv["dO"],
-                     outs=(ov["dq"], ov["dk"], ov["dv"]), workspace=ws)
+                     outs=(ov["dq"], ov["dk"], ov["dv"]), workspace=ws,
+                     reuse_forward_states=ws_need > 0)
 
     for _ in range(args.warmup):
         for Bn, L in SWEEP:
@@ -363,7 +365,8 @@ def run_e2e(args, la2, lam, ws, dev, world):
             ov = sweep_views(dout[buf], Bn, L)
             la2.forward(xv["q"], xv["k"], xv["v"], lam, out=ov["o"], workspace=ws)
             la2.backward(xv["q"], xv["k"], xv["v"], lam, xv["dO"],
-                         outs=(ov["dq"], ov["dk"], ov["dv"]), workspace=ws)
+                         outs=(ov["dq"], ov["dk"], ov["dv"]), workspace=ws,
+                         reuse_forward_states=ws.numel() > 16)
             ev_done[i].record(comp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_done[i])

@@ -54,6 +54,9 @@ def library():
         lib.la2_backward.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I64, I, I, I,
                                      P, SZ, P]
         lib.la2_backward.restype = I
+        lib.la2_backward_ex.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I64, I, I, I,
+                                        P, SZ, ctypes.c_uint, P]
+        lib.la2_backward_ex.restype = I
         lib.la2_decode_step.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
         lib.la2_decode_step.restype = I
         lib.la2_last_device_error.argtypes = [P]
@@ -182,8 +185,14 @@ def forward_noalloc(q, k, v, lam, kv0=None, *, want_state: bool = False, out=Non
 
 
 def backward(q, k, v, lam, dO, kv0=None, *, want_dkv0: bool = False, outs=None,
-             workspace=None, stream=None):
-    """Gradients (dq, dk, dv[, dkv0]) of sum(o * dO)."""
+             workspace=None, reuse_forward_states: bool = False, stream=None):
+    """Gradients (dq, dk, dv[, dkv0]) of sum(o * dO).
+
+    reuse_forward_states: `workspace` (sized for the backward) was passed to
+    forward() with the same inputs and still holds the chunk states it wrote,
+    so the backward does not recompute them."""
+    if reuse_forward_states and workspace is None:
+        raise ValueError("reuse_forward_states needs the forward's workspace")
     lib = library()
     for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam), ("dO", dO)):
         _dev(t, name)
@@ -205,9 +214,10 @@ def backward(q, k, v, lam, dO, kv0=None, *, want_dkv0: bool = False, outs=None,
     ws = workspace
     if ws is None:
         ws = _workspace(workspace_size(LA2_OP_BACKWARD, B, H, L, d, e, q.dtype), q.device)
-    code = lib.la2_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(dO),
-                            _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dkv0), B, H, L, d, e, _dt(q),
-                            _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream))
+    code = lib.la2_backward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(dO),
+                               _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dkv0), B, H, L, d, e, _dt(q),
+                               _ptr(ws), 0 if ws is None else ws.numel(),
+                               1 if reuse_forward_states else 0, _stream(stream))
     _check(code, "la2_backward")
     return (dq, dk, dv, dkv0) if want_dkv0 else (dq, dk, dv)
 

@@ -210,14 +210,14 @@ template <typename T, int D, int E>
 cudaError_t simt_backward(const void *q, const void *k, const void *v,
                           const float *lam, const float *kv0, const void *dO,
                           void *dq, void *dk, void *dv, float *dkv0, float *ws,
-                          const Geo &g, cudaStream_t st) {
+                          const Geo &g, bool reuse_fwd, cudaStream_t st) {
   using namespace la2::simt;
   const T *Q = (const T *)q, *K = (const T *)k, *V = (const T *)v, *G = (const T *)dO;
   const int64_t BH = (int64_t)g.B * g.H;
   float *wsf = ws;
   float *wsr = ws ? ws + (size_t)BH * g.S * D * E : nullptr;
   cudaError_t err = cudaSuccess;
-  if (g.S > 1) {
+  if (g.S > 1 && !reuse_fwd) {
     auto kst = fwd_kernel<T, D, E, false>;
     cudaFuncSetAttribute(kst, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fwd_smem<D, E>());
     err = timed(K_SIMT_FWD_STATE, st, [&] {
@@ -229,6 +229,8 @@ cudaError_t simt_backward(const void *q, const void *k, const void *v,
       scan_fwd_kernel<D, E><<<dim3((D * E + NT - 1) / NT, (unsigned)BH), NT, 0, st>>>(wsf, kv0, lam, g);
     });
     if (err) return err;
+  }
+  if (g.S > 1) {
     auto krs = rev_state_kernel<T, D, E>;
     cudaFuncSetAttribute(krs, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rev_smem<D, E>());
     err = timed(K_SIMT_REV_STATE, st, [&] {
@@ -363,6 +365,18 @@ la2_status la2_backward(const void *q, const void *k, const void *v,
                         void *dq, void *dk, void *dv, float *dkv0,
                         int B, int H, int64_t L, int d, int e, la2_dtype dt,
                         void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return la2_backward_ex(q, k, v, lambda, kv0, dO, dq, dk, dv, dkv0, B, H, L, d, e, dt, workspace,
+                         workspace_bytes, 0u, stream);
+}
+
+la2_status la2_backward_ex(const void *q, const void *k, const void *v,
+                           const float *lambda, const float *kv0, const void *dO,
+                           void *dq, void *dk, void *dv, float *dkv0,
+                           int B, int H, int64_t L, int d, int e, la2_dtype dt,
+                           void *workspace, size_t workspace_bytes, unsigned flags,
+                           cudaStream_t stream) {
+  if (flags & ~(unsigned)LA2_BWD_REUSE_FORWARD_STATES) return LA2_ERR_INVALID;
+  const bool reuse = (flags & LA2_BWD_REUSE_FORWARD_STATES) != 0;
   if (B < 0 || H < 0 || L < 0) return LA2_ERR_INVALID;
   if (dt != LA2_F32 && dt != LA2_BF16) return LA2_ERR_UNSUPPORTED;
   if (!shape_supported(d, e, dt)) return LA2_ERR_UNSUPPORTED;
@@ -396,7 +410,7 @@ la2_status la2_backward(const void *q, const void *k, const void *v,
   float *ws = (float *)workspace;
   cudaError_t err;
   if (p == PATH_TC) {
-    err = la2::tc::backward(q, k, v, lambda, kv0, dO, dq, dk, dv, dkv0, ws, g, stream,
+    err = la2::tc::backward(q, k, v, lambda, kv0, dO, dq, dk, dv, dkv0, ws, g, reuse, stream,
                             [&](int which, auto &&fn) {
                               static const int ids[] = {K_TC_FWD_STATE, K_SCAN_FWD, K_TC_DQ,
                                                         K_TC_REV_STATE, K_SCAN_REV, K_TC_DV,
@@ -405,10 +419,10 @@ la2_status la2_backward(const void *q, const void *k, const void *v,
                             });
   } else if (dt == LA2_F32) {
     err = LA2_DISPATCH_DE(d, e, simt_backward, float, q, k, v, lambda, kv0, dO, dq, dk, dv, dkv0,
-                          ws, g, stream);
+                          ws, g, reuse, stream);
   } else {
     err = LA2_DISPATCH_DE(d, e, simt_backward, __nv_bfloat16, q, k, v, lambda, kv0, dO, dq, dk,
-                          dv, dkv0, ws, g, stream);
+                          dv, dkv0, ws, g, reuse, stream);
   }
   return to_status(err);
 }

@@ -77,28 +77,18 @@ template <int MODE> struct Layout {
 
 inline bool supports(int d, int e, bool bf16) { return bf16 && d == 128 && e == 128; }
 
-// Chunks per (b,h).  One CTA per SM at a time (each uses all of TMEM), so a
-// pass over BH*S chunks of ceil(nblk/S) blocks takes
-//   ceil(BH*S / sms) waves x (blocks per chunk + ~1 block of pipeline fill),
-// and a split (S > 1) adds the chunk-state pre-pass over S-1 chunks, which
-// moves half the bytes per block.  Pick the S with the smallest estimate.
+// Chunks per (b,h).  One CTA per SM at a time (each uses all of TMEM), and
+// a block's time is set mostly by its latency chain, not by its share of
+// HBM bandwidth, so a single wave of long chunks beats several waves of
+// short ones: when B*H leaves SMs idle, split each sequence into
+// floor(SMs / (B*H)) chunks, else not at all.  (Measured on the H = 32
+// length sweep: L = 32K, B*H = 64 is fastest at S = 2, L = 64K, B*H = 32 at
+// S = 4; more chunks, or two waves, were slower because the chunk-state
+// pre-pass grows with S.)
 inline int64_t auto_split(int64_t BH, int64_t nblk, int sms) {
-  int64_t best_s = 1;
-  double best = 1e300;
-  const int64_t smax = nblk < 256 ? nblk : 256;
-  for (int64_t S = 1; S <= smax; S++) {
-    const int64_t per = (nblk + S - 1) / S;
-    const int64_t s_eff = (nblk + per - 1) / per;
-    if (s_eff != S) continue;  // same plan as a smaller S
-    const double blocks = (double)per + 1.0;
-    double cost = (double)((BH * S + sms - 1) / sms) * blocks;
-    if (S > 1) cost += 0.5 * (double)((BH * (S - 1) + sms - 1) / sms) * blocks;
-    if (cost < best * 0.999) {
-      best = cost;
-      best_s = S;
-    }
-  }
-  return best_s;
+  (void)nblk;
+  if (BH >= sms) return 1;
+  return sms / BH;
 }
 
 using namespace la2::sm100;
@@ -1026,7 +1016,7 @@ cudaError_t forward(const void *q, const void *k, const void *v, const float *la
 template <typename Timed>
 cudaError_t backward(const void *q, const void *k, const void *v, const float *lam,
                      const float *kv0, const void *dO, void *dq, void *dk, void *dv, float *dkv0,
-                     float *ws, const Geo &g, cudaStream_t st, Timed &&timed) {
+                     float *ws, const Geo &g, bool reuse_fwd, cudaStream_t st, Timed &&timed) {
   if (!geometry_ok(g)) return cudaErrorInvalidValue;
   const int64_t BH = (int64_t)g.B * g.H;
   CUtensorMap mq, mk, mv, mg, mdq, mdk, mdv;
@@ -1038,7 +1028,8 @@ cudaError_t backward(const void *q, const void *k, const void *v, const float *l
   float *wsr = ws ? ws + (size_t)BH * g.S * 128 * 128 : nullptr;
   const dim3 sgrid(128 * 128 / la2::simt::NT, (unsigned)BH);
   cudaError_t err = cudaSuccess;
-  if (g.S > 1) {
+  // the forward pass leaves the same chunk entry states in the same place
+  if (g.S > 1 && !reuse_fwd) {
     err = timed(0, [&] { launch_chunk<MODE_STATE>(mk, mk, mv, mk, lam, nullptr, wsf, nullptr, g, st); });
     if (err) return err;
     err = timed(1, [&] {

@@ -146,6 +146,24 @@ la2_status la2_backward(const void *q, const void *k, const void *v,
                         cudaStream_t stream);
 
 /*
+ * la2_backward with flags.  LA2_BWD_REUSE_FORWARD_STATES: `workspace`
+ * already holds the chunk entry states that la2_forward wrote for the same
+ * q, k, v, lambda, kv0 and sizes -- the caller gave la2_forward this same
+ * workspace (sized for LA2_OP_BACKWARD) and has not touched it since, with
+ * the same split option in force -- so the backward skips recomputing them
+ * (one pass over k and v fewer for long sequences).  With stale or foreign
+ * contents the gradients are wrong; the library cannot check this.  Unknown
+ * flag bits return LA2_ERR_INVALID.  flags = 0 is la2_backward.
+ */
+enum { LA2_BWD_REUSE_FORWARD_STATES = 1 };
+la2_status la2_backward_ex(const void *q, const void *k, const void *v,
+                           const float *lambda, const float *kv0, const void *dO,
+                           void *dq, void *dk, void *dv, float *dkv0,
+                           int B, int H, int64_t L, int d, int e, la2_dtype dt,
+                           void *workspace, size_t workspace_bytes, unsigned flags,
+                           cudaStream_t stream);
+
+/*
  * One recurrent decode step for one new token per (b,h):
  *     kv <- lambda kv + k^T v,    o = q kv
  * q, k [B,H,d], v, o [B,H,e] of type dt; kv fp32 [B,H,d,e] updated IN PLACE

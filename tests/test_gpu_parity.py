@@ -132,6 +132,33 @@ def test_tc_phase_serial_variant(orc, L, split):
     compare(got, oracle_all(orc, x, lam, x["kv0"]), torch.bfloat16, f"v1 L={L} S={split}")
 
 
+@pytest.mark.parametrize("path", ["simt", "tc"])
+def test_backward_reuses_forward_states(orc, path):
+    """A training step that hands the forward's workspace to the backward
+    (LA2_BWD_REUSE_FORWARD_STATES) gives the same gradients as a backward
+    that recomputes the chunk states, and the oracle's."""
+    B, H, L = 1, 3, 1000
+    x = inputs.make_inputs(B, H, L, 128, 128, dtype=torch.bfloat16, device=DEV, seed=13,
+                           with_kv0=True)
+    lam = inputs.fixed_lambdas((1.0, 0.95, 0.5), DEV)
+    with options(path=path, split=4):
+        n = la2.workspace_size(la2.LA2_OP_BACKWARD, B, H, L, 128, 128, torch.bfloat16)
+        assert n > 0
+        ws = torch.empty(n, dtype=torch.uint8, device=DEV)
+        o = la2.forward(x["q"], x["k"], x["v"], lam, x["kv0"], workspace=ws)
+        got = la2.backward(x["q"], x["k"], x["v"], lam, x["dO"], x["kv0"], want_dkv0=True,
+                           workspace=ws, reuse_forward_states=True)
+        ref = la2.backward(x["q"], x["k"], x["v"], lam, x["dO"], x["kv0"], want_dkv0=True)
+        torch.cuda.synchronize()
+    assert la2.last_device_error() == 0
+    for a, b in zip(got, ref):
+        assert torch.equal(a, b)
+    want = oracle_all(orc, x, lam, x["kv0"])
+    for name, a, r in zip(("dq", "dk", "dv", "dkv0"), got, want[2:]):
+        check(f"reuse {path} {name}", a, r, torch.bfloat16)
+    check(f"reuse {path} o", o, want[0], torch.bfloat16)
+
+
 def test_split_invariance_gpu():
     """Different splits agree with each other (same kernels, other chunking)."""
     x = inputs.make_inputs(2, 2, 2048, 128, 128, dtype=torch.bfloat16, device=DEV, seed=5)
