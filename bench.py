@@ -133,12 +133,21 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest of every rank's value (timings: the job is as slow as its
+    slowest rank).  NCCL reduces a device tensor, gloo a host one."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank processed `units_per_rank` units in
+    at most `ms_max` milliseconds."""
+    return world * units_per_rank / (ms_max / 1e3)
 
 
 # ------------------------------------------------------------- workloads
@@ -273,7 +282,7 @@ def run_la2(args, world, rank, local):
                  for i in range(len(SWEEP))]
 
     tokens_step = TOKENS * len(SWEEP)
-    value = world * tokens_step * args.steps / (ms / 1e3)
+    value = weak_scaling_value(tokens_step * args.steps, world, ms)
     sweep = [{"B": Bn, "L": L, "tokens_per_s": TOKENS / (t / 1e3), "ms": t}
              for (Bn, L), t in zip(SWEEP, per_shape)]
     rates = [s["tokens_per_s"] for s in sweep]
