@@ -473,6 +473,37 @@ __device__ __forceinline__ void scale_row_sw128_bf16(uint8_t *box, int row, __nv
   }
 }
 
+// One 128-element bf16 row of a two-box tile (d 0..63 in the first 128-byte
+// swizzled box, 64..127 in the second) as sixteen 16-byte chunks, chunk c
+// holding elements 8c..8c+7.  All loads are issued before any result is
+// used.
+__device__ __forceinline__ void ld_row_sw128(const uint8_t *tile, int row, uint4 (&w)[16]) {
+#pragma unroll
+  for (int c = 0; c < 16; c++)
+    w[c] = *reinterpret_cast<const uint4 *>(tile + (c >> 3) * BOX + row * 128 +
+                                            (((c & 7) ^ (row & 7)) << 4));
+}
+__device__ __forceinline__ void st_row_sw128(uint8_t *tile, int row, const uint4 (&w)[16]) {
+#pragma unroll
+  for (int c = 0; c < 16; c++)
+    *reinterpret_cast<uint4 *>(tile + (c >> 3) * BOX + row * 128 + (((c & 7) ^ (row & 7)) << 4)) =
+        w[c];
+}
+
+// Multiply one 128-element row of a two-box tile by f2 in place, the whole
+// row in flight at once (packed bf16x2 multiplies: f rounded once to bf16).
+__device__ __forceinline__ void scale_row2_sw128(uint8_t *tile, int row, __nv_bfloat162 f2) {
+  uint4 w[16];
+  ld_row_sw128(tile, row, w);
+#pragma unroll
+  for (int c = 0; c < 16; c++) {
+    __nv_bfloat162 *u = reinterpret_cast<__nv_bfloat162 *>(&w[c]);
+#pragma unroll
+    for (int m = 0; m < 4; m++) u[m] = __hmul2(u[m], f2);
+  }
+  st_row_sw128(tile, row, w);
+}
+
 template <int MODE> struct Layout2 {
   static constexpr bool OUT = Traits<MODE>::OUT;
   static constexpr int NSTAGE = OUT ? 2 : 3;
@@ -516,6 +547,14 @@ __device__ __forceinline__ void role_sync(int id, int n) {
   do {                                                                                    \
     if (tracing && (blk) < kTraceBlocks) g_trace[(ev) * kTraceBlocks + (blk)] = globaltimer(); \
   } while (0)
+
+// The MMA issuer's pause between idle probe rounds.
+constexpr uint32_t kIdlePauseCycles = 64;
+__device__ __forceinline__ uint32_t clock_u32() {
+  uint32_t c;
+  asm volatile("mov.u32 %0, %%clock;" : "=r"(c));
+  return c;
+}
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
@@ -576,9 +615,13 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   };
   // trace events: 0 load issued, 1 S issued, 2 P.B2/X/state issued, 3 mask
   // start, 4 mask done, 5 epilogue start, 6 state handed back, 7 store read
-  // done, 8 kernel entry, 9 set-up done
+  // done, 8 kernel entry, 9 set-up done, 12 S issue begins, 13 products
+  // issue begin, 14 row decays done, 15 output tile staged
   const bool tracing = g.trace == MODE && blockIdx.x == 0;
+  const bool tracing_all = g.trace == MODE;  // per-CTA entry / exit (events 10, 11)
   if (tid == 0) LA2_TRACE(8, 0);
+  if (tid == 0 && tracing_all && blockIdx.x < kTraceBlocks)
+    g_trace[10 * kTraceBlocks + blockIdx.x] = globaltimer();
 
   if (tid <= BLOCK) pw[tid] = (float)pow_int((double)lambda[h], tid);
   if (tid < BLOCK) pwz[tid] = 0.f;
@@ -589,13 +632,13 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       mbar_init(b_eab + 8 * s, 1);
       mbar_init(b_ec + 8 * s, 1);
       // P written (mask warps, output passes) and the A0 / B1 row decays
-      // applied (decay warps)
-      mbar_init(b_pfull + 8 * s, OUT ? 256 : 128);
+      // applied (decay warps); one arrival per warp
+      mbar_init(b_pfull + 8 * s, OUT ? 8 : 4);
     }
     mbar_init(b_sfull, 1);
     mbar_init(b_sfull + 8, 1);
     mbar_init(b_ofull, 1);
-    mbar_init(b_oempty, 128);
+    mbar_init(b_oempty, 4);
     mbar_init(b_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -705,12 +748,14 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       // S of block j needs products j-2 done, so no waiter can fall two
       // phases behind a barrier.
       int nS = 0, nP = 0, seen = 0;
+      uint32_t idle = 0;
       uint64_t t_last = globaltimer();
       while (nP < nblk) {
         bool did = false;
         if (OUT && nS < nblk && seen >= nS - 1 &&
             mbar_test(b_fab + 8 * (nS % NS), (uint32_t)((nS / NS) & 1))) {
           tc_fence_after();
+          LA2_TRACE(12, nS);
           issue_S(nS);
           nS++;
           did = true;
@@ -720,6 +765,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
             mbar_test(b_fc + 8 * (nP % NS), (uint32_t)((nP / NS) & 1)) &&
             mbar_test(b_oempty, (uint32_t)(nP & 1))) {
           tc_fence_after();
+          LA2_TRACE(13, nP);
           issue_P3(nP);
           nP++;
           did = true;
@@ -729,13 +775,22 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
           did = true;
         }
         if (did) {
-          t_last = globaltimer();
-        } else if (*abort_flag) {
-          break;
-        } else if (globaltimer() - t_last > kWaitTimeoutNs) {
-          *abort_flag = 1;
-          raise_error(ERR_TIMEOUT);
-          break;
+          idle = 0;
+        } else if ((++idle & 63) == 0) {
+          // an idle probe round costs shared-memory cycles the other roles
+          // need, so the abort flag and the clock are read every 64th round
+          if (*abort_flag) break;
+          const uint64_t now = globaltimer();
+          if (idle == 64) t_last = now;
+          if (now - t_last > kWaitTimeoutNs) {
+            *abort_flag = 1;
+            raise_error(ERR_TIMEOUT);
+            break;
+          }
+        } else {
+          const uint32_t c0 = clock_u32();
+          while (clock_u32() - c0 < kIdlePauseCycles) {
+          }
         }
       }
       // all MMAs issued by this thread have finished before TMEM is freed
@@ -745,8 +800,18 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
     }
   } else if (warp < 6) {
     // -------------------------------------------------------- mask warps
-    const int row = (warp & 3) * 32 + lane;
-    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    // Warp quarter q owns rows 32q..32q+31 and splits S into four 32-column
+    // parts p.  Parts wholly above the diagonal (below it in the reverse
+    // passes) are zero; the diagonal part p == q looks its factors up in the
+    // zero-extended table; in the other parts the factor of column 32p + k
+    // is a * lambda^(31-k) with a = lambda^(row-32p-31) (reverse: a *
+    // lambda^k, a = lambda^(32p-row)), a <= 1, generated by two chains of
+    // multiplications by lambda^2 from the largest factor down: no
+    // shared-memory lookup per element, and at most 16 roundings per factor.
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+    const float lam1 = pw[1], lam2 = pw[2];
     for (int i = 0; OUT && i < nblk; i++) {
       const int st = i % NS;
       bool ok = mbar_wait(b_sfull + 8 * (i & 1), (uint32_t)((i >> 1) & 1), abort_flag);
@@ -756,25 +821,43 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       const uint32_t sb = 128u * (uint32_t)(i & 1);
 #pragma unroll
       for (int part = 0; part < 4; part++) {
-        uint32_t r[32];
-        tmem_ld32(tl + sb + part * 32, r);
-        tmem_wait_ld();
         uint32_t pk[16];
+        if (REV ? part < q : part > q) {
 #pragma unroll
-        for (int j = 0; j < 16; j++) {
-          const int t0 = part * 32 + 2 * j;
-          // causal mask and decay in one lookup: distance < 0 reads 0
-          const int n0 = REV ? t0 - row : row - t0;
-          const float f0 = __uint_as_float(r[2 * j]) * pw[n0];
-          const float f1 = __uint_as_float(r[2 * j + 1]) * pw[REV ? n0 + 1 : n0 - 1];
-          pk[j] = pack_bf16x2(f0, f1);
+          for (int j = 0; j < 16; j++) pk[j] = 0u;
+        } else {
+          uint32_t r[32];
+          tmem_ld32(tl + sb + part * 32, r);
+          tmem_wait_ld();
+          if (part == q) {
+#pragma unroll
+            for (int j = 0; j < 16; j++) {
+              // distance < 0 reads 0 from the table: the causal mask
+              const int n0 = REV ? 2 * j - lane : lane - 2 * j;
+              const float f0 = __uint_as_float(r[2 * j]) * pw[n0];
+              const float f1 = __uint_as_float(r[2 * j + 1]) * pw[REV ? n0 + 1 : n0 - 1];
+              pk[j] = pack_bf16x2(f0, f1);
+            }
+          } else {
+            const float a = REV ? pw[32 * part - row] : pw[row - 32 * part - 31];
+            // xe, xo: factors of the pair's even and odd column
+            float xe = REV ? a : a * lam1, xo = REV ? a * lam1 : a;
+#pragma unroll
+            for (int jj = 0; jj < 16; jj++) {
+              const int j = REV ? jj : 15 - jj;
+              pk[j] = pack_bf16x2(__uint_as_float(r[2 * j]) * xe, __uint_as_float(r[2 * j + 1]) * xo);
+              xe *= lam2;
+              xo *= lam2;
+            }
+          }
         }
         tmem_st16(tl + sb + part * 16, pk);
       }
       tmem_wait_st();
       tc_fence_before();
       if (row == 0) LA2_TRACE(4, i);
-      mbar_arrive(b_pfull + 8 * st);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_pfull + 8 * st);
     }
   } else if (warp < 10) {
     // ---------------------------------------------------- epilogue warps
@@ -815,7 +898,8 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(b_oempty);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_oempty);
     }
     float *dst = nullptr;
     float dscale = 1.f;
@@ -844,6 +928,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
           st_row_bf16_sw128(stg + pair * BOX, row, 4, reinterpret_cast<const float *>(&r[32]));
         }
       }
+      if (wtid == 0) LA2_TRACE(15, i);
       const bool last = i == nblk - 1;
       const float dec = last ? 1.f : pw[cb_of(i + 1)];
 #pragma unroll
@@ -873,7 +958,8 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       fence_proxy_async_smem();
       tc_fence_before();
       if (wtid == 0) LA2_TRACE(6, i);
-      mbar_arrive(b_oempty);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_oempty);
       if (OUT) role_sync(BAR_EPI, 128);  // the whole output tile is in shared memory
       if (wtid == 0) {
         if (OUT) {
@@ -903,22 +989,22 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       uint8_t *stage = smem + st * LY::STAGE;
       if (OUT) {
         const float f = REV ? (row < cbj ? pw[cbj - row] : 0.f) : pw[row + 1];
-        const __nv_bfloat162 f2 = __float2bfloat162_rn(f);
-        scale_row_sw128_bf16(stage, row, f2);
-        scale_row_sw128_bf16(stage + BOX, row, f2);
+        scale_row2_sw128(stage, row, __float2bfloat162_rn(f));
       }
       uint8_t *B1 = OUT ? stage + TILE : stage;
       const float fb = row < cbj ? (REV ? pw[row] : pw[cbj - 1 - row]) : 0.f;
-      const __nv_bfloat162 fb2 = __float2bfloat162_rn(fb);
-      scale_row_sw128_bf16(B1, row, fb2);
-      scale_row_sw128_bf16(B1 + BOX, row, fb2);
+      scale_row2_sw128(B1, row, __float2bfloat162_rn(fb));
       fence_proxy_async_smem();
-      mbar_arrive(b_pfull + 8 * st);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_pfull + 8 * st);
+      if (row == 0) LA2_TRACE(14, j);
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  if (tid == 0 && tracing_all && blockIdx.x < kTraceBlocks)
+    g_trace[11 * kTraceBlocks + blockIdx.x] = globaltimer();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, LY::TMEM_COLS);

@@ -217,7 +217,9 @@ enum {
  * Events: 0 loads issued, 1 S = A0 B1^T issued, 2 P.B2 / state term / state
  * update issued, 3 mask start, 4 mask done, 5 epilogue start, 6 state handed
  * back to the MMA issuer, 7 output tile read by the store, 8 kernel entry,
- * 9 set-up done.  With out == NULL returns the buffer's entry count.
+ * 9 set-up done (all of CTA 0, indexed by block); 10 entry and 11 exit of
+ * every CTA (indexed by CTA, first 512).  With out == NULL returns the
+ * buffer's entry count.
  */
 size_t la2_trace_read(uint64_t *out, size_t n);
 int la2_set_option(int option, int value);
