@@ -560,7 +560,10 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-template <int MODE>
+// TRACE: the instantiation that records the trace stamps (LA2_OPT_TRACE);
+// the stamps' branches cost a few percent, so the other launches compile
+// without them.
+template <int MODE, bool TRACE>
 __global__ void __launch_bounds__(NT2, 1)
 chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
               const __grid_constant__ CUtensorMap tm2, const __grid_constant__ CUtensorMap tmo,
@@ -617,8 +620,8 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   // start, 4 mask done, 5 epilogue start, 6 state handed back, 7 store read
   // done, 8 kernel entry, 9 set-up done, 12 S issue begins, 13 products
   // issue begin, 14 row decays done, 15 output tile staged
-  const bool tracing = g.trace == MODE && blockIdx.x == 0;
-  const bool tracing_all = g.trace == MODE;  // per-CTA entry / exit (events 10, 11)
+  const bool tracing = TRACE && blockIdx.x == 0;
+  const bool tracing_all = TRACE;  // per-CTA entry / exit (events 10, 11)
   if (tid == 0) LA2_TRACE(8, 0);
   if (tid == 0 && tracing_all && blockIdx.x < kTraceBlocks)
     g_trace[10 * kTraceBlocks + blockIdx.x] = globaltimer();
@@ -1061,7 +1064,7 @@ cudaError_t launch_chunk(const CUtensorMap &m0, const CUtensorMap &m1, const CUt
     return cudaGetLastError();
   }
   using LY = Layout2<MODE>;
-  auto k = chunk_kernel2<MODE>;
+  auto k = g.trace == MODE ? chunk_kernel2<MODE, true> : chunk_kernel2<MODE, false>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::SMEM);
   if (e != cudaSuccess) return e;
   k<<<(unsigned)grid, NT2, LY::SMEM, st>>>(m0, m1, m2, mo, lam, kv0, ws, kv_out, g);

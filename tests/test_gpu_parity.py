@@ -120,6 +120,21 @@ def test_forced_split(orc, path, split):
 
 
 @pytest.mark.parametrize("split", [1, 3])
+@pytest.mark.parametrize("L", [129, 1000])
+def test_tc_decay_range(orc, L, split):
+    """Heads across the range of lambda, from fast decay (lambda^128 far
+    below fp32's normal range) to none, agree with the oracle on the
+    tensor-core path (ragged block, forced chunk split, initial state and
+    dkv0)."""
+    x = inputs.make_inputs(2, 6, L, 128, 128, dtype=torch.bfloat16, device=DEV, seed=L + split,
+                           with_kv0=True)
+    lam = inputs.fixed_lambdas((0.3, 0.8, 0.81, 0.9, 0.999, 1.0), DEV)
+    with options(path="tc", split=split):
+        got = run_fwd_bwd(x, lam, x["kv0"])
+    compare(got, oracle_all(orc, x, lam, x["kv0"]), torch.bfloat16, f"decay range L={L} S={split}")
+
+
+@pytest.mark.parametrize("split", [1, 3])
 @pytest.mark.parametrize("L", [200, 1000])
 def test_tc_phase_serial_variant(orc, L, split):
     """The simpler phase-serial form of the tensor-core kernel (kept for
@@ -339,3 +354,35 @@ def test_bounded_wait_reports_timeout():
         torch.cuda.synchronize()
         assert la2.last_device_error() == 0
     assert torch.equal(again, ref)
+
+
+# ----------------------------------------------------------------- tracing
+def test_trace_instantiation_matches():
+    """LA2_OPT_TRACE runs the tensor-core forward through its traced
+    instantiation: bit-identical output, an entry/exit stamp for every CTA,
+    and per-block stamps of CTA 0 in causal order (S issued after its tiles
+    were loaded, the mask after S, the products after the mask, the output
+    staged after the products)."""
+    B, H, L = 2, 4, 1000
+    x = inputs.make_inputs(B, H, L, 128, 128, dtype=torch.bfloat16, device=DEV, seed=21)
+    lam = inputs.decay_lambdas(H, DEV)
+    with options(path="tc", split=1):
+        ref = la2.forward(x["q"], x["k"], x["v"], lam)
+        torch.cuda.synchronize()
+        la2.trace_read()  # clears
+        old = la2.set_option(la2.LA2_OPT_TRACE, 1)  # mode 0: forward
+        try:
+            got = la2.forward(x["q"], x["k"], x["v"], lam)
+            torch.cuda.synchronize()
+        finally:
+            la2.set_option(la2.LA2_OPT_TRACE, old)
+    assert torch.equal(got, ref)
+    t = la2.trace_read()
+    n_cta, nblk = B * H, (L + 127) // 128
+    entry, exit_ = t[10, :n_cta], t[11, :n_cta]
+    assert bool((entry > 0).all()) and bool((exit_ > entry).all())
+    assert int((t[10, n_cta:] > 0).sum()) == 0
+    for i in range(nblk):
+        s_end, mask_e, p_end, epi_s, oempty = (int(t[e, i]) for e in (1, 4, 2, 5, 6))
+        assert 0 < s_end <= mask_e <= p_end, (i, s_end, mask_e, p_end)
+        assert p_end <= epi_s <= oempty, (i, p_end, epi_s, oempty)
