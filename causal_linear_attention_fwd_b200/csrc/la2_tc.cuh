@@ -578,7 +578,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   constexpr uint32_t IDESC_X = idesc_bf16(128, 128, false, TR::X_MN);
   constexpr uint32_t IDESC_Y = idesc_bf16(128, 128, false, true);
   constexpr uint32_t IDESC_D = idesc_bf16(128, 128, true, true);
-  constexpr int BAR_MASK = 1, BAR_EPI = 2, BAR_DECAY = 3;
+  constexpr int BAR_EPI = 2;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -818,7 +818,8 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
     for (int i = 0; OUT && i < nblk; i++) {
       const int st = i % NS;
       bool ok = mbar_wait(b_sfull + 8 * (i & 1), (uint32_t)((i >> 1) & 1), abort_flag);
-      if (role_any(!ok, BAR_MASK, 128)) break;
+      // a warp vote suffices: no later step syncs the mask warps together
+      if (__any_sync(0xffffffffu, !ok)) break;
       tc_fence_after();
       if (row == 0) LA2_TRACE(3, i);
       const uint32_t sb = 128u * (uint32_t)(i & 1);
@@ -988,7 +989,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       const int cbj = cb_of(j);
       const bool ok = OUT ? mbar_wait(b_sfull + 8 * (j & 1), (uint32_t)((j >> 1) & 1), abort_flag)
                           : mbar_wait(b_fab + 8 * st, (uint32_t)((j / NS) & 1), abort_flag);
-      if (role_any(!ok, BAR_DECAY, 128)) break;
+      if (__any_sync(0xffffffffu, !ok)) break;  // as for the mask warps
       uint8_t *stage = smem + st * LY::STAGE;
       if (OUT) {
         const float f = REV ? (row < cbj ? pw[cbj - row] : 0.f) : pw[row + 1];
