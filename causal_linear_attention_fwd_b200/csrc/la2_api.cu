@@ -166,6 +166,35 @@ Geo plan(int B, int H, int64_t L, int blk, Path path) {
   g.Lc = per * blk;
   g.S = (int)((L + g.Lc - 1) / g.Lc);
   if (g.S < 1) g.S = 1;
+  // Sub-chunks for the tensor-core chunk-state pre-passes: those passes
+  // have B*H*(S-1) chunks, fewer than the SMs when the split exists at all,
+  // so each chunk is cut into M sub-chunks, M minimising (waves of CTAs) x
+  // (blocks per CTA).  Lc becomes M * Ls with Ls a multiple of the block.
+  int64_t M = 1;
+  if (path == PATH_TC && g.S > 1) {
+    const int sms = device_sms();
+    const int64_t work = (int64_t)B * H * (g.S - 1);
+    int64_t best = -1;
+    for (int64_t m = 1; m <= 8 && m <= per; m++) {
+      const int64_t cost = ((work * m + sms - 1) / sms) * ((per + m - 1) / m);
+      if (best < 0 || cost < best) {
+        best = cost;
+        M = m;
+      }
+    }
+    g.Lc = M * (((per + M - 1) / M) * blk);
+    g.S = (int)((L + g.Lc - 1) / g.Lc);
+    if (g.S <= 1) {
+      g.S = 1;
+      M = 1;
+    }
+  }
+  g.M = (int)M;
+  g.Ls = g.Lc / M;
+  g.Ssub = (int)((L + g.Ls - 1) / g.Ls);
+  g.wsS = g.Ssub;
+  g.nst = g.S - 1;
+  g.c0 = 0;
   return g;
 }
 
@@ -173,7 +202,7 @@ int block_rows(Path p) { return p == PATH_TC ? la2::tc::BLOCK : la2::simt::C; }
 
 size_t ws_bytes(int op, const Geo &g, int d, int e) {
   if (g.S <= 1) return 0;
-  size_t one = (size_t)g.B * g.H * g.S * d * e * sizeof(float);
+  size_t one = (size_t)g.B * g.H * g.wsS * d * e * sizeof(float);
   return op == LA2_OP_BACKWARD ? 2 * one : one;
 }
 
@@ -195,7 +224,8 @@ cudaError_t simt_forward(const void *q, const void *k, const void *v,
     });
     if (err) return err;
     err = timed(K_SIMT_FWD_SCAN, st, [&] {
-      scan_fwd_kernel<D, E><<<dim3((D * E + NT - 1) / NT, (unsigned)BH), NT, 0, st>>>(ws, kv0, lam, g);
+      scan_fwd_kernel<D, E><<<dim3((D * E + NT - 1) / NT, (unsigned)BH), NT, 0, st>>>(
+          ws, kv0, lam, la2::state_geo(g, false));
     });
     if (err) return err;
   }
@@ -215,7 +245,7 @@ cudaError_t simt_backward(const void *q, const void *k, const void *v,
   const T *Q = (const T *)q, *K = (const T *)k, *V = (const T *)v, *G = (const T *)dO;
   const int64_t BH = (int64_t)g.B * g.H;
   float *wsf = ws;
-  float *wsr = ws ? ws + (size_t)BH * g.S * D * E : nullptr;
+  float *wsr = ws ? ws + (size_t)BH * g.wsS * D * E : nullptr;
   cudaError_t err = cudaSuccess;
   if (g.S > 1 && !reuse_fwd) {
     auto kst = fwd_kernel<T, D, E, false>;
@@ -226,7 +256,8 @@ cudaError_t simt_backward(const void *q, const void *k, const void *v,
     });
     if (err) return err;
     err = timed(K_SIMT_FWD_SCAN, st, [&] {
-      scan_fwd_kernel<D, E><<<dim3((D * E + NT - 1) / NT, (unsigned)BH), NT, 0, st>>>(wsf, kv0, lam, g);
+      scan_fwd_kernel<D, E><<<dim3((D * E + NT - 1) / NT, (unsigned)BH), NT, 0, st>>>(
+          wsf, kv0, lam, la2::state_geo(g, false));
     });
     if (err) return err;
   }
@@ -238,7 +269,8 @@ cudaError_t simt_backward(const void *q, const void *k, const void *v,
     });
     if (err) return err;
     err = timed(K_SIMT_REV_SCAN, st, [&] {
-      scan_rev_kernel<D, E><<<dim3((D * E + NT - 1) / NT, (unsigned)BH), NT, 0, st>>>(wsr, lam, g);
+      scan_rev_kernel<D, E><<<dim3((D * E + NT - 1) / NT, (unsigned)BH), NT, 0, st>>>(
+          wsr, lam, la2::state_geo(g, true));
     });
     if (err) return err;
   }

@@ -33,11 +33,35 @@ struct Geo {
   int64_t L;
   int S;        // chunks per (b,h)
   int64_t Lc;   // rows per chunk (multiple of the block size); last may be short
+  // The chunk-state pre-passes may run on a finer split: M sub-chunks of Ls
+  // rows per chunk (Lc = M * Ls), Ssub of them over the sequence, so that
+  // they fill the GPU too.  The workspace holds wsS d x e states per (b,h)
+  // (one per sub-chunk); a chunk-state pass processes nst (sub-)chunks
+  // starting at index c0.  M = 1 is the plain split.
+  int M;
+  int64_t Ls;
+  int Ssub;
+  int wsS;
+  int nst;
+  int c0;
   int inject;   // test hook: CTA 0 of a tensor-core pass withholds one MMA
                 // completion signal so that its bounded wait runs out
   int variant;  // tensor-core kernel form (0: warp-specialised, 1: phase-serial)
   int trace;    // tensor-core pass whose CTA 0 stamps the trace buffer (-1: none)
 };
+
+// Geometry of a chunk-state pre-pass and its scan: the (sub-)chunk split,
+// forward (chunks 0 .. S-2 of the main split, as (S-1)*M sub-chunks from
+// index 0) or reverse (everything after chunk 0: sub-chunks M .. Ssub-1).
+inline Geo state_geo(const Geo &g, bool reverse) {
+  Geo s = g;
+  s.S = g.Ssub;
+  s.Lc = g.Ls;
+  s.M = 1;
+  s.nst = reverse ? g.Ssub - g.M : (g.S - 1) * g.M;
+  s.c0 = reverse ? g.M : 0;
+  return s;
+}
 
 namespace simt {
 
@@ -155,8 +179,9 @@ scan_fwd_kernel(float *__restrict__ ws, const float *__restrict__ kv0,
   if (idx >= D * E) return;
   const float decay = (float)pow_int((double)lambda[bh % g.H], g.Lc);
   float run = kv0 ? kv0[bh * D * E + idx] : 0.f;
-  for (int c = 1; c < g.S; c++) {
-    float *p = ws + (bh * g.S + c) * (int64_t)D * E + idx;
+  // slot c holds the contribution of (sub-)chunk c-1, c = 1..nst (all full)
+  for (int c = 1; c <= g.nst; c++) {
+    float *p = ws + (bh * g.wsS + c) * (int64_t)D * E + idx;
     run = decay * run + *p;
     *p = run;
   }
@@ -286,8 +311,9 @@ scan_rev_kernel(float *__restrict__ ws, const float *__restrict__ lambda, Geo g)
   const float full = (float)pow_int(lam, g.Lc);
   const float last = (float)pow_int(lam, g.L - (int64_t)(g.S - 1) * g.Lc);
   float run = 0.f;
-  for (int c = g.S - 2; c >= 0; c--) {
-    float *p = ws + (bh * g.S + c) * (int64_t)D * E + idx;
+  // slot c holds the contribution of (sub-)chunk c+1, c+1 = c0..S-1
+  for (int c = g.S - 2; c >= g.c0 - 1; c--) {
+    float *p = ws + (bh * g.wsS + c) * (int64_t)D * E + idx;
     run = (c + 1 == g.S - 1 ? last : full) * run + *p;
     *p = run;
   }

@@ -156,9 +156,9 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quarter = warp & 3, half = warp >> 2;
   const int row = quarter * 32 + lane;
-  const int nch = OUT ? g.S : g.S - 1;
+  const int nch = OUT ? g.S : g.nst;
   const int64_t bh = blockIdx.x / nch;
-  const int c = blockIdx.x % nch + (MODE == MODE_RSTATE ? 1 : 0);
+  const int c = blockIdx.x % nch + (OUT ? 0 : g.c0);
   const int h = (int)(bh % g.H);
   const int64_t a = (int64_t)c * g.Lc;
   const int64_t b = g.L < a + g.Lc ? g.L : a + g.Lc;
@@ -212,9 +212,9 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
     const float *init = nullptr;
     if (MODE == MODE_FWD || MODE == MODE_DQ) {
       if (c == 0) init = kv0 ? kv0 + bh * 128 * 128 : nullptr;
-      else init = ws + (bh * g.S + c) * (int64_t)128 * 128;
+      else init = ws + (bh * g.wsS + (int64_t)c * g.M) * (int64_t)128 * 128;
     } else if (MODE == MODE_DV || MODE == MODE_DK) {
-      if (c != g.S - 1) init = ws + (bh * g.S + c) * (int64_t)128 * 128;
+      if (c != g.S - 1) init = ws + (bh * g.wsS + (int64_t)(c + 1) * g.M - 1) * (int64_t)128 * 128;
     }
     uint8_t *kvbf = smem + LY::KVBF + half * BOX;
 #pragma unroll
@@ -407,8 +407,8 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
     float *dst = nullptr;
     float scale = 1.f;
     if (MODE == MODE_FWD) dst = (kv_out && c == g.S - 1) ? kv_out + bh * 128 * 128 : nullptr;
-    if (MODE == MODE_STATE) dst = ws + (bh * g.S + c + 1) * (int64_t)128 * 128;
-    if (MODE == MODE_RSTATE) dst = ws + (bh * g.S + c - 1) * (int64_t)128 * 128;
+    if (MODE == MODE_STATE) dst = ws + (bh * g.wsS + c + 1) * (int64_t)128 * 128;
+    if (MODE == MODE_RSTATE) dst = ws + (bh * g.wsS + c - 1) * (int64_t)128 * 128;
     if (MODE == MODE_DV && c == 0 && kv_out) {  // dkv0 = lambda * D(0)
       dst = kv_out + bh * 128 * 128;
       scale = lambda[h];
@@ -603,9 +603,9 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   const uint32_t b_done = b_oempty + 8;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nch = OUT ? g.S : g.S - 1;
+  const int nch = OUT ? g.S : g.nst;
   const int64_t bh = blockIdx.x / nch;
-  const int c = blockIdx.x % nch + (MODE == MODE_RSTATE ? 1 : 0);
+  const int c = blockIdx.x % nch + (OUT ? 0 : g.c0);
   const int h = (int)(bh % g.H);
   const int64_t a = (int64_t)c * g.Lc;
   const int64_t b = g.L < a + g.Lc ? g.L : a + g.Lc;
@@ -874,9 +874,9 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       const float *init = nullptr;
       if (MODE == MODE_FWD || MODE == MODE_DQ) {
         if (c == 0) init = kv0 ? kv0 + bh * 128 * 128 : nullptr;
-        else init = ws + (bh * g.S + c) * (int64_t)128 * 128;
+        else init = ws + (bh * g.wsS + (int64_t)c * g.M) * (int64_t)128 * 128;
       } else if (MODE == MODE_DV || MODE == MODE_DK) {
-        if (c != g.S - 1) init = ws + (bh * g.S + c) * (int64_t)128 * 128;
+        if (c != g.S - 1) init = ws + (bh * g.wsS + (int64_t)(c + 1) * g.M - 1) * (int64_t)128 * 128;
       }
       const float dec = pw[nblk > 0 ? cb_of(0) : 0];
 #pragma unroll
@@ -908,8 +908,8 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
     float *dst = nullptr;
     float dscale = 1.f;
     if (MODE == MODE_FWD) dst = (kv_out && c == g.S - 1) ? kv_out + bh * 128 * 128 : nullptr;
-    if (MODE == MODE_STATE) dst = ws + (bh * g.S + c + 1) * (int64_t)128 * 128;
-    if (MODE == MODE_RSTATE) dst = ws + (bh * g.S + c - 1) * (int64_t)128 * 128;
+    if (MODE == MODE_STATE) dst = ws + (bh * g.wsS + c + 1) * (int64_t)128 * 128;
+    if (MODE == MODE_RSTATE) dst = ws + (bh * g.wsS + c - 1) * (int64_t)128 * 128;
     if (MODE == MODE_DV && c == 0 && kv_out) {  // dkv0 = lambda * D(0)
       dst = kv_out + bh * 128 * 128;
       dscale = lambda[h];
@@ -1054,7 +1054,7 @@ template <int MODE>
 cudaError_t launch_chunk(const CUtensorMap &m0, const CUtensorMap &m1, const CUtensorMap &m2,
                          const CUtensorMap &mo, const float *lam, const float *kv0, float *ws,
                          float *kv_out, const Geo &g, cudaStream_t st) {
-  const int64_t nch = Layout<MODE>::OUT ? g.S : g.S - 1;
+  const int64_t nch = Layout<MODE>::OUT ? g.S : g.nst;
   const int64_t grid = (int64_t)g.B * g.H * nch;
   if (g.variant == 1) {  // first (phase-serial) form of the kernel
     using LY = Layout<MODE>;
@@ -1089,11 +1089,12 @@ cudaError_t forward(const void *q, const void *k, const void *v, const float *la
     return cudaErrorInvalidValue;
   cudaError_t err = cudaSuccess;
   if (g.S > 1) {
-    err = timed(0, [&] { launch_chunk<MODE_STATE>(mk, mk, mv, mk, lam, nullptr, ws, nullptr, g, st); });
+    const Geo gs = state_geo(g, false);
+    err = timed(0, [&] { launch_chunk<MODE_STATE>(mk, mk, mv, mk, lam, nullptr, ws, nullptr, gs, st); });
     if (err) return err;
     err = timed(1, [&] {
       la2::simt::scan_fwd_kernel<128, 128>
-          <<<dim3(128 * 128 / la2::simt::NT, (unsigned)BH), la2::simt::NT, 0, st>>>(ws, kv0, lam, g);
+          <<<dim3(128 * 128 / la2::simt::NT, (unsigned)BH), la2::simt::NT, 0, st>>>(ws, kv0, lam, gs);
     });
     if (err) return err;
   }
@@ -1115,25 +1116,26 @@ cudaError_t backward(const void *q, const void *k, const void *v, const float *l
       !make_map(&mdk, dk, BH, g.L) || !make_map(&mdv, dv, BH, g.L))
     return cudaErrorInvalidValue;
   float *wsf = ws;
-  float *wsr = ws ? ws + (size_t)BH * g.S * 128 * 128 : nullptr;
+  float *wsr = ws ? ws + (size_t)BH * g.wsS * 128 * 128 : nullptr;
   const dim3 sgrid(128 * 128 / la2::simt::NT, (unsigned)BH);
+  const Geo gf = state_geo(g, false), gr = state_geo(g, true);
   cudaError_t err = cudaSuccess;
   // the forward pass leaves the same chunk entry states in the same place
   if (g.S > 1 && !reuse_fwd) {
-    err = timed(0, [&] { launch_chunk<MODE_STATE>(mk, mk, mv, mk, lam, nullptr, wsf, nullptr, g, st); });
+    err = timed(0, [&] { launch_chunk<MODE_STATE>(mk, mk, mv, mk, lam, nullptr, wsf, nullptr, gf, st); });
     if (err) return err;
     err = timed(1, [&] {
-      la2::simt::scan_fwd_kernel<128, 128><<<sgrid, la2::simt::NT, 0, st>>>(wsf, kv0, lam, g);
+      la2::simt::scan_fwd_kernel<128, 128><<<sgrid, la2::simt::NT, 0, st>>>(wsf, kv0, lam, gf);
     });
     if (err) return err;
   }
   err = timed(2, [&] { launch_chunk<MODE_DQ>(mg, mv, mk, mdq, lam, kv0, wsf, nullptr, g, st); });
   if (err) return err;
   if (g.S > 1) {
-    err = timed(3, [&] { launch_chunk<MODE_RSTATE>(mq, mq, mg, mq, lam, nullptr, wsr, nullptr, g, st); });
+    err = timed(3, [&] { launch_chunk<MODE_RSTATE>(mq, mq, mg, mq, lam, nullptr, wsr, nullptr, gr, st); });
     if (err) return err;
     err = timed(4, [&] {
-      la2::simt::scan_rev_kernel<128, 128><<<sgrid, la2::simt::NT, 0, st>>>(wsr, lam, g);
+      la2::simt::scan_rev_kernel<128, 128><<<sgrid, la2::simt::NT, 0, st>>>(wsr, lam, gr);
     });
     if (err) return err;
   }
