@@ -179,11 +179,20 @@ scan_fwd_kernel(float *__restrict__ ws, const float *__restrict__ kv0,
   if (idx >= D * E) return;
   const float decay = (float)pow_int((double)lambda[bh % g.H], g.Lc);
   float run = kv0 ? kv0[bh * D * E + idx] : 0.f;
-  // slot c holds the contribution of (sub-)chunk c-1, c = 1..nst (all full)
-  for (int c = 1; c <= g.nst; c++) {
-    float *p = ws + (bh * g.wsS + c) * (int64_t)D * E + idx;
-    run = decay * run + *p;
-    *p = run;
+  // slot c holds the contribution of (sub-)chunk c-1, c = 1..nst (all full);
+  // eight slots' loads are issued before the running sum walks them
+  float *base = ws + bh * g.wsS * (int64_t)D * E + idx;
+  for (int c0 = 1; c0 <= g.nst; c0 += 8) {
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; j++)
+      if (c0 + j <= g.nst) v[j] = base[(int64_t)(c0 + j) * D * E];
+#pragma unroll
+    for (int j = 0; j < 8; j++)
+      if (c0 + j <= g.nst) {
+        run = decay * run + v[j];
+        base[(int64_t)(c0 + j) * D * E] = run;
+      }
   }
 }
 
@@ -311,11 +320,22 @@ scan_rev_kernel(float *__restrict__ ws, const float *__restrict__ lambda, Geo g)
   const float full = (float)pow_int(lam, g.Lc);
   const float last = (float)pow_int(lam, g.L - (int64_t)(g.S - 1) * g.Lc);
   float run = 0.f;
-  // slot c holds the contribution of (sub-)chunk c+1, c+1 = c0..S-1
-  for (int c = g.S - 2; c >= g.c0 - 1; c--) {
-    float *p = ws + (bh * g.wsS + c) * (int64_t)D * E + idx;
-    run = (c + 1 == g.S - 1 ? last : full) * run + *p;
-    *p = run;
+  // slot c holds the contribution of (sub-)chunk c+1, c+1 = c0..S-1, walked
+  // downwards with eight slots' loads in flight
+  float *base = ws + bh * g.wsS * (int64_t)D * E + idx;
+  const int lo = g.c0 - 1;
+  for (int c1 = g.S - 2; c1 >= lo; c1 -= 8) {
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; j++)
+      if (c1 - j >= lo) v[j] = base[(int64_t)(c1 - j) * D * E];
+#pragma unroll
+    for (int j = 0; j < 8; j++)
+      if (c1 - j >= lo) {
+        const int c = c1 - j;
+        run = (c + 1 == g.S - 1 ? last : full) * run + v[j];
+        base[(int64_t)c * D * E] = run;
+      }
   }
 }
 
