@@ -57,6 +57,11 @@ def library():
         lib.la2_backward_ex.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I64, I, I, I,
                                         P, SZ, ctypes.c_uint, P]
         lib.la2_backward_ex.restype = I
+        lib.la2_forward_varlen.argtypes = [P, P, P, P, P, P, P, P, I, I, I64, I, I, I, P]
+        lib.la2_forward_varlen.restype = I
+        lib.la2_backward_varlen.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, I, I64, I, I,
+                                            I, P]
+        lib.la2_backward_varlen.restype = I
         lib.la2_decode_step.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
         lib.la2_decode_step.restype = I
         lib.la2_last_device_error.argtypes = [P]
@@ -219,6 +224,61 @@ def backward(q, k, v, lam, dO, kv0=None, *, want_dkv0: bool = False, outs=None,
                                _ptr(ws), 0 if ws is None else ws.numel(),
                                1 if reuse_forward_states else 0, _stream(stream))
     _check(code, "la2_backward")
+    return (dq, dk, dv, dkv0) if want_dkv0 else (dq, dk, dv)
+
+
+def _varlen_args(q, k, v, lam, cu_seqlens, kv0):
+    for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam), ("cu_seqlens", cu_seqlens)):
+        _dev(t, name)
+    H, T, d = q.shape
+    e = v.shape[-1]
+    if k.shape != q.shape or v.shape[:2] != (H, T):
+        raise ValueError("q, k must be [H, T, d] and v [H, T, e]")
+    if lam.dtype != torch.float32 or lam.numel() != H:
+        raise ValueError("lam must be float32 [H]")
+    if cu_seqlens.dtype != torch.int64 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+        raise ValueError("cu_seqlens must be int64 [N+1]")
+    N = cu_seqlens.numel() - 1
+    if kv0 is not None:
+        _dev(kv0, "kv0")
+        if kv0.dtype != torch.float32 or kv0.shape != (N, H, d, e):
+            raise ValueError("kv0 must be float32 [N,H,d,e]")
+    return N, H, T, d, e
+
+
+def forward_varlen(q, k, v, lam, cu_seqlens, kv0=None, *, want_state: bool = False,
+                   out=None, stream=None):
+    """Packed variable-length forward: q, k [H,T,d], v [H,T,e], sequence n on
+    rows cu_seqlens[n]..cu_seqlens[n+1] of every head; per-sequence states
+    [N,H,d,e].  Returns o [H,T,e] (and the final states)."""
+    lib = library()
+    N, H, T, d, e = _varlen_args(q, k, v, lam, cu_seqlens, kv0)
+    o = out if out is not None else torch.empty((H, T, e), dtype=q.dtype, device=q.device)
+    st = torch.empty((N, H, d, e), dtype=torch.float32, device=q.device) if want_state else None
+    code = lib.la2_forward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(cu_seqlens),
+                                  _ptr(kv0), _ptr(o), _ptr(st), N, H, T, d, e, _dt(q),
+                                  _stream(stream))
+    _check(code, "la2_forward_varlen")
+    return (o, st) if want_state else o
+
+
+def backward_varlen(q, k, v, lam, cu_seqlens, dO, kv0=None, *, want_dkv0: bool = False,
+                    outs=None, stream=None):
+    """Gradients (dq, dk, dv[, dkv0]) of sum(o * dO) for forward_varlen."""
+    lib = library()
+    N, H, T, d, e = _varlen_args(q, k, v, lam, cu_seqlens, kv0)
+    _dev(dO, "dO")
+    if dO.shape != v.shape:
+        raise ValueError("dO must match v")
+    if outs is not None:
+        dq, dk, dv = outs
+    else:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dkv0 = torch.empty((N, H, d, e), dtype=torch.float32, device=q.device) if want_dkv0 else None
+    code = lib.la2_backward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(cu_seqlens),
+                                   _ptr(kv0), _ptr(dO), _ptr(dq), _ptr(dk), _ptr(dv),
+                                   _ptr(dkv0), N, H, T, d, e, _dt(q), _stream(stream))
+    _check(code, "la2_backward_varlen")
     return (dq, dk, dv, dkv0) if want_dkv0 else (dq, dk, dv)
 
 

@@ -146,6 +146,7 @@ Path choose_path(int d, int e, la2_dtype dt) {
 // multiple of the block size `blk`) so that B*H*S CTAs fill the GPU.
 Geo plan(int B, int H, int64_t L, int blk, Path path) {
   Geo g;
+  g.cu = nullptr;
   g.inject = 0;
   g.variant = g_opt_variant.load();
   g.trace = g_opt_trace.load() - 1;
@@ -459,6 +460,125 @@ la2_status la2_backward_ex(const void *q, const void *k, const void *v,
   return to_status(err);
 }
 
+// ------------------------------------------------------- packed varlen
+namespace {
+
+// One CTA per (sequence, head) over the sequence's rows; no chunk split.
+Geo plan_varlen(int N, int H, int64_t T, const int64_t *cu) {
+  Geo g;
+  g.B = N;
+  g.H = H;
+  g.L = T;
+  g.S = 1;
+  g.Lc = T;
+  g.M = 1;
+  g.Ls = T;
+  g.Ssub = 1;
+  g.wsS = 1;
+  g.nst = 0;
+  g.c0 = 0;
+  g.cu = cu;
+  g.inject = 0;
+  g.variant = 0;  // the packed form exists in the warp-specialised kernel only
+  g.trace = -1;
+  return g;
+}
+
+// Shared argument checks of the packed entry points: sizes, null and
+// alignment rules, and no output overlapping any argument.
+la2_status check_varlen(int N, int H, int64_t T, int d, int e, la2_dtype dt, const int64_t *cu,
+                        const float *lambda, std::vector<Span> ins, std::vector<Span> outs,
+                        bool need_tensors) {
+  if (N < 0 || H < 0 || T < 0) return LA2_ERR_INVALID;
+  if (dt != LA2_F32 && dt != LA2_BF16) return LA2_ERR_UNSUPPORTED;
+  if (!shape_supported(d, e, dt)) return LA2_ERR_UNSUPPORTED;
+  if (!lambda || !cu || need_tensors) return LA2_ERR_INVALID;
+  if (reinterpret_cast<uintptr_t>(cu) % 8 != 0) return LA2_ERR_INVALID;
+  for (const Span &sp : ins)
+    if (sp.p && sp.p != (const void *)cu && !aligned16(sp.p)) return LA2_ERR_INVALID;
+  for (const Span &sp : outs)
+    if (sp.p && !aligned16(sp.p)) return LA2_ERR_INVALID;
+  std::vector<Span> all = ins;
+  all.insert(all.end(), outs.begin(), outs.end());
+  if (any_overlap(outs, all)) return LA2_ERR_INVALID;
+  return LA2_OK;
+}
+
+}  // namespace
+
+la2_status la2_forward_varlen(const void *q, const void *k, const void *v, const float *lambda,
+                              const int64_t *cu_seqlens, const float *kv0, void *o,
+                              float *kv_out, int N, int H, int64_t T, int d, int e,
+                              la2_dtype dt, cudaStream_t stream) {
+  if (N == 0 || H == 0) return (N < 0 || H < 0 || T < 0) ? LA2_ERR_INVALID : LA2_OK;
+  const size_t es = (dt == LA2_F32 || dt == LA2_BF16) ? esize(dt) : 0;
+  const size_t nq = (size_t)H * T * d * es, nv = (size_t)H * T * e * es;
+  const size_t ns = (size_t)N * H * d * e * sizeof(float);
+  if (kv_out && kv_out == kv0) return LA2_ERR_INVALID;
+  la2_status st = check_varlen(
+      N, H, T, d, e, dt, cu_seqlens, lambda,
+      {{q, nq}, {k, nq}, {v, nv}, {lambda, (size_t)H * 4}, {kv0, kv0 ? ns : 0},
+       {cu_seqlens, (size_t)(N + 1) * 8}},
+      {{o, nv}, {kv_out, kv_out ? ns : 0}}, T > 0 && (!q || !k || !v || !o));
+  if (st != LA2_OK) return st;
+  if (T == 0) {  // every sequence is empty
+    if (!kv_out) return LA2_OK;
+    return to_status(kv0 ? cudaMemcpyAsync(kv_out, kv0, ns, cudaMemcpyDeviceToDevice, stream)
+                         : cudaMemsetAsync(kv_out, 0, ns, stream));
+  }
+  Path p = choose_path(d, e, dt);
+  if (p == PATH_NONE) return LA2_ERR_UNSUPPORTED;
+  Geo g = plan_varlen(N, H, T, cu_seqlens);
+  cudaError_t err;
+  if (p == PATH_TC) {
+    err = la2::tc::forward_varlen(q, k, v, lambda, kv0, o, kv_out, g, stream,
+                                  [&](int, auto &&fn) { return timed(K_TC_FWD, stream, fn); });
+  } else if (dt == LA2_F32) {
+    err = LA2_DISPATCH_DE(d, e, simt_forward, float, q, k, v, lambda, kv0, o, kv_out, nullptr, g,
+                          stream);
+  } else {
+    err = LA2_DISPATCH_DE(d, e, simt_forward, __nv_bfloat16, q, k, v, lambda, kv0, o, kv_out,
+                          nullptr, g, stream);
+  }
+  return to_status(err);
+}
+
+la2_status la2_backward_varlen(const void *q, const void *k, const void *v, const float *lambda,
+                               const int64_t *cu_seqlens, const float *kv0, const void *dO,
+                               void *dq, void *dk, void *dv, float *dkv0, int N, int H,
+                               int64_t T, int d, int e, la2_dtype dt, cudaStream_t stream) {
+  if (N == 0 || H == 0) return (N < 0 || H < 0 || T < 0) ? LA2_ERR_INVALID : LA2_OK;
+  const size_t es = (dt == LA2_F32 || dt == LA2_BF16) ? esize(dt) : 0;
+  const size_t nq = (size_t)H * T * d * es, nv = (size_t)H * T * e * es;
+  const size_t ns = (size_t)N * H * d * e * sizeof(float);
+  la2_status st = check_varlen(
+      N, H, T, d, e, dt, cu_seqlens, lambda,
+      {{q, nq}, {k, nq}, {v, nv}, {dO, nv}, {lambda, (size_t)H * 4}, {kv0, kv0 ? ns : 0},
+       {cu_seqlens, (size_t)(N + 1) * 8}},
+      {{dq, nq}, {dk, nq}, {dv, nv}, {dkv0, dkv0 ? ns : 0}},
+      T > 0 && (!q || !k || !v || !dO || !dq || !dk || !dv));
+  if (st != LA2_OK) return st;
+  if (T == 0) return dkv0 ? to_status(cudaMemsetAsync(dkv0, 0, ns, stream)) : LA2_OK;
+  Path p = choose_path(d, e, dt);
+  if (p == PATH_NONE) return LA2_ERR_UNSUPPORTED;
+  Geo g = plan_varlen(N, H, T, cu_seqlens);
+  cudaError_t err;
+  if (p == PATH_TC) {
+    err = la2::tc::backward_varlen(q, k, v, lambda, kv0, dO, dq, dk, dv, dkv0, g, stream,
+                                   [&](int which, auto &&fn) {
+                                     return timed(which == 2 ? K_TC_DQ : which == 5 ? K_TC_DV : K_TC_DK,
+                                                  stream, fn);
+                                   });
+  } else if (dt == LA2_F32) {
+    err = LA2_DISPATCH_DE(d, e, simt_backward, float, q, k, v, lambda, kv0, dO, dq, dk, dv, dkv0,
+                          nullptr, g, false, stream);
+  } else {
+    err = LA2_DISPATCH_DE(d, e, simt_backward, __nv_bfloat16, q, k, v, lambda, kv0, dO, dq, dk,
+                          dv, dkv0, nullptr, g, false, stream);
+  }
+  return to_status(err);
+}
+
 la2_status la2_decode_step(const void *q, const void *k, const void *v, const float *lambda,
                            float *kv, void *o, int B, int H, int d, int e, la2_dtype dt,
                            cudaStream_t stream) {
@@ -493,6 +613,7 @@ la2_status la2_last_device_error(cudaStream_t stream) {
   if (word && cudaMemcpyToSymbol(la2::g_error_word, &zero, sizeof(zero)) != cudaSuccess)
     return LA2_ERR_CUDA;
   if (word & la2::ERR_TIMEOUT) return LA2_ERR_TIMEOUT;
+  if (word & la2::ERR_BOUNDS) return LA2_ERR_INVALID;  // e.g. bad varlen offsets
   if (word) return LA2_ERR_CUDA;
   return LA2_OK;
 }

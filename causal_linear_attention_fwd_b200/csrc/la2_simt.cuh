@@ -44,11 +44,46 @@ struct Geo {
   int wsS;
   int nst;
   int c0;
+  // Packed variable-length batch (NULL otherwise): B = N sequences, sequence
+  // n owning rows [cu[n], cu[n+1]) of every head's slab of L rows; tensors
+  // are [H, L, d|e], states [N, H, d, e]; S = 1.
+  const int64_t *cu;
   int inject;   // test hook: CTA 0 of a tensor-core pass withholds one MMA
                 // completion signal so that its bounded wait runs out
   int variant;  // tensor-core kernel form (0: warp-specialised, 1: phase-serial)
   int trace;    // tensor-core pass whose CTA 0 stamps the trace buffer (-1: none)
 };
+
+// What one CTA of a pass works on: state slot bh (the (b,h) or (sequence,
+// head) index), slab (the outer index of the [.., L, d] tensors), rows
+// [a, b) of that slab, head h and chunk c.  A varlen range that is not
+// inside the slab is recorded as a bounds error and treated as empty.
+struct Span {
+  int64_t bh, slab, a, b;
+  int h, c;
+};
+__device__ __forceinline__ Span span_of(const Geo &g, int nch, int c_first) {
+  Span s;
+  const int64_t q = blockIdx.x / nch;
+  s.bh = q;
+  s.h = (int)(q % g.H);
+  s.c = (int)(blockIdx.x % nch) + c_first;
+  if (g.cu) {
+    int64_t lo = g.cu[q / g.H], hi = g.cu[q / g.H + 1];
+    if (!(0 <= lo && lo <= hi && hi <= g.L)) {
+      if (threadIdx.x == 0) raise_error(ERR_BOUNDS);
+      lo = hi = 0;
+    }
+    s.slab = s.h;
+    s.a = lo;
+    s.b = hi;
+  } else {
+    s.slab = q;
+    s.a = (int64_t)s.c * g.Lc;
+    s.b = g.L < s.a + g.Lc ? g.L : s.a + g.Lc;
+  }
+  return s;
+}
 
 // Geometry of a chunk-state pre-pass and its scan: the (sub-)chunk split,
 // forward (chunks 0 .. S-2 of the main split, as (S-1)*M sub-chunks from
@@ -102,11 +137,9 @@ fwd_kernel(const T *__restrict__ q, const T *__restrict__ k,
   float *pw = Ps + C * LDP;           // C+1
 
   const int nch = OUT ? g.S : g.S - 1;
-  const int64_t bh = blockIdx.x / nch;
-  const int c = blockIdx.x % nch;
-  const int h = (int)(bh % g.H);
-  const int64_t a = (int64_t)c * g.Lc;
-  const int64_t b = g.L < a + g.Lc ? g.L : a + g.Lc;
+  const Span sp = span_of(g, nch, 0);
+  const int64_t bh = sp.bh, a = sp.a, b = sp.b, slab = sp.slab;
+  const int c = sp.c, h = sp.h;
 
   fill_pow(pw, lambda[h]);
   const float *init = nullptr;
@@ -120,9 +153,9 @@ fwd_kernel(const T *__restrict__ q, const T *__restrict__ k,
 
   for (int64_t p = a; p < b; p += C) {
     const int cb = (int)(b - p < C ? b - p : C);
-    if (OUT) load_tile<T, D>(Qs, LDQ, q + (bh * g.L + p) * D, cb);
-    load_tile<T, D>(Ks, LDQ, k + (bh * g.L + p) * D, cb);
-    load_tile<T, E>(Vs, LDV, v + (bh * g.L + p) * E, cb);
+    if (OUT) load_tile<T, D>(Qs, LDQ, q + (slab * g.L + p) * D, cb);
+    load_tile<T, D>(Ks, LDQ, k + (slab * g.L + p) * D, cb);
+    load_tile<T, E>(Vs, LDV, v + (slab * g.L + p) * E, cb);
     __syncthreads();
     if (OUT) {
       // P = (Q K^T) (.) M over the causal triangle
@@ -146,7 +179,7 @@ fwd_kernel(const T *__restrict__ q, const T *__restrict__ k,
         for (int t = 0; t <= s; t++) acc1 += Ps[s * LDP + t] * Vs[t * LDV + j];
 #pragma unroll 8
         for (int i = 0; i < D; i++) acc2 += Qs[s * LDQ + i] * KV[i * LDS + j];
-        io<T>::st(o + (bh * g.L + p + s) * E + j, acc1 + pw[s + 1] * acc2);
+        io<T>::st(o + (slab * g.L + p + s) * E + j, acc1 + pw[s + 1] * acc2);
       }
       __syncthreads();
     }
@@ -212,11 +245,9 @@ dq_kernel(const T *__restrict__ k, const T *__restrict__ v,
   float *Ps = Ks + C * LDK;       // C x (C+1)
   float *pw = Ps + C * LDP;
 
-  const int64_t bh = blockIdx.x / g.S;
-  const int c = blockIdx.x % g.S;
-  const int h = (int)(bh % g.H);
-  const int64_t a = (int64_t)c * g.Lc;
-  const int64_t b = g.L < a + g.Lc ? g.L : a + g.Lc;
+  const Span sp = span_of(g, g.S, 0);
+  const int64_t bh = sp.bh, a = sp.a, b = sp.b, slab = sp.slab;
+  const int c = sp.c, h = sp.h;
   fill_pow(pw, lambda[h]);
   const float *init = c == 0 ? (kv0 ? kv0 + bh * D * E : nullptr)
                              : ws + (bh * g.S + c) * (int64_t)D * E;
@@ -226,9 +257,9 @@ dq_kernel(const T *__restrict__ k, const T *__restrict__ v,
 
   for (int64_t p = a; p < b; p += C) {
     const int cb = (int)(b - p < C ? b - p : C);
-    load_tile<T, E>(Gs, LDG, dO + (bh * g.L + p) * E, cb);
-    load_tile<T, E>(Vs, LDG, v + (bh * g.L + p) * E, cb);
-    load_tile<T, D>(Ks, LDK, k + (bh * g.L + p) * D, cb);
+    load_tile<T, E>(Gs, LDG, dO + (slab * g.L + p) * E, cb);
+    load_tile<T, E>(Vs, LDG, v + (slab * g.L + p) * E, cb);
+    load_tile<T, D>(Ks, LDK, k + (slab * g.L + p) * D, cb);
     __syncthreads();
     for (int idx = threadIdx.x; idx < C * C; idx += NT) {
       int s = idx / C, t = idx % C;
@@ -249,7 +280,7 @@ dq_kernel(const T *__restrict__ k, const T *__restrict__ v,
       for (int t = 0; t <= s; t++) acc1 += Ps[s * LDP + t] * Ks[t * LDK + i];
 #pragma unroll 8
       for (int j = 0; j < E; j++) acc2 += Gs[s * LDG + j] * KV[i * LDS + j];
-      io<T>::st(dq + (bh * g.L + p + s) * D + i, acc1 + pw[s + 1] * acc2);
+      io<T>::st(dq + (slab * g.L + p + s) * D + i, acc1 + pw[s + 1] * acc2);
     }
     __syncthreads();
     for (int idx = threadIdx.x; idx < D * E; idx += NT) {
@@ -279,12 +310,9 @@ rev_state_kernel(const T *__restrict__ q, const T *__restrict__ dO,
   float *Gs = Qs + C * LDQ;      // C x E
   float *pw = Gs + C * LDG;
 
-  const int nch = g.S - 1;
-  const int64_t bh = blockIdx.x / nch;
-  const int c = 1 + blockIdx.x % nch;
-  const int h = (int)(bh % g.H);
-  const int64_t a = (int64_t)c * g.Lc;
-  const int64_t b = g.L < a + g.Lc ? g.L : a + g.Lc;
+  const Span sp = span_of(g, g.S - 1, 1);
+  const int64_t bh = sp.bh, a = sp.a, b = sp.b, slab = sp.slab;
+  const int c = sp.c, h = sp.h;
   fill_pow(pw, lambda[h]);
   for (int idx = threadIdx.x; idx < D * E; idx += NT) Dst[idx] = 0.f;
   __syncthreads();
@@ -292,8 +320,8 @@ rev_state_kernel(const T *__restrict__ q, const T *__restrict__ dO,
   for (int64_t ib = nb - 1; ib >= 0; ib--) {
     const int64_t p = a + ib * C;
     const int cb = (int)(b - p < C ? b - p : C);
-    load_tile<T, D>(Qs, LDQ, q + (bh * g.L + p) * D, cb);
-    load_tile<T, E>(Gs, LDG, dO + (bh * g.L + p) * E, cb);
+    load_tile<T, D>(Qs, LDQ, q + (slab * g.L + p) * D, cb);
+    load_tile<T, E>(Gs, LDG, dO + (slab * g.L + p) * E, cb);
     __syncthreads();
     for (int idx = threadIdx.x; idx < D * E; idx += NT) {
       int i = idx / E, j = idx % E;
@@ -357,11 +385,9 @@ dkdv_kernel(const T *__restrict__ q, const T *__restrict__ k,
   float *dPt = Pt + C * LDP;       // C x (C+1)  (dO V^T (.) M)^T
   float *pw = dPt + C * LDP;
 
-  const int64_t bh = blockIdx.x / g.S;
-  const int c = blockIdx.x % g.S;
-  const int h = (int)(bh % g.H);
-  const int64_t a = (int64_t)c * g.Lc;
-  const int64_t b = g.L < a + g.Lc ? g.L : a + g.Lc;
+  const Span sp = span_of(g, g.S, 0);
+  const int64_t bh = sp.bh, a = sp.a, b = sp.b, slab = sp.slab;
+  const int c = sp.c, h = sp.h;
   fill_pow(pw, lambda[h]);
   const float *init = c == g.S - 1 ? nullptr : ws + (bh * g.S + c) * (int64_t)D * E;
   for (int idx = threadIdx.x; idx < D * E; idx += NT)
@@ -372,10 +398,10 @@ dkdv_kernel(const T *__restrict__ q, const T *__restrict__ k,
   for (int64_t ib = nb - 1; ib >= 0; ib--) {
     const int64_t p = a + ib * C;
     const int cb = (int)(b - p < C ? b - p : C);
-    load_tile<T, D>(Qs, LDQ, q + (bh * g.L + p) * D, cb);
-    load_tile<T, D>(Ks, LDQ, k + (bh * g.L + p) * D, cb);
-    load_tile<T, E>(Vs, LDG, v + (bh * g.L + p) * E, cb);
-    load_tile<T, E>(Gs, LDG, dO + (bh * g.L + p) * E, cb);
+    load_tile<T, D>(Qs, LDQ, q + (slab * g.L + p) * D, cb);
+    load_tile<T, D>(Ks, LDQ, k + (slab * g.L + p) * D, cb);
+    load_tile<T, E>(Vs, LDG, v + (slab * g.L + p) * E, cb);
+    load_tile<T, E>(Gs, LDG, dO + (slab * g.L + p) * E, cb);
     __syncthreads();
     // transposed masked products, [t][s] with s >= t
     for (int idx = threadIdx.x; idx < C * C; idx += NT) {
@@ -401,7 +427,7 @@ dkdv_kernel(const T *__restrict__ q, const T *__restrict__ k,
       for (int s = t; s < cb; s++) acc1 += dPt[t * LDP + s] * Qs[s * LDQ + i];
 #pragma unroll 8
       for (int j = 0; j < E; j++) acc2 += Vs[t * LDG + j] * Dst[i * LDS + j];
-      io<T>::st(dk + (bh * g.L + p + t) * D + i, acc1 + pw[cb - t] * acc2);
+      io<T>::st(dk + (slab * g.L + p + t) * D + i, acc1 + pw[cb - t] * acc2);
     }
     for (int idx = threadIdx.x; idx < C * E; idx += NT) {
       int t = idx / E, j = idx % E;
@@ -410,7 +436,7 @@ dkdv_kernel(const T *__restrict__ q, const T *__restrict__ k,
       for (int s = t; s < cb; s++) acc1 += Pt[t * LDP + s] * Gs[s * LDG + j];
 #pragma unroll 8
       for (int i = 0; i < D; i++) acc2 += Ks[t * LDQ + i] * Dst[i * LDS + j];
-      io<T>::st(dv + (bh * g.L + p + t) * E + j, acc1 + pw[cb - t] * acc2);
+      io<T>::st(dv + (slab * g.L + p + t) * E + j, acc1 + pw[cb - t] * acc2);
     }
     __syncthreads();
     for (int idx = threadIdx.x; idx < D * E; idx += NT) {

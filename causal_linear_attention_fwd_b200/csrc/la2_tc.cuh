@@ -563,12 +563,18 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 // TRACE: the instantiation that records the trace stamps (LA2_OPT_TRACE);
 // the stamps' branches cost a few percent, so the other launches compile
 // without them.
-template <int MODE, bool TRACE>
+// VARLEN: the packed variable-length form (output passes only): one CTA
+// per (sequence, head) over rows [cu[n], cu[n+1]) of the head's slab.  A
+// sequence's last block reads the next sequence's rows, so the reverse
+// passes mask the columns past the block's end and that block's output rows
+// go out by plain stores (`outp`) instead of a TMA box.
+template <int MODE, bool TRACE, bool VARLEN>
 __global__ void __launch_bounds__(NT2, 1)
 chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
               const __grid_constant__ CUtensorMap tm2, const __grid_constant__ CUtensorMap tmo,
               const float *__restrict__ lambda, const float *__restrict__ kv0,
-              float *__restrict__ ws, float *__restrict__ kv_out, Geo g) {
+              float *__restrict__ ws, float *__restrict__ kv_out, __nv_bfloat16 *__restrict__ outp,
+              Geo g) {
   using LY = Layout2<MODE>;
   using TR = Traits<MODE>;
   constexpr bool OUT = LY::OUT;
@@ -604,11 +610,19 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nch = OUT ? g.S : g.nst;
-  const int64_t bh = blockIdx.x / nch;
-  const int c = blockIdx.x % nch + (OUT ? 0 : g.c0);
-  const int h = (int)(bh % g.H);
-  const int64_t a = (int64_t)c * g.Lc;
-  const int64_t b = g.L < a + g.Lc ? g.L : a + g.Lc;
+  int64_t bh, a, b, slab;
+  int c, h;
+  if constexpr (VARLEN) {
+    const Span sp = span_of(g, 1, 0);
+    bh = sp.bh, a = sp.a, b = sp.b, slab = sp.slab, c = sp.c, h = sp.h;
+  } else {
+    bh = blockIdx.x / nch;
+    c = blockIdx.x % nch + (OUT ? 0 : g.c0);
+    h = (int)(bh % g.H);
+    a = (int64_t)c * g.Lc;
+    b = g.L < a + g.Lc ? g.L : a + g.Lc;
+    slab = bh;
+  }
   const int nblk = (int)((b - a + BLOCK - 1) / BLOCK);
   auto block_of = [&](int j) { return REV ? nblk - 1 - j : j; };
   auto p_of = [&](int j) { return a + (int64_t)block_of(j) * BLOCK; };
@@ -667,7 +681,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       for (int j = 0; j < nblk; j++) {
         const int st = j % NS;
         const uint32_t ph = (uint32_t)((j / NS - 1) & 1);
-        const int y = (int)p_of(j), z = (int)bh;
+        const int y = (int)p_of(j), z = (int)slab;
         uint32_t dst = sbase + st * LY::STAGE;
         // (A0, B1): their slots free once block j-NS's products are done
         if (j >= NS && !mbar_wait(b_eab + 8 * st, ph, abort_flag)) break;
@@ -833,6 +847,15 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
           uint32_t r[32];
           tmem_ld32(tl + sb + part * 32, r);
           tmem_wait_ld();
+          if constexpr (VARLEN && REV) {
+            // columns past the block's end belong to the next sequence
+            const int cbi = cb_of(i);
+            if (cbi < BLOCK) {
+#pragma unroll
+              for (int k = 0; k < 32; k++)
+                if (part * 32 + k >= cbi) r[k] = 0u;
+            }
+          }
           if (part == q) {
 #pragma unroll
             for (int j = 0; j < 16; j++) {
@@ -965,10 +988,26 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       __syncwarp();
       if (lane == 0) mbar_arrive(b_oempty);
       if (OUT) role_sync(BAR_EPI, 128);  // the whole output tile is in shared memory
+      bool tail_rows = false;
+      if constexpr (VARLEN) {
+        // the sequence's last, partial block: its rows only, by plain stores
+        const int cbi = cb_of(i);
+        if (cbi < BLOCK) {
+          tail_rows = true;
+          if (row < cbi) {
+            uint4 w[16];
+            ld_row_sw128(stg, row, w);
+            uint4 *gdst = reinterpret_cast<uint4 *>(outp + ((int64_t)slab * g.L + p_of(i) + row) * 128);
+#pragma unroll
+            for (int k = 0; k < 16; k++) gdst[k] = w[k];
+          }
+          role_sync(BAR_EPI, 128);  // the staging tile has been read
+        }
+      }
       if (wtid == 0) {
-        if (OUT) {
+        if (OUT && !tail_rows) {
           const uint32_t sst = sbase + st * LY::STAGE + LY::C_OFF;
-          const int y = (int)p_of(i), z = (int)bh;
+          const int y = (int)p_of(i), z = (int)slab;
           tma_store_3d(&tmo, sst, 0, y, z);
           tma_store_3d(&tmo, sst + BOX, 64, y, z);
           tma_store_commit();
@@ -976,6 +1015,14 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
         }
         LA2_TRACE(7, i);
         mbar_arrive(b_ec + 8 * st);  // B2 slot reusable
+      }
+    }
+    if constexpr (VARLEN) {
+      // an empty sequence: its final state is the initial one, dkv0 is 0
+      if (nblk == 0 && dst) {
+        const float *src0 = (MODE == MODE_FWD && kv0) ? kv0 + bh * 128 * 128 : nullptr;
+        for (int k = 0; k < 128; k++)
+          dst[(int64_t)row * 128 + k] = src0 ? src0[(int64_t)row * 128 + k] : 0.f;
       }
     }
     if (OUT && wtid == 0) tma_store_wait0();
@@ -1053,7 +1100,7 @@ inline bool make_map(CUtensorMap *m, const void *ptr, int64_t BH, int64_t L) {
 template <int MODE>
 cudaError_t launch_chunk(const CUtensorMap &m0, const CUtensorMap &m1, const CUtensorMap &m2,
                          const CUtensorMap &mo, const float *lam, const float *kv0, float *ws,
-                         float *kv_out, const Geo &g, cudaStream_t st) {
+                         float *kv_out, const Geo &g, cudaStream_t st, void *outp = nullptr) {
   const int64_t nch = Layout<MODE>::OUT ? g.S : g.nst;
   const int64_t grid = (int64_t)g.B * g.H * nch;
   if (g.variant == 1) {  // first (phase-serial) form of the kernel
@@ -1065,10 +1112,14 @@ cudaError_t launch_chunk(const CUtensorMap &m0, const CUtensorMap &m1, const CUt
     return cudaGetLastError();
   }
   using LY = Layout2<MODE>;
-  auto k = g.trace == MODE ? chunk_kernel2<MODE, true> : chunk_kernel2<MODE, false>;
+  auto k = g.trace == MODE ? chunk_kernel2<MODE, true, false> : chunk_kernel2<MODE, false, false>;
+  if constexpr (LY::OUT) {
+    if (g.cu) k = chunk_kernel2<MODE, false, true>;
+  }
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::SMEM);
   if (e != cudaSuccess) return e;
-  k<<<(unsigned)grid, NT2, LY::SMEM, st>>>(m0, m1, m2, mo, lam, kv0, ws, kv_out, g);
+  k<<<(unsigned)grid, NT2, LY::SMEM, st>>>(m0, m1, m2, mo, lam, kv0, ws, kv_out,
+                                          static_cast<__nv_bfloat16 *>(outp), g);
   return cudaGetLastError();
 }
 
@@ -1142,6 +1193,40 @@ cudaError_t backward(const void *q, const void *k, const void *v, const float *l
   err = timed(5, [&] { launch_chunk<MODE_DV>(mk, mq, mg, mdv, lam, nullptr, wsr, dkv0, g, st); });
   if (err) return err;
   return timed(6, [&] { launch_chunk<MODE_DK>(mv, mg, mq, mdk, lam, nullptr, wsr, nullptr, g, st); });
+}
+
+// Packed variable-length batch: g.B = N sequences, g.L = T rows per head
+// slab, g.cu the device offsets, S = 1 (one CTA per (sequence, head)).
+// Tensor maps run over [H, T, 128].
+template <typename Timed>
+cudaError_t forward_varlen(const void *q, const void *k, const void *v, const float *lam,
+                           const float *kv0, void *o, float *kv_out, const Geo &g,
+                           cudaStream_t st, Timed &&timed) {
+  if (!geometry_ok(g) || !g.cu || g.S != 1) return cudaErrorInvalidValue;
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map(&mq, q, g.H, g.L) || !make_map(&mk, k, g.H, g.L) || !make_map(&mv, v, g.H, g.L) ||
+      !make_map(&mo, o, g.H, g.L))
+    return cudaErrorInvalidValue;
+  return timed(2, [&] { launch_chunk<MODE_FWD>(mq, mk, mv, mo, lam, kv0, nullptr, kv_out, g, st, o); });
+}
+
+template <typename Timed>
+cudaError_t backward_varlen(const void *q, const void *k, const void *v, const float *lam,
+                            const float *kv0, const void *dO, void *dq, void *dk, void *dv,
+                            float *dkv0, const Geo &g, cudaStream_t st, Timed &&timed) {
+  if (!geometry_ok(g) || !g.cu || g.S != 1) return cudaErrorInvalidValue;
+  CUtensorMap mq, mk, mv, mg, mdq, mdk, mdv;
+  if (!make_map(&mq, q, g.H, g.L) || !make_map(&mk, k, g.H, g.L) || !make_map(&mv, v, g.H, g.L) ||
+      !make_map(&mg, dO, g.H, g.L) || !make_map(&mdq, dq, g.H, g.L) ||
+      !make_map(&mdk, dk, g.H, g.L) || !make_map(&mdv, dv, g.H, g.L))
+    return cudaErrorInvalidValue;
+  cudaError_t err = timed(2, [&] {
+    launch_chunk<MODE_DQ>(mg, mv, mk, mdq, lam, kv0, nullptr, nullptr, g, st, dq);
+  });
+  if (err) return err;
+  err = timed(5, [&] { launch_chunk<MODE_DV>(mk, mq, mg, mdv, lam, nullptr, nullptr, dkv0, g, st, dv); });
+  if (err) return err;
+  return timed(6, [&] { launch_chunk<MODE_DK>(mv, mg, mq, mdk, lam, nullptr, nullptr, nullptr, g, st, dk); });
 }
 
 }  // namespace tc

@@ -164,6 +164,44 @@ la2_status la2_backward_ex(const void *q, const void *k, const void *v,
                            cudaStream_t stream);
 
 /*
+ * Packed variable-length batches: N sequences of different lengths stored
+ * back to back.  q, k [H, T, d] and v, o [H, T, e] (row-major; the slab of
+ * head h holds all sequences' rows for that head), cu_seqlens device int64
+ * [N+1] (8-byte aligned) with 0 = cu[0] <= cu[1] <= ... <= cu[N] = T:
+ * sequence n owns rows [cu[n], cu[n+1]) of every head's slab.  Each
+ * sequence is an independent problem with its own decay state, reset at its
+ * first row: kv0 / kv_out (and dkv0 in the backward) are fp32 [N, H, d, e],
+ * kv0 may be NULL (zero), kv_out / dkv0 may be NULL (not written); an empty
+ * sequence passes kv0 through to kv_out (its dkv0 is 0).  lambda [H] as for
+ * la2_forward.  The forward computes, per sequence, what la2_forward does
+ * for B = 1, L = its length; the backward, what la2_backward does.  One CTA
+ * per (sequence, head) walks the whole sequence (no chunk split, so no
+ * workspace): a batch with a few very long sequences runs at the speed of
+ * its longest one.  No synchronisation.
+ * Errors: LA2_ERR_INVALID for negative sizes, a NULL lambda or cu_seqlens,
+ * NULL tensors with T > 0, misaligned pointers, an output overlapping any
+ * argument, kv_out == kv0; LA2_ERR_UNSUPPORTED for an unknown dtype or a
+ * (d, e) outside the supported set.  Offsets outside [0, T] or decreasing
+ * are not checked on the host (that would synchronise): the kernel treats
+ * such a sequence as empty and sets the bounds bit (2) of the device error
+ * word, which la2_last_device_error() reports as LA2_ERR_INVALID.
+ * Source: the Lightning Attention-2 notes page, "Tiling." paragraph, applied
+ * to each sequence of the batch; the pages describe no packed form (it is
+ * the batching the parallel training form needs).
+ */
+la2_status la2_forward_varlen(const void *q, const void *k, const void *v,
+                              const float *lambda, const int64_t *cu_seqlens,
+                              const float *kv0, void *o, float *kv_out,
+                              int N, int H, int64_t T, int d, int e, la2_dtype dt,
+                              cudaStream_t stream);
+la2_status la2_backward_varlen(const void *q, const void *k, const void *v,
+                               const float *lambda, const int64_t *cu_seqlens,
+                               const float *kv0, const void *dO,
+                               void *dq, void *dk, void *dv, float *dkv0,
+                               int N, int H, int64_t T, int d, int e, la2_dtype dt,
+                               cudaStream_t stream);
+
+/*
  * One recurrent decode step for one new token per (b,h):
  *     kv <- lambda kv + k^T v,    o = q kv
  * q, k [B,H,d], v, o [B,H,e] of type dt; kv fp32 [B,H,d,e] updated IN PLACE
@@ -179,8 +217,10 @@ la2_status la2_decode_step(const void *q, const void *k, const void *v,
 
 /*
  * Synchronises `stream`, then reports and clears the device error word that
- * the kernels' bounded waits set when a wait gives up (LA2_ERR_TIMEOUT), or
- * LA2_ERR_CUDA if the synchronisation itself fails.  LA2_OK otherwise.
+ * the kernels set: LA2_ERR_TIMEOUT when a bounded wait gave up,
+ * LA2_ERR_INVALID when a kernel met out-of-range data it could not use (a
+ * packed-batch offset outside [0, T]); LA2_ERR_CUDA if the synchronisation
+ * itself fails.  LA2_OK otherwise.
  */
 la2_status la2_last_device_error(cudaStream_t stream);
 

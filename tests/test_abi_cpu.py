@@ -53,7 +53,7 @@ def test_set_option_roundtrip(lib):
 
 # fake, 16-byte aligned, non-overlapping device addresses
 MB = 1 << 20
-Q, K, V, O, LAM, KV0, KVO, WS, DO, DQ, DK, DV, DKV = [(i + 1) * 64 * MB for i in range(13)]
+Q, K, V, O, LAM, KV0, KVO, WS, DO, DQ, DK, DV, DKV, CU = [(i + 1) * 64 * MB for i in range(14)]
 
 
 def fwd(lib, q=Q, k=K, v=V, lam=LAM, kv0=None, o=O, kvo=None, Bn=1, H=2, L=100, d=64, e=64,
@@ -105,6 +105,37 @@ def test_decode_validation(lib):
     assert f(Q, K, V, LAM, KV0 + 4, O, 2, 2, 64, 64, B.LA2_BF16, None) == INV
     assert f(Q, K, V, LAM, KV0, O, 2, 2, 64, 80, B.LA2_BF16, None) == B.LA2_ERR_UNSUPPORTED
     assert f(Q, K, V, LAM, KV0, O, 0, 2, 64, 64, B.LA2_BF16, None) == B.LA2_OK
+
+
+def test_varlen_validation(lib):
+    INV, UNS, OK = B.LA2_ERR_INVALID, B.LA2_ERR_UNSUPPORTED, B.LA2_OK
+
+    def fwdv(q=Q, k=K, v=V, lam=LAM, cu=CU, kv0=None, o=O, kvo=None, N=3, H=2, T=100, d=64,
+             e=64, dt=B.LA2_BF16):
+        return lib.la2_forward_varlen(q, k, v, lam, cu, kv0, o, kvo, N, H, T, d, e, dt, None)
+
+    def bwdv(q=Q, k=K, v=V, lam=LAM, cu=CU, kv0=None, dO=DO, dq=DQ, dk=DK, dv=DV, dkv=None, N=3,
+             H=2, T=100, d=64, e=64, dt=B.LA2_BF16):
+        return lib.la2_backward_varlen(q, k, v, lam, cu, kv0, dO, dq, dk, dv, dkv, N, H, T, d, e,
+                                       dt, None)
+
+    assert fwdv(cu=None) == INV
+    assert fwdv(cu=CU + 4) == INV                    # offsets not 8-byte aligned
+    assert fwdv(lam=None) == INV
+    assert fwdv(q=None) == INV
+    assert fwdv(N=-1) == INV and fwdv(T=-1) == INV and fwdv(H=-2) == INV
+    assert fwdv(d=96) == UNS and fwdv(dt=5) == UNS
+    assert fwdv(kv0=KV0, kvo=KV0) == INV             # kv_out == kv0
+    assert fwdv(o=Q + 64) == INV                     # o overlaps q
+    assert fwdv(kvo=CU) == INV                       # kv_out overlaps the offsets
+    assert fwdv(q=Q + 8) == INV                      # not 16-byte aligned
+    assert fwdv(N=0) == OK and fwdv(H=0) == OK       # empty batch
+    assert fwdv(T=0, q=None, k=None, v=None, o=None) == OK  # all sequences empty, no state out
+    assert bwdv(dO=None) == INV
+    assert bwdv(dk=DQ) == INV                        # two outputs at one address
+    assert bwdv(dv=CU) == INV                        # output over the offsets
+    assert bwdv(d=128, e=80) == UNS
+    assert bwdv(N=0) == OK
 
 
 def test_workspace_rules(lib):

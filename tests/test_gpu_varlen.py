@@ -1,0 +1,117 @@
+"""GPU parity of the packed variable-length entry points against the oracle.
+
+Each sequence of a packed batch is an independent problem with its own state,
+so the reference is the oracle run on each sequence's rows alone (B = 1), its
+initial state the sequence's slice of kv0.  The lengths mix empty, single-row,
+block-sized, ragged and multi-block sequences; every sequence but the last is
+followed by another one's rows, which its last block reads and must ignore."""
+import numpy as np
+import pytest
+import torch
+
+import causal_linear_attention_fwd_b200 as la2
+from causal_linear_attention_fwd_b200 import inputs
+from gpu_util import check, host
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+PATHS = {"simt": 1, "tc": 2}
+LENS = [300, 0, 1, 127, 128, 129, 1000, 5, 256]
+
+
+def packed_inputs(lens, H, d, e, dtype, seed):
+    T = sum(lens)
+    N = len(lens)
+    x = inputs.make_inputs(1, H, T, d, e, dtype=dtype, device=DEV, seed=seed)
+    x = {n: t[0] for n, t in x.items()}  # [H, T, .]
+    kv0 = inputs.make_inputs(N, H, 1, d, e, dtype=dtype, device=DEV, seed=seed + 1,
+                             with_dO=False, with_kv0=True)["kv0"]
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int64, device=DEV)
+    return x, kv0, cu
+
+
+def reference(orc, x, kv0, cu, lam):
+    """Per-sequence oracle results scattered back to the packed layout."""
+    H, T, d = x["q"].shape
+    e = x["v"].shape[-1]
+    N = cu.numel() - 1
+    h = {n: host(t) for n, t in x.items()}
+    lam_h = lam.double().cpu().numpy()
+    s0 = kv0.double().cpu().numpy()
+    o = np.zeros((H, T, e)); dq = np.zeros((H, T, d)); dk = np.zeros((H, T, d))
+    dv = np.zeros((H, T, e))
+    st = np.zeros((N, H, d, e)); dkv0 = np.zeros((N, H, d, e))
+    offs = cu.cpu().numpy()
+    for n in range(N):
+        a, b = int(offs[n]), int(offs[n + 1])
+        if a == b:
+            st[n] = s0[n]
+            continue
+        sl = {k: v[None, :, a:b] for k, v in h.items()}
+        on, sn = orc.forward(sl["q"], sl["k"], sl["v"], lam_h, s0[n:n + 1], want_state=True)
+        g = orc.backward(sl["q"], sl["k"], sl["v"], lam_h, sl["dO"], s0[n:n + 1])
+        o[:, a:b] = on[0]
+        st[n] = sn[0]
+        dq[:, a:b], dk[:, a:b], dv[:, a:b] = g[0][0], g[1][0], g[2][0]
+        dkv0[n] = g[3][0]
+    return o, st, dq, dk, dv, dkv0
+
+
+@pytest.mark.parametrize("path,dtype,de", [("tc", torch.bfloat16, (128, 128)),
+                                           ("simt", torch.float32, (64, 64)),
+                                           ("simt", torch.bfloat16, (64, 128))])
+def test_varlen_matches_oracle(orc, path, dtype, de):
+    d, e = de
+    H = 3
+    x, kv0, cu = packed_inputs(LENS, H, d, e, dtype, seed=5)
+    lam = inputs.fixed_lambdas((1.0, 0.97, 0.0), DEV)
+    old = la2.set_option(la2.LA2_OPT_PATH, PATHS[path])
+    try:
+        o, st = la2.forward_varlen(x["q"], x["k"], x["v"], lam, cu, kv0, want_state=True)
+        dq, dk, dv, dkv0 = la2.backward_varlen(x["q"], x["k"], x["v"], lam, cu, x["dO"], kv0,
+                                               want_dkv0=True)
+        torch.cuda.synchronize()
+    finally:
+        la2.set_option(la2.LA2_OPT_PATH, old)
+    assert la2.last_device_error() == 0
+    ref = reference(orc, x, kv0, cu, lam)
+    for name, got, r in zip(("o", "kv_out", "dq", "dk", "dv", "dkv0"),
+                            (o, st, dq, dk, dv, dkv0), ref):
+        check(f"varlen {path} {name}", got, r, dtype)
+
+
+def test_varlen_equals_batched_call():
+    """Equal-length sequences packed give what the [B,H,L,d] call gives for
+    the same rows (the tensor-core path in both)."""
+    Bn, H, L = 3, 2, 700
+    x = inputs.make_inputs(Bn, H, L, 128, 128, dtype=torch.bfloat16, device=DEV, seed=9,
+                           with_kv0=True)
+    lam = inputs.decay_lambdas(H, DEV)
+    o_b, st_b = la2.forward(x["q"], x["k"], x["v"], lam, x["kv0"], want_state=True)
+    pack = {n: x[n].permute(1, 0, 2, 3).reshape(H, Bn * L, -1).contiguous()
+            for n in ("q", "k", "v")}
+    cu = torch.arange(0, (Bn + 1) * L, L, dtype=torch.int64, device=DEV)
+    o_v, st_v = la2.forward_varlen(pack["q"], pack["k"], pack["v"], lam, cu, x["kv0"],
+                                   want_state=True)
+    torch.cuda.synchronize()
+    o_v = o_v.reshape(H, Bn, L, -1).permute(1, 0, 2, 3)
+    # the batched call may split each sequence into chunks (another
+    # summation order), so the two agree to the parity tolerance
+    check("packed vs batched o", o_v, host(o_b), torch.bfloat16)
+    check("packed vs batched state", st_v, host(st_b), torch.bfloat16)
+
+
+def test_varlen_bad_offsets_reported():
+    """Offsets outside [0, T] or decreasing: that sequence is treated as
+    empty and the device error word reports LA2_ERR_INVALID; nothing faults."""
+    H, T = 2, 600
+    x = inputs.make_inputs(1, H, T, 128, 128, dtype=torch.bfloat16, device=DEV, seed=3)
+    lam = inputs.decay_lambdas(H, DEV)
+    la2.last_device_error()  # clear
+    for bad in ([0, 400, 200, 600], [0, 300, 900]):
+        cu = torch.tensor(bad, dtype=torch.int64, device=DEV)
+        la2.forward_varlen(x["q"][0], x["k"][0], x["v"][0], lam, cu)
+        torch.cuda.synchronize()
+        assert la2.last_device_error() == 1  # LA2_ERR_INVALID
+    assert la2.last_device_error() == 0
