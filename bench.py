@@ -512,6 +512,81 @@ def run_long(args, world, rank, local):
                     "hbm_frac_fwd_min": round(1024 * Hh * value / world / 1e9 / pk["hbm_gbs"], 4)})
 
 
+def varlen_lengths(total, seed=0, lo=64, hi=8192):
+    """Document lengths of a packed training batch: log-uniform in [lo, hi]
+    rows, drawn from a seeded generator until `total` rows are filled (the
+    last one cut to fit)."""
+    rng = np.random.default_rng(seed)
+    lens = []
+    while sum(lens) < total:
+        n = int(round(float(np.exp(rng.uniform(np.log(lo), np.log(hi))))))
+        lens.append(min(n, total - sum(lens)))
+    return lens
+
+
+def run_varlen(args, world, rank, local):
+    """Packed variable-length batch, 65,536 rows per head slab, H=32,
+    d=e=128, bf16, fwd+bwd (secondary workload)."""
+    import causal_linear_attention_fwd_b200 as la2
+    from causal_linear_attention_fwd_b200 import inputs
+    dev = torch.device("cuda", local)
+    pk = peaks()
+    Hh, T = H, TOKENS
+    lens = varlen_lengths(T, seed=0)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int64, device=dev)
+    x = inputs.make_inputs(1, Hh, T, D, E, dtype=torch.bfloat16, device=dev, seed=0)
+    x = {n: t[0] for n, t in x.items()}
+    lam = inputs.decay_lambdas(Hh, dev)
+    o = torch.empty_like(x["v"])
+    outs = (torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"]))
+
+    def step():
+        la2.forward_varlen(x["q"], x["k"], x["v"], lam, cu, out=o)
+        la2.backward_varlen(x["q"], x["k"], x["v"], lam, cu, x["dO"], outs=outs)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert la2.last_device_error() == 0
+    clocks = ClockSampler(local)
+    la2.profile_enable(True)
+    la2.profile_report()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    prof = la2.profile_report()
+    la2.profile_enable(False)
+    assert la2.last_device_error() == 0
+    ms = max_over_ranks(a.elapsed_time(b), world)
+    value = world * T * args.steps / (ms / 1e3)
+    name, rec = max(prof.items(), key=lambda kv: kv[1]["ms"])
+    avg = rec["ms"] / rec["launches"]
+    alg = 1024 * Hh * T
+    ach = alg / (avg / 1e3) / 1e9
+    roof = {"kernel": name, "bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"],
+            "unit": "GB/s", "frac": round(ach / pk["hbm_gbs"], 4), "traffic": None,
+            "alg_bytes_per_launch": alg, "avg_launch_ms": avg,
+            "note": "traffic not captured for the packed instantiation"}
+    return _common(world, args.steps, args.warmup, value, "tokens/s",
+                   "packed varlen fwd+bwd tokens/s (H=32, d=e=128, bf16)",
+                   {"workload": f"packed variable-length batch, {len(lens)} sequences "
+                                f"(log-uniform 64..8192 rows, seed 0, longest {max(lens)}), "
+                                f"65,536 rows per head, H=32, d=e=128, bf16, fwd+bwd",
+                    "l2": "inputs 512 MiB per tensor, larger than L2; no flush"}, ms,
+                   {"dtype": "bf16", "roofline": roof, "kernels": prof,
+                    "gpu_launches": sum(v["launches"] for v in prof.values()), "clocks": clk,
+                    "sequences": len(lens)})
+
+
 def run_decode(args, world, rank, local):
     """Recurrent decode, batch 256, H=64, d=e=128, fp32 state; one step of
     this workload = `--decode-steps` consecutive decode steps replayed from a
@@ -583,8 +658,10 @@ def main():
     ap.add_argument("--impl", default="la2", choices=["la2", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--workload", default="sweep", choices=["sweep", "long", "decode"],
-                    help="sweep (the metric; default), long (1M-token forward), decode")
+    ap.add_argument("--workload", default="sweep",
+                    choices=["sweep", "long", "decode", "varlen"],
+                    help="sweep (the metric; default), long (1M-token forward), decode, "
+                         "varlen (packed variable-length fwd+bwd)")
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--only", default=None,
                     help="B:L -- time a single sweep point instead of the whole sweep "
@@ -605,7 +682,8 @@ def main():
         return
     world, rank, local = dist_setup(args.gpus)
     try:
-        fn = {"sweep": run_la2, "long": run_long, "decode": run_decode}[args.workload]
+        fn = {"sweep": run_la2, "long": run_long, "decode": run_decode,
+              "varlen": run_varlen}[args.workload]
         line = fn(args, world, rank, local)
         if rank == 0:
             print(json.dumps(line), flush=True)
