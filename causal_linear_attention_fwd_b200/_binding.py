@@ -62,6 +62,11 @@ def library():
         lib.la2_backward_varlen.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, I, I64, I, I,
                                             I, P]
         lib.la2_backward_varlen.restype = I
+        lib.la2_forward_pool.argtypes = [P, P, P, P, P, P, I, P, ctypes.c_uint, I, I, I64, I,
+                                         I, I, P, SZ, P]
+        lib.la2_forward_pool.restype = I
+        lib.la2_decode_tokens.argtypes = [P, P, P, P, P, P, I, P, I, I, I, I, I, I, P]
+        lib.la2_decode_tokens.restype = I
         lib.la2_decode_step.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
         lib.la2_decode_step.restype = I
         lib.la2_last_device_error.argtypes = [P]
@@ -280,6 +285,69 @@ def backward_varlen(q, k, v, lam, cu_seqlens, dO, kv0=None, *, want_dkv0: bool =
                                    _ptr(dkv0), N, H, T, d, e, _dt(q), _stream(stream))
     _check(code, "la2_backward_varlen")
     return (dq, dk, dv, dkv0) if want_dkv0 else (dq, dk, dv)
+
+
+LA2_POOL_CONTINUE = 1
+
+
+def _slots(slots, B):
+    if slots is None:
+        return None
+    _dev(slots, "slots")
+    if slots.dtype != torch.int32 or slots.shape != (B,):
+        raise ValueError("slots must be int32 [B]")
+    return slots
+
+
+def forward_pool(q, k, v, lam, pool, slots, *, continue_state: bool = False, out=None,
+                 workspace=None, stream=None):
+    """Prefill into a state pool [P,H,d,e]: request b starts from zero (or,
+    with continue_state, from pool[slots[b]]) and leaves its final state in
+    pool[slots[b]].  Returns o [B,H,L,e]."""
+    lib = library()
+    for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam), ("pool", pool)):
+        _dev(t, name)
+    B, H, L, d = q.shape
+    e = v.shape[-1]
+    if k.shape != q.shape or v.shape[:3] != (B, H, L):
+        raise ValueError("shape mismatch among q, k, v")
+    if pool.dtype != torch.float32 or pool.dim() != 4 or pool.shape[1:] != (H, d, e):
+        raise ValueError("pool must be float32 [P,H,d,e]")
+    slots = _slots(slots, B)
+    if slots is None:
+        raise ValueError("forward_pool needs a slot table")
+    o = out if out is not None else torch.empty((B, H, L, e), dtype=q.dtype, device=q.device)
+    ws = workspace
+    if ws is None:
+        ws = _workspace(workspace_size(LA2_OP_FORWARD, B, H, L, d, e, q.dtype), q.device)
+    code = lib.la2_forward_pool(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(pool), _ptr(slots),
+                                pool.shape[0], _ptr(o),
+                                LA2_POOL_CONTINUE if continue_state else 0, B, H, L, d, e,
+                                _dt(q), _ptr(ws), 0 if ws is None else ws.numel(),
+                                _stream(stream))
+    _check(code, "la2_forward_pool")
+    return o
+
+
+def decode_tokens(q, k, v, lam, pool, slots=None, *, out=None, stream=None):
+    """T tokens per request at once: q, k [B,H,T,d], v [B,H,T,e]; the state
+    of request b is pool[slots[b]] (pool[b] without a slot table), updated
+    in place; returns o [B,H,T,e]."""
+    lib = library()
+    for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam), ("pool", pool)):
+        _dev(t, name)
+    B, H, T, d = q.shape
+    e = v.shape[-1]
+    if k.shape != q.shape or v.shape[:3] != (B, H, T):
+        raise ValueError("shape mismatch among q, k, v")
+    if pool.dtype != torch.float32 or pool.dim() != 4 or pool.shape[1:] != (H, d, e):
+        raise ValueError("pool must be float32 [P,H,d,e]")
+    slots = _slots(slots, B)
+    o = out if out is not None else torch.empty((B, H, T, e), dtype=q.dtype, device=q.device)
+    code = lib.la2_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(pool), _ptr(slots),
+                                 pool.shape[0], _ptr(o), B, H, T, d, e, _dt(q), _stream(stream))
+    _check(code, "la2_decode_tokens")
+    return o
 
 
 def decode_step(q, k, v, lam, kv, *, out=None, stream=None):

@@ -147,6 +147,8 @@ Path choose_path(int d, int e, la2_dtype dt) {
 Geo plan(int B, int H, int64_t L, int blk, Path path) {
   Geo g;
   g.cu = nullptr;
+  g.slots = nullptr;
+  g.pool = 0;
   g.inject = 0;
   g.variant = g_opt_variant.load();
   g.trace = g_opt_trace.load() - 1;
@@ -291,10 +293,11 @@ cudaError_t simt_backward(const void *q, const void *k, const void *v,
 
 template <typename T, int D, int E>
 cudaError_t decode(const void *q, const void *k, const void *v, const float *lam,
-                   float *kv, void *o, int B, int H, cudaStream_t st) {
+                   float *pool, const int *slots, int pool_size, void *o, int B, int H,
+                   int ntok, cudaStream_t st) {
   return timed(K_DECODE, st, [&] {
     la2::dec::decode_kernel<T, D, E><<<(unsigned)((int64_t)B * H), la2::dec::NT, 0, st>>>(
-        (const T *)q, (const T *)k, (const T *)v, lam, kv, (T *)o, H);
+        (const T *)q, (const T *)k, (const T *)v, lam, pool, slots, pool_size, (T *)o, H, ntok);
   });
 }
 
@@ -478,6 +481,8 @@ Geo plan_varlen(int N, int H, int64_t T, const int64_t *cu) {
   g.nst = 0;
   g.c0 = 0;
   g.cu = cu;
+  g.slots = nullptr;
+  g.pool = 0;
   g.inject = 0;
   g.variant = 0;  // the packed form exists in the warp-specialised kernel only
   g.trace = -1;
@@ -579,6 +584,59 @@ la2_status la2_backward_varlen(const void *q, const void *k, const void *v, cons
   return to_status(err);
 }
 
+la2_status la2_forward_pool(const void *q, const void *k, const void *v, const float *lambda,
+                            float *kv_pool, const int32_t *slots, int pool_size, void *o,
+                            unsigned flags, int B, int H, int64_t L, int d, int e, la2_dtype dt,
+                            void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (flags & ~(unsigned)LA2_POOL_CONTINUE) return LA2_ERR_INVALID;
+  if (B < 0 || H < 0 || L < 1 || pool_size < 0) return LA2_ERR_INVALID;
+  if (dt != LA2_F32 && dt != LA2_BF16) return LA2_ERR_UNSUPPORTED;
+  if (!shape_supported(d, e, dt)) return LA2_ERR_UNSUPPORTED;
+  const int64_t BH = (int64_t)B * H;
+  if (BH == 0) return LA2_OK;
+  if (!q || !k || !v || !lambda || !kv_pool || !slots || !o) return LA2_ERR_INVALID;
+  for (const void *p : std::initializer_list<const void *>{
+           (const void *)q, (const void *)k, (const void *)v, (const void *)lambda,
+           (const void *)kv_pool, (const void *)o, workspace})
+    if (p && !aligned16(p)) return LA2_ERR_INVALID;
+  if (reinterpret_cast<uintptr_t>(slots) % 4 != 0) return LA2_ERR_INVALID;
+  const size_t es = esize(dt);
+  const size_t nq = (size_t)BH * L * d * es, nv = (size_t)BH * L * e * es;
+  std::vector<Span> ins = {{q, nq}, {k, nq}, {v, nv}, {lambda, (size_t)H * 4},
+                           {slots, (size_t)B * 4}};
+  std::vector<Span> outs = {{o, nv},
+                            {kv_pool, (size_t)pool_size * H * d * e * sizeof(float)},
+                            {workspace, workspace_bytes}};
+  std::vector<Span> all = ins;
+  all.insert(all.end(), outs.begin(), outs.end());
+  if (any_overlap(outs, all)) return LA2_ERR_INVALID;
+  Path p = choose_path(d, e, dt);
+  if (p == PATH_NONE) return LA2_ERR_UNSUPPORTED;
+  Geo g = plan(B, H, L, block_rows(p), p);
+  g.slots = slots;
+  g.pool = pool_size;
+  g.variant = 0;  // the slot table exists in the warp-specialised kernel only
+  const size_t need = ws_bytes(LA2_OP_FORWARD, g, d, e);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return LA2_ERR_INVALID;
+  float *ws = (float *)workspace;
+  const float *kv0 = (flags & LA2_POOL_CONTINUE) ? kv_pool : nullptr;
+  cudaError_t err;
+  if (p == PATH_TC) {
+    err = la2::tc::forward(q, k, v, lambda, kv0, o, kv_pool, ws, g, stream,
+                           [&](int which, auto &&fn) {
+                             return timed(which == 0 ? K_TC_FWD_STATE : which == 1 ? K_SCAN_FWD : K_TC_FWD,
+                                          stream, fn);
+                           });
+  } else if (dt == LA2_F32) {
+    err = LA2_DISPATCH_DE(d, e, simt_forward, float, q, k, v, lambda, kv0, o, kv_pool, ws, g,
+                          stream);
+  } else {
+    err = LA2_DISPATCH_DE(d, e, simt_forward, __nv_bfloat16, q, k, v, lambda, kv0, o, kv_pool,
+                          ws, g, stream);
+  }
+  return to_status(err);
+}
+
 la2_status la2_decode_step(const void *q, const void *k, const void *v, const float *lambda,
                            float *kv, void *o, int B, int H, int d, int e, la2_dtype dt,
                            cudaStream_t stream) {
@@ -598,10 +656,43 @@ la2_status la2_decode_step(const void *q, const void *k, const void *v, const fl
   std::vector<Span> all = ins;
   all.insert(all.end(), outs.begin(), outs.end());
   if (any_overlap(outs, all)) return LA2_ERR_INVALID;
-  cudaError_t err = dt == LA2_F32
-                        ? LA2_DISPATCH_DE(d, e, decode, float, q, k, v, lambda, kv, o, B, H, stream)
-                        : LA2_DISPATCH_DE(d, e, decode, __nv_bfloat16, q, k, v, lambda, kv, o, B, H,
-                                          stream);
+  cudaError_t err =
+      dt == LA2_F32
+          ? LA2_DISPATCH_DE(d, e, decode, float, q, k, v, lambda, kv, nullptr, B, o, B, H, 1, stream)
+          : LA2_DISPATCH_DE(d, e, decode, __nv_bfloat16, q, k, v, lambda, kv, nullptr, B, o, B, H,
+                            1, stream);
+  return to_status(err);
+}
+
+la2_status la2_decode_tokens(const void *q, const void *k, const void *v, const float *lambda,
+                             float *kv_pool, const int32_t *slots, int pool_size, void *o,
+                             int B, int H, int T, int d, int e, la2_dtype dt,
+                             cudaStream_t stream) {
+  if (B < 0 || H < 0 || T < 0 || pool_size < 0) return LA2_ERR_INVALID;
+  if (dt != LA2_F32 && dt != LA2_BF16) return LA2_ERR_UNSUPPORTED;
+  if (!shape_supported(d, e, dt)) return LA2_ERR_UNSUPPORTED;
+  const int64_t BH = (int64_t)B * H;
+  if (BH == 0 || T == 0) return LA2_OK;
+  if (!slots && pool_size < B) return LA2_ERR_INVALID;
+  if (!q || !k || !v || !lambda || !kv_pool || !o) return LA2_ERR_INVALID;
+  for (const void *p : std::initializer_list<const void *>{
+           (const void *)q, (const void *)k, (const void *)v, (const void *)lambda,
+           (const void *)kv_pool, (const void *)o})
+    if (!aligned16(p)) return LA2_ERR_INVALID;
+  if (slots && reinterpret_cast<uintptr_t>(slots) % 4 != 0) return LA2_ERR_INVALID;
+  const size_t es = esize(dt);
+  std::vector<Span> ins = {{q, BH * T * d * es}, {k, BH * T * d * es}, {v, BH * T * e * es},
+                           {lambda, (size_t)H * 4}, {slots, slots ? (size_t)B * 4 : 0}};
+  std::vector<Span> outs = {{kv_pool, (size_t)pool_size * H * d * e * sizeof(float)},
+                            {o, BH * T * e * es}};
+  std::vector<Span> all = ins;
+  all.insert(all.end(), outs.begin(), outs.end());
+  if (any_overlap(outs, all)) return LA2_ERR_INVALID;
+  cudaError_t err =
+      dt == LA2_F32 ? LA2_DISPATCH_DE(d, e, decode, float, q, k, v, lambda, kv_pool, slots,
+                                      pool_size, o, B, H, T, stream)
+                    : LA2_DISPATCH_DE(d, e, decode, __nv_bfloat16, q, k, v, lambda, kv_pool, slots,
+                                      pool_size, o, B, H, T, stream);
   return to_status(err);
 }
 

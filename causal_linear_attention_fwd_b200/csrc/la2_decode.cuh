@@ -1,6 +1,8 @@
-// la2_decode.cuh -- one recurrent decode step, HBM-bound.
+// la2_decode.cuh -- recurrent decode steps, HBM-bound.
 //
 //   kv <- lambda kv + k^T v,   o = q kv        (per (b,h), kv fp32 d x e)
+//
+// applied to T consecutive tokens per call (T = 1: one step).
 //
 // The recurrent form with a fixed-size state (Lightning Attention glossary
 // page, section "主な特徴・仕組み").  Each step must read and write the whole
@@ -48,11 +50,18 @@ template <> struct vec_t<2> {
   }
 };
 
+// T tokens per (b,h) in order: the state is read once, updated T times in
+// registers (o_t from the state after token t), and written back once.  The
+// state of request b lives at pool[slot], slot = slots[b] (slots NULL: slot =
+// b); a negative slot marks an inactive request (nothing read or written), a
+// slot >= pool_size is recorded as a bounds error and skipped.  q, k
+// [B,H,T,D], v, o [B,H,T,E]; T = 1 is the single decode step.
 template <typename T, int D, int E>
 __global__ void __launch_bounds__(NT)
 decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
               const T *__restrict__ v, const float *__restrict__ lambda,
-              float *__restrict__ kv, T *__restrict__ o, int H) {
+              float *__restrict__ pool, const int *__restrict__ slots, int pool_size,
+              T *__restrict__ o, int H, int ntok) {
   constexpr int ROWS = D / NW;   // rows per warp
   constexpr int VEC = E / 32;    // columns per lane
   using V = vec_t<VEC>;
@@ -60,46 +69,60 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
   __shared__ float red[NW][E];
 
   const int64_t bh = blockIdx.x;
+  const int64_t b = bh / H;
+  const int h = (int)(bh % H);
   const int tid = threadIdx.x, w = tid / 32, l = tid % 32;
-  if (tid < D) {
-    qs[tid] = io<T>::ld(q + bh * D + tid);
-    ks[tid] = io<T>::ld(k + bh * D + tid);
+  int64_t slot = b;
+  if (slots) {
+    slot = slots[b];
+    if (slot < 0) return;  // inactive request
+    if (slot >= pool_size) {
+      if (tid == 0) raise_error(ERR_BOUNDS);
+      return;
+    }
   }
-  if (tid < E) vs[tid] = io<T>::ld(v + bh * E + tid);
-  const float lam = lambda[bh % H];
-
-  float *base = kv + bh * (int64_t)D * E + (int64_t)(w * ROWS) * E + l * VEC;
+  const float lam = lambda[h];
+  float *base = pool + (slot * H + h) * (int64_t)D * E + (int64_t)(w * ROWS) * E + l * VEC;
   typename V::type x[ROWS];
 #pragma unroll
   for (int r = 0; r < ROWS; r++) x[r] = V::ld(base + (int64_t)r * E);
-  __syncthreads();
 
-  float vv[VEC], acc[VEC];
-#pragma unroll
-  for (int c = 0; c < VEC; c++) {
-    vv[c] = vs[l * VEC + c];
-    acc[c] = 0.f;
-  }
-#pragma unroll
-  for (int r = 0; r < ROWS; r++) {
-    const int i = w * ROWS + r;
-    const float ki = ks[i], qi = qs[i];
+  for (int t = 0; t < ntok; t++) {
+    const int64_t tok = bh * ntok + t;
+    if (tid < D) {
+      qs[tid] = io<T>::ld(q + tok * D + tid);
+      ks[tid] = io<T>::ld(k + tok * D + tid);
+    }
+    if (tid < E) vs[tid] = io<T>::ld(v + tok * E + tid);
+    __syncthreads();  // this token's q, k, v in; the last one's sums read out
+
+    float vv[VEC], acc[VEC];
 #pragma unroll
     for (int c = 0; c < VEC; c++) {
-      float s = fmaf(lam, V::at(x[r], c), ki * vv[c]);
-      V::at(x[r], c) = s;
-      acc[c] = fmaf(qi, s, acc[c]);
+      vv[c] = vs[l * VEC + c];
+      acc[c] = 0.f;
     }
-    V::st(base + (int64_t)r * E, x[r]);
-  }
 #pragma unroll
-  for (int c = 0; c < VEC; c++) red[w][l * VEC + c] = acc[c];
-  __syncthreads();
-  if (tid < E) {
-    float s = 0.f;
+    for (int r = 0; r < ROWS; r++) {
+      const int i = w * ROWS + r;
+      const float ki = ks[i], qi = qs[i];
 #pragma unroll
-    for (int ww = 0; ww < NW; ww++) s += red[ww][tid];
-    io<T>::st(o + bh * E + tid, s);
+      for (int c = 0; c < VEC; c++) {
+        float s = fmaf(lam, V::at(x[r], c), ki * vv[c]);
+        V::at(x[r], c) = s;
+        acc[c] = fmaf(qi, s, acc[c]);
+      }
+      if (t == ntok - 1) V::st(base + (int64_t)r * E, x[r]);
+    }
+#pragma unroll
+    for (int c = 0; c < VEC; c++) red[w][l * VEC + c] = acc[c];
+    __syncthreads();  // every warp's partial sums in
+    if (tid < E) {
+      float sum = 0.f;
+#pragma unroll
+      for (int ww = 0; ww < NW; ww++) sum += red[ww][tid];
+      io<T>::st(o + tok * E + tid, sum);
+    }
   }
 }
 

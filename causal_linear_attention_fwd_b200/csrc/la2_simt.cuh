@@ -48,6 +48,11 @@ struct Geo {
   // n owning rows [cu[n], cu[n+1]) of every head's slab of L rows; tensors
   // are [H, L, d|e], states [N, H, d, e]; S = 1.
   const int64_t *cu;
+  // State pool (NULL otherwise): the initial / final state of (b,h) is
+  // pool state slots[b] * H + h of the kv0 / kv_out arrays, [pool, H, d, e];
+  // a negative slot means none (zero initial state, final state dropped).
+  const int *slots;
+  int pool;
   int inject;   // test hook: CTA 0 of a tensor-core pass withholds one MMA
                 // completion signal so that its bounded wait runs out
   int variant;  // tensor-core kernel form (0: warp-specialised, 1: phase-serial)
@@ -83,6 +88,20 @@ __device__ __forceinline__ Span span_of(const Geo &g, int nch, int c_first) {
     s.b = g.L < s.a + g.Lc ? g.L : s.a + g.Lc;
   }
   return s;
+}
+
+// Index of (b,h)'s state in the kv0 / kv_out arrays: bh itself, or through
+// the state pool's slot table; -1 for none.  A slot past the pool is a
+// bounds error and treated as none.
+__device__ __forceinline__ int64_t state_slot(const Geo &g, int64_t bh) {
+  if (!g.slots) return bh;
+  const int64_t s = g.slots[bh / g.H];
+  if (s < 0) return -1;
+  if (s >= g.pool) {
+    raise_error(ERR_BOUNDS);
+    return -1;
+  }
+  return s * g.H + bh % g.H;
 }
 
 // Geometry of a chunk-state pre-pass and its scan: the (sub-)chunk split,
@@ -143,9 +162,10 @@ fwd_kernel(const T *__restrict__ q, const T *__restrict__ k,
 
   fill_pow(pw, lambda[h]);
   const float *init = nullptr;
+  const int64_t so = state_slot(g, bh);
   if (OUT) {
-    if (c == 0) init = kv0 ? kv0 + bh * D * E : nullptr;
-    else init = ws + (bh * g.S + c) * (int64_t)D * E;
+    if (g.S > 1) init = ws + (bh * g.S + c) * (int64_t)D * E;
+    else init = (kv0 && so >= 0) ? kv0 + so * D * E : nullptr;
   }
   for (int idx = threadIdx.x; idx < D * E; idx += NT)
     KV[(idx / E) * LDS + idx % E] = init ? init[idx] : 0.f;
@@ -194,7 +214,7 @@ fwd_kernel(const T *__restrict__ q, const T *__restrict__ k,
     __syncthreads();
   }
   float *dst = nullptr;
-  if (OUT) dst = (kv_out && c == g.S - 1) ? kv_out + bh * D * E : nullptr;
+  if (OUT) dst = (kv_out && c == g.S - 1 && so >= 0) ? kv_out + so * D * E : nullptr;
   else dst = ws + (bh * g.S + c + 1) * (int64_t)D * E;
   if (dst)
     for (int idx = threadIdx.x; idx < D * E; idx += NT)
@@ -211,10 +231,14 @@ scan_fwd_kernel(float *__restrict__ ws, const float *__restrict__ kv0,
   const int idx = blockIdx.x * NT + threadIdx.x;
   if (idx >= D * E) return;
   const float decay = (float)pow_int((double)lambda[bh % g.H], g.Lc);
-  float run = kv0 ? kv0[bh * D * E + idx] : 0.f;
+  const int64_t so = state_slot(g, bh);
+  float run = (kv0 && so >= 0) ? kv0[so * D * E + idx] : 0.f;
   // slot c holds the contribution of (sub-)chunk c-1, c = 1..nst (all full);
   // eight slots' loads are issued before the running sum walks them
   float *base = ws + bh * g.wsS * (int64_t)D * E + idx;
+  // slot 0 takes the initial state itself: the split passes read every
+  // chunk's entry state here, never kv0, so kv_out may be kv0's storage
+  base[0] = run;
   for (int c0 = 1; c0 <= g.nst; c0 += 8) {
     float v[8];
 #pragma unroll
@@ -249,8 +273,8 @@ dq_kernel(const T *__restrict__ k, const T *__restrict__ v,
   const int64_t bh = sp.bh, a = sp.a, b = sp.b, slab = sp.slab;
   const int c = sp.c, h = sp.h;
   fill_pow(pw, lambda[h]);
-  const float *init = c == 0 ? (kv0 ? kv0 + bh * D * E : nullptr)
-                             : ws + (bh * g.S + c) * (int64_t)D * E;
+  const float *init = g.S > 1 ? ws + (bh * g.S + c) * (int64_t)D * E
+                              : (kv0 ? kv0 + bh * D * E : nullptr);
   for (int idx = threadIdx.x; idx < D * E; idx += NT)
     KV[(idx / E) * LDS + idx % E] = init ? init[idx] : 0.f;
   __syncthreads();

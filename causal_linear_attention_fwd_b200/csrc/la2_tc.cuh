@@ -211,8 +211,14 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
   {
     const float *init = nullptr;
     if (MODE == MODE_FWD || MODE == MODE_DQ) {
-      if (c == 0) init = kv0 ? kv0 + bh * 128 * 128 : nullptr;
-      else init = ws + (bh * g.wsS + (int64_t)c * g.M) * (int64_t)128 * 128;
+      // a split pass reads every chunk's entry state from the workspace (the
+      // scan put the initial one in slot 0), never kv0, which kv_out may reuse
+      if (g.S > 1) {
+        init = ws + (bh * g.wsS + (int64_t)c * g.M) * (int64_t)128 * 128;
+      } else {
+        const int64_t so = state_slot(g, bh);
+        init = (kv0 && so >= 0) ? kv0 + so * 128 * 128 : nullptr;
+      }
     } else if (MODE == MODE_DV || MODE == MODE_DK) {
       if (c != g.S - 1) init = ws + (bh * g.wsS + (int64_t)(c + 1) * g.M - 1) * (int64_t)128 * 128;
     }
@@ -406,7 +412,10 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
     // final state of the chunk
     float *dst = nullptr;
     float scale = 1.f;
-    if (MODE == MODE_FWD) dst = (kv_out && c == g.S - 1) ? kv_out + bh * 128 * 128 : nullptr;
+    if (MODE == MODE_FWD) {
+      const int64_t so = state_slot(g, bh);
+      dst = (kv_out && c == g.S - 1 && so >= 0) ? kv_out + so * 128 * 128 : nullptr;
+    }
     if (MODE == MODE_STATE) dst = ws + (bh * g.wsS + c + 1) * (int64_t)128 * 128;
     if (MODE == MODE_RSTATE) dst = ws + (bh * g.wsS + c - 1) * (int64_t)128 * 128;
     if (MODE == MODE_DV && c == 0 && kv_out) {  // dkv0 = lambda * D(0)
@@ -896,8 +905,14 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
     {
       const float *init = nullptr;
       if (MODE == MODE_FWD || MODE == MODE_DQ) {
-        if (c == 0) init = kv0 ? kv0 + bh * 128 * 128 : nullptr;
-        else init = ws + (bh * g.wsS + (int64_t)c * g.M) * (int64_t)128 * 128;
+        // a split pass reads every chunk's entry state from the workspace (the
+        // scan put the initial one in slot 0), never kv0, which kv_out may reuse
+        if (g.S > 1) {
+          init = ws + (bh * g.wsS + (int64_t)c * g.M) * (int64_t)128 * 128;
+        } else {
+          const int64_t so = state_slot(g, bh);
+          init = (kv0 && so >= 0) ? kv0 + so * 128 * 128 : nullptr;
+        }
       } else if (MODE == MODE_DV || MODE == MODE_DK) {
         if (c != g.S - 1) init = ws + (bh * g.wsS + (int64_t)(c + 1) * g.M - 1) * (int64_t)128 * 128;
       }
@@ -930,7 +945,10 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
     }
     float *dst = nullptr;
     float dscale = 1.f;
-    if (MODE == MODE_FWD) dst = (kv_out && c == g.S - 1) ? kv_out + bh * 128 * 128 : nullptr;
+    if (MODE == MODE_FWD) {
+      const int64_t so = state_slot(g, bh);
+      dst = (kv_out && c == g.S - 1 && so >= 0) ? kv_out + so * 128 * 128 : nullptr;
+    }
     if (MODE == MODE_STATE) dst = ws + (bh * g.wsS + c + 1) * (int64_t)128 * 128;
     if (MODE == MODE_RSTATE) dst = ws + (bh * g.wsS + c - 1) * (int64_t)128 * 128;
     if (MODE == MODE_DV && c == 0 && kv_out) {  // dkv0 = lambda * D(0)

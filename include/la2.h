@@ -216,6 +216,52 @@ la2_status la2_decode_step(const void *q, const void *k, const void *v,
                            cudaStream_t stream);
 
 /*
+ * State pool for serving: the recurrent states of many requests live in one
+ * fp32 array kv_pool [pool_size, H, d, e]; request b of a call uses state
+ * slots[b] (device int32 [B], 4-byte aligned).  A negative slot marks an
+ * inactive request: its state is neither read nor written (and decode
+ * leaves its outputs untouched).  A slot >= pool_size is not checked on the
+ * host (that would synchronise): the kernel skips that request and sets the
+ * bounds bit of the device error word (la2_last_device_error ->
+ * LA2_ERR_INVALID).  Two active requests of one call sharing a slot race:
+ * the caller keeps the active slots of a call distinct.
+ *
+ * la2_forward_pool: prefill straight into the pool.  As la2_forward for q,
+ * k, v [B,H,L,d|e] (L >= 1), o [B,H,L,e] and the workspace (sized by
+ * la2_workspace_size(LA2_OP_FORWARD, ...)), with the initial state zero, or
+ * with flags = LA2_POOL_CONTINUE the slot's current state (a chunked
+ * prefill continuing a request, or several tokens decoded at once through
+ * the block schedule); the final state is written back to the slot.  Reading
+ * and writing one slot in one call is safe: a split sequence reads its
+ * entry states from the workspace, never from the pool.
+ *
+ * la2_decode_tokens: T >= 0 new tokens per request at once, q, k [B,H,T,d],
+ * v, o [B,H,T,e]: for t = 0..T-1, kv <- lambda kv + k_t^T v_t, o_t = q_t kv
+ * (the la2_decode_step recurrence applied T times), reading and writing the
+ * slot's state once per call instead of once per token.  slots may be NULL:
+ * request b then uses state b (pool_size >= B).  la2_decode_step is this
+ * with T = 1, slots NULL.
+ *
+ * Errors as for la2_forward / la2_decode_step (LA2_ERR_INVALID also for
+ * unknown flag bits, L < 1 in la2_forward_pool, a NULL slot table in
+ * la2_forward_pool).  The pages describe the recurrent form and the hand-off
+ * from the parallel (training / prefill) form only in words; the pool, its
+ * slot table and the multi-token call are this library's serving interface.
+ * Source: glossary page, section "主な特徴・仕組み" (parallel form for
+ * training, recurrent form with a constant-size state for inference).
+ */
+enum { LA2_POOL_CONTINUE = 1 };
+la2_status la2_forward_pool(const void *q, const void *k, const void *v,
+                            const float *lambda, float *kv_pool, const int32_t *slots,
+                            int pool_size, void *o, unsigned flags,
+                            int B, int H, int64_t L, int d, int e, la2_dtype dt,
+                            void *workspace, size_t workspace_bytes, cudaStream_t stream);
+la2_status la2_decode_tokens(const void *q, const void *k, const void *v,
+                             const float *lambda, float *kv_pool, const int32_t *slots,
+                             int pool_size, void *o, int B, int H, int T, int d, int e,
+                             la2_dtype dt, cudaStream_t stream);
+
+/*
  * Synchronises `stream`, then reports and clears the device error word that
  * the kernels set: LA2_ERR_TIMEOUT when a bounded wait gave up,
  * LA2_ERR_INVALID when a kernel met out-of-range data it could not use (a

@@ -138,6 +138,36 @@ def test_varlen_validation(lib):
     assert bwdv(N=0) == OK
 
 
+def test_pool_validation(lib):
+    INV, UNS, OK = B.LA2_ERR_INVALID, B.LA2_ERR_UNSUPPORTED, B.LA2_OK
+    SL = CU  # a fake slot table address
+
+    def fwdp(q=Q, k=K, v=V, lam=LAM, pool=KV0, slots=SL, P=8, o=O, flags=0, Bn=2, H=2, L=100,
+             d=64, e=64, dt=B.LA2_BF16, ws=None, wsb=0):
+        return lib.la2_forward_pool(q, k, v, lam, pool, slots, P, o, flags, Bn, H, L, d, e, dt,
+                                    ws, wsb, None)
+
+    def dect(q=Q, k=K, v=V, lam=LAM, pool=KV0, slots=SL, P=8, o=O, Bn=2, H=2, T=4, d=64, e=64,
+             dt=B.LA2_BF16):
+        return lib.la2_decode_tokens(q, k, v, lam, pool, slots, P, o, Bn, H, T, d, e, dt, None)
+
+    assert fwdp(flags=2) == INV                      # unknown flag bit
+    assert fwdp(L=0) == INV                          # a prefill has at least one row
+    assert fwdp(slots=None) == INV
+    assert fwdp(slots=SL + 2) == INV                 # slot table not 4-byte aligned
+    assert fwdp(pool=None) == INV
+    assert fwdp(o=KV0 + 64) == INV                   # o inside the pool
+    assert fwdp(P=-1) == INV
+    assert fwdp(d=96) == UNS
+    assert fwdp(Bn=0) == OK
+    assert dect(T=-1) == INV
+    assert dect(slots=None, P=1) == INV              # no slot table: pool must hold B states
+    assert dect(o=KV0) == INV                        # o overlaps the pool
+    assert dect(q=None) == INV
+    assert dect(e=80) == UNS
+    assert dect(T=0) == OK and dect(Bn=0) == OK
+
+
 def test_workspace_rules(lib):
     # a long sequence with few (b,h) pairs is split, so scratch is needed ...
     need = lib.la2_workspace_size(B.LA2_OP_FORWARD, 1, 2, 1 << 16, 64, 64, B.LA2_BF16)

@@ -1,0 +1,112 @@
+"""GPU parity of the state-pool serving calls against the oracle: multi-token
+decode through a slot table (with inactive requests), prefill straight into
+the pool, and a chunked continuation that reads and writes the same slots
+(also with the sequence split across CTAs)."""
+import numpy as np
+import pytest
+import torch
+
+import causal_linear_attention_fwd_b200 as la2
+from causal_linear_attention_fwd_b200 import inputs
+from gpu_util import check, host
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+PATHS = {"simt": 1, "tc": 2}
+CASES = [("tc", torch.bfloat16, (128, 128)), ("simt", torch.float32, (64, 64))]
+
+
+def tokens(B, H, T, d, e, dtype, seed):
+    """T decode tokens per request, [B,H,T,d|e], from the seeded decode stream."""
+    gen = inputs.DecodeStream(B, H, d, e, dtype=dtype, device=DEV, seed=seed)
+    steps = [gen.next() for _ in range(T)]
+    return tuple(torch.stack([s[i] for s in steps], dim=2).contiguous() for i in range(3))
+
+
+@pytest.mark.parametrize("T", [1, 3, 8])
+@pytest.mark.parametrize("dtype,de", [(torch.bfloat16, (128, 128)), (torch.float32, (64, 64))])
+def test_decode_tokens_matches_oracle(orc, T, dtype, de):
+    d, e = de
+    B, H, P = 6, 3, 10
+    slots_h = [7, -1, 2, 9, 0, 4]
+    pool = inputs.decode_state0(P, H, d, e, device=DEV, seed=4)
+    pool0 = pool.clone()
+    slots = torch.tensor(slots_h, dtype=torch.int32, device=DEV)
+    lam = inputs.fixed_lambdas((1.0, 0.99, 0.5), DEV)
+    q, k, v = tokens(B, H, T, d, e, dtype, seed=T)
+    o = torch.full((B, H, T, e), 7.0, dtype=dtype, device=DEV)
+    la2.decode_tokens(q, k, v, lam, pool, slots, out=o)
+    torch.cuda.synchronize()
+    assert la2.last_device_error() == 0
+    lam_h = lam.double().cpu().numpy()
+    for b, s in enumerate(slots_h):
+        if s < 0:
+            assert bool((o[b] == 7.0).all())  # inactive: outputs untouched
+            continue
+        kv = pool0[s:s + 1].double().cpu().numpy().copy()
+        ref = np.stack([orc.decode_step(host(q[b:b + 1, :, t]), host(k[b:b + 1, :, t]),
+                                        host(v[b:b + 1, :, t]), lam_h, kv)[0]
+                        for t in range(T)], axis=1)
+        check(f"decode T={T} req {b} o", o[b], ref, dtype)
+        check(f"decode T={T} req {b} state", pool[s], kv[0], dtype)
+    untouched = [i for i in range(P) if i not in slots_h]
+    assert torch.equal(pool[untouched], pool0[untouched])
+
+
+@pytest.mark.parametrize("split", [1, 3])
+@pytest.mark.parametrize("path,dtype,de", CASES)
+def test_prefill_decode_continue_matches_forward(orc, path, dtype, de, split):
+    """prefill (L1 rows) into fresh slots, decode T tokens, continue with L2
+    rows in place: every output equals the oracle's forward over the
+    concatenated sequence, and the slot holds its final state."""
+    d, e = de
+    B, H, P, L1, T, L2 = 4, 2, 6, 300, 5, 200
+    slots_h = [3, 0, 5, 1]
+    slots = torch.tensor(slots_h, dtype=torch.int32, device=DEV)
+    lam = inputs.decay_lambdas(H, DEV)
+    x = inputs.make_inputs(B, H, L1 + T + L2, d, e, dtype=dtype, device=DEV, seed=split,
+                           with_dO=False)
+    pool = torch.full((P, H, d, e), 3.0, dtype=torch.float32, device=DEV)  # stale contents
+    cut = lambda t, a, b: t[:, :, a:b].contiguous()
+    old_p = la2.set_option(la2.LA2_OPT_PATH, PATHS[path])
+    old_s = la2.set_option(la2.LA2_OPT_SPLIT, split)
+    try:
+        o1 = la2.forward_pool(cut(x["q"], 0, L1), cut(x["k"], 0, L1), cut(x["v"], 0, L1), lam,
+                              pool, slots)
+        o2 = la2.decode_tokens(cut(x["q"], L1, L1 + T), cut(x["k"], L1, L1 + T),
+                               cut(x["v"], L1, L1 + T), lam, pool, slots)
+        n = L1 + T
+        o3 = la2.forward_pool(cut(x["q"], n, n + L2), cut(x["k"], n, n + L2),
+                              cut(x["v"], n, n + L2), lam, pool, slots, continue_state=True)
+        torch.cuda.synchronize()
+    finally:
+        la2.set_option(la2.LA2_OPT_PATH, old_p)
+        la2.set_option(la2.LA2_OPT_SPLIT, old_s)
+    assert la2.last_device_error() == 0
+    o_ref, st_ref = orc.forward(host(x["q"]), host(x["k"]), host(x["v"]),
+                                lam.double().cpu().numpy(), None, want_state=True)
+    got = torch.cat([o1, o2, o3], dim=2)
+    check(f"{path} S={split} o", got, o_ref, dtype)
+    check(f"{path} S={split} final states", pool[slots_h], st_ref, dtype)
+    assert bool((pool[[2, 4]] == 3.0).all())  # slots no request uses
+
+
+def test_pool_slot_past_end_reported():
+    """A slot >= pool_size: that request is skipped, the device error word
+    reports LA2_ERR_INVALID, nothing faults."""
+    B, H, P = 2, 2, 3
+    pool = torch.zeros((P, H, 128, 128), dtype=torch.float32, device=DEV)
+    slots = torch.tensor([1, 3], dtype=torch.int32, device=DEV)
+    lam = inputs.decay_lambdas(H, DEV)
+    q, k, v = tokens(B, H, 2, 128, 128, torch.bfloat16, seed=1)
+    la2.last_device_error()
+    la2.decode_tokens(q, k, v, lam, pool, slots)
+    torch.cuda.synchronize()
+    assert la2.last_device_error() == 1
+    x = inputs.make_inputs(B, H, 200, 128, 128, dtype=torch.bfloat16, device=DEV, seed=2,
+                           with_dO=False)
+    la2.forward_pool(x["q"], x["k"], x["v"], lam, pool, slots)
+    torch.cuda.synchronize()
+    assert la2.last_device_error() == 1
+    assert la2.last_device_error() == 0
