@@ -589,28 +589,43 @@ def run_varlen(args, world, rank, local):
 
 def run_decode(args, world, rank, local):
     """Recurrent decode, batch 256, H=64, d=e=128, fp32 state; one step of
-    this workload = `--decode-steps` consecutive decode steps replayed from a
-    CUDA graph (secondary workload)."""
+    this workload = `--decode-steps` consecutive tokens per request replayed
+    from a CUDA graph, `--decode-tokens` T of them per call (T = 1: one
+    la2_decode_step per token; T > 1: la2_decode_tokens, the state read and
+    written once per T tokens) (secondary workload)."""
     import causal_linear_attention_fwd_b200 as la2
     from causal_linear_attention_fwd_b200 import inputs
     dev = torch.device("cuda", local)
     pk = peaks()
-    Bn, Hh, n = 256, 64, args.decode_steps
+    Bn, Hh, n, T = 256, 64, args.decode_steps, args.decode_tokens
+    assert n % T == 0, "--decode-steps must be a multiple of --decode-tokens"
+    calls = n // T
     lam = inputs.decay_lambdas(Hh, dev)
     kv = inputs.decode_state0(Bn, Hh, D, E, device=dev, seed=0)
     gen = inputs.DecodeStream(Bn, Hh, D, E, device=dev, seed=0)
     toks = [gen.next() for _ in range(n)]
-    outs = torch.empty((n, Bn, Hh, E), dtype=torch.bfloat16, device=dev)
+    if T > 1:  # [B,H,T,d|e] per call
+        toks = [tuple(torch.stack([toks[c * T + t][i] for t in range(T)], dim=2).contiguous()
+                      for i in range(3)) for c in range(calls)]
+    outs = torch.empty((calls, Bn, Hh, T, E) if T > 1 else (n, Bn, Hh, E), dtype=torch.bfloat16,
+                       device=dev)
+
+    def call(c, stream):
+        if T > 1:
+            la2.decode_tokens(*toks[c], lam, kv, out=outs[c], stream=stream)
+        else:
+            la2.decode_step(*toks[c], lam, kv, out=outs[c], stream=stream)
+
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
-        for t in range(min(n, 8)):  # eager warm-up launches
-            la2.decode_step(*toks[t], lam, kv, out=outs[t], stream=s)
+        for c in range(min(calls, 8)):  # eager warm-up launches
+            call(c, s)
     s.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
-        for t in range(n):
-            la2.decode_step(*toks[t], lam, kv, out=outs[t], stream=s)
+        for c in range(calls):
+            call(c, s)
     for _ in range(args.warmup):
         g.replay()
     torch.cuda.synchronize()
@@ -631,20 +646,22 @@ def run_decode(args, world, rank, local):
     clk = clocks.stop()
     ms = max_over_ranks(a.elapsed_time(b), world)
     value = world * Bn * n * args.steps / (ms / 1e3)
-    per_launch_ms = ms / (n * args.steps)
-    bytes_launch = Bn * Hh * (2 * D * E * 4 + (2 * D + 2 * E) * 2)
+    per_launch_ms = ms / (calls * args.steps)
+    bytes_launch = Bn * Hh * (2 * D * E * 4 + T * (2 * D + 2 * E) * 2)
     ach = bytes_launch / (per_launch_ms / 1e3) / 1e9
     roof = {"kernel": "decode_step", "bound": "hbm", "achieved": round(ach, 1),
             "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(ach / pk["hbm_gbs"], 4),
             "traffic": traffic_for("decode_step", Bn * Hh), "alg_bytes_per_launch": bytes_launch,
             "avg_launch_ms": per_launch_ms,
-            "note": "launch time = graph replay time / launches (1024 launches per replay)"}
+            "note": f"launch time = graph replay time / launches ({calls} launches per replay)"}
+    what = ("one decode step per call" if T == 1 else
+            f"{T} tokens per call (la2_decode_tokens)")
     line = _common(world, args.steps, args.warmup, value, "tokens/s",
                    "decode tokens/s (batch 256, H=64, d=e=128, fp32 state); % of HBM bandwidth",
                    {"workload": f"recurrent decode, batch 256, H=64, d=e=128, fp32 state "
-                                f"(1 GiB), {n} steps per graph replay",
+                                f"(1 GiB), {n} tokens per request per graph replay, {what}",
                     "l2": "state 1 GiB, larger than L2; no flush"}, ms,
-                   {"dtype": "f32", "roofline": roof, "gpu_launches": n * args.steps,
+                   {"dtype": "f32", "roofline": roof, "gpu_launches": calls * args.steps,
                     "clocks": clk})
     del g
     return line
@@ -663,6 +680,8 @@ def main():
                     help="sweep (the metric; default), long (1M-token forward), decode, "
                          "varlen (packed variable-length fwd+bwd)")
     ap.add_argument("--decode-steps", type=int, default=1024)
+    ap.add_argument("--decode-tokens", type=int, default=1,
+                    help="decode workload: tokens per request per call (1 = decode_step)")
     ap.add_argument("--only", default=None,
                     help="B:L -- time a single sweep point instead of the whole sweep "
                          "(profiling aid; not the metric)")
