@@ -56,7 +56,9 @@ template <> struct vec_t<2> {
 // b); a negative slot marks an inactive request (nothing read or written), a
 // slot >= pool_size is recorded as a bounds error and skipped.  q, k
 // [B,H,T,D], v, o [B,H,T,E]; T = 1 is the single decode step.
-template <typename T, int D, int E>
+// G: tokens per group (1 for single-token calls, which then compile to the
+// plain one-token loop; 4 for multi-token calls).
+template <typename T, int D, int E, int G>
 __global__ void __launch_bounds__(NT)
 decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
               const T *__restrict__ v, const float *__restrict__ lambda,
@@ -65,8 +67,10 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
   constexpr int ROWS = D / NW;   // rows per warp
   constexpr int VEC = E / 32;    // columns per lane
   using V = vec_t<VEC>;
-  __shared__ float qs[D], ks[D], vs[E];
-  __shared__ float red[NW][E];
+  // tokens go in groups of G: one load of their q, k, v and one cross-warp
+  // reduction of their outputs per group (two block syncs per G tokens)
+  __shared__ float qs[G][D], ks[G][D], vs[G][E];
+  __shared__ float red[NW][G][E];
 
   const int64_t bh = blockIdx.x;
   const int64_t b = bh / H;
@@ -87,41 +91,49 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
 #pragma unroll
   for (int r = 0; r < ROWS; r++) x[r] = V::ld(base + (int64_t)r * E);
 
-  for (int t = 0; t < ntok; t++) {
-    const int64_t tok = bh * ntok + t;
-    if (tid < D) {
-      qs[tid] = io<T>::ld(q + tok * D + tid);
-      ks[tid] = io<T>::ld(k + tok * D + tid);
+  for (int t0 = 0; t0 < ntok; t0 += G) {
+    const int ng = ntok - t0 < G ? ntok - t0 : G;
+    const int64_t tok0 = bh * ntok + t0;
+    for (int idx = tid; idx < ng * D; idx += NT) {
+      qs[idx / D][idx % D] = io<T>::ld(q + tok0 * D + idx);
+      ks[idx / D][idx % D] = io<T>::ld(k + tok0 * D + idx);
     }
-    if (tid < E) vs[tid] = io<T>::ld(v + tok * E + tid);
-    __syncthreads();  // this token's q, k, v in; the last one's sums read out
+    for (int idx = tid; idx < ng * E; idx += NT) vs[idx / E][idx % E] = io<T>::ld(v + tok0 * E + idx);
+    __syncthreads();  // this group's q, k, v in; the last group's sums read out
 
-    float vv[VEC], acc[VEC];
+    float acc[G][VEC];
 #pragma unroll
-    for (int c = 0; c < VEC; c++) {
-      vv[c] = vs[l * VEC + c];
-      acc[c] = 0.f;
-    }
-#pragma unroll
-    for (int r = 0; r < ROWS; r++) {
-      const int i = w * ROWS + r;
-      const float ki = ks[i], qi = qs[i];
+    for (int g = 0; g < G; g++) {
+      if (g >= ng) break;
+      float vv[VEC];
 #pragma unroll
       for (int c = 0; c < VEC; c++) {
-        float s = fmaf(lam, V::at(x[r], c), ki * vv[c]);
-        V::at(x[r], c) = s;
-        acc[c] = fmaf(qi, s, acc[c]);
+        vv[c] = vs[g][l * VEC + c];
+        acc[g][c] = 0.f;
       }
-      if (t == ntok - 1) V::st(base + (int64_t)r * E, x[r]);
-    }
 #pragma unroll
-    for (int c = 0; c < VEC; c++) red[w][l * VEC + c] = acc[c];
-    __syncthreads();  // every warp's partial sums in
-    if (tid < E) {
+      for (int r = 0; r < ROWS; r++) {
+        const int i = w * ROWS + r;
+        const float ki = ks[g][i], qi = qs[g][i];
+#pragma unroll
+        for (int c = 0; c < VEC; c++) {
+          float sv = fmaf(lam, V::at(x[r], c), ki * vv[c]);
+          V::at(x[r], c) = sv;
+          acc[g][c] = fmaf(qi, sv, acc[g][c]);
+        }
+        // the last token's row goes out as soon as it is final
+        if (t0 + g == ntok - 1) V::st(base + (int64_t)r * E, x[r]);
+      }
+#pragma unroll
+      for (int c = 0; c < VEC; c++) red[w][g][l * VEC + c] = acc[g][c];
+    }
+    __syncthreads();  // every warp's partial sums of the group in
+    for (int idx = tid; idx < ng * E; idx += NT) {
+      const int g = idx / E, j = idx % E;
       float sum = 0.f;
 #pragma unroll
-      for (int ww = 0; ww < NW; ww++) sum += red[ww][tid];
-      io<T>::st(o + tok * E + tid, sum);
+      for (int ww = 0; ww < NW; ww++) sum += red[ww][g][j];
+      io<T>::st(o + (tok0 + g) * E + j, sum);
     }
   }
 }
