@@ -54,9 +54,12 @@ class Oracle:
         self._lib.oracle_forward.argtypes = [i, i, l, i, i, P, P, P, P, P, P, P]
         self._lib.oracle_backward.argtypes = [i, i, l, i, i, P, P, P, P, P, P,
                                               P, P, P, P]
+        self._lib.oracle_backward_end.argtypes = [i, i, l, i, i, P, P, P, P, P, P,
+                                                  P, P, P, P, P]
         self._lib.oracle_decode_step.argtypes = [i, i, i, i, P, P, P, P, P, P]
         self._lib.oracle_num_threads.restype = ctypes.c_int
-        for f in ("oracle_forward", "oracle_backward", "oracle_decode_step"):
+        for f in ("oracle_forward", "oracle_backward", "oracle_backward_end",
+                  "oracle_decode_step"):
             getattr(self._lib, f).restype = None
 
     @staticmethod
@@ -90,8 +93,10 @@ class Oracle:
                                  self._p(o), self._p(st))
         return (o, st) if want_state else o
 
-    def backward(self, q, k, v, lam, dO, kv0=None):
-        """Gradients (dq, dk, dv, dkv0) of sum(o * dO); all fp64."""
+    def backward(self, q, k, v, lam, dO, kv0=None, dstate_end=None):
+        """Gradients (dq, dk, dv, dkv0) of sum(o * dO); all fp64.
+        dstate_end [B,H,d,e]: terminal adjoint G_L (the reverse state flowing
+        in from rows after these; default zero)."""
         q, k, v, dO = self._f32(q), self._f32(k), self._f32(v), self._f32(dO)
         B, H, L, d = q.shape
         e = v.shape[-1]
@@ -102,10 +107,11 @@ class Oracle:
         dk = np.empty((B, H, L, d), np.float64)
         dv = np.empty((B, H, L, e), np.float64)
         dkv0 = np.empty((B, H, d, e), np.float64)
-        self._lib.oracle_backward(B, H, L, d, e, self._p(q), self._p(k),
-                                  self._p(v), self._p(lam), self._p(kv0),
-                                  self._p(dO), self._p(dq), self._p(dk),
-                                  self._p(dv), self._p(dkv0))
+        gend = None if dstate_end is None else self._f64(dstate_end).reshape(B, H, d, e)
+        self._lib.oracle_backward_end(B, H, L, d, e, self._p(q), self._p(k),
+                                      self._p(v), self._p(lam), self._p(kv0),
+                                      self._p(dO), self._p(gend), self._p(dq),
+                                      self._p(dk), self._p(dv), self._p(dkv0))
         return dq, dk, dv, dkv0
 
     def decode_step(self, q, k, v, lam, kv):

@@ -94,11 +94,17 @@ void oracle_forward(int B, int H, long L, int d, int e,
  *
  * The "tiling in both forward and backward" of the Lightning Attention-2 notes
  * page ("Tiling." paragraph) is a faster schedule of exactly these sums.
+ *
+ * oracle_backward_end takes a terminal adjoint G_L = gend [B,H,d,e] (NULL:
+ * zero): the part of the loss that depends on the state after the last
+ * token through tokens that come later (the rows after a shard of a longer
+ * sequence: G_L = sum_{s >= L} lambda^(s-L) q_s^T dO_s).  Same chain rule.
  */
-void oracle_backward(int B, int H, long L, int d, int e,
-                     const float *q, const float *k, const float *v,
-                     const double *lambda, const double *kv0, const float *dO,
-                     double *dq, double *dk, double *dv, double *dkv0)
+void oracle_backward_end(int B, int H, long L, int d, int e,
+                         const float *q, const float *k, const float *v,
+                         const double *lambda, const double *kv0, const float *dO,
+                         const double *gend,
+                         double *dq, double *dk, double *dv, double *dkv0)
 {
     long BH = (long)B * H;
 #pragma omp parallel for schedule(dynamic, 1)
@@ -124,8 +130,9 @@ void oracle_backward(int B, int H, long L, int d, int e,
             }
         }
 
-        /* reverse sweep: G_t = q_t^T dO_t + lambda G_{t+1} */
-        memset(st, 0, sizeof(double) * d * e);
+        /* reverse sweep: G_t = q_t^T dO_t + lambda G_{t+1}, from G_L */
+        if (gend) memcpy(st, gend + bh * d * e, sizeof(double) * d * e);
+        else memset(st, 0, sizeof(double) * d * e);
         for (long t = L - 1; t >= 0; t--) {
             const float *qt = qb + t * d, *kt = kb + t * d, *vt = vb + t * e, *gt = gb + t * e;
             for (int i = 0; i < d; i++)
@@ -146,6 +153,14 @@ void oracle_backward(int B, int H, long L, int d, int e,
             for (int i = 0; i < d * e; i++) dkv0[bh * d * e + i] = lam * st[i];
         free(st);
     }
+}
+
+void oracle_backward(int B, int H, long L, int d, int e,
+                     const float *q, const float *k, const float *v,
+                     const double *lambda, const double *kv0, const float *dO,
+                     double *dq, double *dk, double *dv, double *dkv0)
+{
+    oracle_backward_end(B, H, L, d, e, q, k, v, lambda, kv0, dO, NULL, dq, dk, dv, dkv0);
 }
 
 /*

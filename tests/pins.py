@@ -214,6 +214,51 @@ def pin_adjoint(orc):
         assert abs(val - ref) <= 1e-11 * max(1.0, abs(ref)), (name, val, ref)
 
 
+def pin_backward_terminal_closed_form(orc):
+    """A terminal adjoint G_L (the reverse state flowing in from rows after
+    the sequence) adds to the closed form: G_t gains lam^(L-t) G_L, so
+    dk_t += lam^(L-t) G_L v_t, dv_t += lam^(L-t) k_t G_L, dkv0 += lam^(L+1)
+    G_L; dq does not change."""
+    q, k, v, dO, lam, s0 = small_case(kv0=True)
+    B, H, L, d = q.shape
+    e = v.shape[-1]
+    gend = bf16_exact((B, H, d, e), 17, 0.4).astype(np.float64)
+    got = orc.backward(q, k, v, lam, dO, s0, dstate_end=gend)
+    dq, dk, dv, dkv0 = quadratic_backward(q, k, v, lam, dO, s0)
+    for b in range(B):
+        for h in range(H):
+            w = np.power(float(lam[h]), L - np.arange(L))  # lam^(L-t)
+            G = gend[b, h]
+            dk[b, h] += w[:, None] * (v[b, h].astype(np.float64) @ G.T)
+            dv[b, h] += w[:, None] * (k[b, h].astype(np.float64) @ G)
+            dkv0[b, h] += float(lam[h]) ** (L + 1) * G
+    for name, x, r in zip(("dq", "dk", "dv", "dkv0"), got, (dq, dk, dv, dkv0)):
+        assert_close(x, r, 1e-12, f"{name} with a terminal adjoint vs closed form")
+
+
+def pin_backward_split(orc):
+    """A sequence cut at L1: the second part's backward from the forward state
+    at L1, and the first part's backward with the terminal adjoint sum_{s >=
+    L1} lam^(s-L1) q_s^T dO_s (the plain sum), reproduce the whole backward."""
+    q, k, v, dO, lam, s0 = small_case(L=30, kv0=True)
+    full = orc.backward(q, k, v, lam, dO, s0)
+    L1 = 13
+    _, st1 = orc.forward(q[:, :, :L1], k[:, :, :L1], v[:, :, :L1], lam, s0, want_state=True)
+    part2 = orc.backward(q[:, :, L1:], k[:, :, L1:], v[:, :, L1:], lam, dO[:, :, L1:], st1)
+    B, H, L, d = q.shape
+    e = v.shape[-1]
+    gend = np.zeros((B, H, d, e))
+    for b in range(B):
+        for h in range(H):
+            w = np.power(float(lam[h]), np.arange(L - L1))
+            gend[b, h] = (q[b, h, L1:].astype(np.float64) * w[:, None]).T @ dO[b, h, L1:]
+    part1 = orc.backward(q[:, :, :L1], k[:, :, :L1], v[:, :, :L1], lam, dO[:, :, :L1], s0,
+                         dstate_end=gend)
+    for i, name in enumerate(("dq", "dk", "dv")):
+        assert_close(np.concatenate([part1[i], part2[i]], 2), full[i], 1e-12, f"split {name}")
+    assert_close(part1[3], full[3], 1e-12, "split dkv0")
+
+
 # --------------------------------------------------------------- state pins
 def pin_state_handoff(orc):
     q, k, v, dO, lam, s0 = small_case(L=30, kv0=True)
@@ -258,5 +303,6 @@ def pin_golden(orc):
 
 
 ALL_PINS = [pin_bruteforce, pin_prefix_sum, pin_lambda_zero, pin_length_one,
-            pin_backward_closed_form, pin_finite_difference, pin_adjoint,
+            pin_backward_closed_form, pin_backward_terminal_closed_form, pin_backward_split,
+            pin_finite_difference, pin_adjoint,
             pin_state_handoff, pin_decode_equals_forward, pin_golden]

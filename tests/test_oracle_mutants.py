@@ -42,6 +42,12 @@ MUTANTS = [
     ("backward_dkv0_missing_lambda",
      "dkv0[bh * d * e + i] = lam * st[i];",
      "dkv0[bh * d * e + i] = st[i];"),
+    ("backward_ignores_terminal_adjoint",
+     "if (gend) memcpy(st, gend + bh * d * e, sizeof(double) * d * e);",
+     "if (0) memcpy(st, gend + bh * d * e, sizeof(double) * d * e);"),
+    ("backward_terminal_adjoint_wrong_head",
+     "if (gend) memcpy(st, gend + bh * d * e, sizeof(double) * d * e);",
+     "if (gend) memcpy(st, gend + (bh % H) * d * e, sizeof(double) * d * e);"),
     ("decode_drops_new_token",
      "s[i * e + j] = lam * s[i * e + j] + (double)kt[i] * (double)vt[j];",
      "s[i * e + j] = lam * s[i * e + j] + (double)kt[i] * (double)vt[j] * (double)(lam != lam);"),
