@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(HERE, "libla2.so")
 
 LA2_OK, LA2_ERR_INVALID, LA2_ERR_UNSUPPORTED, LA2_ERR_CUDA, LA2_ERR_TIMEOUT = range(5)
 LA2_F32, LA2_BF16 = 0, 1
-LA2_OP_FORWARD, LA2_OP_BACKWARD = 0, 1
+LA2_OP_FORWARD, LA2_OP_BACKWARD, LA2_OP_SHARD_STATE = 0, 1, 2
 LA2_OPT_SPLIT, LA2_OPT_PATH, LA2_OPT_INJECT_TIMEOUT, LA2_OPT_VARIANT, LA2_OPT_TRACE = 0, 1, 2, 3, 4
 
 _lock = threading.Lock()
@@ -67,6 +67,13 @@ def library():
         lib.la2_forward_pool.restype = I
         lib.la2_decode_tokens.argtypes = [P, P, P, P, P, P, I, P, I, I, I, I, I, I, P]
         lib.la2_decode_tokens.restype = I
+        lib.la2_shard_state.argtypes = [P, P, P, P, I, I, I64, I, I, I, I, P, SZ, P]
+        lib.la2_shard_state.restype = I
+        lib.la2_state_prefix.argtypes = [P, P, P, P, I, I, I, I64, I, I, I, P]
+        lib.la2_state_prefix.restype = I
+        lib.la2_backward_shard.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, I, I64, I, I, I,
+                                           P, SZ, ctypes.c_uint, P]
+        lib.la2_backward_shard.restype = I
         lib.la2_decode_step.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
         lib.la2_decode_step.restype = I
         lib.la2_last_device_error.argtypes = [P]
@@ -348,6 +355,79 @@ def decode_tokens(q, k, v, lam, pool, slots=None, *, out=None, stream=None):
                                  pool.shape[0], _ptr(o), B, H, T, d, e, _dt(q), _stream(stream))
     _check(code, "la2_decode_tokens")
     return o
+
+
+def shard_state(a, b, lam, *, reverse: bool = False, workspace=None, stream=None):
+    """One shard's d x e summary: forward (a = k, b = v) sum_t
+    lam^(L-1-t) k_t^T v_t, reverse (a = q, b = dO) sum_t lam^t q_t^T dO_t;
+    fp32 [B,H,d,e]."""
+    lib = library()
+    for name, t in (("a", a), ("b", b), ("lam", lam)):
+        _dev(t, name)
+    B, H, L, d = a.shape
+    e = b.shape[-1]
+    if b.shape[:3] != (B, H, L):
+        raise ValueError("shape mismatch between a and b")
+    out = torch.empty((B, H, d, e), dtype=torch.float32, device=a.device)
+    ws = workspace
+    if ws is None:
+        ws = _workspace(workspace_size(LA2_OP_SHARD_STATE, B, H, L, d, e, a.dtype), a.device)
+    code = lib.la2_shard_state(_ptr(a), _ptr(b), _ptr(lam), _ptr(out), B, H, L, d, e, _dt(a),
+                               1 if reverse else 0, _ptr(ws), 0 if ws is None else ws.numel(),
+                               _stream(stream))
+    _check(code, "la2_shard_state")
+    return out
+
+
+def state_prefix(delta, lam, L_shard: int, kv0=None, *, reverse: bool = False, stream=None):
+    """Every shard's boundary state from the R shards' deltas [R,B,H,d,e]:
+    forward, the state entering shard r (from kv0); reverse, the reverse
+    state flowing into shard r from the rows after it."""
+    lib = library()
+    for name, t in (("delta", delta), ("lam", lam)):
+        _dev(t, name)
+    if delta.dtype != torch.float32 or delta.dim() != 5:
+        raise ValueError("delta must be float32 [R,B,H,d,e]")
+    R, B, H, d, e = delta.shape
+    if kv0 is not None:
+        _dev(kv0, "kv0")
+    out = torch.empty_like(delta)
+    code = lib.la2_state_prefix(_ptr(delta), _ptr(kv0), _ptr(lam), _ptr(out), R, B, H,
+                                int(L_shard), d, e, 1 if reverse else 0, _stream(stream))
+    _check(code, "la2_state_prefix")
+    return out
+
+
+def backward_shard(q, k, v, lam, dO, kv0=None, dstate_end=None, *, want_dkv0: bool = False,
+                   outs=None, workspace=None, stream=None):
+    """backward() of one shard of a longer sequence: kv0 its entry state,
+    dstate_end the reverse state flowing in from the rows after it."""
+    lib = library()
+    for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam), ("dO", dO)):
+        _dev(t, name)
+    B, H, L, d = q.shape
+    e = v.shape[-1]
+    if k.shape != q.shape or v.shape[:3] != (B, H, L) or dO.shape != v.shape:
+        raise ValueError("shape mismatch among q, k, v, dO")
+    for name, t in (("kv0", kv0), ("dstate_end", dstate_end)):
+        if t is not None:
+            _dev(t, name)
+            if t.dtype != torch.float32 or t.shape != (B, H, d, e):
+                raise ValueError(f"{name} must be float32 [B,H,d,e]")
+    if outs is not None:
+        dq, dk, dv = outs
+    else:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dkv0 = torch.empty((B, H, d, e), dtype=torch.float32, device=q.device) if want_dkv0 else None
+    ws = workspace
+    if ws is None:
+        ws = _workspace(workspace_size(LA2_OP_BACKWARD, B, H, L, d, e, q.dtype), q.device)
+    code = lib.la2_backward_shard(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(dO),
+                                  _ptr(dstate_end), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dkv0),
+                                  B, H, L, d, e, _dt(q), _ptr(ws),
+                                  0 if ws is None else ws.numel(), 0, _stream(stream))
+    _check(code, "la2_backward_shard")
+    return (dq, dk, dv, dkv0) if want_dkv0 else (dq, dk, dv)
 
 
 def decode_step(q, k, v, lam, kv, *, out=None, stream=None):

@@ -14,6 +14,7 @@
 #include "../../include/la2.h"
 #include "la2_common.cuh"
 #include "la2_decode.cuh"
+#include "la2_shard.cuh"
 #include "la2_simt.cuh"
 #include "la2_tc.cuh"
 
@@ -204,6 +205,8 @@ Geo plan(int B, int H, int64_t L, int blk, Path path) {
 int block_rows(Path p) { return p == PATH_TC ? la2::tc::BLOCK : la2::simt::C; }
 
 size_t ws_bytes(int op, const Geo &g, int d, int e) {
+  if (op == LA2_OP_SHARD_STATE)  // one delta per sub-chunk plus one spare slot
+    return (size_t)g.B * g.H * (g.Ssub + 1) * d * e * sizeof(float);
   if (g.S <= 1) return 0;
   size_t one = (size_t)g.B * g.H * g.wsS * d * e * sizeof(float);
   return op == LA2_OP_BACKWARD ? 2 * one : one;
@@ -223,7 +226,7 @@ cudaError_t simt_forward(const void *q, const void *k, const void *v,
     cudaFuncSetAttribute(kst, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fwd_smem<D, E>());
     err = timed(K_SIMT_FWD_STATE, st, [&] {
       kst<<<(unsigned)(BH * (g.S - 1)), NT, fwd_smem<D, E>(), st>>>(
-          Q, K, V, lam, nullptr, nullptr, nullptr, ws, g);
+          Q, K, V, lam, nullptr, nullptr, nullptr, ws, la2::state_geo(g, false));
     });
     if (err) return err;
     err = timed(K_SIMT_FWD_SCAN, st, [&] {
@@ -243,7 +246,8 @@ template <typename T, int D, int E>
 cudaError_t simt_backward(const void *q, const void *k, const void *v,
                           const float *lam, const float *kv0, const void *dO,
                           void *dq, void *dk, void *dv, float *dkv0, float *ws,
-                          const Geo &g, bool reuse_fwd, cudaStream_t st) {
+                          const Geo &g, bool reuse_fwd, cudaStream_t st,
+                          const float *dend = nullptr) {
   using namespace la2::simt;
   const T *Q = (const T *)q, *K = (const T *)k, *V = (const T *)v, *G = (const T *)dO;
   const int64_t BH = (int64_t)g.B * g.H;
@@ -255,7 +259,7 @@ cudaError_t simt_backward(const void *q, const void *k, const void *v,
     cudaFuncSetAttribute(kst, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fwd_smem<D, E>());
     err = timed(K_SIMT_FWD_STATE, st, [&] {
       kst<<<(unsigned)(BH * (g.S - 1)), NT, fwd_smem<D, E>(), st>>>(
-          Q, K, V, lam, nullptr, nullptr, nullptr, wsf, g);
+          Q, K, V, lam, nullptr, nullptr, nullptr, wsf, la2::state_geo(g, false));
     });
     if (err) return err;
     err = timed(K_SIMT_FWD_SCAN, st, [&] {
@@ -268,12 +272,13 @@ cudaError_t simt_backward(const void *q, const void *k, const void *v,
     auto krs = rev_state_kernel<T, D, E>;
     cudaFuncSetAttribute(krs, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rev_smem<D, E>());
     err = timed(K_SIMT_REV_STATE, st, [&] {
-      krs<<<(unsigned)(BH * (g.S - 1)), NT, rev_smem<D, E>(), st>>>(Q, G, lam, wsr, g);
+      krs<<<(unsigned)(BH * (g.S - 1)), NT, rev_smem<D, E>(), st>>>(Q, G, lam, wsr,
+                                                                    la2::state_geo(g, true));
     });
     if (err) return err;
     err = timed(K_SIMT_REV_SCAN, st, [&] {
       scan_rev_kernel<D, E><<<dim3((D * E + NT - 1) / NT, (unsigned)BH), NT, 0, st>>>(
-          wsr, lam, la2::state_geo(g, true));
+          wsr, lam, dend, la2::state_geo(g, true));
     });
     if (err) return err;
   }
@@ -287,7 +292,7 @@ cudaError_t simt_backward(const void *q, const void *k, const void *v,
   cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dkdv_smem<D, E>());
   return timed(K_SIMT_DKDV, st, [&] {
     kk<<<(unsigned)(BH * g.S), NT, dkdv_smem<D, E>(), st>>>(Q, K, V, G, lam, (T *)dk, (T *)dv,
-                                                           dkv0, wsr, g);
+                                                           dkv0, wsr, dend, g);
   });
 }
 
@@ -311,6 +316,49 @@ cudaError_t decode(const void *q, const void *k, const void *v, const float *lam
 la2_status to_status(cudaError_t e) { return e == cudaSuccess ? LA2_OK : LA2_ERR_CUDA; }
 
 }  // namespace
+
+// ------------------------------------------------------- shard helpers
+template <typename T, int D, int E>
+cudaError_t simt_shard_state(const void *a, const void *b, const float *lam, float *ws,
+                             const Geo &gs, bool reverse, cudaStream_t st) {
+  using namespace la2::simt;
+  const int64_t BH = (int64_t)gs.B * gs.H;
+  if (!reverse) {
+    auto kst = fwd_kernel<T, D, E, false>;
+    cudaFuncSetAttribute(kst, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fwd_smem<D, E>());
+    return timed(K_SIMT_FWD_STATE, st, [&] {
+      kst<<<(unsigned)(BH * gs.nst), NT, fwd_smem<D, E>(), st>>>(
+          nullptr, (const T *)a, (const T *)b, lam, nullptr, nullptr, nullptr, ws, gs);
+    });
+  }
+  auto krs = rev_state_kernel<T, D, E>;
+  cudaFuncSetAttribute(krs, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rev_smem<D, E>());
+  return timed(K_SIMT_REV_STATE, st, [&] {
+    krs<<<(unsigned)(BH * gs.nst), NT, rev_smem<D, E>(), st>>>((const T *)a, (const T *)b, lam,
+                                                              ws + (size_t)D * E, gs);
+  });
+}
+
+template <typename T, int D, int E>
+cudaError_t combine(const float *ws, const Geo &gs, const float *lam, bool reverse, float *out,
+                    cudaStream_t st) {
+  const int64_t BH = (int64_t)gs.B * gs.H;
+  la2::shard::combine_kernel<D, E>
+      <<<dim3((D * E + la2::shard::NT - 1) / la2::shard::NT, (unsigned)BH), la2::shard::NT, 0, st>>>(
+          ws, gs.wsS, reverse ? 0 : 1, gs.nst, gs.Lc, gs.L, lam, gs.H, reverse ? 1 : 0, out);
+  return cudaGetLastError();
+}
+
+template <typename T, int D, int E>
+cudaError_t prefix(const float *delta, const float *kv0, const float *lam, int R, int B, int H,
+                   int64_t Ls, bool reverse, float *out, cudaStream_t st) {
+  const int64_t BH = (int64_t)B * H;
+  la2::shard::prefix_kernel<D, E>
+      <<<dim3((D * E + la2::shard::NT - 1) / la2::shard::NT, (unsigned)BH), la2::shard::NT, 0, st>>>(
+          delta, kv0, lam, H, R, BH, Ls, reverse ? 1 : 0, out);
+  return cudaGetLastError();
+}
+
 
 extern "C" {
 
@@ -338,7 +386,7 @@ int la2_set_option(int option, int value) {
 
 size_t la2_workspace_size(int op, int B, int H, int64_t L, int d, int e, la2_dtype dt) {
   if (B <= 0 || H <= 0 || L <= 0 || !shape_supported(d, e, dt)) return 0;
-  if (op != LA2_OP_FORWARD && op != LA2_OP_BACKWARD) return 0;
+  if (op != LA2_OP_FORWARD && op != LA2_OP_BACKWARD && op != LA2_OP_SHARD_STATE) return 0;
   Path p = choose_path(d, e, dt);
   if (p == PATH_NONE) return 0;
   Geo g = plan(B, H, L, block_rows(p), p);
@@ -634,6 +682,142 @@ la2_status la2_forward_pool(const void *q, const void *k, const void *v, const f
   } else {
     err = LA2_DISPATCH_DE(d, e, simt_forward, __nv_bfloat16, q, k, v, lambda, kv0, o, kv_pool,
                           ws, g, stream);
+  }
+  return to_status(err);
+}
+
+// ------------------------------------------------------------ shards
+namespace {
+
+// The chunk-state passes over every sub-chunk of one shard.
+Geo shard_geo(const Geo &g) {
+  Geo s = g;
+  s.S = g.Ssub;
+  s.Lc = g.Ls;
+  s.M = 1;
+  s.nst = g.Ssub;
+  s.c0 = 0;
+  s.wsS = g.Ssub + 1;
+  s.variant = 0;
+  return s;
+}
+
+}  // namespace
+
+la2_status la2_shard_state(const void *a, const void *b, const float *lambda, float *out,
+                           int B, int H, int64_t L, int d, int e, la2_dtype dt, int reverse,
+                           void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (B < 0 || H < 0 || L < 1) return LA2_ERR_INVALID;
+  if (dt != LA2_F32 && dt != LA2_BF16) return LA2_ERR_UNSUPPORTED;
+  if (!shape_supported(d, e, dt)) return LA2_ERR_UNSUPPORTED;
+  const int64_t BH = (int64_t)B * H;
+  if (BH == 0) return LA2_OK;
+  if (!a || !b || !lambda || !out || !workspace) return LA2_ERR_INVALID;
+  for (const void *p : std::initializer_list<const void *>{a, b, (const void *)lambda,
+                                                          (const void *)out, workspace})
+    if (!aligned16(p)) return LA2_ERR_INVALID;
+  const size_t es = esize(dt);
+  std::vector<Span> ins = {{a, (size_t)BH * L * d * es}, {b, (size_t)BH * L * e * es},
+                           {lambda, (size_t)H * 4}};
+  std::vector<Span> outs = {{out, (size_t)BH * d * e * 4}, {workspace, workspace_bytes}};
+  std::vector<Span> all = ins;
+  all.insert(all.end(), outs.begin(), outs.end());
+  if (any_overlap(outs, all)) return LA2_ERR_INVALID;
+  Path p = choose_path(d, e, dt);
+  if (p == PATH_NONE) return LA2_ERR_UNSUPPORTED;
+  const Geo g = plan(B, H, L, block_rows(p), p);
+  if (workspace_bytes < ws_bytes(LA2_OP_SHARD_STATE, g, d, e)) return LA2_ERR_INVALID;
+  const Geo gs = shard_geo(g);
+  float *ws = (float *)workspace;
+  cudaError_t err;
+  if (p == PATH_TC) {
+    err = la2::tc::shard_state(a, b, lambda, ws, gs, reverse != 0, stream,
+                               [&](int which, auto &&fn) {
+                                 return timed(which == 0 ? K_TC_FWD_STATE : K_TC_REV_STATE, stream, fn);
+                               });
+  } else if (dt == LA2_F32) {
+    err = LA2_DISPATCH_DE(d, e, simt_shard_state, float, a, b, lambda, ws, gs, reverse != 0, stream);
+  } else {
+    err = LA2_DISPATCH_DE(d, e, simt_shard_state, __nv_bfloat16, a, b, lambda, ws, gs, reverse != 0,
+                          stream);
+  }
+  if (err == cudaSuccess)
+    err = LA2_DISPATCH_DE(d, e, combine, float, ws, gs, lambda, reverse != 0, out, stream);
+  return to_status(err);
+}
+
+la2_status la2_state_prefix(const float *delta, const float *kv0, const float *lambda,
+                            float *out, int R, int B, int H, int64_t L_shard, int d, int e,
+                            int reverse, cudaStream_t stream) {
+  if (R < 0 || B < 0 || H < 0 || L_shard < 0) return LA2_ERR_INVALID;
+  if (!shape_supported(d, e, LA2_F32)) return LA2_ERR_UNSUPPORTED;
+  const int64_t BH = (int64_t)B * H;
+  if (BH == 0 || R == 0) return LA2_OK;
+  if (!delta || !lambda || !out) return LA2_ERR_INVALID;
+  for (const void *p : std::initializer_list<const void *>{(const void *)delta, (const void *)kv0,
+                                                          (const void *)lambda, (const void *)out})
+    if (p && !aligned16(p)) return LA2_ERR_INVALID;
+  const size_t all_states = (size_t)R * BH * d * e * 4;
+  std::vector<Span> ins = {{delta, all_states}, {kv0, kv0 ? (size_t)BH * d * e * 4 : 0},
+                           {lambda, (size_t)H * 4}};
+  std::vector<Span> outs = {{out, all_states}};
+  std::vector<Span> all = ins;
+  all.insert(all.end(), outs.begin(), outs.end());
+  if (any_overlap(outs, all)) return LA2_ERR_INVALID;
+  return to_status(LA2_DISPATCH_DE(d, e, prefix, float, delta, reverse ? nullptr : kv0, lambda, R,
+                                   B, H, L_shard, reverse != 0, out, stream));
+}
+
+la2_status la2_backward_shard(const void *q, const void *k, const void *v, const float *lambda,
+                              const float *kv0, const void *dO, const float *dstate_end,
+                              void *dq, void *dk, void *dv, float *dkv0, int B, int H,
+                              int64_t L, int d, int e, la2_dtype dt, void *workspace,
+                              size_t workspace_bytes, unsigned flags, cudaStream_t stream) {
+  if (flags & ~(unsigned)LA2_BWD_REUSE_FORWARD_STATES) return LA2_ERR_INVALID;
+  const bool reuse = (flags & LA2_BWD_REUSE_FORWARD_STATES) != 0;
+  if (B < 0 || H < 0 || L < 1) return LA2_ERR_INVALID;
+  if (dt != LA2_F32 && dt != LA2_BF16) return LA2_ERR_UNSUPPORTED;
+  if (!shape_supported(d, e, dt)) return LA2_ERR_UNSUPPORTED;
+  const int64_t BH = (int64_t)B * H;
+  if (BH == 0) return LA2_OK;
+  const size_t es = esize(dt);
+  const size_t nq = (size_t)BH * L * d * es, nv = (size_t)BH * L * e * es;
+  const size_t ns = (size_t)BH * d * e * sizeof(float);
+  if (!lambda || !q || !k || !v || !dO || !dq || !dk || !dv) return LA2_ERR_INVALID;
+  for (const void *p : std::initializer_list<const void *>{
+           (const void *)q, (const void *)k, (const void *)v, (const void *)lambda,
+           (const void *)kv0, (const void *)dO, (const void *)dstate_end, (const void *)dq,
+           (const void *)dk, (const void *)dv, (const void *)dkv0, workspace})
+    if (p && !aligned16(p)) return LA2_ERR_INVALID;
+  std::vector<Span> ins = {{q, nq}, {k, nq}, {v, nv}, {dO, nv}, {lambda, (size_t)H * 4},
+                           {kv0, kv0 ? ns : 0}, {dstate_end, dstate_end ? ns : 0}};
+  std::vector<Span> outs = {{dq, nq}, {dk, nq}, {dv, nv}, {dkv0, dkv0 ? ns : 0},
+                            {workspace, workspace_bytes}};
+  std::vector<Span> all = ins;
+  all.insert(all.end(), outs.begin(), outs.end());
+  if (any_overlap(outs, all)) return LA2_ERR_INVALID;
+  Path p = choose_path(d, e, dt);
+  if (p == PATH_NONE) return LA2_ERR_UNSUPPORTED;
+  Geo g = plan(B, H, L, block_rows(p), p);
+  const size_t need = ws_bytes(LA2_OP_BACKWARD, g, d, e);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return LA2_ERR_INVALID;
+  float *ws = (float *)workspace;
+  cudaError_t err;
+  if (p == PATH_TC) {
+    err = la2::tc::backward(q, k, v, lambda, kv0, dO, dq, dk, dv, dkv0, ws, g, reuse, stream,
+                            [&](int which, auto &&fn) {
+                              static const int ids[] = {K_TC_FWD_STATE, K_SCAN_FWD, K_TC_DQ,
+                                                        K_TC_REV_STATE, K_SCAN_REV, K_TC_DV,
+                                                        K_TC_DK};
+                              return timed(ids[which], stream, fn);
+                            },
+                            dstate_end);
+  } else if (dt == LA2_F32) {
+    err = LA2_DISPATCH_DE(d, e, simt_backward, float, q, k, v, lambda, kv0, dO, dq, dk, dv, dkv0,
+                          ws, g, reuse, stream, dstate_end);
+  } else {
+    err = LA2_DISPATCH_DE(d, e, simt_backward, __nv_bfloat16, q, k, v, lambda, kv0, dO, dq, dk,
+                          dv, dkv0, ws, g, reuse, stream, dstate_end);
   }
   return to_status(err);
 }

@@ -155,8 +155,9 @@ fwd_kernel(const T *__restrict__ q, const T *__restrict__ k,
   float *Ps = Vs + C * LDV;           // C x (C+1)
   float *pw = Ps + C * LDP;           // C+1
 
-  const int nch = OUT ? g.S : g.S - 1;
-  const Span sp = span_of(g, nch, 0);
+  // output pass: one CTA per chunk; state pass: g.nst (sub-)chunks from c0
+  const int nch = OUT ? g.S : g.nst;
+  const Span sp = span_of(g, nch, OUT ? 0 : g.c0);
   const int64_t bh = sp.bh, a = sp.a, b = sp.b, slab = sp.slab;
   const int c = sp.c, h = sp.h;
 
@@ -215,7 +216,7 @@ fwd_kernel(const T *__restrict__ q, const T *__restrict__ k,
   }
   float *dst = nullptr;
   if (OUT) dst = (kv_out && c == g.S - 1 && so >= 0) ? kv_out + so * D * E : nullptr;
-  else dst = ws + (bh * g.S + c + 1) * (int64_t)D * E;
+  else dst = ws + (bh * g.wsS + c + 1) * (int64_t)D * E;
   if (dst)
     for (int idx = threadIdx.x; idx < D * E; idx += NT)
       dst[idx] = KV[(idx / E) * LDS + idx % E];
@@ -334,7 +335,7 @@ rev_state_kernel(const T *__restrict__ q, const T *__restrict__ dO,
   float *Gs = Qs + C * LDQ;      // C x E
   float *pw = Gs + C * LDG;
 
-  const Span sp = span_of(g, g.S - 1, 1);
+  const Span sp = span_of(g, g.nst, g.c0);
   const int64_t bh = sp.bh, a = sp.a, b = sp.b, slab = sp.slab;
   const int c = sp.c, h = sp.h;
   fill_pow(pw, lambda[h]);
@@ -355,7 +356,7 @@ rev_state_kernel(const T *__restrict__ q, const T *__restrict__ dO,
     }
     __syncthreads();
   }
-  float *dst = ws + (bh * g.S + c - 1) * (int64_t)D * E;
+  float *dst = ws + (bh * g.wsS + c - 1) * (int64_t)D * E;
   for (int idx = threadIdx.x; idx < D * E; idx += NT) dst[idx] = Dst[idx];
 }
 
@@ -364,14 +365,16 @@ rev_state_kernel(const T *__restrict__ q, const T *__restrict__ dO,
 // the right (the state at its last row + 1).
 template <int D, int E>
 __global__ void __launch_bounds__(NT)
-scan_rev_kernel(float *__restrict__ ws, const float *__restrict__ lambda, Geo g) {
+scan_rev_kernel(float *__restrict__ ws, const float *__restrict__ lambda,
+                const float *__restrict__ dend, Geo g) {
   const int64_t bh = blockIdx.y;
   const int idx = blockIdx.x * NT + threadIdx.x;
   if (idx >= D * E) return;
   const double lam = (double)lambda[bh % g.H];
   const float full = (float)pow_int(lam, g.Lc);
   const float last = (float)pow_int(lam, g.L - (int64_t)(g.S - 1) * g.Lc);
-  float run = 0.f;
+  // the reverse state past the sequence end (NULL: zero)
+  float run = dend ? dend[bh * D * E + idx] : 0.f;
   // slot c holds the contribution of (sub-)chunk c+1, c+1 = c0..S-1, walked
   // downwards with eight slots' loads in flight
   float *base = ws + bh * g.wsS * (int64_t)D * E + idx;
@@ -397,7 +400,7 @@ dkdv_kernel(const T *__restrict__ q, const T *__restrict__ k,
             const T *__restrict__ v, const T *__restrict__ dO,
             const float *__restrict__ lambda, T *__restrict__ dk,
             T *__restrict__ dv, float *__restrict__ dkv0,
-            const float *__restrict__ ws, Geo g) {
+            const float *__restrict__ ws, const float *__restrict__ dend, Geo g) {
   constexpr int LDQ = D + 1, LDG = E + 1, LDS = E + 1, LDP = C + 1;
   extern __shared__ float sm[];
   float *Dst = sm;                 // D x (E+1)
@@ -413,7 +416,8 @@ dkdv_kernel(const T *__restrict__ q, const T *__restrict__ k,
   const int64_t bh = sp.bh, a = sp.a, b = sp.b, slab = sp.slab;
   const int c = sp.c, h = sp.h;
   fill_pow(pw, lambda[h]);
-  const float *init = c == g.S - 1 ? nullptr : ws + (bh * g.S + c) * (int64_t)D * E;
+  const float *init = c == g.S - 1 ? (dend ? dend + bh * D * E : nullptr)
+                                   : ws + (bh * g.S + c) * (int64_t)D * E;
   for (int idx = threadIdx.x; idx < D * E; idx += NT)
     Dst[(idx / E) * LDS + idx % E] = init ? init[idx] : 0.f;
   __syncthreads();

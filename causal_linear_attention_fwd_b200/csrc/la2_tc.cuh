@@ -221,6 +221,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
       }
     } else if (MODE == MODE_DV || MODE == MODE_DK) {
       if (c != g.S - 1) init = ws + (bh * g.wsS + (int64_t)(c + 1) * g.M - 1) * (int64_t)128 * 128;
+      else init = kv0 ? kv0 + bh * 128 * 128 : nullptr;
     }
     uint8_t *kvbf = smem + LY::KVBF + half * BOX;
 #pragma unroll
@@ -914,7 +915,10 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
           init = (kv0 && so >= 0) ? kv0 + so * 128 * 128 : nullptr;
         }
       } else if (MODE == MODE_DV || MODE == MODE_DK) {
+        // the last chunk starts from the reverse state past the sequence end
+        // (kv0 carries it in the reverse passes; NULL: zero)
         if (c != g.S - 1) init = ws + (bh * g.wsS + (int64_t)(c + 1) * g.M - 1) * (int64_t)128 * 128;
+        else init = kv0 ? kv0 + bh * 128 * 128 : nullptr;
       }
       const float dec = pw[nblk > 0 ? cb_of(0) : 0];
 #pragma unroll
@@ -1176,7 +1180,8 @@ cudaError_t forward(const void *q, const void *k, const void *v, const float *la
 template <typename Timed>
 cudaError_t backward(const void *q, const void *k, const void *v, const float *lam,
                      const float *kv0, const void *dO, void *dq, void *dk, void *dv, float *dkv0,
-                     float *ws, const Geo &g, bool reuse_fwd, cudaStream_t st, Timed &&timed) {
+                     float *ws, const Geo &g, bool reuse_fwd, cudaStream_t st, Timed &&timed,
+                     const float *dend = nullptr) {
   if (!geometry_ok(g)) return cudaErrorInvalidValue;
   const int64_t BH = (int64_t)g.B * g.H;
   CUtensorMap mq, mk, mv, mg, mdq, mdk, mdv;
@@ -1204,13 +1209,31 @@ cudaError_t backward(const void *q, const void *k, const void *v, const float *l
     err = timed(3, [&] { launch_chunk<MODE_RSTATE>(mq, mq, mg, mq, lam, nullptr, wsr, nullptr, gr, st); });
     if (err) return err;
     err = timed(4, [&] {
-      la2::simt::scan_rev_kernel<128, 128><<<sgrid, la2::simt::NT, 0, st>>>(wsr, lam, gr);
+      la2::simt::scan_rev_kernel<128, 128><<<sgrid, la2::simt::NT, 0, st>>>(wsr, lam, dend, gr);
     });
     if (err) return err;
   }
-  err = timed(5, [&] { launch_chunk<MODE_DV>(mk, mq, mg, mdv, lam, nullptr, wsr, dkv0, g, st); });
+  err = timed(5, [&] { launch_chunk<MODE_DV>(mk, mq, mg, mdv, lam, dend, wsr, dkv0, g, st); });
   if (err) return err;
-  return timed(6, [&] { launch_chunk<MODE_DK>(mv, mg, mq, mdk, lam, nullptr, wsr, nullptr, g, st); });
+  return timed(6, [&] { launch_chunk<MODE_DK>(mv, mg, mq, mdk, lam, dend, wsr, nullptr, g, st); });
+}
+
+// Chunk-state pass over every sub-chunk of a shard (a: K or Q, b: V or dO):
+// forward deltas into workspace slots 1..nst, reverse deltas into slots
+// 0..nst-1 (the reverse pass writes slot c-1 for sub-chunk c, so its base is
+// one slot further on).
+template <typename Timed>
+cudaError_t shard_state(const void *a, const void *b, const float *lam, float *ws,
+                        const Geo &gs, bool reverse, cudaStream_t st, Timed &&timed) {
+  if (!geometry_ok(gs)) return cudaErrorInvalidValue;
+  const int64_t BH = (int64_t)gs.B * gs.H;
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, a, BH, gs.L) || !make_map(&mb, b, BH, gs.L)) return cudaErrorInvalidValue;
+  if (!reverse)
+    return timed(0, [&] { launch_chunk<MODE_STATE>(ma, ma, mb, ma, lam, nullptr, ws, nullptr, gs, st); });
+  return timed(3, [&] {
+    launch_chunk<MODE_RSTATE>(ma, ma, mb, ma, lam, nullptr, ws + 128 * 128, nullptr, gs, st);
+  });
 }
 
 // Packed variable-length batch: g.B = N sequences, g.L = T rows per head

@@ -74,12 +74,12 @@ typedef enum {
 typedef enum { LA2_F32 = 0, LA2_BF16 = 1 } la2_dtype;
 
 /* Operation codes for la2_workspace_size(). */
-enum { LA2_OP_FORWARD = 0, LA2_OP_BACKWARD = 1 };
+enum { LA2_OP_FORWARD = 0, LA2_OP_BACKWARD = 1, LA2_OP_SHARD_STATE = 2 };
 
 /*
- * Bytes of device scratch that la2_forward (op = LA2_OP_FORWARD) or
- * la2_backward (op = LA2_OP_BACKWARD) needs for these sizes on the CURRENT
- * device.  The scratch holds the fp32 d x e states at the boundaries of the
+ * Bytes of device scratch that la2_forward (op = LA2_OP_FORWARD),
+ * la2_backward (op = LA2_OP_BACKWARD) or la2_shard_state (op =
+ * LA2_OP_SHARD_STATE) needs for these sizes on the CURRENT device.  The scratch holds the fp32 d x e states at the boundaries of the
  * sequence chunks that run in parallel (the split of one long sequence over
  * several CTAs); it may be 0 when the sequence is not split.  Returns 0 for
  * unsupported arguments as well; the call then reports the error.
@@ -260,6 +260,51 @@ la2_status la2_decode_tokens(const void *q, const void *k, const void *v,
                              const float *lambda, float *kv_pool, const int32_t *slots,
                              int pool_size, void *o, int B, int H, int T, int d, int e,
                              la2_dtype dt, cudaStream_t stream);
+
+/*
+ * Sequence sharding: a sequence of R * L rows cut into R shards of L rows
+ * (one per GPU, in order) needs, per shard, only two d x e summaries of the
+ * other shards -- an exact reassociation of the block recurrence.
+ *
+ * la2_shard_state: one shard's summary, fp32 out [B,H,d,e]: reverse = 0
+ * (a = k [B,H,L,d], b = v [B,H,L,e]) the forward delta sum_t
+ * lambda^(L-1-t) k_t^T v_t (the shard's final state from a zero start);
+ * reverse = 1 (a = q, b = dO) the reverse delta sum_t lambda^t q_t^T dO_t.
+ * Workspace: la2_workspace_size(LA2_OP_SHARD_STATE, ...) bytes (required).
+ *
+ * la2_state_prefix: from the R shards' deltas delta [R,B,H,d,e] (gathered
+ * from every rank), every shard's boundary state, out [R,B,H,d,e]: forward
+ * out[0] = kv0 (NULL: zero), out[r] = lambda^L out[r-1] + delta[r-1] (the
+ * state entering shard r); reverse out[R-1] = 0, out[r] = lambda^L out[r+1]
+ * + delta[r+1] (the reverse state flowing into shard r from the rows after
+ * it; kv0 ignored).  fp32 throughout; d, e as elsewhere.
+ *
+ * la2_backward_shard: la2_backward_ex for one shard, with dstate_end [B,H,d,e]
+ * (NULL: zero) the reverse state flowing in from the rows after it, i.e. its
+ * out[r] of the reverse prefix; kv0 is the shard's entry state (the forward
+ * prefix's out[r]).  Its dq, dk, dv are those rows' slices of the gradients
+ * of the whole sequence; on the first shard dkv0 is the whole sequence's.
+ *
+ * A rank then computes its shard's outputs with la2_forward(kv0 = entry
+ * state) and its gradients with la2_backward_shard, after one all-gather of
+ * the R deltas per direction (the only exchange; see the package's
+ * seqpar module).  Errors as for la2_forward / la2_backward.  The pages do
+ * not discuss sharding a sequence across devices; the reassociation is the
+ * tiling one (Lightning Attention-2 notes page, "Tiling." paragraph) applied
+ * to shards.
+ */
+la2_status la2_shard_state(const void *a, const void *b, const float *lambda, float *out,
+                           int B, int H, int64_t L, int d, int e, la2_dtype dt, int reverse,
+                           void *workspace, size_t workspace_bytes, cudaStream_t stream);
+la2_status la2_state_prefix(const float *delta, const float *kv0, const float *lambda,
+                            float *out, int R, int B, int H, int64_t L_shard, int d, int e,
+                            int reverse, cudaStream_t stream);
+la2_status la2_backward_shard(const void *q, const void *k, const void *v,
+                              const float *lambda, const float *kv0, const void *dO,
+                              const float *dstate_end, void *dq, void *dk, void *dv,
+                              float *dkv0, int B, int H, int64_t L, int d, int e,
+                              la2_dtype dt, void *workspace, size_t workspace_bytes,
+                              unsigned flags, cudaStream_t stream);
 
 /*
  * Synchronises `stream`, then reports and clears the device error word that

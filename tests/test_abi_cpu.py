@@ -168,6 +168,30 @@ def test_pool_validation(lib):
     assert dect(T=0) == OK and dect(Bn=0) == OK
 
 
+def test_shard_validation(lib):
+    INV, UNS, OK = B.LA2_ERR_INVALID, B.LA2_ERR_UNSUPPORTED, B.LA2_OK
+    ss = lambda a=K, b=V, lam=LAM, out=KVO, Bn=1, H=2, L=100, d=64, e=64, rev=0, ws=WS, wsb=MB: \
+        lib.la2_shard_state(a, b, lam, out, Bn, H, L, d, e, B.LA2_BF16, rev, ws, wsb, None)
+    assert ss(L=0) == INV
+    assert ss(ws=None) == INV                        # the workspace is required
+    assert ss(out=K + 256) == INV                    # out overlaps an input
+    assert ss(d=96) == UNS
+    assert ss(wsb=16) == INV                         # workspace too small
+    assert ss(Bn=0) == OK
+    sp = lambda dl=DQ, kv0=None, lam=LAM, out=DK, R=3, Bn=1, H=2, L=100, d=64, e=64, rev=0: \
+        lib.la2_state_prefix(dl, kv0, lam, out, R, Bn, H, L, d, e, rev, None)
+    assert sp(R=-1) == INV
+    assert sp(out=DQ + 16) == INV                    # out overlaps the deltas
+    assert sp(d=96) == UNS
+    assert sp(R=0) == OK
+    bs = lambda flags=0, dend=None, dq=DQ, L=100: lib.la2_backward_shard(
+        Q, K, V, LAM, None, DO, dend, dq, DK, DV, None, 1, 2, L, 64, 64, B.LA2_BF16, None, 0,
+        flags, None)
+    assert bs(flags=2) == INV
+    assert bs(dend=DQ) == INV                        # an output over dstate_end
+    assert bs(L=0) == INV
+
+
 def test_workspace_rules(lib):
     # a long sequence with few (b,h) pairs is split, so scratch is needed ...
     need = lib.la2_workspace_size(B.LA2_OP_FORWARD, 1, 2, 1 << 16, 64, 64, B.LA2_BF16)
