@@ -158,7 +158,11 @@ fwd_kernel(const T *__restrict__ q, const T *__restrict__ k,
   // output pass: one CTA per chunk; state pass: g.nst (sub-)chunks from c0
   const int nch = OUT ? g.S : g.nst;
   const Span sp = span_of(g, nch, OUT ? 0 : g.c0);
-  const int64_t bh = sp.bh, a = sp.a, b = sp.b, slab = sp.slab;
+  const int64_t bh = sp.bh, a = sp.a, slab = sp.slab;
+  // a state-pool request that is inactive (negative slot) or out of the
+  // pool (reported by state_slot): no rows
+  const int64_t b =
+      (OUT && g.slots && (unsigned)g.slots[bh / g.H] >= (unsigned)g.pool) ? a : sp.b;
   const int c = sp.c, h = sp.h;
 
   fill_pow(pw, lambda[h]);

@@ -632,6 +632,9 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
     a = (int64_t)c * g.Lc;
     b = g.L < a + g.Lc ? g.L : a + g.Lc;
     slab = bh;
+    // a state-pool request that is inactive (negative slot) or out of the
+    // pool (reported by state_slot): no rows
+    if (MODE == MODE_FWD && g.slots && (unsigned)g.slots[bh / g.H] >= (unsigned)g.pool) b = a;
   }
   const int nblk = (int)((b - a + BLOCK - 1) / BLOCK);
   auto block_of = [&](int j) { return REV ? nblk - 1 - j : j; };

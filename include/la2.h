@@ -219,10 +219,10 @@ la2_status la2_decode_step(const void *q, const void *k, const void *v,
  * State pool for serving: the recurrent states of many requests live in one
  * fp32 array kv_pool [pool_size, H, d, e]; request b of a call uses state
  * slots[b] (device int32 [B], 4-byte aligned).  A negative slot marks an
- * inactive request: its state is neither read nor written (and decode
- * leaves its outputs untouched).  A slot >= pool_size is not checked on the
- * host (that would synchronise): the kernel skips that request and sets the
- * bounds bit of the device error word (la2_last_device_error ->
+ * inactive request: its state is neither read nor written and its outputs
+ * are left untouched.  A slot >= pool_size is not checked on the host (that
+ * would synchronise): the kernel skips that request the same way and sets
+ * the bounds bit of the device error word (la2_last_device_error ->
  * LA2_ERR_INVALID).  Two active requests of one call sharing a slot race:
  * the caller keeps the active slots of a call distinct.
  *
@@ -239,8 +239,11 @@ la2_status la2_decode_step(const void *q, const void *k, const void *v,
  * v, o [B,H,T,e]: for t = 0..T-1, kv <- lambda kv + k_t^T v_t, o_t = q_t kv
  * (the la2_decode_step recurrence applied T times), reading and writing the
  * slot's state once per call instead of once per token.  slots may be NULL:
- * request b then uses state b (pool_size >= B).  la2_decode_step is this
- * with T = 1, slots NULL.
+ * request b then uses state b (pool_size >= B).  From 32 tokens per request
+ * on (bf16, d = e = 128) the call runs them as one block of the chunk
+ * schedule on the tensor cores (la2_forward_pool's path, one chunk per
+ * request); below that, or for other shapes, token by token in registers.
+ * la2_decode_step is this with T = 1, slots NULL.
  *
  * Errors as for la2_forward / la2_decode_step (LA2_ERR_INVALID also for
  * unknown flag bits, L < 1 in la2_forward_pool, a NULL slot table in

@@ -24,7 +24,7 @@ def tokens(B, H, T, d, e, dtype, seed):
     return tuple(torch.stack([s[i] for s in steps], dim=2).contiguous() for i in range(3))
 
 
-@pytest.mark.parametrize("T", [1, 3, 8])
+@pytest.mark.parametrize("T", [1, 3, 8, 40])
 @pytest.mark.parametrize("dtype,de", [(torch.bfloat16, (128, 128)), (torch.float32, (64, 64))])
 def test_decode_tokens_matches_oracle(orc, T, dtype, de):
     d, e = de
