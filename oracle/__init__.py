@@ -56,10 +56,11 @@ class Oracle:
                                               P, P, P, P]
         self._lib.oracle_backward_end.argtypes = [i, i, l, i, i, P, P, P, P, P, P,
                                                   P, P, P, P, P]
+        self._lib.oracle_dlambda.argtypes = [i, i, l, i, i, P, P, P, P, P, P, P]
         self._lib.oracle_decode_step.argtypes = [i, i, i, i, P, P, P, P, P, P]
         self._lib.oracle_num_threads.restype = ctypes.c_int
         for f in ("oracle_forward", "oracle_backward", "oracle_backward_end",
-                  "oracle_decode_step"):
+                  "oracle_dlambda", "oracle_decode_step"):
             getattr(self._lib, f).restype = None
 
     @staticmethod
@@ -113,6 +114,19 @@ class Oracle:
                                       self._p(dO), self._p(gend), self._p(dq),
                                       self._p(dk), self._p(dv), self._p(dkv0))
         return dq, dk, dv, dkv0
+
+    def dlambda(self, q, k, v, lam, dO, kv0=None):
+        """Gradient of sum(o * dO) with respect to lam [H], summed over the
+        batch (fp64 [H])."""
+        q, k, v, dO = self._f32(q), self._f32(k), self._f32(v), self._f32(dO)
+        B, H, L, d = q.shape
+        e = v.shape[-1]
+        lam = self._f64(lam).reshape(H)
+        kv0 = None if kv0 is None else self._f64(kv0).reshape(B, H, d, e)
+        out = np.empty(H, np.float64)
+        self._lib.oracle_dlambda(B, H, L, d, e, self._p(q), self._p(k), self._p(v),
+                                 self._p(lam), self._p(kv0), self._p(dO), self._p(out))
+        return out
 
     def decode_step(self, q, k, v, lam, kv):
         """One step; kv [B,H,d,e] fp64 is updated IN PLACE; returns o [B,H,e]."""

@@ -192,3 +192,55 @@ void oracle_decode_step(int B, int H, int d, int e,
         }
     }
 }
+
+/*
+ * Gradient of the loss sum(o * dO) with respect to each head's decay
+ * lambda_h, summed over the batch: the chain rule through the recurrence
+ * (the running state of the Lightning Attention-2 notes page, opening
+ * paragraph, with the decay factor).  With kv_t = lambda kv_{t-1} + k_t^T
+ * v_t (kv_{-1} = kv0, a constant) its derivative R_t = d kv_t / d lambda
+ * obeys
+ *   R_t = kv_{t-1} + lambda R_{t-1},   R_{-1} = 0,
+ * and o_t = q_t kv_t gives d o_t / d lambda = q_t R_t, so
+ *   dlambda_h = sum_b sum_t dO_t . (q_t R_t).
+ * dlam [H] double (written, not accumulated).
+ */
+void oracle_dlambda(int B, int H, long L, int d, int e,
+                    const float *q, const float *k, const float *v,
+                    const double *lambda, const double *kv0, const float *dO,
+                    double *dlam)
+{
+    long BH = (long)B * H;
+    double *part = (double *)calloc((size_t)BH, sizeof(double));
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; bh++) {
+        int h = (int)(bh % H);
+        double lam = lambda[h];
+        double *st = (double *)malloc(sizeof(double) * d * e);
+        double *rt = (double *)calloc((size_t)d * e, sizeof(double));
+        const float *qb = q + bh * L * d, *kb = k + bh * L * d, *vb = v + bh * L * e;
+        const float *gb = dO + bh * L * e;
+        if (kv0) memcpy(st, kv0 + bh * d * e, sizeof(double) * d * e);
+        else memset(st, 0, sizeof(double) * d * e);
+        double acc = 0.0;
+        for (long t = 0; t < L; t++) {
+            const float *qt = qb + t * d, *kt = kb + t * d, *vt = vb + t * e, *gt = gb + t * e;
+            for (int i = 0; i < d; i++)
+                for (int j = 0; j < e; j++) {
+                    rt[i * e + j] = st[i * e + j] + lam * rt[i * e + j];   /* uses kv_{t-1} */
+                    st[i * e + j] = lam * st[i * e + j] + (double)kt[i] * (double)vt[j];
+                }
+            for (int j = 0; j < e; j++) {
+                double s = 0.0;
+                for (int i = 0; i < d; i++) s += (double)qt[i] * rt[i * e + j];
+                acc += (double)gt[j] * s;
+            }
+        }
+        part[bh] = acc;
+        free(st);
+        free(rt);
+    }
+    for (int h = 0; h < H; h++) dlam[h] = 0.0;
+    for (long bh = 0; bh < BH; bh++) dlam[bh % H] += part[bh];
+    free(part);
+}

@@ -259,6 +259,46 @@ def pin_backward_split(orc):
     assert_close(part1[3], full[3], 1e-12, "split dkv0")
 
 
+def pin_dlambda_closed_form(orc):
+    """dlambda_h = sum_b sum_t dO_t . [ sum_{j<t} (t-j) lam^(t-j-1) (q_t.k_j) v_j
+    + (t+1) lam^t q_t kv0 ]: the derivative of the quadratic form entry by
+    entry (the diagonal's weight 1 does not depend on lambda); lambda = 0 keeps
+    only the j = t-1 terms and, with kv0, the t = 0 one."""
+    for lams in ((1.0, 0.9, 0.37), (0.0, 0.5, 1.0)):
+        q, k, v, dO, lam, s0 = small_case(lams=lams, kv0=True)
+        got = orc.dlambda(q, k, v, lam, dO, s0)
+        B, H, L, d = q.shape
+        ref = np.zeros(H)
+        n = np.arange(L)[:, None] - np.arange(L)[None, :]
+        for h in range(H):
+            lm = float(lam[h])
+            with np.errstate(divide="ignore", invalid="ignore"):
+                W = np.where(n >= 1, n * np.power(lm, np.maximum(n - 1, 0)), 0.0)
+            a = (np.arange(L) + 1) * np.power(lm, np.arange(L))  # (t+1) lam^t, 0^0 = 1
+            for b in range(B):
+                Q, K, V, G = (x[b, h].astype(np.float64) for x in (q, k, v, dO))
+                ref[h] += np.sum(((Q @ K.T) * W) @ V * G)
+                ref[h] += np.sum(a[:, None] * (Q @ s0[b, h]) * G)
+        assert_close(got, ref, 1e-12, f"dlambda vs closed form {lams}")
+
+
+def pin_dlambda_finite_difference(orc):
+    """sum(o * dO) as a function of one head's lambda: a central difference
+    with step 2^-10 around lambda (a polynomial of degree L in lambda, so the
+    error is O(h^2) times its third derivative)."""
+    q, k, v, dO, lam, s0 = small_case(B=1, H=2, L=9, d=3, e=4, lams=(0.75, 0.5))
+    got = orc.dlambda(q, k, v, lam, dO, s0)
+    h = 2.0 ** -10
+    for i in range(2):
+        lp, lm = lam.copy(), lam.copy()
+        lp[i] += h
+        lm[i] -= h
+        fp = float(np.sum(orc.forward(q, k, v, lp, s0) * dO))
+        fm = float(np.sum(orc.forward(q, k, v, lm, s0) * dO))
+        fd = (fp - fm) / (2 * h)
+        assert abs(fd - got[i]) <= 1e-5 * max(1.0, abs(fd)), (i, fd, got[i])
+
+
 # --------------------------------------------------------------- state pins
 def pin_state_handoff(orc):
     q, k, v, dO, lam, s0 = small_case(L=30, kv0=True)
@@ -304,5 +344,6 @@ def pin_golden(orc):
 
 ALL_PINS = [pin_bruteforce, pin_prefix_sum, pin_lambda_zero, pin_length_one,
             pin_backward_closed_form, pin_backward_terminal_closed_form, pin_backward_split,
+            pin_dlambda_closed_form, pin_dlambda_finite_difference,
             pin_finite_difference, pin_adjoint,
             pin_state_handoff, pin_decode_equals_forward, pin_golden]

@@ -48,6 +48,12 @@ MUTANTS = [
     ("backward_terminal_adjoint_wrong_head",
      "if (gend) memcpy(st, gend + bh * d * e, sizeof(double) * d * e);",
      "if (gend) memcpy(st, gend + (bh % H) * d * e, sizeof(double) * d * e);"),
+    ("dlambda_derivative_missing_decay",
+     "rt[i * e + j] = st[i * e + j] + lam * rt[i * e + j];",
+     "rt[i * e + j] = st[i * e + j] + rt[i * e + j];"),
+    ("dlambda_sign",
+     "part[bh] = acc;",
+     "part[bh] = -acc;"),
     ("decode_drops_new_token",
      "s[i * e + j] = lam * s[i * e + j] + (double)kt[i] * (double)vt[j];",
      "s[i * e + j] = lam * s[i * e + j] + (double)kt[i] * (double)vt[j] * (double)(lam != lam);"),
