@@ -114,15 +114,15 @@ bool overlaps(Span x, Span y) {
   uintptr_t b0 = reinterpret_cast<uintptr_t>(y.p), b1 = b0 + y.n;
   return a0 < b1 && b0 < a1;
 }
-bool any_overlap(const std::vector<Span> &outs, const std::vector<Span> &all) {
-  for (size_t i = 0; i < outs.size(); i++)
-    for (size_t j = 0; j < all.size(); j++)
-      if (outs[i].p != all[j].p || outs[i].n != all[j].n)
-        if (overlaps(outs[i], all[j])) return true;
-  // two outputs at the same address also overlap
-  for (size_t i = 0; i < outs.size(); i++)
+// An output sharing any byte with an input (an exact alias included) or
+// with another output.
+bool any_overlap(const std::vector<Span> &outs, const std::vector<Span> &ins) {
+  for (size_t i = 0; i < outs.size(); i++) {
+    for (size_t j = 0; j < ins.size(); j++)
+      if (overlaps(outs[i], ins[j])) return true;
     for (size_t j = i + 1; j < outs.size(); j++)
       if (overlaps(outs[i], outs[j])) return true;
+  }
   return false;
 }
 
@@ -323,6 +323,24 @@ la2_status to_status(cudaError_t e) { return e == cudaSuccess ? LA2_OK : LA2_ERR
 // 1.8 ms for 32 tokens by the register kernel).
 constexpr int kDecodeBlockTokens = 32;
 
+// ------------------------------------------------------- d lambda helper
+template <typename T, int D, int E>
+cudaError_t simt_dlambda(const void *q, const void *k, const void *v, const void *dO,
+                         const float *lam, const float *kv0, float *dlam, const Geo &g,
+                         cudaStream_t st) {
+  using namespace la2::simt;
+  auto kd = dlambda_kernel<T, D, E>;
+  cudaError_t e = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)dlam_smem<D, E>());
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(dlam, 0, (size_t)g.H * sizeof(float), st);
+  if (e != cudaSuccess) return e;
+  return timed(K_SIMT_DKDV, st, [&] {
+    kd<<<(unsigned)((int64_t)g.B * g.H), NT, dlam_smem<D, E>(), st>>>(
+        (const T *)q, (const T *)k, (const T *)v, (const T *)dO, lam, kv0, dlam, g);
+  });
+}
+
 // ------------------------------------------------------- shard helpers
 template <typename T, int D, int E>
 cudaError_t simt_shard_state(const void *a, const void *b, const float *lam, float *ws,
@@ -418,9 +436,7 @@ la2_status la2_forward(const void *q, const void *k, const void *v,
   if (kv_out && kv_out == kv0) return LA2_ERR_INVALID;
   std::vector<Span> ins = {{q, nq}, {k, nq}, {v, nv}, {lambda, (size_t)H * 4}, {kv0, kv0 ? ns : 0}};
   std::vector<Span> outs = {{o, nv}, {kv_out, kv_out ? ns : 0}, {workspace, workspace_bytes}};
-  std::vector<Span> all = ins;
-  all.insert(all.end(), outs.begin(), outs.end());
-  if (any_overlap(outs, all)) return LA2_ERR_INVALID;
+  if (any_overlap(outs, ins)) return LA2_ERR_INVALID;
 
   if (L == 0) {
     if (!kv_out) return LA2_OK;
@@ -485,9 +501,7 @@ la2_status la2_backward_ex(const void *q, const void *k, const void *v,
                            {kv0, kv0 ? ns : 0}};
   std::vector<Span> outs = {{dq, nq}, {dk, nq}, {dv, nv}, {dkv0, dkv0 ? ns : 0},
                             {workspace, workspace_bytes}};
-  std::vector<Span> all = ins;
-  all.insert(all.end(), outs.begin(), outs.end());
-  if (any_overlap(outs, all)) return LA2_ERR_INVALID;
+  if (any_overlap(outs, ins)) return LA2_ERR_INVALID;
 
   if (L == 0) {
     if (!dkv0) return LA2_OK;
@@ -558,9 +572,7 @@ la2_status check_varlen(int N, int H, int64_t T, int d, int e, la2_dtype dt, con
     if (sp.p && sp.p != (const void *)cu && !aligned16(sp.p)) return LA2_ERR_INVALID;
   for (const Span &sp : outs)
     if (sp.p && !aligned16(sp.p)) return LA2_ERR_INVALID;
-  std::vector<Span> all = ins;
-  all.insert(all.end(), outs.begin(), outs.end());
-  if (any_overlap(outs, all)) return LA2_ERR_INVALID;
+  if (any_overlap(outs, ins)) return LA2_ERR_INVALID;
   return LA2_OK;
 }
 
@@ -662,9 +674,7 @@ la2_status la2_forward_pool(const void *q, const void *k, const void *v, const f
   std::vector<Span> outs = {{o, nv},
                             {kv_pool, (size_t)pool_size * H * d * e * sizeof(float)},
                             {workspace, workspace_bytes}};
-  std::vector<Span> all = ins;
-  all.insert(all.end(), outs.begin(), outs.end());
-  if (any_overlap(outs, all)) return LA2_ERR_INVALID;
+  if (any_overlap(outs, ins)) return LA2_ERR_INVALID;
   Path p = choose_path(d, e, dt);
   if (p == PATH_NONE) return LA2_ERR_UNSUPPORTED;
   Geo g = plan(B, H, L, block_rows(p), p);
@@ -726,9 +736,7 @@ la2_status la2_shard_state(const void *a, const void *b, const float *lambda, fl
   std::vector<Span> ins = {{a, (size_t)BH * L * d * es}, {b, (size_t)BH * L * e * es},
                            {lambda, (size_t)H * 4}};
   std::vector<Span> outs = {{out, (size_t)BH * d * e * 4}, {workspace, workspace_bytes}};
-  std::vector<Span> all = ins;
-  all.insert(all.end(), outs.begin(), outs.end());
-  if (any_overlap(outs, all)) return LA2_ERR_INVALID;
+  if (any_overlap(outs, ins)) return LA2_ERR_INVALID;
   Path p = choose_path(d, e, dt);
   if (p == PATH_NONE) return LA2_ERR_UNSUPPORTED;
   const Geo g = plan(B, H, L, block_rows(p), p);
@@ -767,9 +775,7 @@ la2_status la2_state_prefix(const float *delta, const float *kv0, const float *l
   std::vector<Span> ins = {{delta, all_states}, {kv0, kv0 ? (size_t)BH * d * e * 4 : 0},
                            {lambda, (size_t)H * 4}};
   std::vector<Span> outs = {{out, all_states}};
-  std::vector<Span> all = ins;
-  all.insert(all.end(), outs.begin(), outs.end());
-  if (any_overlap(outs, all)) return LA2_ERR_INVALID;
+  if (any_overlap(outs, ins)) return LA2_ERR_INVALID;
   return to_status(LA2_DISPATCH_DE(d, e, prefix, float, delta, reverse ? nullptr : kv0, lambda, R,
                                    B, H, L_shard, reverse != 0, out, stream));
 }
@@ -799,9 +805,7 @@ la2_status la2_backward_shard(const void *q, const void *k, const void *v, const
                            {kv0, kv0 ? ns : 0}, {dstate_end, dstate_end ? ns : 0}};
   std::vector<Span> outs = {{dq, nq}, {dk, nq}, {dv, nv}, {dkv0, dkv0 ? ns : 0},
                             {workspace, workspace_bytes}};
-  std::vector<Span> all = ins;
-  all.insert(all.end(), outs.begin(), outs.end());
-  if (any_overlap(outs, all)) return LA2_ERR_INVALID;
+  if (any_overlap(outs, ins)) return LA2_ERR_INVALID;
   Path p = choose_path(d, e, dt);
   if (p == PATH_NONE) return LA2_ERR_UNSUPPORTED;
   Geo g = plan(B, H, L, block_rows(p), p);
@@ -828,6 +832,38 @@ la2_status la2_backward_shard(const void *q, const void *k, const void *v, const
   return to_status(err);
 }
 
+la2_status la2_backward_dlambda(const void *q, const void *k, const void *v,
+                                const float *lambda, const float *kv0, const void *dO,
+                                float *dlambda, int B, int H, int64_t L, int d, int e,
+                                la2_dtype dt, cudaStream_t stream) {
+  if (B < 0 || H < 0 || L < 0) return LA2_ERR_INVALID;
+  if (dt != LA2_F32 && dt != LA2_BF16) return LA2_ERR_UNSUPPORTED;
+  if (!shape_supported(d, e, dt)) return LA2_ERR_UNSUPPORTED;
+  const int64_t BH = (int64_t)B * H;
+  if (H == 0) return LA2_OK;
+  if (!lambda || !dlambda || (BH > 0 && L > 0 && (!q || !k || !v || !dO))) return LA2_ERR_INVALID;
+  for (const void *p : std::initializer_list<const void *>{
+           (const void *)q, (const void *)k, (const void *)v, (const void *)lambda,
+           (const void *)kv0, (const void *)dO, (const void *)dlambda})
+    if (p && !aligned16(p)) return LA2_ERR_INVALID;
+  const size_t es = esize(dt);
+  const size_t nq = (size_t)BH * L * d * es, nv = (size_t)BH * L * e * es;
+  std::vector<Span> ins = {{q, nq}, {k, nq}, {v, nv}, {dO, nv}, {lambda, (size_t)H * 4},
+                           {kv0, kv0 ? (size_t)BH * d * e * 4 : 0}};
+  std::vector<Span> outs = {{dlambda, (size_t)H * 4}};
+  if (any_overlap(outs, ins)) return LA2_ERR_INVALID;
+  if (BH == 0 || L == 0) {  // no token depends on lambda
+    return to_status(cudaMemsetAsync(dlambda, 0, (size_t)H * sizeof(float), stream));
+  }
+  Geo g = plan(B, H, L, la2::simt::C, PATH_SIMT);
+  cudaError_t err =
+      dt == LA2_F32
+          ? LA2_DISPATCH_DE(d, e, simt_dlambda, float, q, k, v, dO, lambda, kv0, dlambda, g, stream)
+          : LA2_DISPATCH_DE(d, e, simt_dlambda, __nv_bfloat16, q, k, v, dO, lambda, kv0, dlambda,
+                            g, stream);
+  return to_status(err);
+}
+
 la2_status la2_decode_step(const void *q, const void *k, const void *v, const float *lambda,
                            float *kv, void *o, int B, int H, int d, int e, la2_dtype dt,
                            cudaStream_t stream) {
@@ -844,9 +880,7 @@ la2_status la2_decode_step(const void *q, const void *k, const void *v, const fl
   std::vector<Span> ins = {{q, BH * d * es}, {k, BH * d * es}, {v, BH * e * es},
                            {lambda, (size_t)H * 4}};
   std::vector<Span> outs = {{kv, BH * d * e * sizeof(float)}, {o, BH * e * es}};
-  std::vector<Span> all = ins;
-  all.insert(all.end(), outs.begin(), outs.end());
-  if (any_overlap(outs, all)) return LA2_ERR_INVALID;
+  if (any_overlap(outs, ins)) return LA2_ERR_INVALID;
   cudaError_t err =
       dt == LA2_F32
           ? LA2_DISPATCH_DE(d, e, decode, float, q, k, v, lambda, kv, nullptr, B, o, B, H, 1, stream)
@@ -876,9 +910,7 @@ la2_status la2_decode_tokens(const void *q, const void *k, const void *v, const 
                            {lambda, (size_t)H * 4}, {slots, slots ? (size_t)B * 4 : 0}};
   std::vector<Span> outs = {{kv_pool, (size_t)pool_size * H * d * e * sizeof(float)},
                             {o, BH * T * e * es}};
-  std::vector<Span> all = ins;
-  all.insert(all.end(), outs.begin(), outs.end());
-  if (any_overlap(outs, all)) return LA2_ERR_INVALID;
+  if (any_overlap(outs, ins)) return LA2_ERR_INVALID;
   // From kDecodeBlockTokens tokens per request on, one block of the chunk
   // schedule (tensor cores, the state read and written once) beats the
   // token-by-token register update; the [B,H,T,.] layout is the forward's.

@@ -81,6 +81,8 @@ def test_forward_validation(lib):
     assert fwd(lib, kv0=KV0, kvo=KV0) == INV         # kv_out == kv0
     assert fwd(lib, o=Q + 64) == INV                 # o overlaps q
     assert fwd(lib, kvo=V + 1024) == INV             # kv_out overlaps v
+    assert fwd(lib, o=V) == INV                      # o exactly aliases v (same span)
+    assert fwd(lib, kv0=KV0, kvo=KV0 + 0) == INV
     assert fwd(lib, Bn=0) == B.LA2_OK                # empty batch: nothing to do
     assert fwd(lib, H=0) == B.LA2_OK
 
@@ -91,6 +93,8 @@ def test_backward_validation(lib):
     assert bwd(lib, dq=None) == INV
     assert bwd(lib, dk=DQ) == INV                    # two outputs at one address
     assert bwd(lib, dv=DO) == INV                    # output aliases an input
+    assert bwd(lib, dq=DO) == INV                    # dq exactly aliases dO (d = e)
+    assert bwd(lib, dk=K) == INV                     # dk exactly aliases k
     assert bwd(lib, dkv=DQ + 16) == INV              # dkv0 inside dq
     assert bwd(lib, d=128, e=96) == UNS
     assert bwd(lib, H=-1) == INV
@@ -190,6 +194,18 @@ def test_shard_validation(lib):
     assert bs(flags=2) == INV
     assert bs(dend=DQ) == INV                        # an output over dstate_end
     assert bs(L=0) == INV
+
+
+def test_dlambda_validation(lib):
+    INV, UNS, OK = B.LA2_ERR_INVALID, B.LA2_ERR_UNSUPPORTED, B.LA2_OK
+    f = lambda q=Q, dl=KVO, L=100, d=64, H=2: lib.la2_backward_dlambda(
+        q, K, V, LAM, None, DO, dl, 1, H, L, d, 64, B.LA2_BF16, None)
+    assert f(L=-1) == INV
+    assert f(dl=None) == INV
+    assert f(dl=LAM) == INV                          # output over lambda
+    assert f(q=None) == INV
+    assert f(d=96) == UNS
+    assert f(H=0) == OK
 
 
 def test_workspace_rules(lib):
