@@ -12,7 +12,7 @@ its absence raises an error: there is no CPU fallback.
 from ._binding import (  # noqa: F401
     LA2Error, LA2_OP_BACKWARD, LA2_OP_FORWARD, LA2_OPT_INJECT_TIMEOUT, LA2_OPT_PATH,
     LA2_POOL_CONTINUE, LA2_OP_SHARD_STATE, backward_shard, decode_tokens, forward_pool,
-    shard_state, state_prefix,
+    shard_state, state_prefix, dlambda,
     LA2_OPT_SPLIT, LA2_OPT_TRACE, LA2_OPT_VARIANT, trace_read,
     backward, backward_varlen, decode_step, forward, forward_noalloc, forward_varlen,
     last_device_error, library, profile_enable, profile_report, set_option, status_string,
@@ -20,6 +20,6 @@ from ._binding import (  # noqa: F401
 
 __all__ = ["forward", "forward_noalloc", "backward", "forward_varlen", "backward_varlen",
            "forward_pool", "decode_step", "decode_tokens", "shard_state", "state_prefix",
-           "backward_shard", "workspace_size",
+           "backward_shard", "dlambda", "workspace_size",
            "last_device_error", "set_option", "profile_enable", "profile_report",
            "status_string", "version", "library", "LA2Error"]

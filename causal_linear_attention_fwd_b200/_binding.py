@@ -74,6 +74,8 @@ def library():
         lib.la2_backward_shard.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, I, I64, I, I, I,
                                            P, SZ, ctypes.c_uint, P]
         lib.la2_backward_shard.restype = I
+        lib.la2_backward_dlambda.argtypes = [P, P, P, P, P, P, P, I, I, I64, I, I, I, P]
+        lib.la2_backward_dlambda.restype = I
         lib.la2_decode_step.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
         lib.la2_decode_step.restype = I
         lib.la2_last_device_error.argtypes = [P]
@@ -428,6 +430,25 @@ def backward_shard(q, k, v, lam, dO, kv0=None, dstate_end=None, *, want_dkv0: bo
                                   0 if ws is None else ws.numel(), 0, _stream(stream))
     _check(code, "la2_backward_shard")
     return (dq, dk, dv, dkv0) if want_dkv0 else (dq, dk, dv)
+
+
+def dlambda(q, k, v, lam, dO, kv0=None, *, stream=None):
+    """Gradient of sum(o * dO) with respect to lam [H] (float32 [H], summed
+    over the batch)."""
+    lib = library()
+    for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam), ("dO", dO)):
+        _dev(t, name)
+    B, H, L, d = q.shape
+    e = v.shape[-1]
+    if k.shape != q.shape or v.shape[:3] != (B, H, L) or dO.shape != v.shape:
+        raise ValueError("shape mismatch among q, k, v, dO")
+    if kv0 is not None:
+        _dev(kv0, "kv0")
+    out = torch.empty(H, dtype=torch.float32, device=q.device)
+    code = lib.la2_backward_dlambda(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(dO),
+                                    _ptr(out), B, H, L, d, e, _dt(q), _stream(stream))
+    _check(code, "la2_backward_dlambda")
+    return out
 
 
 def decode_step(q, k, v, lam, kv, *, out=None, stream=None):

@@ -501,5 +501,109 @@ template <int D, int E> constexpr size_t dkdv_smem() {
                           2 * C * (C + 1) + C + 1);
 }
 
+// ------------------------------------------------------------ d lambda
+// Gradient of sum(o * dO) with respect to lambda_h, one CTA per (b,h) over
+// the whole sequence, added into dlam[h].  With the carried states, per
+// block of rows p.. (local t, j):
+//   KV = sum_{j<p} lambda^(p-1-j) k_j^T v_j,
+//   W  = sum_{j<p} (p-1-j) lambda^(p-1-j) k_j^T v_j,
+// the derivative of o_t splits into the block's own pairs
+//   sum_{j<t} (t-j) lambda^(t-j-1) (q_t . k_j) v_j
+// and the earlier rows  lambda^t ((t+1) q_t KV + q_t W)  (with KV = kv0,
+// W = 0 before the first block: d/dlambda of lambda^(t+1) q_t kv0); both
+// are dotted with dO_t.  Then W <- lambda^cb (cb KV + W) + sum_j (cb-1-j)
+// lambda^(cb-1-j) k_j^T v_j and KV <- lambda^cb KV + sum_j lambda^(cb-1-j)
+// k_j^T v_j.  No division by lambda, so lambda = 0 is exact.
+template <int D, int E>
+constexpr size_t dlam_smem() {
+  return sizeof(float) * (2 * D * (E + 1) + 2 * C * (D + 1) + 2 * C * (E + 1) + (C + 1) + NT / 32);
+}
+
+template <typename T, int D, int E>
+__global__ void __launch_bounds__(NT)
+dlambda_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+               const T *__restrict__ dO, const float *__restrict__ lambda,
+               const float *__restrict__ kv0, float *__restrict__ dlam, Geo g) {
+  constexpr int LDS = E + 1, LDQ = D + 1, LDV = E + 1;
+  extern __shared__ float sm[];
+  float *KV = sm;                  // D x (E+1)
+  float *Wst = KV + D * LDS;       // D x (E+1)
+  float *Qs = Wst + D * LDS;       // C x (D+1)
+  float *Ks = Qs + C * LDQ;        // C x (D+1)
+  float *Vs = Ks + C * LDQ;        // C x (E+1)
+  float *Gs = Vs + C * LDV;        // C x (E+1)   dO
+  float *pw = Gs + C * LDV;        // C+1
+  float *red = pw + (C + 1);       // NT/32
+
+  const int64_t bh = blockIdx.x;
+  const int h = (int)(bh % g.H);
+  fill_pow(pw, lambda[h]);
+  for (int idx = threadIdx.x; idx < D * E; idx += NT) {
+    KV[(idx / E) * LDS + idx % E] = kv0 ? kv0[bh * D * E + idx] : 0.f;
+    Wst[(idx / E) * LDS + idx % E] = 0.f;
+  }
+  double acc = 0.0;
+  __syncthreads();
+
+  for (int64_t p = 0; p < g.L; p += C) {
+    const int cb = (int)(g.L - p < C ? g.L - p : C);
+    load_tile<T, D>(Qs, LDQ, q + (bh * g.L + p) * D, cb);
+    load_tile<T, D>(Ks, LDQ, k + (bh * g.L + p) * D, cb);
+    load_tile<T, E>(Vs, LDV, v + (bh * g.L + p) * E, cb);
+    load_tile<T, E>(Gs, LDV, dO + (bh * g.L + p) * E, cb);
+    __syncthreads();
+    // the block's own pairs j < t
+    for (int idx = threadIdx.x; idx < C * C; idx += NT) {
+      const int t = idx / C, j = idx % C;
+      if (j < t && t < cb) {
+        float s = 0.f, gv = 0.f;
+#pragma unroll 8
+        for (int i = 0; i < D; i++) s += Qs[t * LDQ + i] * Ks[j * LDQ + i];
+#pragma unroll 8
+        for (int c = 0; c < E; c++) gv += Gs[t * LDV + c] * Vs[j * LDV + c];
+        acc += (double)((float)(t - j) * pw[t - j - 1] * s * gv);
+      }
+    }
+    // the earlier rows through the carried states
+    for (int idx = threadIdx.x; idx < C * E; idx += NT) {
+      const int t = idx / E, c = idx % E;
+      if (t < cb) {
+        float x = 0.f, y = 0.f;
+#pragma unroll 8
+        for (int i = 0; i < D; i++) {
+          x += Qs[t * LDQ + i] * KV[i * LDS + c];
+          y += Qs[t * LDQ + i] * Wst[i * LDS + c];
+        }
+        acc += (double)(pw[t] * ((float)(t + 1) * x + y) * Gs[t * LDV + c]);
+      }
+    }
+    __syncthreads();
+    // W from the old KV, then KV
+    for (int idx = threadIdx.x; idx < D * E; idx += NT) {
+      const int i = idx / E, c = idx % E;
+      float dkv = 0.f, dw = 0.f;
+      for (int j = 0; j < cb; j++) {
+        const float kvj = pw[cb - 1 - j] * Ks[j * LDQ + i] * Vs[j * LDV + c];
+        dkv += kvj;
+        dw += (float)(cb - 1 - j) * kvj;
+      }
+      const float kv_old = KV[i * LDS + c];
+      Wst[i * LDS + c] = pw[cb] * ((float)cb * kv_old + Wst[i * LDS + c]) + dw;
+      KV[i * LDS + c] = pw[cb] * kv_old + dkv;
+    }
+    __syncthreads();
+  }
+  // block sum, then one atomic add per CTA
+  float a = (float)acc;
+  for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int w = 0; w < NT / 32; w++) t += red[w];
+    atomicAdd(dlam + h, t);
+  }
+}
+
 }  // namespace simt
 }  // namespace la2

@@ -216,6 +216,27 @@ la2_status la2_decode_step(const void *q, const void *k, const void *v,
                            cudaStream_t stream);
 
 /*
+ * Gradient of sum(o * dO) with respect to each head's decay: dlambda fp32
+ * [H] (written), summed over the batch -- for training a learnable decay.
+ * Inputs as for la2_backward (kv0 may be NULL).  Per head
+ *   dlambda_h = sum_b sum_t dO_t . ( sum_{j<t} (t-j) lambda^(t-j-1)
+ *               (q_t . k_j) v_j + (t+1) lambda^t q_t kv0 ),
+ * computed block by block with a second carried state (the position-
+ * weighted sum of k^T v) next to the usual one; exact at lambda = 0.  One
+ * CTA per (b,h) walks the whole sequence on the fp32-FMA path (a
+ * functional path: no chunk split and no tensor cores); the batch sum is
+ * made with atomics, so it is not bitwise reproducible across runs.
+ * Errors as for la2_backward (dlambda overlapping an input:
+ * LA2_ERR_INVALID).  The pages do not treat the decay as learnable; the
+ * derivative is the chain rule through the recurrence of the Lightning
+ * Attention-2 notes page (opening paragraph's running state, with decay).
+ */
+la2_status la2_backward_dlambda(const void *q, const void *k, const void *v,
+                                const float *lambda, const float *kv0, const void *dO,
+                                float *dlambda, int B, int H, int64_t L, int d, int e,
+                                la2_dtype dt, cudaStream_t stream);
+
+/*
  * State pool for serving: the recurrent states of many requests live in one
  * fp32 array kv_pool [pool_size, H, d, e]; request b of a call uses state
  * slots[b] (device int32 [B], 4-byte aligned).  A negative slot marks an

@@ -386,3 +386,19 @@ def test_trace_instantiation_matches():
         s_end, mask_e, p_end, epi_s, oempty = (int(t[e, i]) for e in (1, 4, 2, 5, 6))
         assert 0 < s_end <= mask_e <= p_end, (i, s_end, mask_e, p_end)
         assert p_end <= epi_s <= oempty, (i, p_end, epi_s, oempty)
+
+
+# --------------------------------------------------- gradient w.r.t. lambda
+@pytest.mark.parametrize("dtype,de,L", [(torch.bfloat16, (128, 128), 300),
+                                        (torch.float32, (64, 64), 257),
+                                        (torch.bfloat16, (64, 128), 33)])
+def test_dlambda_matches_oracle(orc, dtype, de, L):
+    d, e = de
+    x = inputs.make_inputs(2, 3, L, d, e, dtype=dtype, device=DEV, seed=L, with_kv0=True)
+    lam = inputs.fixed_lambdas((1.0, 0.9, 0.0), DEV)
+    got = la2.dlambda(x["q"], x["k"], x["v"], lam, x["dO"], x["kv0"])
+    torch.cuda.synchronize()
+    h = {n: host(t) for n, t in x.items()}
+    ref = orc.dlambda(h["q"], h["k"], h["v"], lam.double().cpu().numpy(), h["dO"], h["kv0"])
+    err = np.max(np.abs(got.double().cpu().numpy() - ref))
+    assert err <= 1e-3 * max(float(np.max(np.abs(ref))), 1e-6), (got, ref)
