@@ -512,18 +512,6 @@ def run_long(args, world, rank, local):
                     "hbm_frac_fwd_min": round(1024 * Hh * value / world / 1e9 / pk["hbm_gbs"], 4)})
 
 
-def varlen_lengths(total, seed=0, lo=64, hi=8192):
-    """Document lengths of a packed training batch: log-uniform in [lo, hi]
-    rows, drawn from a seeded generator until `total` rows are filled (the
-    last one cut to fit)."""
-    rng = np.random.default_rng(seed)
-    lens = []
-    while sum(lens) < total:
-        n = int(round(float(np.exp(rng.uniform(np.log(lo), np.log(hi))))))
-        lens.append(min(n, total - sum(lens)))
-    return lens
-
-
 def run_varlen(args, world, rank, local):
     """Packed variable-length batch, 65,536 rows per head slab, H=32,
     d=e=128, bf16, fwd+bwd (secondary workload)."""
@@ -532,7 +520,7 @@ def run_varlen(args, world, rank, local):
     dev = torch.device("cuda", local)
     pk = peaks()
     Hh, T = H, TOKENS
-    lens = varlen_lengths(T, seed=0)
+    lens = inputs.varlen_lengths(T, seed=0)
     cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int64, device=dev)
     x = inputs.make_inputs(1, Hh, T, D, E, dtype=torch.bfloat16, device=dev, seed=0)
     x = {n: t[0] for n, t in x.items()}
@@ -667,6 +655,77 @@ def run_decode(args, world, rank, local):
     return line
 
 
+def run_dlambda(args, world, rank, local):
+    """Gradient with respect to the decay, la2_backward_dlambda, on the
+    B=4, H=16, L=2048 training shape (bf16 inputs, fp32-FMA arithmetic)
+    (secondary workload)."""
+    import causal_linear_attention_fwd_b200 as la2
+    from causal_linear_attention_fwd_b200 import inputs
+    dev = torch.device("cuda", local)
+    Bn, Hh, L = 4, 16, 2048
+    x = inputs.make_inputs(Bn, Hh, L, D, E, dtype=torch.bfloat16, device=dev, seed=0)
+    lam = inputs.decay_lambdas(Hh, dev)
+    ws_n = la2.workspace_size(la2.LA2_OP_DLAMBDA, Bn, Hh, L, D, E, torch.bfloat16)
+    ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        la2.dlambda(x["q"], x["k"], x["v"], lam, x["dO"], workspace=ws)
+    torch.cuda.synchronize()
+    assert la2.last_device_error() == 0
+    clocks = ClockSampler(local)
+    la2.profile_enable(True)
+    la2.profile_report()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        la2.dlambda(x["q"], x["k"], x["v"], lam, x["dO"], workspace=ws)
+    b.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    prof = la2.profile_report()
+    la2.profile_enable(False)
+    assert la2.last_device_error() == 0
+    ms = max_over_ranks(a.elapsed_time(b), world)
+    value = world * Bn * L * args.steps / (ms / 1e3)
+    name, rec = max(prof.items(), key=lambda kv: kv[1]["ms"])
+    avg = rec["ms"] / rec["launches"]
+    # fp32 FMA work of the block schedule per token-head (C = 32 rows): the
+    # state terms q KV and q W, the updates of KV and W (2 d e flops each),
+    # and the block's own pairs, (C-1)/2 of them per row at 2 (d + e) flops
+    fl_th = 8 * D * E + (32 - 1) * (D + E)
+    alg = fl_th * Bn * Hh * L
+    ach = alg / (avg / 1e3) / 1e12
+    with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+        mhz = float(json.load(f).get("sm_max_mhz", 1965.0))
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    peak = sms * 128 * 2 * mhz * 1e6 / 1e12  # fp32 lanes x FMA x max SM clock
+    roof = {"kernel": name, "bound": "alu", "achieved": round(ach, 2), "peak": round(peak, 1),
+            "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
+            "alg_flops_per_launch": alg, "avg_launch_ms": avg,
+            "peak_source": f"{sms} SMs x 128 fp32 lanes x 2 flops x {mhz:.0f} MHz (max SM clock)"}
+    extra = {"dtype": "f32", "roofline": roof, "kernels": prof,
+             "gpu_launches": sum(v["launches"] for v in prof.values()), "clocks": clk}
+    if rank == 0 and not args.no_cpu:
+        import oracle
+        orc = oracle.load()
+        h = {n: t[:1].double().cpu().numpy() for n, t in x.items()}
+        t0 = time.perf_counter()
+        orc.dlambda(h["q"], h["k"], h["v"], lam.double().cpu().numpy(), h["dO"])
+        dt = time.perf_counter() - t0
+        extra["cpu_baseline"] = {"value": round(L / dt, 1), "unit": "tokens/s",
+                                 "cores": orc.num_threads(), "kind": "oracle",
+                                 "sample": f"one batch row (16 heads x {L} rows) of the workload"}
+    return _common(world, args.steps, args.warmup, value, "tokens/s",
+                   "dlambda tokens/s (B=4,H=16,L=2048,d=e=128, bf16 inputs, fp32 FMA)",
+                   {"workload": "gradient w.r.t. the decay, B=4, H=16, L=2,048, d=e=128, bf16 "
+                                "inputs",
+                    "l2": "inputs 32 MiB (fit in L2); the pass is arithmetic-bound"}, ms, extra)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -676,9 +735,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--workload", default="sweep",
-                    choices=["sweep", "long", "decode", "varlen"],
+                    choices=["sweep", "long", "decode", "varlen", "dlambda"],
                     help="sweep (the metric; default), long (1M-token forward), decode, "
-                         "varlen (packed variable-length fwd+bwd)")
+                         "varlen (packed variable-length fwd+bwd), dlambda (decay gradient)")
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--decode-tokens", type=int, default=1,
                     help="decode workload: tokens per request per call (1 = decode_step)")
@@ -702,7 +761,7 @@ def main():
     world, rank, local = dist_setup(args.gpus)
     try:
         fn = {"sweep": run_la2, "long": run_long, "decode": run_decode,
-              "varlen": run_varlen}[args.workload]
+              "varlen": run_varlen, "dlambda": run_dlambda}[args.workload]
         line = fn(args, world, rank, local)
         if rank == 0:
             print(json.dumps(line), flush=True)

@@ -11,7 +11,7 @@ its absence raises an error: there is no CPU fallback.
 """
 from ._binding import (  # noqa: F401
     LA2Error, LA2_OP_BACKWARD, LA2_OP_FORWARD, LA2_OPT_INJECT_TIMEOUT, LA2_OPT_PATH,
-    LA2_POOL_CONTINUE, LA2_OP_SHARD_STATE, backward_shard, decode_tokens, forward_pool,
+    LA2_POOL_CONTINUE, LA2_OP_SHARD_STATE, LA2_OP_DLAMBDA, backward_shard, decode_tokens, forward_pool,
     shard_state, state_prefix, dlambda,
     LA2_OPT_SPLIT, LA2_OPT_TRACE, LA2_OPT_VARIANT, trace_read,
     backward, backward_varlen, decode_step, forward, forward_noalloc, forward_varlen,

@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(HERE, "libla2.so")
 
 LA2_OK, LA2_ERR_INVALID, LA2_ERR_UNSUPPORTED, LA2_ERR_CUDA, LA2_ERR_TIMEOUT = range(5)
 LA2_F32, LA2_BF16 = 0, 1
-LA2_OP_FORWARD, LA2_OP_BACKWARD, LA2_OP_SHARD_STATE = 0, 1, 2
+LA2_OP_FORWARD, LA2_OP_BACKWARD, LA2_OP_SHARD_STATE, LA2_OP_DLAMBDA = 0, 1, 2, 3
 LA2_OPT_SPLIT, LA2_OPT_PATH, LA2_OPT_INJECT_TIMEOUT, LA2_OPT_VARIANT, LA2_OPT_TRACE = 0, 1, 2, 3, 4
 
 _lock = threading.Lock()
@@ -76,6 +76,8 @@ def library():
         lib.la2_backward_shard.restype = I
         lib.la2_backward_dlambda.argtypes = [P, P, P, P, P, P, P, I, I, I64, I, I, I, P]
         lib.la2_backward_dlambda.restype = I
+        lib.la2_backward_dlambda_ex.argtypes = [P, P, P, P, P, P, P, I, I, I64, I, I, I, P, SZ, P]
+        lib.la2_backward_dlambda_ex.restype = I
         lib.la2_decode_step.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
         lib.la2_decode_step.restype = I
         lib.la2_last_device_error.argtypes = [P]
@@ -432,9 +434,11 @@ def backward_shard(q, k, v, lam, dO, kv0=None, dstate_end=None, *, want_dkv0: bo
     return (dq, dk, dv, dkv0) if want_dkv0 else (dq, dk, dv)
 
 
-def dlambda(q, k, v, lam, dO, kv0=None, *, stream=None):
+def dlambda(q, k, v, lam, dO, kv0=None, *, workspace=None, chunked: bool = True, stream=None):
     """Gradient of sum(o * dO) with respect to lam [H] (float32 [H], summed
-    over the batch)."""
+    over the batch).  chunked: split the sequences over several CTAs
+    (la2_backward_dlambda_ex with `workspace`, allocated here when None);
+    False: one CTA per (b,h), no workspace (la2_backward_dlambda)."""
     lib = library()
     for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam), ("dO", dO)):
         _dev(t, name)
@@ -445,9 +449,18 @@ def dlambda(q, k, v, lam, dO, kv0=None, *, stream=None):
     if kv0 is not None:
         _dev(kv0, "kv0")
     out = torch.empty(H, dtype=torch.float32, device=q.device)
-    code = lib.la2_backward_dlambda(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(dO),
-                                    _ptr(out), B, H, L, d, e, _dt(q), _stream(stream))
-    _check(code, "la2_backward_dlambda")
+    if not chunked:
+        code = lib.la2_backward_dlambda(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(dO),
+                                        _ptr(out), B, H, L, d, e, _dt(q), _stream(stream))
+        _check(code, "la2_backward_dlambda")
+        return out
+    if workspace is None:
+        workspace = _workspace(workspace_size(LA2_OP_DLAMBDA, B, H, L, d, e, q.dtype), q.device)
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    code = lib.la2_backward_dlambda_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(dO),
+                                       _ptr(out), B, H, L, d, e, _dt(q), _ptr(workspace), nbytes,
+                                       _stream(stream))
+    _check(code, "la2_backward_dlambda_ex")
     return out
 
 

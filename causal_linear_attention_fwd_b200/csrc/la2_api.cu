@@ -32,13 +32,14 @@ std::atomic<int> g_opt_trace{0};
 enum KernelId {
   K_SIMT_FWD_STATE, K_SIMT_FWD_SCAN, K_SIMT_FWD, K_SIMT_DQ, K_SIMT_REV_STATE,
   K_SIMT_REV_SCAN, K_SIMT_DKDV, K_DECODE, K_TC_FWD_STATE, K_TC_FWD, K_TC_DQ,
-  K_TC_REV_STATE, K_TC_DV, K_TC_DK, K_SCAN_FWD, K_SCAN_REV, K_COUNT
+  K_TC_REV_STATE, K_TC_DV, K_TC_DK, K_SCAN_FWD, K_SCAN_REV, K_SIMT_DLAMBDA,
+  K_SIMT_DLAMBDA_STATE, K_SIMT_DLAMBDA_SCAN, K_COUNT
 };
 const char *kKernelName[K_COUNT] = {
     "simt_fwd_chunk_state", "simt_scan_fwd", "simt_fwd", "simt_dq",
     "simt_rev_chunk_state", "simt_scan_rev", "simt_dkdv", "decode_step",
     "tc_fwd_chunk_state", "tc_fwd", "tc_dq", "tc_rev_chunk_state", "tc_dv", "tc_dk",
-    "scan_fwd", "scan_rev"};
+    "scan_fwd", "scan_rev", "simt_dlambda", "simt_dlambda_chunk_state", "simt_dlambda_scan"};
 
 struct ProfRec {
   int kid;
@@ -204,7 +205,51 @@ Geo plan(int B, int H, int64_t L, int blk, Path path) {
 
 int block_rows(Path p) { return p == PATH_TC ? la2::tc::BLOCK : la2::simt::C; }
 
+// Chunk plan of the decay gradient (fp32-FMA kernel, one CTA per SM): at
+// most one wave, S = floor(SMs / (B*H)) chunks per sequence when B*H is
+// below the SM count (LA2_OPT_SPLIT overrides), Lc a multiple of the block.
+// The chunk-state pre-pass covers chunks 0..S-2 only, so it runs on M
+// sub-chunks of Ls rows per chunk (Lc = M Ls), M filling the SMs (at most
+// 8); the workspace holds (S-1) M + 1 (KV, W) pairs per (b,h).
+Geo plan_dlambda(int B, int H, int64_t L, bool split_ok) {
+  Geo g = plan(B, H, L, la2::simt::C, PATH_SIMT);
+  const int64_t blk = la2::simt::C, nblk = (L + blk - 1) / blk;
+  const int64_t BH = (int64_t)B * H;
+  const int sms = device_sms();
+  int64_t S = g_opt_split.load();
+  if (S <= 0) S = BH >= sms ? 1 : sms / BH;
+  if (!split_ok || S > nblk) S = split_ok ? nblk : 1;
+  if (S < 1) S = 1;
+  int64_t per = (nblk + S - 1) / S;  // blocks per chunk
+  S = (nblk + per - 1) / per;
+  int64_t M = 1;
+  if (S > 1) {
+    // the largest M <= min(8, SMs / (B*H*(S-1))) whose whole sub-chunks
+    // keep S chunks
+    int64_t want = sms / (BH * (S - 1));
+    if (want > 8) want = 8;
+    for (int64_t m = want; m > 1; m--) {
+      const int64_t p = ((per + m - 1) / m) * m;
+      if ((nblk + p - 1) / p == S) {
+        M = m;
+        per = p;
+        break;
+      }
+    }
+  }
+  g.S = (int)S;
+  g.Lc = per * blk;
+  g.M = (int)M;
+  g.Ls = g.Lc / M;
+  g.nst = (int)((S - 1) * M);
+  g.wsS = g.nst + 1;
+  g.Ssub = g.wsS;
+  return g;
+}
+
 size_t ws_bytes(int op, const Geo &g, int d, int e) {
+  if (op == LA2_OP_DLAMBDA)  // (KV, W) per sub-chunk boundary
+    return g.S > 1 ? (size_t)g.B * g.H * g.wsS * 2 * d * e * sizeof(float) : 0;
   if (op == LA2_OP_SHARD_STATE)  // one delta per sub-chunk plus one spare slot
     return (size_t)g.B * g.H * (g.Ssub + 1) * d * e * sizeof(float);
   if (g.S <= 1) return 0;
@@ -324,20 +369,38 @@ la2_status to_status(cudaError_t e) { return e == cudaSuccess ? LA2_OK : LA2_ERR
 constexpr int kDecodeBlockTokens = 32;
 
 // ------------------------------------------------------- d lambda helper
+// dlam = 0; split: chunk-state pre-pass over the sub-chunks of chunks
+// 0..S-2, the scan of the (KV, W) pairs, then the gradient pass over every
+// chunk.
 template <typename T, int D, int E>
 cudaError_t simt_dlambda(const void *q, const void *k, const void *v, const void *dO,
-                         const float *lam, const float *kv0, float *dlam, const Geo &g,
-                         cudaStream_t st) {
+                         const float *lam, const float *kv0, float *dlam, float *ws,
+                         const Geo &g, cudaStream_t st) {
   using namespace la2::simt;
-  auto kd = dlambda_kernel<T, D, E>;
+  auto kd = dlambda_kernel<T, D, E, false>;
+  auto ks = dlambda_kernel<T, D, E, true>;
   cudaError_t e = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)dlam_smem<D, E>());
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dlam_smem<D, E>());
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(dlam, 0, (size_t)g.H * sizeof(float), st);
   if (e != cudaSuccess) return e;
-  return timed(K_SIMT_DKDV, st, [&] {
-    kd<<<(unsigned)((int64_t)g.B * g.H), NT, dlam_smem<D, E>(), st>>>(
-        (const T *)q, (const T *)k, (const T *)v, (const T *)dO, lam, kv0, dlam, g);
+  const int64_t BH = (int64_t)g.B * g.H;
+  const T *Q = (const T *)q, *K = (const T *)k, *V = (const T *)v, *G = (const T *)dO;
+  if (g.S > 1) {
+    e = timed(K_SIMT_DLAMBDA_STATE, st, [&] {
+      ks<<<(unsigned)(BH * g.nst), NT, dlam_smem<D, E>(), st>>>(Q, K, V, G, lam, nullptr, ws,
+                                                                  nullptr, g);
+    });
+    if (e != cudaSuccess) return e;
+    e = timed(K_SIMT_DLAMBDA_SCAN, st, [&] {
+      dlam_scan_kernel<D, E><<<dim3(D * E / NT, (unsigned)BH), NT, 0, st>>>(ws, kv0, lam, g);
+    });
+    if (e != cudaSuccess) return e;
+  }
+  return timed(K_SIMT_DLAMBDA, st, [&] {
+    kd<<<(unsigned)(BH * g.S), NT, dlam_smem<D, E>(), st>>>(Q, K, V, G, lam, kv0, ws, dlam, g);
   });
 }
 
@@ -410,6 +473,7 @@ int la2_set_option(int option, int value) {
 
 size_t la2_workspace_size(int op, int B, int H, int64_t L, int d, int e, la2_dtype dt) {
   if (B <= 0 || H <= 0 || L <= 0 || !shape_supported(d, e, dt)) return 0;
+  if (op == LA2_OP_DLAMBDA) return ws_bytes(op, plan_dlambda(B, H, L, true), d, e);
   if (op != LA2_OP_FORWARD && op != LA2_OP_BACKWARD && op != LA2_OP_SHARD_STATE) return 0;
   Path p = choose_path(d, e, dt);
   if (p == PATH_NONE) return 0;
@@ -832,10 +896,13 @@ la2_status la2_backward_shard(const void *q, const void *k, const void *v, const
   return to_status(err);
 }
 
-la2_status la2_backward_dlambda(const void *q, const void *k, const void *v,
-                                const float *lambda, const float *kv0, const void *dO,
-                                float *dlambda, int B, int H, int64_t L, int d, int e,
-                                la2_dtype dt, cudaStream_t stream) {
+namespace {
+// split: chunk the sequences as la2_workspace_size(LA2_OP_DLAMBDA) planned
+// (the workspace must then hold that much); otherwise one chunk per (b,h).
+la2_status dlambda_call(const void *q, const void *k, const void *v, const float *lambda,
+                        const float *kv0, const void *dO, float *dlambda, int B, int H,
+                        int64_t L, int d, int e, la2_dtype dt, void *workspace,
+                        size_t workspace_bytes, bool split, cudaStream_t stream) {
   if (B < 0 || H < 0 || L < 0) return LA2_ERR_INVALID;
   if (dt != LA2_F32 && dt != LA2_BF16) return LA2_ERR_UNSUPPORTED;
   if (!shape_supported(d, e, dt)) return LA2_ERR_UNSUPPORTED;
@@ -844,24 +911,46 @@ la2_status la2_backward_dlambda(const void *q, const void *k, const void *v,
   if (!lambda || !dlambda || (BH > 0 && L > 0 && (!q || !k || !v || !dO))) return LA2_ERR_INVALID;
   for (const void *p : std::initializer_list<const void *>{
            (const void *)q, (const void *)k, (const void *)v, (const void *)lambda,
-           (const void *)kv0, (const void *)dO, (const void *)dlambda})
+           (const void *)kv0, (const void *)dO, (const void *)dlambda, workspace})
     if (p && !aligned16(p)) return LA2_ERR_INVALID;
   const size_t es = esize(dt);
   const size_t nq = (size_t)BH * L * d * es, nv = (size_t)BH * L * e * es;
   std::vector<Span> ins = {{q, nq}, {k, nq}, {v, nv}, {dO, nv}, {lambda, (size_t)H * 4},
                            {kv0, kv0 ? (size_t)BH * d * e * 4 : 0}};
-  std::vector<Span> outs = {{dlambda, (size_t)H * 4}};
+  std::vector<Span> outs = {{dlambda, (size_t)H * 4}, {workspace, workspace ? workspace_bytes : 0}};
   if (any_overlap(outs, ins)) return LA2_ERR_INVALID;
   if (BH == 0 || L == 0) {  // no token depends on lambda
     return to_status(cudaMemsetAsync(dlambda, 0, (size_t)H * sizeof(float), stream));
   }
-  Geo g = plan(B, H, L, la2::simt::C, PATH_SIMT);
+  const Geo g = plan_dlambda(B, H, L, split);
+  const size_t need = ws_bytes(LA2_OP_DLAMBDA, g, d, e);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return LA2_ERR_INVALID;
+  float *ws = (float *)workspace;
   cudaError_t err =
       dt == LA2_F32
-          ? LA2_DISPATCH_DE(d, e, simt_dlambda, float, q, k, v, dO, lambda, kv0, dlambda, g, stream)
+          ? LA2_DISPATCH_DE(d, e, simt_dlambda, float, q, k, v, dO, lambda, kv0, dlambda, ws, g,
+                            stream)
           : LA2_DISPATCH_DE(d, e, simt_dlambda, __nv_bfloat16, q, k, v, dO, lambda, kv0, dlambda,
-                            g, stream);
+                            ws, g, stream);
   return to_status(err);
+}
+}  // namespace
+
+la2_status la2_backward_dlambda(const void *q, const void *k, const void *v,
+                                const float *lambda, const float *kv0, const void *dO,
+                                float *dlambda, int B, int H, int64_t L, int d, int e,
+                                la2_dtype dt, cudaStream_t stream) {
+  return dlambda_call(q, k, v, lambda, kv0, dO, dlambda, B, H, L, d, e, dt, nullptr, 0, false,
+                      stream);
+}
+
+la2_status la2_backward_dlambda_ex(const void *q, const void *k, const void *v,
+                                   const float *lambda, const float *kv0, const void *dO,
+                                   float *dlambda, int B, int H, int64_t L, int d, int e,
+                                   la2_dtype dt, void *workspace, size_t workspace_bytes,
+                                   cudaStream_t stream) {
+  return dlambda_call(q, k, v, lambda, kv0, dO, dlambda, B, H, L, d, e, dt, workspace,
+                      workspace_bytes, true, stream);
 }
 
 la2_status la2_decode_step(const void *q, const void *k, const void *v, const float *lambda,

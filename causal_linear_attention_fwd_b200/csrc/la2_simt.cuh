@@ -502,106 +502,219 @@ template <int D, int E> constexpr size_t dkdv_smem() {
 }
 
 // ------------------------------------------------------------ d lambda
-// Gradient of sum(o * dO) with respect to lambda_h, one CTA per (b,h) over
-// the whole sequence, added into dlam[h].  With the carried states, per
-// block of rows p.. (local t, j):
+// Gradient of sum(o * dO) with respect to lambda_h, added into dlam[h].
+// With the carried states at the start of a block of rows p.. (local t, j):
 //   KV = sum_{j<p} lambda^(p-1-j) k_j^T v_j,
 //   W  = sum_{j<p} (p-1-j) lambda^(p-1-j) k_j^T v_j,
 // the derivative of o_t splits into the block's own pairs
 //   sum_{j<t} (t-j) lambda^(t-j-1) (q_t . k_j) v_j
-// and the earlier rows  lambda^t ((t+1) q_t KV + q_t W)  (with KV = kv0,
-// W = 0 before the first block: d/dlambda of lambda^(t+1) q_t kv0); both
-// are dotted with dO_t.  Then W <- lambda^cb (cb KV + W) + sum_j (cb-1-j)
-// lambda^(cb-1-j) k_j^T v_j and KV <- lambda^cb KV + sum_j lambda^(cb-1-j)
-// k_j^T v_j.  No division by lambda, so lambda = 0 is exact.
+// and the earlier rows  lambda^t ((t+1) q_t KV + q_t W)  (KV = kv0, W = 0
+// before the first row: d/dlambda of lambda^(t+1) q_t kv0); both are dotted
+// with dO_t.  Then W <- lambda^cb (cb KV + W) + sum_j (cb-1-j) lambda^(cb-1-j)
+// k_j^T v_j and KV <- lambda^cb KV + sum_j lambda^(cb-1-j) k_j^T v_j.  No
+// division by lambda, so lambda = 0 is exact.  The same pair of updates over
+// a whole chunk of Lc rows composes chunks:  W' = lambda^Lc (Lc KV + W) + dW,
+// KV' = lambda^Lc KV + dKV.
+//
+// Layout: the 256 threads form a 16 x 16 grid; thread (ti, tc) keeps the
+// entries (ti + 16 i, tc + 16 j) of KV and of W, i < D/16, j < E/16, in
+// registers for the whole chunk, so the per-row work is outer products of a
+// q (k) row slice with a dO (v) row slice read from shared memory (the 16
+// threads of a row read 16 consecutive words: no bank conflicts).  The
+// block's own pairs take 2 x 2 tiles of S = Q K^T and G = dO V^T per thread.
+// STATE = true: the chunk-state pre-pass (from zero, no gradient) over the
+// g.nst sub-chunks of Ls rows before the last chunk: writes sub-chunk u's
+// (dKV, dW) to workspace slot u+1 of the (b,h)'s wsS slots.  The gradient
+// pass's chunk c (Lc = M Ls rows) enters with the pair in slot c M.
 template <int D, int E>
 constexpr size_t dlam_smem() {
-  return sizeof(float) * (2 * D * (E + 1) + 2 * C * (D + 1) + 2 * C * (E + 1) + (C + 1) + NT / 32);
+  return sizeof(float) * (2 * C * (D + 1) + 2 * C * (E + 1) + (C + 2)) + sizeof(double) * (NT / 32);
 }
 
-template <typename T, int D, int E>
-__global__ void __launch_bounds__(NT)
+template <typename T, int D, int E, bool STATE>
+__global__ void __launch_bounds__(NT, 1)
 dlambda_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                const T *__restrict__ dO, const float *__restrict__ lambda,
-               const float *__restrict__ kv0, float *__restrict__ dlam, Geo g) {
-  constexpr int LDS = E + 1, LDQ = D + 1, LDV = E + 1;
+               const float *__restrict__ kv0, float *__restrict__ ws, float *__restrict__ dlam,
+               Geo g) {
+  constexpr int LQ = D + 1, LV = E + 1;  // odd row strides: row r starts at bank r
+  constexpr int TI = D / 16, TC = E / 16;
   extern __shared__ float sm[];
-  float *KV = sm;                  // D x (E+1)
-  float *Wst = KV + D * LDS;       // D x (E+1)
-  float *Qs = Wst + D * LDS;       // C x (D+1)
-  float *Ks = Qs + C * LDQ;        // C x (D+1)
-  float *Vs = Ks + C * LDQ;        // C x (E+1)
-  float *Gs = Vs + C * LDV;        // C x (E+1)   dO
-  float *pw = Gs + C * LDV;        // C+1
-  float *red = pw + (C + 1);       // NT/32
+  float *Qs = sm;                  // C x LQ
+  float *Ks = Qs + C * LQ;         // C x LQ
+  float *Vs = Ks + C * LQ;         // C x LV
+  float *Gs = Vs + C * LV;         // C x LV   dO
+  float *pw = Gs + C * LV;         // C+1
+  double *red = reinterpret_cast<double *>(pw + C + 2);  // NT/32
 
-  const int64_t bh = blockIdx.x;
+  const int nch = STATE ? g.nst : g.S;
+  const int64_t len = STATE ? g.Ls : g.Lc;
+  const int64_t bh = blockIdx.x / nch;
+  const int c = blockIdx.x % nch;
   const int h = (int)(bh % g.H);
+  const int64_t a = (int64_t)c * len;
+  const int64_t b = g.L < a + len ? g.L : a + len;
+  const int tid = threadIdx.x;
+  const int ti = tid >> 4, tc = tid & 15;
   fill_pow(pw, lambda[h]);
-  for (int idx = threadIdx.x; idx < D * E; idx += NT) {
-    KV[(idx / E) * LDS + idx % E] = kv0 ? kv0[bh * D * E + idx] : 0.f;
-    Wst[(idx / E) * LDS + idx % E] = 0.f;
+
+  float KV[TI][TC], Wt[TI][TC];
+  {
+    const float *ikv = nullptr, *iw = nullptr;
+    if (!STATE) {
+      if (g.S > 1) {
+        ikv = ws + ((bh * g.wsS + (int64_t)c * g.M) * 2) * (int64_t)D * E;
+        iw = ikv + D * E;
+      } else if (kv0) {
+        ikv = kv0 + bh * (int64_t)D * E;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < TI; i++)
+#pragma unroll
+      for (int j = 0; j < TC; j++) {
+        KV[i][j] = ikv ? ikv[(ti + 16 * i) * E + tc + 16 * j] : 0.f;
+        Wt[i][j] = iw ? iw[(ti + 16 * i) * E + tc + 16 * j] : 0.f;
+      }
   }
   double acc = 0.0;
   __syncthreads();
 
-  for (int64_t p = 0; p < g.L; p += C) {
-    const int cb = (int)(g.L - p < C ? g.L - p : C);
-    load_tile<T, D>(Qs, LDQ, q + (bh * g.L + p) * D, cb);
-    load_tile<T, D>(Ks, LDQ, k + (bh * g.L + p) * D, cb);
-    load_tile<T, E>(Vs, LDV, v + (bh * g.L + p) * E, cb);
-    load_tile<T, E>(Gs, LDV, dO + (bh * g.L + p) * E, cb);
+  for (int64_t p = a; p < b; p += C) {
+    const int cb = (int)(b - p < C ? b - p : C);
+    if (!STATE) load_tile<T, D>(Qs, LQ, q + (bh * g.L + p) * D, cb);
+    load_tile<T, D>(Ks, LQ, k + (bh * g.L + p) * D, cb);
+    load_tile<T, E>(Vs, LV, v + (bh * g.L + p) * E, cb);
+    if (!STATE) load_tile<T, E>(Gs, LV, dO + (bh * g.L + p) * E, cb);
     __syncthreads();
-    // the block's own pairs j < t
-    for (int idx = threadIdx.x; idx < C * C; idx += NT) {
-      const int t = idx / C, j = idx % C;
-      if (j < t && t < cb) {
-        float s = 0.f, gv = 0.f;
-#pragma unroll 8
-        for (int i = 0; i < D; i++) s += Qs[t * LDQ + i] * Ks[j * LDQ + i];
-#pragma unroll 8
-        for (int c = 0; c < E; c++) gv += Gs[t * LDV + c] * Vs[j * LDV + c];
-        acc += (double)((float)(t - j) * pw[t - j - 1] * s * gv);
-      }
-    }
-    // the earlier rows through the carried states
-    for (int idx = threadIdx.x; idx < C * E; idx += NT) {
-      const int t = idx / E, c = idx % E;
-      if (t < cb) {
-        float x = 0.f, y = 0.f;
-#pragma unroll 8
-        for (int i = 0; i < D; i++) {
-          x += Qs[t * LDQ + i] * KV[i * LDS + c];
-          y += Qs[t * LDQ + i] * Wst[i * LDS + c];
+    if (!STATE) {
+      float part = 0.f;
+      // the earlier rows: lambda^t ((t+1) q_t KV dO_t + q_t W dO_t), the
+      // thread's tile of the double sums
+      for (int t = 0; t < cb; t++) {
+        float qv[TI], gv[TC];
+#pragma unroll
+        for (int i = 0; i < TI; i++) qv[i] = Qs[t * LQ + ti + 16 * i];
+#pragma unroll
+        for (int j = 0; j < TC; j++) gv[j] = Gs[t * LV + tc + 16 * j];
+        float s1 = 0.f, s0 = 0.f;
+#pragma unroll
+        for (int i = 0; i < TI; i++) {
+          float r1 = 0.f, r0 = 0.f;
+#pragma unroll
+          for (int j = 0; j < TC; j++) {
+            r1 = fmaf(KV[i][j], gv[j], r1);
+            r0 = fmaf(Wt[i][j], gv[j], r0);
+          }
+          s1 = fmaf(qv[i], r1, s1);
+          s0 = fmaf(qv[i], r0, s0);
         }
-        acc += (double)(pw[t] * ((float)(t + 1) * x + y) * Gs[t * LDV + c]);
+        part += pw[t] * fmaf((float)(t + 1), s1, s0);
       }
+      // the block's own pairs j < t: 2 x 2 of S = Q K^T and G = dO V^T
+      {
+        const int t0 = 2 * ti, j0 = 2 * tc;
+        float S[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, G[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+        if (j0 < t0 + 1 && t0 < cb) {
+#pragma unroll 4
+          for (int x = 0; x < D; x++) {
+            const float qa = Qs[t0 * LQ + x], qb = Qs[(t0 + 1) * LQ + x];
+            const float ka = Ks[j0 * LQ + x], kb = Ks[(j0 + 1) * LQ + x];
+            S[0][0] = fmaf(qa, ka, S[0][0]); S[0][1] = fmaf(qa, kb, S[0][1]);
+            S[1][0] = fmaf(qb, ka, S[1][0]); S[1][1] = fmaf(qb, kb, S[1][1]);
+          }
+#pragma unroll 4
+          for (int x = 0; x < E; x++) {
+            const float ga = Gs[t0 * LV + x], gb = Gs[(t0 + 1) * LV + x];
+            const float va = Vs[j0 * LV + x], vb = Vs[(j0 + 1) * LV + x];
+            G[0][0] = fmaf(ga, va, G[0][0]); G[0][1] = fmaf(ga, vb, G[0][1]);
+            G[1][0] = fmaf(gb, va, G[1][0]); G[1][1] = fmaf(gb, vb, G[1][1]);
+          }
+#pragma unroll
+          for (int u = 0; u < 2; u++)
+#pragma unroll
+            for (int w = 0; w < 2; w++) {
+              const int t = t0 + u, j = j0 + w;
+              if (j < t && t < cb) part += (float)(t - j) * pw[t - j - 1] * S[u][w] * G[u][w];
+            }
+        }
+      }
+      acc += (double)part;
     }
-    __syncthreads();
-    // W from the old KV, then KV
-    for (int idx = threadIdx.x; idx < D * E; idx += NT) {
-      const int i = idx / E, c = idx % E;
-      float dkv = 0.f, dw = 0.f;
-      for (int j = 0; j < cb; j++) {
-        const float kvj = pw[cb - 1 - j] * Ks[j * LDQ + i] * Vs[j * LDV + c];
-        dkv += kvj;
-        dw += (float)(cb - 1 - j) * kvj;
+    // W from the old KV, then KV; then the block's rows
+    const float dec = pw[cb];
+#pragma unroll
+    for (int i = 0; i < TI; i++)
+#pragma unroll
+      for (int j = 0; j < TC; j++) {
+        Wt[i][j] = dec * fmaf((float)cb, KV[i][j], Wt[i][j]);
+        KV[i][j] = dec * KV[i][j];
       }
-      const float kv_old = KV[i * LDS + c];
-      Wst[i * LDS + c] = pw[cb] * ((float)cb * kv_old + Wst[i * LDS + c]) + dw;
-      KV[i * LDS + c] = pw[cb] * kv_old + dkv;
+    for (int jr = 0; jr < cb; jr++) {
+      const float bj = pw[cb - 1 - jr], wj = (float)(cb - 1 - jr) * bj;
+      float kv_[TI], vv[TC];
+#pragma unroll
+      for (int i = 0; i < TI; i++) kv_[i] = Ks[jr * LQ + ti + 16 * i];
+#pragma unroll
+      for (int j = 0; j < TC; j++) vv[j] = Vs[jr * LV + tc + 16 * j];
+#pragma unroll
+      for (int i = 0; i < TI; i++) {
+        const float kb = bj * kv_[i], kw = wj * kv_[i];
+#pragma unroll
+        for (int j = 0; j < TC; j++) {
+          KV[i][j] = fmaf(kb, vv[j], KV[i][j]);
+          Wt[i][j] = fmaf(kw, vv[j], Wt[i][j]);
+        }
+      }
     }
     __syncthreads();
   }
-  // block sum, then one atomic add per CTA
-  float a = (float)acc;
-  for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float t = 0.f;
-    for (int w = 0; w < NT / 32; w++) t += red[w];
-    atomicAdd(dlam + h, t);
+  if constexpr (STATE) {
+    float *okv = ws + ((bh * g.wsS + c + 1) * 2) * (int64_t)D * E, *ow = okv + D * E;
+#pragma unroll
+    for (int i = 0; i < TI; i++)
+#pragma unroll
+      for (int j = 0; j < TC; j++) {
+        okv[(ti + 16 * i) * E + tc + 16 * j] = KV[i][j];
+        ow[(ti + 16 * i) * E + tc + 16 * j] = Wt[i][j];
+      }
+  } else {
+    // block sum, then one atomic add per CTA
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if ((tid & 31) == 0) red[tid >> 5] = acc;
+    __syncthreads();
+    if (tid == 0) {
+      double t = 0.0;
+      for (int w = 0; w < NT / 32; w++) t += red[w];
+      atomicAdd(dlam + h, (float)t);
+    }
+  }
+}
+
+// Sub-chunk entry states of the decay gradient, in place over the
+// workspace's [B*H, wsS, 2, D, E] slots: slot u+1 holds sub-chunk u's (dKV,
+// dW) (all Ls rows); afterwards slot u holds the (KV, W) entering sub-chunk
+// u, slot 0 the initial (kv0 or 0, 0).
+template <int D, int E>
+__global__ void __launch_bounds__(NT)
+dlam_scan_kernel(float *__restrict__ ws, const float *__restrict__ kv0,
+                 const float *__restrict__ lambda, Geo g) {
+  const int64_t bh = blockIdx.y;
+  const int idx = blockIdx.x * NT + threadIdx.x;
+  if (idx >= D * E) return;
+  const float f = (float)pow_int((double)lambda[bh % g.H], g.Ls);
+  const float n = (float)g.Ls;
+  float *base = ws + bh * g.wsS * 2 * (int64_t)D * E + idx;
+  float kv = kv0 ? kv0[bh * D * E + idx] : 0.f, w = 0.f;
+  base[0] = kv;
+  base[D * E] = w;
+  for (int c = 1; c <= g.nst; c++) {
+    float *s = base + (int64_t)c * 2 * D * E;
+    const float dkv = s[0], dw = s[D * E];
+    w = fmaf(f, fmaf(n, kv, w), dw);
+    kv = fmaf(f, kv, dkv);
+    s[0] = kv;
+    s[D * E] = w;
   }
 }
 

@@ -102,3 +102,16 @@ def decode_state0(B, H, d, e, *, device="cpu", seed: int = 0) -> torch.Tensor:
     """Initial decode state kv0 ~ 0.01 * N(0,1), fp32 [B,H,d,e]."""
     return randn((B, H, d, e), dtype=torch.float32, device=device, seed=seed,
                  tid=TENSOR_ID["kv0"], scale=0.01)
+
+
+def varlen_lengths(total: int, seed: int = 0, lo: int = 64, hi: int = 8192) -> list:
+    """Document lengths of a packed training batch: log-uniform in [lo, hi]
+    rows, drawn from a seeded numpy generator until `total` rows are filled
+    (the last one cut to fit)."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    lens = []
+    while sum(lens) < total:
+        n = int(round(float(np.exp(rng.uniform(np.log(lo), np.log(hi))))))
+        lens.append(min(n, total - sum(lens)))
+    return lens

@@ -74,12 +74,14 @@ typedef enum {
 typedef enum { LA2_F32 = 0, LA2_BF16 = 1 } la2_dtype;
 
 /* Operation codes for la2_workspace_size(). */
-enum { LA2_OP_FORWARD = 0, LA2_OP_BACKWARD = 1, LA2_OP_SHARD_STATE = 2 };
+enum { LA2_OP_FORWARD = 0, LA2_OP_BACKWARD = 1, LA2_OP_SHARD_STATE = 2, LA2_OP_DLAMBDA = 3 };
 
 /*
  * Bytes of device scratch that la2_forward (op = LA2_OP_FORWARD),
- * la2_backward (op = LA2_OP_BACKWARD) or la2_shard_state (op =
- * LA2_OP_SHARD_STATE) needs for these sizes on the CURRENT device.  The scratch holds the fp32 d x e states at the boundaries of the
+ * la2_backward (op = LA2_OP_BACKWARD), la2_shard_state (op =
+ * LA2_OP_SHARD_STATE) or la2_backward_dlambda_ex (op = LA2_OP_DLAMBDA)
+ * needs for these sizes on the CURRENT device.  The scratch holds the fp32
+ * d x e states at the boundaries of the
  * sequence chunks that run in parallel (the split of one long sequence over
  * several CTAs); it may be 0 when the sequence is not split.  Returns 0 for
  * unsupported arguments as well; the call then reports the error.
@@ -222,19 +224,35 @@ la2_status la2_decode_step(const void *q, const void *k, const void *v,
  *   dlambda_h = sum_b sum_t dO_t . ( sum_{j<t} (t-j) lambda^(t-j-1)
  *               (q_t . k_j) v_j + (t+1) lambda^t q_t kv0 ),
  * computed block by block with a second carried state (the position-
- * weighted sum of k^T v) next to the usual one; exact at lambda = 0.  One
- * CTA per (b,h) walks the whole sequence on the fp32-FMA path (a
- * functional path: no chunk split and no tensor cores); the batch sum is
- * made with atomics, so it is not bitwise reproducible across runs.
- * Errors as for la2_backward (dlambda overlapping an input:
- * LA2_ERR_INVALID).  The pages do not treat the decay as learnable; the
- * derivative is the chain rule through the recurrence of the Lightning
- * Attention-2 notes page (opening paragraph's running state, with decay).
+ * weighted sum of k^T v) next to the usual one; exact at lambda = 0.  It
+ * runs on the fp32-FMA path (no tensor cores), one CTA per (b,h) over the
+ * whole sequence; the batch sum is made with atomics, so it is not bitwise
+ * reproducible across runs.  Errors as for la2_backward (dlambda
+ * overlapping an input: LA2_ERR_INVALID).  The pages do not treat the decay
+ * as learnable; the derivative is the chain rule through the recurrence of
+ * the Lightning Attention-2 notes page (opening paragraph's running state,
+ * with decay).
  */
 la2_status la2_backward_dlambda(const void *q, const void *k, const void *v,
                                 const float *lambda, const float *kv0, const void *dO,
                                 float *dlambda, int B, int H, int64_t L, int d, int e,
                                 la2_dtype dt, cudaStream_t stream);
+
+/*
+ * la2_backward_dlambda with a workspace of la2_workspace_size(
+ * LA2_OP_DLAMBDA, ...) bytes (16-byte aligned; caller-owned; it may not
+ * overlap an input): when B*H is below the number of SMs each sequence is
+ * split into chunks that run in parallel, their entry states (KV, W) coming
+ * from a chunk-state pre-pass and a scan over the chunks (the pair composes
+ * as W' = lambda^Lc (Lc KV + W) + dW, KV' = lambda^Lc KV + dKV).  A size of
+ * 0 means no split; workspace may then be NULL.  A workspace smaller than
+ * needed: LA2_ERR_INVALID.
+ */
+la2_status la2_backward_dlambda_ex(const void *q, const void *k, const void *v,
+                                   const float *lambda, const float *kv0, const void *dO,
+                                   float *dlambda, int B, int H, int64_t L, int d, int e,
+                                   la2_dtype dt, void *workspace, size_t workspace_bytes,
+                                   cudaStream_t stream);
 
 /*
  * State pool for serving: the recurrent states of many requests live in one

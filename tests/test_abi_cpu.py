@@ -208,6 +208,32 @@ def test_dlambda_validation(lib):
     assert f(H=0) == OK
 
 
+def test_dlambda_ex_workspace_rules(lib):
+    """The chunked decay gradient: scratch (KV, W) per chunk when the
+    sequences are split; too little scratch, or scratch over an input, is
+    rejected before any launch."""
+    INV = B.LA2_ERR_INVALID
+    need = lib.la2_workspace_size(B.LA2_OP_DLAMBDA, 1, 2, 1 << 16, 64, 64, B.LA2_BF16)
+    assert need > 0 and need % (2 * 64 * 64 * 4) == 0
+    old = la2.set_option(la2.LA2_OPT_SPLIT, 3)
+    try:
+        n = lib.la2_workspace_size(B.LA2_OP_DLAMBDA, 2, 3, 1000, 64, 128, B.LA2_F32)
+        # (KV, W) pairs at the sub-chunk boundaries of the first two chunks
+        # plus the initial pair: an odd number of pairs, at least 3
+        pairs = n // (2 * 3 * 2 * 64 * 128 * 4)
+        assert n == pairs * 2 * 3 * 2 * 64 * 128 * 4 and pairs >= 3 and pairs % 2 == 1
+        la2.set_option(la2.LA2_OPT_SPLIT, 1)
+        assert lib.la2_workspace_size(B.LA2_OP_DLAMBDA, 2, 3, 1000, 64, 128, B.LA2_F32) == 0
+    finally:
+        la2.set_option(la2.LA2_OPT_SPLIT, old)
+    f = lambda ws=WS, wsb=need, L=1 << 16: lib.la2_backward_dlambda_ex(
+        Q, K, V, LAM, None, DO, KVO, 1, 2, L, 64, 64, B.LA2_BF16, ws, wsb, None)
+    assert f(wsb=need - 1) == INV
+    assert f(ws=None, wsb=0) == INV
+    assert f(ws=Q) == INV                            # scratch over an input
+    assert f(ws=KVO) == INV                          # scratch over the output
+
+
 def test_workspace_rules(lib):
     # a long sequence with few (b,h) pairs is split, so scratch is needed ...
     need = lib.la2_workspace_size(B.LA2_OP_FORWARD, 1, 2, 1 << 16, 64, 64, B.LA2_BF16)

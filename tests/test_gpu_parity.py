@@ -389,16 +389,42 @@ def test_trace_instantiation_matches():
 
 
 # --------------------------------------------------- gradient w.r.t. lambda
+@pytest.mark.parametrize("split", [0, 1, 3, 7, None])
 @pytest.mark.parametrize("dtype,de,L", [(torch.bfloat16, (128, 128), 300),
                                         (torch.float32, (64, 64), 257),
-                                        (torch.bfloat16, (64, 128), 33)])
-def test_dlambda_matches_oracle(orc, dtype, de, L):
+                                        (torch.bfloat16, (64, 128), 33),
+                                        (torch.float32, (128, 64), 1000)])
+def test_dlambda_matches_oracle(orc, dtype, de, L, split):
+    """split: chunks per sequence (0 = the library's choice; None = the
+    workspace-free entry point, one chunk per sequence)."""
     d, e = de
     x = inputs.make_inputs(2, 3, L, d, e, dtype=dtype, device=DEV, seed=L, with_kv0=True)
     lam = inputs.fixed_lambdas((1.0, 0.9, 0.0), DEV)
-    got = la2.dlambda(x["q"], x["k"], x["v"], lam, x["dO"], x["kv0"])
-    torch.cuda.synchronize()
+    old = la2.set_option(la2.LA2_OPT_SPLIT, split or 0)
+    try:
+        got = la2.dlambda(x["q"], x["k"], x["v"], lam, x["dO"], x["kv0"],
+                          chunked=split is not None)
+        torch.cuda.synchronize()
+    finally:
+        la2.set_option(la2.LA2_OPT_SPLIT, old)
+    assert la2.last_device_error() == 0
     h = {n: host(t) for n, t in x.items()}
     ref = orc.dlambda(h["q"], h["k"], h["v"], lam.double().cpu().numpy(), h["dO"], h["kv0"])
     err = np.max(np.abs(got.double().cpu().numpy() - ref))
     assert err <= 1e-3 * max(float(np.max(np.abs(ref))), 1e-6), (got, ref)
+
+
+def test_dlambda_b4_h16_l2048(orc):
+    """The decay gradient on the training shape the bench times (B=4, H=16,
+    L=2,048, bf16 inputs, the recipe's decays), every head against the
+    oracle."""
+    B, H, L = 4, 16, 2048
+    x = inputs.make_inputs(B, H, L, 128, 128, dtype=torch.bfloat16, device=DEV, seed=0)
+    lam = inputs.decay_lambdas(H, DEV)
+    got = la2.dlambda(x["q"], x["k"], x["v"], lam, x["dO"])
+    torch.cuda.synchronize()
+    assert la2.last_device_error() == 0
+    h = {n: host(t) for n, t in x.items()}
+    ref = orc.dlambda(h["q"], h["k"], h["v"], lam.double().cpu().numpy(), h["dO"])
+    err = np.max(np.abs(got.double().cpu().numpy() - ref))
+    assert err <= 1e-3 * float(np.max(np.abs(ref))), (got, ref)

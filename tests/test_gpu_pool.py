@@ -110,3 +110,28 @@ def test_pool_slot_past_end_reported():
     torch.cuda.synchronize()
     assert la2.last_device_error() == 1
     assert la2.last_device_error() == 0
+
+
+@pytest.mark.parametrize("T", [4, 64])
+def test_decode_tokens_bench_batch_sampled(orc, T):
+    """Multi-token decode on the batch the bench times (256 requests x H 64,
+    d = e = 128, bf16 tokens, fp32 state of 1 GiB): two calls of T tokens,
+    token by token below 32 per call and through the tensor-core block path
+    from 32; sampled requests against the oracle's decode steps."""
+    B, H, d, e = 256, 64, 128, 128
+    kv = inputs.decode_state0(B, H, d, e, device=DEV, seed=0)
+    kv0 = kv[[0, 77, 255]].double().cpu().numpy()
+    lam = inputs.decay_lambdas(H, DEV)
+    calls = [tokens(B, H, T, d, e, torch.bfloat16, seed=10 + c) for c in range(2)]
+    outs = [la2.decode_tokens(q, k, v, lam, kv) for q, k, v in calls]
+    torch.cuda.synchronize()
+    assert la2.last_device_error() == 0
+    lam_h = lam.double().cpu().numpy()
+    for i, b in enumerate((0, 77, 255)):
+        st = kv0[i:i + 1].copy()
+        for c, (q, k, v) in enumerate(calls):
+            ref = np.stack([orc.decode_step(host(q[b:b + 1, :, t]), host(k[b:b + 1, :, t]),
+                                            host(v[b:b + 1, :, t]), lam_h, st)[0]
+                            for t in range(T)], axis=1)
+            check(f"T={T} call {c} request {b} o", outs[c][b], ref, torch.bfloat16)
+        check(f"T={T} request {b} state", kv[b], st[0], torch.bfloat16)

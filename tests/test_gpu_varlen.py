@@ -115,3 +115,34 @@ def test_varlen_bad_offsets_reported():
         torch.cuda.synchronize()
         assert la2.last_device_error() == 1  # LA2_ERR_INVALID
     assert la2.last_device_error() == 0
+
+
+def test_varlen_bench_batch_sampled(orc):
+    """The packed batch the bench times (35 sequences of 64..8,082 rows,
+    65,536 rows per head, H = 32, bf16, seed 0), forward and backward in one
+    launch each; sampled (sequence, head) pairs -- the longest, the shortest,
+    the first and the last sequence, heads 0, 17 and 31 -- against the oracle
+    on that sequence's rows alone."""
+    H, T = 32, 65536
+    lens = inputs.varlen_lengths(T, seed=0)
+    offs = np.concatenate([[0], np.cumsum(lens)])
+    cu = torch.tensor(offs, dtype=torch.int64, device=DEV)
+    x = inputs.make_inputs(1, H, T, 128, 128, dtype=torch.bfloat16, device=DEV, seed=0)
+    x = {n: t[0] for n, t in x.items()}
+    lam = inputs.decay_lambdas(H, DEV)
+    o = la2.forward_varlen(x["q"], x["k"], x["v"], lam, cu)
+    dq, dk, dv = la2.backward_varlen(x["q"], x["k"], x["v"], lam, cu, x["dO"])
+    torch.cuda.synchronize()
+    assert la2.last_device_error() == 0
+    lam_h = lam.double().cpu().numpy()
+    seqs = sorted({int(np.argmax(lens)), int(np.argmin(lens)), 0, len(lens) - 1})
+    for n in seqs:
+        a, b = int(offs[n]), int(offs[n + 1])
+        for hh in (0, 17, 31):
+            sl = {k: host(t[hh:hh + 1, a:b])[None] for k, t in x.items()}
+            o_ref = orc.forward(sl["q"], sl["k"], sl["v"], lam_h[hh:hh + 1])
+            g = orc.backward(sl["q"], sl["k"], sl["v"], lam_h[hh:hh + 1], sl["dO"])
+            tag = f"seq {n} ({b - a} rows) head {hh}"
+            check(f"{tag} o", o[hh, a:b], o_ref[0, 0], torch.bfloat16)
+            for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), g[:3]):
+                check(f"{tag} {name}", got[hh, a:b], ref[0, 0], torch.bfloat16)
