@@ -380,9 +380,9 @@ cudaError_t simt_dlambda(const void *q, const void *k, const void *v, const void
   auto kd = dlambda_kernel<T, D, E, false>;
   auto ks = dlambda_kernel<T, D, E, true>;
   cudaError_t e = cudaFuncSetAttribute(kd, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)dlam_smem<D, E>());
+                                       (int)dlam_smem<T, D, E>());
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dlam_smem<D, E>());
+    e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dlam_smem<T, D, E>());
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(dlam, 0, (size_t)g.H * sizeof(float), st);
   if (e != cudaSuccess) return e;
@@ -390,7 +390,7 @@ cudaError_t simt_dlambda(const void *q, const void *k, const void *v, const void
   const T *Q = (const T *)q, *K = (const T *)k, *V = (const T *)v, *G = (const T *)dO;
   if (g.S > 1) {
     e = timed(K_SIMT_DLAMBDA_STATE, st, [&] {
-      ks<<<(unsigned)(BH * g.nst), NT, dlam_smem<D, E>(), st>>>(Q, K, V, G, lam, nullptr, ws,
+      ks<<<(unsigned)(BH * g.nst), NT, dlam_smem<T, D, E>(), st>>>(Q, K, V, G, lam, nullptr, ws,
                                                                   nullptr, g);
     });
     if (e != cudaSuccess) return e;
@@ -400,7 +400,7 @@ cudaError_t simt_dlambda(const void *q, const void *k, const void *v, const void
     if (e != cudaSuccess) return e;
   }
   return timed(K_SIMT_DLAMBDA, st, [&] {
-    kd<<<(unsigned)(BH * g.S), NT, dlam_smem<D, E>(), st>>>(Q, K, V, G, lam, kv0, ws, dlam, g);
+    kd<<<(unsigned)(BH * g.S), NT, dlam_smem<T, D, E>(), st>>>(Q, K, V, G, lam, kv0, ws, dlam, g);
   });
 }
 

@@ -501,6 +501,33 @@ template <int D, int E> constexpr size_t dkdv_smem() {
                           2 * C * (C + 1) + C + 1);
 }
 
+// Asynchronous copy of rows [0, cb) of a C-row tile (row length W, type T)
+// into `raw` (C x W, dense), 16 bytes per copy; rows >= cb are filled with
+// zeros (a zero-byte source read from row 0, which exists).
+template <typename T, int W>
+__device__ __forceinline__ void stage_tile(T *raw, const T *src, int cb) {
+  constexpr int PER = 16 / (int)sizeof(T), CH = W / PER;
+  for (int idx = threadIdx.x; idx < C * CH; idx += NT) {
+    const int r = idx / CH, ch = idx % CH;
+    const T *s = src + (int64_t)(r < cb ? r : 0) * W + ch * PER;
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(raw + r * W + ch * PER);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(s),
+                 "r"(r < cb ? 16 : 0)
+                 : "memory");
+  }
+}
+__device__ __forceinline__ void stage_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void stage_wait() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// fp32 copy of a staged tile into a padded tile (row stride ld).
+template <typename T, int W>
+__device__ __forceinline__ void unstage_tile(float *dst, int ld, const T *raw) {
+  for (int idx = threadIdx.x; idx < C * W; idx += NT) {
+    const int r = idx / W, c = idx % W;
+    dst[r * ld + c] = io<T>::ld(raw + idx);
+  }
+}
+
 // ------------------------------------------------------------ d lambda
 // Gradient of sum(o * dO) with respect to lambda_h, added into dlam[h].
 // With the carried states at the start of a block of rows p.. (local t, j):
@@ -526,9 +553,10 @@ template <int D, int E> constexpr size_t dkdv_smem() {
 // g.nst sub-chunks of Ls rows before the last chunk: writes sub-chunk u's
 // (dKV, dW) to workspace slot u+1 of the (b,h)'s wsS slots.  The gradient
 // pass's chunk c (Lc = M Ls rows) enters with the pair in slot c M.
-template <int D, int E>
+template <typename T, int D, int E>
 constexpr size_t dlam_smem() {
-  return sizeof(float) * (2 * C * (D + 1) + 2 * C * (E + 1) + (C + 2)) + sizeof(double) * (NT / 32);
+  return sizeof(float) * (2 * C * (D + 1) + 2 * C * (E + 1) + (C + 2)) + sizeof(double) * (NT / 32) +
+         16 + sizeof(T) * (2 * C * D + 2 * C * E);
 }
 
 template <typename T, int D, int E, bool STATE>
@@ -546,6 +574,11 @@ dlambda_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__rest
   float *Gs = Vs + C * LV;         // C x LV   dO
   float *pw = Gs + C * LV;         // C+1
   double *red = reinterpret_cast<double *>(pw + C + 2);  // NT/32
+  // the next block's rows in flight while the current one is computed (16-
+  // byte aligned: the copies move 16 bytes; every row is a multiple of 16)
+  T *rQ = reinterpret_cast<T *>((reinterpret_cast<uintptr_t>(red + NT / 32) + 15) &
+                                ~static_cast<uintptr_t>(15));  // C x D each, then C x E
+  T *rK = rQ + C * D, *rV = rK + C * D, *rG = rV + C * E;
 
   const int nch = STATE ? g.nst : g.S;
   const int64_t len = STATE ? g.Ls : g.Lc;
@@ -578,15 +611,26 @@ dlambda_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__rest
       }
   }
   double acc = 0.0;
-  __syncthreads();
+  auto stage = [&](int64_t p) {
+    const int cb = (int)(b - p < C ? b - p : C);
+    if (!STATE) stage_tile<T, D>(rQ, q + (bh * g.L + p) * D, cb);
+    stage_tile<T, D>(rK, k + (bh * g.L + p) * D, cb);
+    stage_tile<T, E>(rV, v + (bh * g.L + p) * E, cb);
+    if (!STATE) stage_tile<T, E>(rG, dO + (bh * g.L + p) * E, cb);
+    stage_commit();
+  };
+  if (a < b) stage(a);
 
   for (int64_t p = a; p < b; p += C) {
     const int cb = (int)(b - p < C ? b - p : C);
-    if (!STATE) load_tile<T, D>(Qs, LQ, q + (bh * g.L + p) * D, cb);
-    load_tile<T, D>(Ks, LQ, k + (bh * g.L + p) * D, cb);
-    load_tile<T, E>(Vs, LV, v + (bh * g.L + p) * E, cb);
-    if (!STATE) load_tile<T, E>(Gs, LV, dO + (bh * g.L + p) * E, cb);
+    stage_wait();
+    __syncthreads();  // the block's rows have landed; the previous block is done
+    if (!STATE) unstage_tile<T, D>(Qs, LQ, rQ);
+    unstage_tile<T, D>(Ks, LQ, rK);
+    unstage_tile<T, E>(Vs, LV, rV);
+    if (!STATE) unstage_tile<T, E>(Gs, LV, rG);
     __syncthreads();
+    if (p + C < b) stage(p + C);
     if (!STATE) {
       float part = 0.f;
       // the earlier rows: lambda^t ((t+1) q_t KV dO_t + q_t W dO_t), the
@@ -667,7 +711,6 @@ dlambda_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__rest
         }
       }
     }
-    __syncthreads();
   }
   if constexpr (STATE) {
     float *okv = ws + ((bh * g.wsS + c + 1) * 2) * (int64_t)D * E, *ow = okv + D * E;
