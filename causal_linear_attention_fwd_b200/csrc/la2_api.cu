@@ -27,6 +27,7 @@ std::atomic<int> g_opt_path{0};
 std::atomic<int> g_opt_inject{0};
 std::atomic<int> g_opt_variant{0};
 std::atomic<int> g_opt_trace{0};
+std::atomic<int> g_opt_varlen_order{0};
 
 // ------------------------------------------------------------ profiling
 enum KernelId {
@@ -149,6 +150,7 @@ Path choose_path(int d, int e, la2_dtype dt) {
 Geo plan(int B, int H, int64_t L, int blk, Path path) {
   Geo g;
   g.cu = nullptr;
+  g.lpt = 0;
   g.slots = nullptr;
   g.pool = 0;
   g.inject = 0;
@@ -468,6 +470,7 @@ int la2_set_option(int option, int value) {
   if (option == LA2_OPT_INJECT_TIMEOUT) return g_opt_inject.exchange(value);
   if (option == LA2_OPT_VARIANT) return g_opt_variant.exchange(value);
   if (option == LA2_OPT_TRACE) return g_opt_trace.exchange(value);
+  if (option == LA2_OPT_VARLEN_ORDER) return g_opt_varlen_order.exchange(value);
   return -1;
 }
 
@@ -614,6 +617,7 @@ Geo plan_varlen(int N, int H, int64_t T, const int64_t *cu) {
   g.nst = 0;
   g.c0 = 0;
   g.cu = cu;
+  g.lpt = N <= 64 && g_opt_varlen_order.load() == 0;
   g.slots = nullptr;
   g.pool = 0;
   g.inject = 0;

@@ -48,6 +48,10 @@ struct Geo {
   // n owning rows [cu[n], cu[n+1]) of every head's slab of L rows; tensors
   // are [H, L, d|e], states [N, H, d, e]; S = 1.
   const int64_t *cu;
+  // Packed batch of at most 64 sequences: the tensor-core passes take the
+  // sequences longest first (list scheduling of unequal CTAs), see
+  // lpt_sequence.
+  int lpt;
   // State pool (NULL otherwise): the initial / final state of (b,h) is
   // pool state slots[b] * H + h of the kv0 / kv_out arrays, [pool, H, d, e];
   // a negative slot means none (zero initial state, final state dropped).
@@ -67,9 +71,11 @@ struct Span {
   int64_t bh, slab, a, b;
   int h, c;
 };
-__device__ __forceinline__ Span span_of(const Geo &g, int nch, int c_first) {
+// seq >= 0 (packed batch, one CTA per (sequence, head)): the CTA serves that
+// sequence and head blockIdx.x % H instead of its own index's sequence.
+__device__ __forceinline__ Span span_of(const Geo &g, int nch, int c_first, int64_t seq = -1) {
   Span s;
-  const int64_t q = blockIdx.x / nch;
+  const int64_t q = seq >= 0 ? seq * g.H + blockIdx.x % g.H : blockIdx.x / nch;
   s.bh = q;
   s.h = (int)(q % g.H);
   s.c = (int)(blockIdx.x % nch) + c_first;
@@ -88,6 +94,26 @@ __device__ __forceinline__ Span span_of(const Geo &g, int nch, int c_first) {
     s.b = g.L < s.a + g.Lc ? g.L : s.a + g.Lc;
   }
   return s;
+}
+
+// Longest-first order of a packed batch of N <= 64 sequences (ties in index
+// order), computed by one warp from the offsets: the index of the sequence
+// whose rank is R.  The lengths stay in registers (lane i holds sequences i
+// and i + 32) and each lane counts the sequences that precede its own in
+// the order; the order is total, so every rank names exactly one sequence.
+__device__ __forceinline__ int lpt_sequence(const int64_t *cu, int N, int R) {
+  const int lane = threadIdx.x & 31;
+  const int64_t l0 = lane < N ? cu[lane + 1] - cu[lane] : -1;
+  const int64_t l1 = lane + 32 < N ? cu[lane + 33] - cu[lane + 32] : -1;
+  int r0 = 0, r1 = 0;
+  for (int m = 0; m < N; m++) {
+    const int64_t lm = __shfl_sync(0xffffffffu, m < 32 ? l0 : l1, m & 31);
+    r0 += (lm > l0) || (lm == l0 && m < lane);
+    r1 += (lm > l1) || (lm == l1 && m < lane + 32);
+  }
+  const unsigned h0 = __ballot_sync(0xffffffffu, lane < N && r0 == R);
+  const unsigned h1 = __ballot_sync(0xffffffffu, lane + 32 < N && r1 == R);
+  return h0 ? __ffs(h0) - 1 : (h1 ? 31 + __ffs(h1) : 0);
 }
 
 // Index of (b,h)'s state in the kv0 / kv_out arrays: bh itself, or through

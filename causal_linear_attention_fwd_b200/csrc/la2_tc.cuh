@@ -623,7 +623,16 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   int64_t bh, a, b, slab;
   int c, h;
   if constexpr (VARLEN) {
-    const Span sp = span_of(g, 1, 0);
+    int64_t seq = -1;
+    if (g.lpt) {  // longest sequences first
+      if (warp == 0) {
+        const int n = lpt_sequence(g.cu, g.B, (int)(blockIdx.x / g.H));
+        if (lane == 0) tmem_slot[2] = (uint32_t)n;
+      }
+      __syncthreads();
+      seq = tmem_slot[2];
+    }
+    const Span sp = span_of(g, 1, 0, seq);
     bh = sp.bh, a = sp.a, b = sp.b, slab = sp.slab, c = sp.c, h = sp.h;
   } else {
     bh = blockIdx.x / nch;

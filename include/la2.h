@@ -376,11 +376,15 @@ const char *la2_status_string(la2_status s);
  * of tensor-core pass p (0 forward, 1 dQ, 2 forward chunk state, 3 dV,
  * 4 dK, 5 reverse chunk state) of the warp-specialised kernel stamps the
  * device clock at fixed points of each block into the trace buffer (see
- * la2_trace_read).  Returns the previous value, or -1 for an unknown option.
+ * la2_trace_read).  LA2_OPT_VARLEN_ORDER: 0 (default) = the tensor-core
+ * passes of a packed batch of at most 64 sequences start the longest
+ * sequences first (each CTA ranks the lengths from cu_seqlens on the device),
+ * so that short ones fill the last wave; 1 = in the given order.  Returns the
+ * previous value, or -1 for an unknown option.
  */
 enum {
     LA2_OPT_SPLIT = 0, LA2_OPT_PATH = 1, LA2_OPT_INJECT_TIMEOUT = 2, LA2_OPT_VARIANT = 3,
-    LA2_OPT_TRACE = 4
+    LA2_OPT_TRACE = 4, LA2_OPT_VARLEN_ORDER = 5
 };
 
 /*

@@ -146,3 +146,52 @@ def test_varlen_bench_batch_sampled(orc):
             check(f"{tag} o", o[hh, a:b], o_ref[0, 0], torch.bfloat16)
             for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), g[:3]):
                 check(f"{tag} {name}", got[hh, a:b], ref[0, 0], torch.bfloat16)
+
+
+def _varlen_all(x, kv0, cu, lam, order):
+    """Every output of a packed forward + backward with the given CTA order
+    option; outputs pre-filled with NaN, so a (sequence, head) that no CTA
+    served would show."""
+    H, T, d = x["q"].shape
+    e = x["v"].shape[-1]
+    N = cu.numel() - 1
+    nan = lambda *s: torch.full(s, float("nan"), dtype=x["q"].dtype, device=DEV)
+    o = nan(H, T, e)
+    outs = (nan(H, T, d), nan(H, T, d), nan(H, T, e))
+    old = la2.set_option(la2.LA2_OPT_VARLEN_ORDER, order)
+    try:
+        _, st = la2.forward_varlen(x["q"], x["k"], x["v"], lam, cu, kv0, want_state=True, out=o)
+        g = la2.backward_varlen(x["q"], x["k"], x["v"], lam, cu, x["dO"], kv0, want_dkv0=True,
+                                outs=outs)
+        torch.cuda.synchronize()
+    finally:
+        la2.set_option(la2.LA2_OPT_VARLEN_ORDER, old)
+    assert la2.last_device_error() == 0
+    assert N > 0
+    return (o, st) + tuple(g)
+
+
+def test_varlen_longest_first_is_a_reordering():
+    """Longest-first CTA order (the default for <= 64 sequences; lengths with
+    ties, an empty and a one-row sequence) serves every (sequence, head) once
+    with the same arithmetic: results bitwise equal to the given order's."""
+    lens = [300, 0, 1, 1000, 128, 1000, 5, 256, 129, 300, 2000, 7]
+    x, kv0, cu = packed_inputs(lens, 4, 128, 128, torch.bfloat16, seed=11)
+    lam = inputs.decay_lambdas(4, DEV)
+    a = _varlen_all(x, kv0, cu, lam, 0)
+    b = _varlen_all(x, kv0, cu, lam, 1)
+    for name, u, w in zip(("o", "kv_out", "dq", "dk", "dv", "dkv0"), a, b):
+        assert not torch.isnan(u).any(), name
+        assert torch.equal(u, w), name
+
+
+def test_varlen_many_sequences_matches_oracle(orc):
+    """70 sequences (above the longest-first limit: the given order), lengths
+    0..400 rows, against the oracle per sequence."""
+    lens = [int(v) for v in np.random.default_rng(70).integers(0, 400, size=70)]
+    x, kv0, cu = packed_inputs(lens, 2, 128, 128, torch.bfloat16, seed=12)
+    lam = inputs.decay_lambdas(2, DEV)
+    got = _varlen_all(x, kv0, cu, lam, 0)
+    ref = reference(orc, x, kv0, cu, lam)
+    for name, u, r in zip(("o", "kv_out", "dq", "dk", "dv", "dkv0"), got, ref):
+        check(f"70 sequences {name}", u, r, torch.bfloat16)
