@@ -28,19 +28,21 @@ std::atomic<int> g_opt_inject{0};
 std::atomic<int> g_opt_variant{0};
 std::atomic<int> g_opt_trace{0};
 std::atomic<int> g_opt_varlen_order{0};
+std::atomic<int> g_opt_decode_block{0};
 
 // ------------------------------------------------------------ profiling
 enum KernelId {
   K_SIMT_FWD_STATE, K_SIMT_FWD_SCAN, K_SIMT_FWD, K_SIMT_DQ, K_SIMT_REV_STATE,
   K_SIMT_REV_SCAN, K_SIMT_DKDV, K_DECODE, K_TC_FWD_STATE, K_TC_FWD, K_TC_DQ,
   K_TC_REV_STATE, K_TC_DV, K_TC_DK, K_SCAN_FWD, K_SCAN_REV, K_SIMT_DLAMBDA,
-  K_SIMT_DLAMBDA_STATE, K_SIMT_DLAMBDA_SCAN, K_COUNT
+  K_SIMT_DLAMBDA_STATE, K_SIMT_DLAMBDA_SCAN, K_TC_DECODE_UNITS, K_COUNT
 };
 const char *kKernelName[K_COUNT] = {
     "simt_fwd_chunk_state", "simt_scan_fwd", "simt_fwd", "simt_dq",
     "simt_rev_chunk_state", "simt_scan_rev", "simt_dkdv", "decode_step",
     "tc_fwd_chunk_state", "tc_fwd", "tc_dq", "tc_rev_chunk_state", "tc_dv", "tc_dk",
-    "scan_fwd", "scan_rev", "simt_dlambda", "simt_dlambda_chunk_state", "simt_dlambda_scan"};
+    "scan_fwd", "scan_rev", "simt_dlambda", "simt_dlambda_chunk_state", "simt_dlambda_scan",
+    "tc_decode_units"};
 
 struct ProfRec {
   int kid;
@@ -364,11 +366,13 @@ la2_status to_status(cudaError_t e) { return e == cudaSuccess ? LA2_OK : LA2_ERR
 
 }  // namespace
 
-// Tokens per request from which la2_decode_tokens runs one block of the
-// chunk schedule instead of the token-by-token kernel (measured crossover
-// on B200: ~1.2 ms per call for the block at batch 256 x 64 heads, against
-// 1.8 ms for 32 tokens by the register kernel).
-constexpr int kDecodeBlockTokens = 32;
+// Tokens per request from which la2_decode_tokens runs the tensor-core
+// block form (one block of the chunk schedule per request) instead of the
+// token-by-token register update.  Measured on B200 at batch 256 x 64 heads:
+// the decode-unit kernel takes ~0.93 ms per call for any T <= 128 (148 CTAs,
+// ~110 units each, set by each unit's state round trip), the token kernel
+// 0.41 ms at T = 4, 0.62 at 8, 0.96 at 16 and 1.77 at 32.
+constexpr int kDecodeBlockTokens = 16;
 
 // ------------------------------------------------------- d lambda helper
 // dlam = 0; split: chunk-state pre-pass over the sub-chunks of chunks
@@ -471,6 +475,7 @@ int la2_set_option(int option, int value) {
   if (option == LA2_OPT_VARIANT) return g_opt_variant.exchange(value);
   if (option == LA2_OPT_TRACE) return g_opt_trace.exchange(value);
   if (option == LA2_OPT_VARLEN_ORDER) return g_opt_varlen_order.exchange(value);
+  if (option == LA2_OPT_DECODE_BLOCK_TOKENS) return g_opt_decode_block.exchange(value);
   return -1;
 }
 
@@ -1005,17 +1010,27 @@ la2_status la2_decode_tokens(const void *q, const void *k, const void *v, const 
                             {o, BH * T * e * es}};
   if (any_overlap(outs, ins)) return LA2_ERR_INVALID;
   // From kDecodeBlockTokens tokens per request on, one block of the chunk
-  // schedule (tensor cores, the state read and written once) beats the
-  // token-by-token register update; the [B,H,T,.] layout is the forward's.
-  if (T >= kDecodeBlockTokens && choose_path(d, e, dt) == PATH_TC) {
+  // schedule (tensor cores, the state read and written once per call) beats
+  // the token-by-token register update; the [B,H,T,.] layout is the
+  // forward's.
+  const int from = g_opt_decode_block.load() > 0 ? g_opt_decode_block.load() : kDecodeBlockTokens;
+  if (T >= from && choose_path(d, e, dt) == PATH_TC) {
     Geo g = plan(B, H, T, block_rows(PATH_TC), PATH_TC);
+    g.slots = slots;
+    g.pool = pool_size;
+    g.variant = 0;
+    // up to one block per request: one CTA per SM walks (request, head)
+    // units back to back (a range of units spans at most two heads)
+    const int64_t P = BH < device_sms() ? BH : device_sms();
+    if (T <= la2::tc::BLOCK && (BH + P - 1) / P <= B) {
+      g.L = T;
+      return to_status(la2::tc::decode_units(q, k, v, lambda, kv_pool, o, g, (int)P, stream,
+                                             [&](int, auto &&fn) { return timed(K_TC_DECODE_UNITS, stream, fn); }));
+    }
     g.S = 1;  // one chunk per request: no workspace
     g.Lc = g.Ls = T;
     g.M = g.Ssub = g.wsS = 1;
     g.nst = 0;
-    g.slots = slots;
-    g.pool = pool_size;
-    g.variant = 0;
     return to_status(la2::tc::forward(q, k, v, lambda, kv_pool, o, kv_pool, nullptr, g, stream,
                                       [&](int, auto &&fn) { return timed(K_TC_FWD, stream, fn); }));
   }

@@ -528,8 +528,8 @@ template <int MODE> struct Layout2 {
   static constexpr uint32_t NBAR = 5 * NSTAGE + 5;
   static constexpr uint32_t AB_BYTES = OUT ? 2 * TILE : TILE;
   static constexpr uint32_t C_OFF = AB_BYTES;
-  // decay table: 128 zeros then lambda^0..lambda^128 (see chunk_kernel2)
-  static constexpr uint32_t MISC_BYTES = 8 * NBAR + 16 + 4 * (2 * BLOCK + 1);
+  // decay tables: twice 32 zeros then lambda^0..lambda^128 (see chunk_kernel2)
+  static constexpr uint32_t MISC_BYTES = 8 * NBAR + 16 + 4 * 2 * (32 + BLOCK + 1);
   static constexpr uint32_t SMEM = MISC + MISC_BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = OUT ? 512 : 128;
   static constexpr uint32_t COL_O = 256;
@@ -578,7 +578,14 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 // sequence's last block reads the next sequence's rows, so the reverse
 // passes mask the columns past the block's end and that block's output rows
 // go out by plain stores (`outp`) instead of a TMA box.
-template <int MODE, bool TRACE, bool VARLEN>
+// KIND: 0 the plain form, 1 the packed (VARLEN) form, 2 the decode-unit form
+// (forward only): the B*H (request, head) units of a call of T <= 128 tokens
+// per request, head-major, cut into gridDim.x contiguous ranges; each unit is
+// one block with its own state, read from and written back to the state
+// pool, so one CTA per SM walks ~B*H/SMs units back to back (a range spans
+// at most two heads: two decay tables).
+constexpr int KIND_PLAIN = 0, KIND_VARLEN = 1, KIND_UNITS = 2;
+template <int MODE, bool TRACE, int KIND>
 __global__ void __launch_bounds__(NT2, 1)
 chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
               const __grid_constant__ CUtensorMap tm2, const __grid_constant__ CUtensorMap tmo,
@@ -587,6 +594,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
               Geo g) {
   using LY = Layout2<MODE>;
   using TR = Traits<MODE>;
+  constexpr bool VARLEN = KIND == KIND_VARLEN, UNITS = KIND == KIND_UNITS;
   constexpr bool OUT = LY::OUT;
   constexpr bool REV = TR::REV;
   constexpr int NS = LY::NSTAGE;
@@ -603,11 +611,14 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + LY::MISC);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + LY::NBAR);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  // pwz[k] = lambda^(k-128) for k >= 128, 0 below: pw = pwz + 128 holds
-  // lambda^0..lambda^128 and pw[n] for n in [-128, 0) reads as 0, which is
-  // the causal mask (a negative distance means a masked entry).
+  // pwz[k] = lambda^(k-32) for 32 <= k <= 160, 0 below: pw = pwz + 32 holds
+  // lambda^0..lambda^128 and pw[n] for n in [-32, 0) reads as 0, which is
+  // the causal mask (a negative distance means a masked entry; the mask
+  // looks up distances down to -31).  pw2, laid out the same way after
+  // another 32 zeros, is the next head's table (decode-unit form).
   float *pwz = reinterpret_cast<float *>(tmem_slot + 4);
-  float *pw = pwz + 128;
+  float *pw = pwz + 32;
+  float *pw2 = pw + (BLOCK + 1) + 32;
   const uint32_t b_fab = smem_u32(bars);
   const uint32_t b_fc = b_fab + 8 * NS;
   const uint32_t b_eab = b_fc + 8 * NS;
@@ -622,7 +633,17 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   const int nch = OUT ? g.S : g.nst;
   int64_t bh, a, b, slab;
   int c, h;
-  if constexpr (VARLEN) {
+  int64_t u0 = 0;  // decode-unit form: the CTA's units [u0, u0 + nblk)
+  if constexpr (UNITS) {
+    const int64_t U = (int64_t)g.B * g.H;
+    u0 = (int64_t)blockIdx.x * U / gridDim.x;
+    const int64_t u1 = ((int64_t)blockIdx.x + 1) * U / gridDim.x;
+    bh = slab = 0;
+    c = 0;
+    h = (int)(u0 / g.B);  // the range's first head
+    a = 0;
+    b = u1 - u0;  // one block per unit
+  } else if constexpr (VARLEN) {
     int64_t seq = -1;
     if (g.lpt) {  // longest sequences first
       if (warp == 0) {
@@ -645,12 +666,27 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
     // pool (reported by state_slot): no rows
     if (MODE == MODE_FWD && g.slots && (unsigned)g.slots[bh / g.H] >= (unsigned)g.pool) b = a;
   }
-  const int nblk = (int)((b - a + BLOCK - 1) / BLOCK);
+  const int nblk = UNITS ? (int)(b - a) : (int)((b - a + BLOCK - 1) / BLOCK);
   auto block_of = [&](int j) { return REV ? nblk - 1 - j : j; };
-  auto p_of = [&](int j) { return a + (int64_t)block_of(j) * BLOCK; };
+  auto p_of = [&](int j) { return UNITS ? (int64_t)0 : a + (int64_t)block_of(j) * BLOCK; };
   auto cb_of = [&](int j) {
-    const int64_t r = b - p_of(j);
+    const int64_t r = (UNITS ? g.L : b) - p_of(j);
     return (int)(r < BLOCK ? r : BLOCK);
+  };
+  // decode-unit form: block j is unit u0 + j = (head, request), head-major
+  auto unit_head = [&](int j) { return (u0 + j) / g.B; };
+  auto slab_of = [&](int j) -> int64_t {
+    if constexpr (UNITS) {
+      const int64_t hh = unit_head(j);
+      return (u0 + j - hh * g.B) * g.H + hh;
+    } else {
+      return slab;
+    }
+  };
+  // the decay table of block j's head
+  auto tab_of = [&](int j) -> const float * {
+    if constexpr (UNITS) return unit_head(j) == h ? pw : pw2;
+    else return pw;
   };
   // trace events: 0 load issued, 1 S issued, 2 P.B2/X/state issued, 3 mask
   // start, 4 mask done, 5 epilogue start, 6 state handed back, 7 store read
@@ -663,7 +699,12 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
     g_trace[10 * kTraceBlocks + blockIdx.x] = globaltimer();
 
   if (tid <= BLOCK) pw[tid] = (float)pow_int((double)lambda[h], tid);
-  if (tid < BLOCK) pwz[tid] = 0.f;
+  if (tid < 32) {
+    pwz[tid] = 0.f;
+    pw[BLOCK + 1 + tid] = 0.f;
+  }
+  if (UNITS && tid > BLOCK && tid <= 2 * BLOCK + 1)
+    pw2[tid - BLOCK - 1] = (float)pow_int((double)lambda[h + 1 < g.H ? h + 1 : h], tid - BLOCK - 1);
   if (tid == 0) {
     for (int s = 0; s < NS; s++) {
       mbar_init(b_fab + 8 * s, 1);
@@ -703,7 +744,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
       for (int j = 0; j < nblk; j++) {
         const int st = j % NS;
         const uint32_t ph = (uint32_t)((j / NS - 1) & 1);
-        const int y = (int)p_of(j), z = (int)slab;
+        const int y = (int)p_of(j), z = (int)slab_of(j);
         uint32_t dst = sbase + st * LY::STAGE;
         // (A0, B1): their slots free once block j-NS's products are done
         if (j >= NS && !mbar_wait(b_eab + 8 * st, ph, abort_flag)) break;
@@ -850,9 +891,14 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
-    const float lam1 = pw[1], lam2 = pw[2];
+    float lam1 = pw[1], lam2 = pw[2];
     for (int i = 0; OUT && i < nblk; i++) {
       const int st = i % NS;
+      const float *pt = tab_of(i);
+      if constexpr (UNITS) {
+        lam1 = pt[1];
+        lam2 = pt[2];
+      }
       bool ok = mbar_wait(b_sfull + 8 * (i & 1), (uint32_t)((i >> 1) & 1), abort_flag);
       // a warp vote suffices: no later step syncs the mask warps together
       if (__any_sync(0xffffffffu, !ok)) break;
@@ -883,12 +929,12 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
             for (int j = 0; j < 16; j++) {
               // distance < 0 reads 0 from the table: the causal mask
               const int n0 = REV ? 2 * j - lane : lane - 2 * j;
-              const float f0 = __uint_as_float(r[2 * j]) * pw[n0];
-              const float f1 = __uint_as_float(r[2 * j + 1]) * pw[REV ? n0 + 1 : n0 - 1];
+              const float f0 = __uint_as_float(r[2 * j]) * pt[n0];
+              const float f1 = __uint_as_float(r[2 * j + 1]) * pt[REV ? n0 + 1 : n0 - 1];
               pk[j] = pack_bf16x2(f0, f1);
             }
           } else {
-            const float a = REV ? pw[32 * part - row] : pw[row - 32 * part - 31];
+            const float a = REV ? pt[32 * part - row] : pt[row - 32 * part - 31];
             // xe, xo: factors of the pair's even and odd column
             float xe = REV ? a : a * lam1, xo = REV ? a * lam1 : a;
 #pragma unroll
@@ -914,25 +960,9 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
     const int wtid = tid - 6 * 32;  // 0..127
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     uint8_t *kvbf = smem + LY::KVBF;
-    // initial state: TMEM (already decayed for block 0's update), bf16 copy
-    {
-      const float *init = nullptr;
-      if (MODE == MODE_FWD || MODE == MODE_DQ) {
-        // a split pass reads every chunk's entry state from the workspace (the
-        // scan put the initial one in slot 0), never kv0, which kv_out may reuse
-        if (g.S > 1) {
-          init = ws + (bh * g.wsS + (int64_t)c * g.M) * (int64_t)128 * 128;
-        } else {
-          const int64_t so = state_slot(g, bh);
-          init = (kv0 && so >= 0) ? kv0 + so * 128 * 128 : nullptr;
-        }
-      } else if (MODE == MODE_DV || MODE == MODE_DK) {
-        // the last chunk starts from the reverse state past the sequence end
-        // (kv0 carries it in the reverse passes; NULL: zero)
-        if (c != g.S - 1) init = ws + (bh * g.wsS + (int64_t)(c + 1) * g.M - 1) * (int64_t)128 * 128;
-        else init = kv0 ? kv0 + bh * 128 * 128 : nullptr;
-      }
-      const float dec = pw[nblk > 0 ? cb_of(0) : 0];
+    // a state into TMEM (already decayed by `dec` for its first block's
+    // update) and, output passes, its bf16 operand copy; NULL: zero
+    auto load_state = [&](const float *init, float dec) {
 #pragma unroll
       for (int part = 0; part < 4; part++) {
         float f[32];
@@ -953,6 +983,33 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
         for (int j = 0; j < 32; j++) r[j] = __float_as_uint(f[j] * dec);
         tmem_st32(tl + LY::COL_KV + part * 32, r);
       }
+    };
+    // decode-unit form: block j's state in the pool (NULL: inactive request)
+    auto unit_state = [&](float *pool, int j) -> float * {
+      const int64_t so = state_slot(g, slab_of(j));
+      return (pool && so >= 0) ? pool + so * 128 * 128 : nullptr;
+    };
+    // initial state: TMEM (already decayed for block 0's update), bf16 copy
+    {
+      const float *init = nullptr;
+      if (UNITS) {
+        init = nblk > 0 ? unit_state(const_cast<float *>(kv0), 0) : nullptr;
+      } else if (MODE == MODE_FWD || MODE == MODE_DQ) {
+        // a split pass reads every chunk's entry state from the workspace (the
+        // scan put the initial one in slot 0), never kv0, which kv_out may reuse
+        if (g.S > 1) {
+          init = ws + (bh * g.wsS + (int64_t)c * g.M) * (int64_t)128 * 128;
+        } else {
+          const int64_t so = state_slot(g, bh);
+          init = (kv0 && so >= 0) ? kv0 + so * 128 * 128 : nullptr;
+        }
+      } else if (MODE == MODE_DV || MODE == MODE_DK) {
+        // the last chunk starts from the reverse state past the sequence end
+        // (kv0 carries it in the reverse passes; NULL: zero)
+        if (c != g.S - 1) init = ws + (bh * g.wsS + (int64_t)(c + 1) * g.M - 1) * (int64_t)128 * 128;
+        else init = kv0 ? kv0 + bh * 128 * 128 : nullptr;
+      }
+      load_state(init, tab_of(0)[nblk > 0 ? cb_of(0) : 0]);
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
@@ -990,8 +1047,11 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
         }
       }
       if (wtid == 0) LA2_TRACE(15, i);
-      const bool last = i == nblk - 1;
-      const float dec = last ? 1.f : pw[cb_of(i + 1)];
+      // every unit of the decode-unit form ends with its only block
+      const bool last = UNITS || i == nblk - 1;
+      const float dec = last ? 1.f : tab_of(i + 1)[cb_of(i + 1)];
+      float *dst_i = dst;
+      if constexpr (UNITS) dst_i = unit_state(kv_out, i);
 #pragma unroll
       for (int pair = 0; pair < 2; pair++) {
         uint32_t r[64];
@@ -1007,12 +1067,25 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
           for (int j = 0; j < 64; j++) r[j] = __float_as_uint(__uint_as_float(r[j]) * dec);
           tmem_st32(tl + LY::COL_KV + pair * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
           tmem_st32(tl + LY::COL_KV + pair * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-        } else if (dst) {
-          float4 *d4 = reinterpret_cast<float4 *>(dst + (int64_t)row * 128 + pair * 64);
+        } else if (dst_i) {
+          float4 *d4 = reinterpret_cast<float4 *>(dst_i + (int64_t)row * 128 + pair * 64);
 #pragma unroll
           for (int j = 0; j < 16; j++)
             d4[j] = make_float4(dscale * __uint_as_float(r[4 * j]), dscale * __uint_as_float(r[4 * j + 1]),
                                 dscale * __uint_as_float(r[4 * j + 2]), dscale * __uint_as_float(r[4 * j + 3]));
+        }
+      }
+      if constexpr (UNITS) {
+        // the next unit's state (its rows were prefetched into L2 a block
+        // ago), and the one after it on its way to L2
+        if (i + 1 < nblk) load_state(unit_state(const_cast<float *>(kv0), i + 1), tab_of(i + 1)[cb_of(i + 1)]);
+        if (i + 2 < nblk) {
+          const float *nx = unit_state(const_cast<float *>(kv0), i + 2);
+          if (nx) {
+#pragma unroll
+            for (int k = 0; k < 4; k++)
+              asm volatile("prefetch.global.L2 [%0];" ::"l"(nx + (int64_t)row * 128 + k * 32));
+          }
         }
       }
       tmem_wait_st();
@@ -1039,9 +1112,10 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
         }
       }
       if (wtid == 0) {
-        if (OUT && !tail_rows) {
+        // (an inactive request of the decode-unit form keeps its outputs)
+        if (OUT && !tail_rows && (!UNITS || unit_state(kv_out, i))) {
           const uint32_t sst = sbase + st * LY::STAGE + LY::C_OFF;
-          const int y = (int)p_of(i), z = (int)slab;
+          const int y = (int)p_of(i), z = (int)slab_of(i);
           tma_store_3d(&tmo, sst, 0, y, z);
           tma_store_3d(&tmo, sst + BOX, 64, y, z);
           tma_store_commit();
@@ -1072,12 +1146,13 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
                           : mbar_wait(b_fab + 8 * st, (uint32_t)((j / NS) & 1), abort_flag);
       if (__any_sync(0xffffffffu, !ok)) break;  // as for the mask warps
       uint8_t *stage = smem + st * LY::STAGE;
+      const float *pt = tab_of(j);
       if (OUT) {
-        const float f = REV ? (row < cbj ? pw[cbj - row] : 0.f) : pw[row + 1];
+        const float f = REV ? (row < cbj ? pt[cbj - row] : 0.f) : pt[row + 1];
         scale_row2_sw128(stage, row, __float2bfloat162_rn(f));
       }
       uint8_t *B1 = OUT ? stage + TILE : stage;
-      const float fb = row < cbj ? (REV ? pw[row] : pw[cbj - 1 - row]) : 0.f;
+      const float fb = row < cbj ? (REV ? pt[row] : pt[cbj - 1 - row]) : 0.f;
       scale_row2_sw128(B1, row, __float2bfloat162_rn(fb));
       fence_proxy_async_smem();
       __syncwarp();
@@ -1146,9 +1221,9 @@ cudaError_t launch_chunk(const CUtensorMap &m0, const CUtensorMap &m1, const CUt
     return cudaGetLastError();
   }
   using LY = Layout2<MODE>;
-  auto k = g.trace == MODE ? chunk_kernel2<MODE, true, false> : chunk_kernel2<MODE, false, false>;
+  auto k = g.trace == MODE ? chunk_kernel2<MODE, true, KIND_PLAIN> : chunk_kernel2<MODE, false, KIND_PLAIN>;
   if constexpr (LY::OUT) {
-    if (g.cu) k = chunk_kernel2<MODE, false, true>;
+    if (g.cu) k = chunk_kernel2<MODE, false, KIND_VARLEN>;
   }
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::SMEM);
   if (e != cudaSuccess) return e;
@@ -1228,6 +1303,31 @@ cudaError_t backward(const void *q, const void *k, const void *v, const float *l
   err = timed(5, [&] { launch_chunk<MODE_DV>(mk, mq, mg, mdv, lam, dend, wsr, dkv0, g, st); });
   if (err) return err;
   return timed(6, [&] { launch_chunk<MODE_DK>(mv, mg, mq, mdk, lam, dend, wsr, nullptr, g, st); });
+}
+
+// Decode units: T <= 128 new tokens for each of B requests x H heads, [B,H,T,.]
+// tensors, the state of (b,h) in the pool at slot slots[b] (b without a
+// table) read and written in place; `ctas` CTAs walk the B*H units, head-
+// major, one block each (the decode-unit form of chunk_kernel2).
+template <typename Timed>
+cudaError_t decode_units(const void *q, const void *k, const void *v, const float *lam,
+                         float *pool, void *o, const Geo &g, int ctas, cudaStream_t st,
+                         Timed &&timed) {
+  const int64_t BH = (int64_t)g.B * g.H;
+  if (!geometry_ok(g) || g.L < 1 || g.L > BLOCK || ctas < 1 || ctas > BH)
+    return cudaErrorInvalidValue;
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map(&mq, q, BH, g.L) || !make_map(&mk, k, BH, g.L) || !make_map(&mv, v, BH, g.L) ||
+      !make_map(&mo, o, BH, g.L))
+    return cudaErrorInvalidValue;
+  using LY = Layout2<MODE_FWD>;
+  auto kern = g.trace == MODE_FWD ? chunk_kernel2<MODE_FWD, true, KIND_UNITS>
+                                  : chunk_kernel2<MODE_FWD, false, KIND_UNITS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::SMEM);
+  if (e != cudaSuccess) return e;
+  return timed(2, [&] {
+    kern<<<(unsigned)ctas, NT2, LY::SMEM, st>>>(mq, mk, mv, mo, lam, pool, nullptr, pool, nullptr, g);
+  });
 }
 
 // Chunk-state pass over every sub-chunk of a shard (a: K or Q, b: V or dO):

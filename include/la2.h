@@ -278,11 +278,14 @@ la2_status la2_backward_dlambda_ex(const void *q, const void *k, const void *v,
  * v, o [B,H,T,e]: for t = 0..T-1, kv <- lambda kv + k_t^T v_t, o_t = q_t kv
  * (the la2_decode_step recurrence applied T times), reading and writing the
  * slot's state once per call instead of once per token.  slots may be NULL:
- * request b then uses state b (pool_size >= B).  From 32 tokens per request
- * on (bf16, d = e = 128) the call runs them as one block of the chunk
- * schedule on the tensor cores (la2_forward_pool's path, one chunk per
- * request); below that, or for other shapes, token by token in registers.
- * la2_decode_step is this with T = 1, slots NULL.
+ * request b then uses state b (pool_size >= B).  From 16 tokens per request
+ * on (bf16, d = e = 128; LA2_OPT_DECODE_BLOCK_TOKENS overrides) the call runs
+ * each request's tokens as one block of the chunk schedule on the tensor
+ * cores: up to 128 tokens, one CTA per SM walks a contiguous range of the
+ * (head, request) units back to back, each unit's state read from and
+ * written back to its slot; beyond 128, la2_forward_pool's path (one chunk
+ * per request).  Below that, or for other shapes, token by token in
+ * registers.  la2_decode_step is this with T = 1, slots NULL.
  *
  * Errors as for la2_forward / la2_decode_step (LA2_ERR_INVALID also for
  * unknown flag bits, L < 1 in la2_forward_pool, a NULL slot table in
@@ -379,12 +382,15 @@ const char *la2_status_string(la2_status s);
  * la2_trace_read).  LA2_OPT_VARLEN_ORDER: 0 (default) = the tensor-core
  * passes of a packed batch of at most 64 sequences start the longest
  * sequences first (each CTA ranks the lengths from cu_seqlens on the device),
- * so that short ones fill the last wave; 1 = in the given order.  Returns the
- * previous value, or -1 for an unknown option.
+ * so that short ones fill the last wave; 1 = in the given order.
+ * LA2_OPT_DECODE_BLOCK_TOKENS: 0 (default) = la2_decode_tokens runs the
+ * tensor-core block form from the library's crossover number of tokens per
+ * request on, the token-by-token kernel below it; n > 0 = from n tokens on.
+ * Returns the previous value, or -1 for an unknown option.
  */
 enum {
     LA2_OPT_SPLIT = 0, LA2_OPT_PATH = 1, LA2_OPT_INJECT_TIMEOUT = 2, LA2_OPT_VARIANT = 3,
-    LA2_OPT_TRACE = 4, LA2_OPT_VARLEN_ORDER = 5
+    LA2_OPT_TRACE = 4, LA2_OPT_VARLEN_ORDER = 5, LA2_OPT_DECODE_BLOCK_TOKENS = 6
 };
 
 /*

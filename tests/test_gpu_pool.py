@@ -24,9 +24,13 @@ def tokens(B, H, T, d, e, dtype, seed):
     return tuple(torch.stack([s[i] for s in steps], dim=2).contiguous() for i in range(3))
 
 
-@pytest.mark.parametrize("T", [1, 3, 8, 40])
+@pytest.mark.parametrize("block_from", [0, 1])
+@pytest.mark.parametrize("T", [1, 3, 8, 40, 128, 129])
 @pytest.mark.parametrize("dtype,de", [(torch.bfloat16, (128, 128)), (torch.float32, (64, 64))])
-def test_decode_tokens_matches_oracle(orc, T, dtype, de):
+def test_decode_tokens_matches_oracle(orc, T, dtype, de, block_from):
+    """block_from: 0 = the library's crossover, 1 = the tensor-core block form
+    for every T (up to 128 tokens the decode-unit kernel, beyond it one
+    chunk-schedule CTA per request; bf16 128 x 128 only)."""
     d, e = de
     B, H, P = 6, 3, 10
     slots_h = [7, -1, 2, 9, 0, 4]
@@ -36,8 +40,12 @@ def test_decode_tokens_matches_oracle(orc, T, dtype, de):
     lam = inputs.fixed_lambdas((1.0, 0.99, 0.5), DEV)
     q, k, v = tokens(B, H, T, d, e, dtype, seed=T)
     o = torch.full((B, H, T, e), 7.0, dtype=dtype, device=DEV)
-    la2.decode_tokens(q, k, v, lam, pool, slots, out=o)
-    torch.cuda.synchronize()
+    old = la2.set_option(la2.LA2_OPT_DECODE_BLOCK_TOKENS, block_from)
+    try:
+        la2.decode_tokens(q, k, v, lam, pool, slots, out=o)
+        torch.cuda.synchronize()
+    finally:
+        la2.set_option(la2.LA2_OPT_DECODE_BLOCK_TOKENS, old)
     assert la2.last_device_error() == 0
     lam_h = lam.double().cpu().numpy()
     for b, s in enumerate(slots_h):
@@ -135,3 +143,44 @@ def test_decode_tokens_bench_batch_sampled(orc, T):
                             for t in range(T)], axis=1)
             check(f"T={T} call {c} request {b} o", outs[c][b], ref, torch.bfloat16)
         check(f"T={T} request {b} state", kv[b], st[0], torch.bfloat16)
+
+
+@pytest.mark.parametrize("T", [5, 64])
+def test_decode_units_many_per_cta(orc, T):
+    """The decode-unit kernel with several (request, head) units per CTA and
+    ranges that cross a head: 300 requests x 3 heads (900 units), a slot
+    table with inactive requests and a permuted pool; every request against
+    the oracle's decode steps, inactive outputs and unused slots untouched."""
+    d = e = 128
+    B, H, P = 300, 3, 320
+    rng = np.random.default_rng(T)
+    perm = rng.permutation(P)[:B]
+    slots_h = [int(s) if rng.random() > 0.1 else -1 for s in perm]
+    pool = inputs.decode_state0(P, H, d, e, device=DEV, seed=5)
+    pool0 = pool.clone()
+    slots = torch.tensor(slots_h, dtype=torch.int32, device=DEV)
+    lam = inputs.decay_lambdas(H, DEV)
+    q, k, v = tokens(B, H, T, d, e, torch.bfloat16, seed=100 + T)
+    o = torch.full((B, H, T, e), 7.0, dtype=torch.bfloat16, device=DEV)
+    old = la2.set_option(la2.LA2_OPT_DECODE_BLOCK_TOKENS, 1)
+    try:
+        la2.decode_tokens(q, k, v, lam, pool, slots, out=o)
+        torch.cuda.synchronize()
+    finally:
+        la2.set_option(la2.LA2_OPT_DECODE_BLOCK_TOKENS, old)
+    assert la2.last_device_error() == 0
+    lam_h = lam.double().cpu().numpy()
+    qh, kh, vh = host(q), host(k), host(v)
+    p0 = pool0.double().cpu().numpy()
+    got_o, got_p = o.float().cpu().numpy(), pool.cpu().numpy()
+    for b, s in enumerate(slots_h):
+        if s < 0:
+            assert bool((o[b] == 7.0).all())
+            continue
+        kv = p0[s:s + 1].copy()
+        ref = np.stack([orc.decode_step(qh[b:b + 1, :, t], kh[b:b + 1, :, t], vh[b:b + 1, :, t],
+                                        lam_h, kv)[0] for t in range(T)], axis=1)
+        check(f"T={T} request {b} o", got_o[b], ref, torch.bfloat16)
+        check(f"T={T} request {b} state", got_p[s], kv[0], torch.bfloat16)
+    untouched = sorted(set(range(P)) - {s for s in slots_h if s >= 0})
+    assert torch.equal(pool[untouched], pool0[untouched])
