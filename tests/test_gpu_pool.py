@@ -184,3 +184,25 @@ def test_decode_units_many_per_cta(orc, T):
         check(f"T={T} request {b} state", got_p[s], kv[0], torch.bfloat16)
     untouched = sorted(set(range(P)) - {s for s in slots_h if s >= 0})
     assert torch.equal(pool[untouched], pool0[untouched])
+
+
+def test_decode_tokens_many_heads_fall_back(orc):
+    """2 requests x 160 heads (320 units over at most one CTA per SM would
+    give a CTA more than two heads): the call falls back to one CTA per
+    (request, head), against the oracle."""
+    B, H, T, d, e = 2, 160, 40, 128, 128
+    pool = inputs.decode_state0(B, H, d, e, device=DEV, seed=6)
+    pool0 = pool.double().cpu().numpy()
+    lam = inputs.decay_lambdas(H, DEV)
+    q, k, v = tokens(B, H, T, d, e, torch.bfloat16, seed=7)
+    o = la2.decode_tokens(q, k, v, lam, pool)
+    torch.cuda.synchronize()
+    assert la2.last_device_error() == 0
+    lam_h = lam.double().cpu().numpy()
+    for b in range(B):
+        kv = pool0[b:b + 1].copy()
+        ref = np.stack([orc.decode_step(host(q[b:b + 1, :, t]), host(k[b:b + 1, :, t]),
+                                        host(v[b:b + 1, :, t]), lam_h, kv)[0]
+                        for t in range(T)], axis=1)
+        check(f"request {b} o", o[b], ref, torch.bfloat16)
+        check(f"request {b} state", pool[b], kv[0], torch.bfloat16)
