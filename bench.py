@@ -512,13 +512,30 @@ def run_long(args, world, rank, local):
                 "unit": "GB/s", "frac": round(ach / pk["hbm_gbs"], 4),
                 "traffic": traffic_for(name, Hh * L), "alg_bytes_per_launch": alg,
                 "avg_launch_ms": avg}
+    extra_cpu = {}
+    if rank == 0 and not args.no_cpu:
+        # the oracle on 16 heads x the first 65,536 rows (a quarter of the
+        # heads, 1/16 of the length): token-heads per second / 64 heads
+        import oracle
+        orc = oracle.load()
+        sl = {n: x[n][:, :16, :65536].float().cpu().numpy() for n in ("q", "k", "v")}
+        t0 = time.perf_counter()
+        orc.forward(sl["q"], sl["k"], sl["v"], lam[:16].double().cpu().numpy())
+        dt = time.perf_counter() - t0
+        extra_cpu = {"cpu_baseline": {
+            "value": round(16 * 65536 / 64 / dt, 1), "unit": "tokens/s", "cores": orc.num_threads(),
+            "kind": "oracle",
+            "sample": "forward of 16 of the 64 heads over the first 65,536 of 1,048,576 rows "
+                      f"({dt:.1f} s); token-heads/s divided by 64 heads, i.e. extrapolated to "
+                      "the full configuration at the same rate per token-head"}}
     return _common(world, args.steps, args.warmup, value, "tokens/s",
                    "long-context forward tokens/s (B=1,H=64,L=1M,d=e=128,bf16)",
                    {"workload": "long-context forward, B=1, H=64, L=1,048,576, d=e=128, bf16",
                     "l2": "inputs 16 GiB per tensor, larger than L2; no flush"}, ms,
                    {"dtype": "bf16", "roofline": roof, "kernels": prof,
                     "gpu_launches": sum(v["launches"] for v in prof.values()), "clocks": clk,
-                    "hbm_frac_fwd_min": round(1024 * Hh * value / world / 1e9 / pk["hbm_gbs"], 4)})
+                    "hbm_frac_fwd_min": round(1024 * Hh * value / world / 1e9 / pk["hbm_gbs"], 4),
+                    **extra_cpu})
 
 
 def run_varlen(args, world, rank, local):
@@ -573,6 +590,31 @@ def run_varlen(args, world, rank, local):
             "unit": "GB/s", "frac": round(ach / pk["hbm_gbs"], 4), "traffic": None,
             "alg_bytes_per_launch": alg, "avg_launch_ms": avg,
             "note": "traffic not captured for the packed instantiation"}
+    extra_cpu = {}
+    if rank == 0 and not args.no_cpu:
+        # the oracle, fwd+bwd, every head, on the documents in batch order
+        # until 8,192 rows (copied to the host before the clock starts)
+        import oracle
+        orc = oracle.load()
+        lam_h = lam.double().cpu().numpy()
+        offs = np.concatenate([[0], np.cumsum(lens)])
+        docs, rows = [], 0
+        for n in range(len(lens)):
+            if rows >= 8192:
+                break
+            a_, b_ = int(offs[n]), int(offs[n + 1])
+            docs.append({k: x[k][:, a_:b_].float().cpu().numpy()[None] for k in ("q", "k", "v", "dO")})
+            rows += b_ - a_
+        t0 = time.perf_counter()
+        for sl in docs:
+            orc.forward(sl["q"], sl["k"], sl["v"], lam_h)
+            orc.backward(sl["q"], sl["k"], sl["v"], lam_h, sl["dO"])
+        dt = time.perf_counter() - t0
+        extra_cpu = {"cpu_baseline": {
+            "value": round(rows / dt, 1), "unit": "tokens/s", "cores": orc.num_threads(),
+            "kind": "oracle",
+            "sample": f"fwd+bwd of the first {len(docs)} documents ({rows} rows x 32 heads, "
+                      f"{dt:.2f} s)"}}
     return _common(world, args.steps, args.warmup, value, "tokens/s",
                    "packed varlen fwd+bwd tokens/s (H=32, d=e=128, bf16)",
                    {"workload": f"packed variable-length batch, {len(lens)} sequences "
@@ -581,7 +623,7 @@ def run_varlen(args, world, rank, local):
                     "l2": "inputs 512 MiB per tensor, larger than L2; no flush"}, ms,
                    {"dtype": "bf16", "roofline": roof, "kernels": prof,
                     "gpu_launches": sum(v["launches"] for v in prof.values()), "clocks": clk,
-                    "sequences": len(lens)})
+                    "sequences": len(lens), **extra_cpu})
 
 
 def run_decode(args, world, rank, local):
@@ -601,6 +643,8 @@ def run_decode(args, world, rank, local):
     kv = inputs.decode_state0(Bn, Hh, D, E, device=dev, seed=0)
     gen = inputs.DecodeStream(Bn, Hh, D, E, device=dev, seed=0)
     toks = [gen.next() for _ in range(n)]
+    # the oracle's sample: requests 0..3 (all 64 heads), every step
+    samp = [tuple(a[:4].float().cpu().numpy() for a in toks[t]) for t in range(n)]
     if T > 1:  # [B,H,T,d|e] per call
         toks = [tuple(torch.stack([toks[c * T + t][i] for t in range(T)], dim=2).contiguous()
                       for i in range(3)) for c in range(calls)]
@@ -653,13 +697,26 @@ def run_decode(args, world, rank, local):
             "note": f"launch time = graph replay time / launches ({calls} launches per replay)"}
     what = ("one decode step per call" if T == 1 else
             f"{T} tokens per call (la2_decode_tokens)")
+    extra = {"dtype": "f32", "roofline": roof, "gpu_launches": calls * args.steps, "clocks": clk}
+    if rank == 0 and not args.no_cpu:
+        import oracle
+        orc = oracle.load()
+        st = kv[:4].double().cpu().numpy().copy()
+        lam_h = lam.double().cpu().numpy()
+        t0 = time.perf_counter()
+        for qt, kt, vt in samp:
+            orc.decode_step(qt, kt, vt, lam_h, st)
+        dt = time.perf_counter() - t0
+        extra["cpu_baseline"] = {
+            "value": round(4 * len(samp) / dt, 1), "unit": "tokens/s", "cores": orc.num_threads(),
+            "kind": "oracle",
+            "sample": f"{len(samp)} decode steps of 4 of the 256 requests (64 heads each, fp64 "
+                      f"state) ({dt:.2f} s); the same rate per request-token as the full batch"}
     line = _common(world, args.steps, args.warmup, value, "tokens/s",
                    "decode tokens/s (batch 256, H=64, d=e=128, fp32 state); % of HBM bandwidth",
                    {"workload": f"recurrent decode, batch 256, H=64, d=e=128, fp32 state "
                                 f"(1 GiB), {n} tokens per request per graph replay, {what}",
-                    "l2": "state 1 GiB, larger than L2; no flush"}, ms,
-                   {"dtype": "f32", "roofline": roof, "gpu_launches": calls * args.steps,
-                    "clocks": clk})
+                    "l2": "state 1 GiB, larger than L2; no flush"}, ms, extra)
     del g
     return line
 
