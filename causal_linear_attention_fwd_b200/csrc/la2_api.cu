@@ -262,6 +262,13 @@ size_t ws_bytes(int op, const Geo &g, int d, int e) {
 }
 
 // ------------------------------------------------------ SIMT dispatch
+// A kernel's dynamic shared memory above the default 48 KB needs an opt-in
+// attribute; its failure is returned rather than left to the launch.
+template <typename K>
+cudaError_t opt_in_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
 template <typename T, int D, int E>
 cudaError_t simt_forward(const void *q, const void *k, const void *v,
                          const float *lam, const float *kv0, void *o,
@@ -272,7 +279,7 @@ cudaError_t simt_forward(const void *q, const void *k, const void *v,
   const int64_t BH = (int64_t)g.B * g.H;
   if (g.S > 1) {
     auto kst = fwd_kernel<T, D, E, false>;
-    cudaFuncSetAttribute(kst, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fwd_smem<D, E>());
+    if (cudaError_t e = opt_in_smem(kst, fwd_smem<D, E>())) return e;
     err = timed(K_SIMT_FWD_STATE, st, [&] {
       kst<<<(unsigned)(BH * (g.S - 1)), NT, fwd_smem<D, E>(), st>>>(
           Q, K, V, lam, nullptr, nullptr, nullptr, ws, la2::state_geo(g, false));
@@ -285,7 +292,7 @@ cudaError_t simt_forward(const void *q, const void *k, const void *v,
     if (err) return err;
   }
   auto kf = fwd_kernel<T, D, E, true>;
-  cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fwd_smem<D, E>());
+  if (cudaError_t e = opt_in_smem(kf, fwd_smem<D, E>())) return e;
   return timed(K_SIMT_FWD, st, [&] {
     kf<<<(unsigned)(BH * g.S), NT, fwd_smem<D, E>(), st>>>(Q, K, V, lam, kv0, (T *)o, kv_out, ws, g);
   });
@@ -305,7 +312,7 @@ cudaError_t simt_backward(const void *q, const void *k, const void *v,
   cudaError_t err = cudaSuccess;
   if (g.S > 1 && !reuse_fwd) {
     auto kst = fwd_kernel<T, D, E, false>;
-    cudaFuncSetAttribute(kst, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fwd_smem<D, E>());
+    if (cudaError_t e = opt_in_smem(kst, fwd_smem<D, E>())) return e;
     err = timed(K_SIMT_FWD_STATE, st, [&] {
       kst<<<(unsigned)(BH * (g.S - 1)), NT, fwd_smem<D, E>(), st>>>(
           Q, K, V, lam, nullptr, nullptr, nullptr, wsf, la2::state_geo(g, false));
@@ -319,7 +326,7 @@ cudaError_t simt_backward(const void *q, const void *k, const void *v,
   }
   if (g.S > 1) {
     auto krs = rev_state_kernel<T, D, E>;
-    cudaFuncSetAttribute(krs, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rev_smem<D, E>());
+    if (cudaError_t e = opt_in_smem(krs, rev_smem<D, E>())) return e;
     err = timed(K_SIMT_REV_STATE, st, [&] {
       krs<<<(unsigned)(BH * (g.S - 1)), NT, rev_smem<D, E>(), st>>>(Q, G, lam, wsr,
                                                                     la2::state_geo(g, true));
@@ -332,13 +339,13 @@ cudaError_t simt_backward(const void *q, const void *k, const void *v,
     if (err) return err;
   }
   auto kq = dq_kernel<T, D, E>;
-  cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dq_smem<D, E>());
+  if (cudaError_t e = opt_in_smem(kq, dq_smem<D, E>())) return e;
   err = timed(K_SIMT_DQ, st, [&] {
     kq<<<(unsigned)(BH * g.S), NT, dq_smem<D, E>(), st>>>(K, V, G, lam, kv0, (T *)dq, wsf, g);
   });
   if (err) return err;
   auto kk = dkdv_kernel<T, D, E>;
-  cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dkdv_smem<D, E>());
+  if (cudaError_t e = opt_in_smem(kk, dkdv_smem<D, E>())) return e;
   return timed(K_SIMT_DKDV, st, [&] {
     kk<<<(unsigned)(BH * g.S), NT, dkdv_smem<D, E>(), st>>>(Q, K, V, G, lam, (T *)dk, (T *)dv,
                                                            dkv0, wsr, dend, g);
@@ -418,14 +425,14 @@ cudaError_t simt_shard_state(const void *a, const void *b, const float *lam, flo
   const int64_t BH = (int64_t)gs.B * gs.H;
   if (!reverse) {
     auto kst = fwd_kernel<T, D, E, false>;
-    cudaFuncSetAttribute(kst, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fwd_smem<D, E>());
+    if (cudaError_t e = opt_in_smem(kst, fwd_smem<D, E>())) return e;
     return timed(K_SIMT_FWD_STATE, st, [&] {
       kst<<<(unsigned)(BH * gs.nst), NT, fwd_smem<D, E>(), st>>>(
           nullptr, (const T *)a, (const T *)b, lam, nullptr, nullptr, nullptr, ws, gs);
     });
   }
   auto krs = rev_state_kernel<T, D, E>;
-  cudaFuncSetAttribute(krs, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rev_smem<D, E>());
+  if (cudaError_t e = opt_in_smem(krs, rev_smem<D, E>())) return e;
   return timed(K_SIMT_REV_STATE, st, [&] {
     krs<<<(unsigned)(BH * gs.nst), NT, rev_smem<D, E>(), st>>>((const T *)a, (const T *)b, lam,
                                                               ws + (size_t)D * E, gs);
