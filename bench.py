@@ -587,9 +587,9 @@ def run_varlen(args, world, rank, local):
     alg = 1024 * Hh * T
     ach = alg / (avg / 1e3) / 1e9
     roof = {"kernel": name, "bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"],
-            "unit": "GB/s", "frac": round(ach / pk["hbm_gbs"], 4), "traffic": None,
-            "alg_bytes_per_launch": alg, "avg_launch_ms": avg,
-            "note": "traffic not captured for the packed instantiation"}
+            "unit": "GB/s", "frac": round(ach / pk["hbm_gbs"], 4),
+            "traffic": traffic_for(name + "_packed", Hh * T),
+            "alg_bytes_per_launch": alg, "avg_launch_ms": avg}
     extra_cpu = {}
     if rank == 0 and not args.no_cpu:
         # the oracle, fwd+bwd, every head, on the documents in batch order
