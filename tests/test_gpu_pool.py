@@ -208,3 +208,37 @@ def test_decode_tokens_many_heads_fall_back(orc):
                         for t in range(T)], axis=1)
         check(f"request {b} o", o[b], ref, torch.bfloat16)
         check(f"request {b} state", pool[b], kv[0], torch.bfloat16)
+
+
+@pytest.mark.parametrize("case", range(12))
+def test_decode_units_agree_with_token_kernel(case):
+    """Seeded random shapes (B up to 300, H up to 20, T up to 128, slot tables
+    with inactive requests): the decode-unit kernel and the token-by-token
+    kernel, two independent paths, give the same outputs and states to the
+    bf16 tolerance."""
+    rng = np.random.default_rng(1000 + case)
+    B, H, T = int(rng.integers(1, 301)), int(rng.integers(1, 21)), int(rng.integers(1, 129))
+    P = B + int(rng.integers(0, 8))
+    perm = rng.permutation(P)[:B]
+    slots_h = [int(s) if rng.random() > 0.15 else -1 for s in perm]
+    slots = torch.tensor(slots_h, dtype=torch.int32, device=DEV)
+    lam = inputs.decay_lambdas(H, DEV)
+    q, k, v = tokens(B, H, T, 128, 128, torch.bfloat16, seed=2000 + case)
+    pool0 = inputs.decode_state0(P, H, 128, 128, device=DEV, seed=case)
+    res = {}
+    for name, frm in (("units", 1), ("token", 100000)):
+        pool = pool0.clone()
+        o = torch.full((B, H, T, 128), 7.0, dtype=torch.bfloat16, device=DEV)
+        old = la2.set_option(la2.LA2_OPT_DECODE_BLOCK_TOKENS, frm)
+        try:
+            la2.decode_tokens(q, k, v, lam, pool, slots, out=o)
+            torch.cuda.synchronize()
+        finally:
+            la2.set_option(la2.LA2_OPT_DECODE_BLOCK_TOKENS, old)
+        assert la2.last_device_error() == 0
+        res[name] = (o, pool)
+    tag = f"B={B} H={H} T={T}"
+    check(f"{tag} o", res["units"][0], host(res["token"][0]), torch.bfloat16)
+    check(f"{tag} pool", res["units"][1], host(res["token"][1]), torch.bfloat16)
+    assert torch.equal(res["units"][0][[b for b, s in enumerate(slots_h) if s < 0]],
+                       res["token"][0][[b for b, s in enumerate(slots_h) if s < 0]])
