@@ -428,3 +428,25 @@ def test_dlambda_b4_h16_l2048(orc):
     ref = orc.dlambda(h["q"], h["k"], h["v"], lam.double().cpu().numpy(), h["dO"])
     err = np.max(np.abs(got.double().cpu().numpy() - ref))
     assert err <= 1e-3 * float(np.max(np.abs(ref))), (got, ref)
+
+
+@pytest.mark.parametrize("case", range(6))
+def test_dlambda_random_splits_agree(case):
+    """Seeded random shapes and forced splits: the chunked decay gradient
+    equals the one-CTA-per-sequence form within the fp32 tolerance."""
+    rng = np.random.default_rng(900 + case)
+    B, H, L = int(rng.integers(1, 4)), int(rng.integers(1, 5)), int(rng.integers(1, 3000))
+    split = int(rng.integers(2, 12))
+    x = inputs.make_inputs(B, H, L, 128, 128, dtype=torch.bfloat16, device=DEV, seed=case,
+                           with_kv0=True)
+    lam = inputs.decay_lambdas(H, DEV)
+    ref = la2.dlambda(x["q"], x["k"], x["v"], lam, x["dO"], x["kv0"], chunked=False)
+    old = la2.set_option(la2.LA2_OPT_SPLIT, split)
+    try:
+        got = la2.dlambda(x["q"], x["k"], x["v"], lam, x["dO"], x["kv0"])
+        torch.cuda.synchronize()
+    finally:
+        la2.set_option(la2.LA2_OPT_SPLIT, old)
+    assert la2.last_device_error() == 0
+    err = float((got.double() - ref.double()).abs().max())
+    assert err <= 1e-3 * float(ref.double().abs().max()), (B, H, L, split, got, ref)

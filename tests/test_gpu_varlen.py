@@ -195,3 +195,34 @@ def test_varlen_many_sequences_matches_oracle(orc):
     ref = reference(orc, x, kv0, cu, lam)
     for name, u, r in zip(("o", "kv_out", "dq", "dk", "dv", "dkv0"), got, ref):
         check(f"70 sequences {name}", u, r, torch.bfloat16)
+
+
+@pytest.mark.parametrize("case", range(8))
+def test_varlen_random_batches_agree_with_per_document_calls(case):
+    """Seeded random packed batches (1..80 documents of 0..700 rows, 1..6
+    heads, both CTA orders by the document count) against the library's
+    batched calls on each document alone, forward and backward, with the
+    documents' own initial states."""
+    rng = np.random.default_rng(500 + case)
+    N, H = int(rng.integers(1, 81)), int(rng.integers(1, 7))
+    lens = [int(x) for x in rng.integers(0, 701, size=N)]
+    if sum(lens) == 0:
+        lens[0] = 1
+    x, kv0, cu = packed_inputs(lens, H, 128, 128, torch.bfloat16, seed=600 + case)
+    lam = inputs.decay_lambdas(H, DEV)
+    got = _varlen_all(x, kv0, cu, lam, 0)
+    offs = cu.cpu().numpy()
+    for n in range(N):
+        a, b = int(offs[n]), int(offs[n + 1])
+        if a == b:
+            continue
+        sl = {k: t[None, :, a:b].contiguous() for k, t in x.items()}
+        s0 = kv0[n:n + 1].contiguous()
+        o, st = la2.forward(sl["q"], sl["k"], sl["v"], lam, s0, want_state=True)
+        dq, dk, dv, dkv0 = la2.backward(sl["q"], sl["k"], sl["v"], lam, sl["dO"], s0,
+                                        want_dkv0=True)
+        tag = f"case {case} doc {n} ({b - a} rows, N={N}, H={H})"
+        for name, u, r in (("o", got[0][:, a:b], o[0]), ("dq", got[2][:, a:b], dq[0]),
+                           ("dk", got[3][:, a:b], dk[0]), ("dv", got[4][:, a:b], dv[0]),
+                           ("kv_out", got[1][n], st[0]), ("dkv0", got[5][n], dkv0[0])):
+            check(f"{tag} {name}", u, host(r), torch.bfloat16)
