@@ -450,3 +450,25 @@ def test_dlambda_random_splits_agree(case):
     assert la2.last_device_error() == 0
     err = float((got.double() - ref.double()).abs().max())
     assert err <= 1e-3 * float(ref.double().abs().max()), (B, H, L, split, got, ref)
+
+
+@pytest.mark.parametrize("case", range(10))
+def test_random_shapes_match_oracle(orc, case):
+    """Seeded random shapes on the tensor-core path (B 1..3, H 1..4, L
+    1..1500 with ragged tails, decays drawn in [0, 1] with one head at 0 and
+    one at 1, an initial state, a random forced split or the library's own):
+    forward, final state and every gradient against the oracle."""
+    rng = np.random.default_rng(4000 + case)
+    B, H, L = int(rng.integers(1, 4)), int(rng.integers(1, 5)), int(rng.integers(1, 1501))
+    vals = [float(v) for v in rng.uniform(0.0, 1.0, size=H)]
+    vals[0] = 0.0
+    if H > 1:
+        vals[-1] = 1.0
+    lam = inputs.fixed_lambdas(tuple(vals), DEV)
+    split = int(rng.integers(0, 9))
+    x = inputs.make_inputs(B, H, L, 128, 128, dtype=torch.bfloat16, device=DEV,
+                           seed=4100 + case, with_kv0=True)
+    with options(path="tc", split=split):
+        got = run_fwd_bwd(x, lam, x["kv0"])
+    compare(got, oracle_all(orc, x, lam, x["kv0"]), torch.bfloat16,
+            f"B={B} H={H} L={L} split={split}")
