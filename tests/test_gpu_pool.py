@@ -114,6 +114,14 @@ def test_pool_slot_past_end_reported():
     la2.decode_tokens(q, k, v, lam, pool, slots)
     torch.cuda.synchronize()
     assert la2.last_device_error() == 1
+    # the same through the decode-unit kernel (20 tokens per request); the
+    # valid request's state still advances
+    before = pool[1].clone()
+    q20, k20, v20 = tokens(B, H, 20, 128, 128, torch.bfloat16, seed=3)
+    la2.decode_tokens(q20, k20, v20, lam, pool, slots)
+    torch.cuda.synchronize()
+    assert la2.last_device_error() == 1
+    assert not torch.equal(pool[1], before)
     x = inputs.make_inputs(B, H, 200, 128, 128, dtype=torch.bfloat16, device=DEV, seed=2,
                            with_dO=False)
     la2.forward_pool(x["q"], x["k"], x["v"], lam, pool, slots)
