@@ -10,7 +10,8 @@ header); this module only compiles it with gcc and marshals numpy arrays.
 Every function here is pinned by tests in ``tests/test_oracle_pins.py``
 (brute-force quadratic attention, the lambda=1 prefix-sum identity, lambda=0,
 block-size invariance of a tiled restatement, finite differences, adjoint
-identities, state hand-off, a hand-derived golden example).
+identities, state hand-off, a hand-derived golden example; for the feature
+map: printed constants, closed forms, its shape, finite differences).
 """
 from __future__ import annotations
 
@@ -37,7 +38,7 @@ def build(src: str = SRC, out: str = LIB, force: bool = False) -> str:
         return out
     tmp = out + f".tmp{os.getpid()}"
     cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99",
-           "-o", tmp, src]
+           "-o", tmp, src, "-lm"]
     subprocess.run(cmd, check=True)
     os.replace(tmp, out)
     return out
@@ -58,9 +59,12 @@ class Oracle:
                                                   P, P, P, P, P]
         self._lib.oracle_dlambda.argtypes = [i, i, l, i, i, P, P, P, P, P, P, P]
         self._lib.oracle_decode_step.argtypes = [i, i, i, i, P, P, P, P, P, P]
+        self._lib.oracle_feature_map.argtypes = [l, P, P]
+        self._lib.oracle_feature_map_grad.argtypes = [l, P, P, P]
         self._lib.oracle_num_threads.restype = ctypes.c_int
         for f in ("oracle_forward", "oracle_backward", "oracle_backward_end",
-                  "oracle_dlambda", "oracle_decode_step"):
+                  "oracle_dlambda", "oracle_decode_step", "oracle_feature_map",
+                  "oracle_feature_map_grad"):
             getattr(self._lib, f).restype = None
 
     @staticmethod
@@ -141,6 +145,23 @@ class Oracle:
                                      self._p(v), self._p(lam), self._p(kv),
                                      self._p(o))
         return o
+
+
+    def feature_map(self, x):
+        """phi(x) = elu(x) + 1 elementwise (fp64, same shape)."""
+        x = self._f32(x)
+        y = np.empty(x.shape, np.float64)
+        self._lib.oracle_feature_map(x.size, self._p(x), self._p(y))
+        return y
+
+    def feature_map_grad(self, x, dy):
+        """dL/dx from dL/dphi(x) = dy: dy * elu'(x) (fp64, same shape)."""
+        x = self._f32(x)
+        dy = self._f64(dy)
+        assert dy.shape == x.shape
+        dx = np.empty(x.shape, np.float64)
+        self._lib.oracle_feature_map_grad(x.size, self._p(x), self._p(dy), self._p(dx))
+        return dx
 
 
 def load(path: str | None = None) -> Oracle:

@@ -24,14 +24,17 @@
  *   o_t  = q_t kv_t                            (the state already holds token t)
  *
  * No blocking, no reordering: one token at a time, fp64 accumulation.
- * The pages give no decay, feature map, normalisation or scaling; inputs are
- * taken as already mapped, and no denominator is applied.
+ * The pages give no decay, feature map, normalisation or scaling; the
+ * attention takes its inputs as already mapped (the optional feature map is
+ * its own pair of functions at the end of this file), and no denominator is
+ * applied.
  *
  * Layout: q,k [B,H,L,d], v [B,H,L,e] contiguous row-major (float, which holds
  * bf16 and fp32 inputs exactly); lambda [H] double; states [B,H,d,e] double;
  * outputs double.  Every (b,h) problem is independent; OpenMP only spreads
  * those independent problems over host cores.
  */
+#include <math.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -243,4 +246,44 @@ void oracle_dlambda(int B, int H, long L, int d, int e,
     for (int h = 0; h < H; h++) dlam[h] = 0.0;
     for (long bh = 0; bh < BH; bh++) dlam[bh % H] += part[bh];
     free(part);
+}
+
+/*
+ * Feature map, the optional prologue applied to q and k before the attention.
+ *
+ * The Lightning Attention glossary page (section "主な特徴・仕組み") has
+ * linear attention replace softmax by a kernel feature map so that K^T V
+ * can be aggregated first, but it names no map.  Reading taken here: the
+ * exponential linear unit plus one, phi(x) = elu(x) + 1, the positive map
+ * of "Transformers are RNNs", one of the works the Luna page lists as its
+ * basis next to the ELU paper.  With elu's own definition (alpha = 1):
+ *
+ *   elu(x) = x              for x > 0,   exp(x) - 1   for x <= 0
+ *   phi(x) = elu(x) + 1
+ *
+ * and, for the chain rule of the backward pass, elu's derivative
+ *
+ *   elu'(x) = 1             for x > 0,   exp(x)       for x <= 0
+ *
+ * so dL/dx = dL/dphi(x) * elu'(x).  Elementwise over n values; x float
+ * (exact bf16 or fp32 inputs), results double.
+ */
+void oracle_feature_map(long n, const float *x, double *y)
+{
+#pragma omp parallel for schedule(static)
+    for (long i = 0; i < n; i++) {
+        double xi = (double)x[i];
+        double elu = xi > 0.0 ? xi : expm1(xi);
+        y[i] = elu + 1.0;
+    }
+}
+
+void oracle_feature_map_grad(long n, const float *x, const double *dy, double *dx)
+{
+#pragma omp parallel for schedule(static)
+    for (long i = 0; i < n; i++) {
+        double xi = (double)x[i];
+        double delu = xi > 0.0 ? 1.0 : exp(xi);
+        dx[i] = dy[i] * delu;
+    }
 }

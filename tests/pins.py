@@ -342,8 +342,61 @@ def pin_golden(orc):
         assert_close(dkv0.reshape(d, e), np.array(c["dkv0"]), 0, c["name"] + " dkv0")
 
 
+# ------------------------------------------------------------- feature map
+def pin_feature_map_values(orc):
+    """phi(x) = elu(x) + 1 at points where it is known without the oracle:
+    exact on the linear side (phi(0) = 1, phi(3) = 4, phi(2.5) = 3.5), and
+    on the exponential side e^-1 and e^-30 (their decimal expansions, to
+    1e-15 absolute) and
+    e^(-ln 2) = 1/2, e^(-ln 4) = 1/4 (the float32 rounding of -ln 2 and
+    -ln 4 moves these by under 1e-7 relative)."""
+    x = np.array([0.0, 3.0, 2.5, -1.0, -30.0, -np.log(2.0), -np.log(4.0)], np.float32)
+    want = np.array([1.0, 4.0, 3.5, 0.36787944117144233, 9.357622968840175e-14, 0.5, 0.25])
+    got = orc.feature_map(x)
+    assert np.array_equal(got[:3], want[:3]), f"feature map, linear side: {got[:3]}"
+    # elu(x) + 1 on the exponential side rounds the sum to 1's spacing, so
+    # its error is absolute, about 1e-16 (e^-30 itself is 9.4e-14)
+    err = np.abs(got - want)
+    assert err[3:5].max() < 1e-15, f"feature map at -1, -30: {got[3:5]} vs {want[3:5]}"
+    assert (err[5:] / want[5:]).max() < 1e-7, f"feature map at -ln 2, -ln 4: {got[5:]}"
+
+
+def pin_feature_map_shape(orc):
+    """The map is positive (what lets the numerator stay a sum of positive
+    weights), equals 1 + x on the positive side and lies in (0, 1] on the
+    other, never below the tangent line 1 + x there (e^x >= 1 + x), and is
+    increasing."""
+    x = bf16_exact((4096,), 91, 3.0)
+    y = orc.feature_map(x)
+    xd = x.astype(np.float64)
+    assert (y > 0).all(), "feature map not positive"
+    pos = xd > 0
+    assert np.array_equal(y[pos], xd[pos] + 1.0), "feature map != 1 + x for x > 0"
+    assert (y[~pos] <= 1.0).all() and (y[~pos] >= 1.0 + xd[~pos]).all(), \
+        "feature map outside [1 + x, 1] for x <= 0"
+    order = np.argsort(xd, kind="stable")
+    assert (np.diff(y[order]) >= 0).all(), "feature map not increasing"
+
+
+def pin_feature_map_finite_difference(orc):
+    """dL/dx = dL/dphi * phi'(x) against central differences of the
+    oracle's own map (the step taken between float32 neighbours of x so
+    both evaluation points are exact inputs)."""
+    g = np.random.default_rng(17)
+    x = (g.standard_normal(512) * 2.0).astype(np.float32)
+    x = x[np.abs(x) > 0.05]
+    dy = g.standard_normal(x.shape)
+    h = np.maximum(1e-3, 1e-3 * np.abs(x)).astype(np.float32)
+    xp, xm = (x + h).astype(np.float32), (x - h).astype(np.float32)
+    slope = (orc.feature_map(xp) - orc.feature_map(xm)) / (xp.astype(np.float64) - xm)
+    got = orc.feature_map_grad(x, dy)
+    err = np.abs(got - dy * slope) / (np.abs(dy * slope) + 1e-12)
+    assert err.max() < 1e-5, f"feature map gradient vs finite differences: {err.max():.3e}"
+
+
 ALL_PINS = [pin_bruteforce, pin_prefix_sum, pin_lambda_zero, pin_length_one,
             pin_backward_closed_form, pin_backward_terminal_closed_form, pin_backward_split,
             pin_dlambda_closed_form, pin_dlambda_finite_difference,
             pin_finite_difference, pin_adjoint,
-            pin_state_handoff, pin_decode_equals_forward, pin_golden]
+            pin_state_handoff, pin_decode_equals_forward, pin_golden,
+            pin_feature_map_values, pin_feature_map_shape, pin_feature_map_finite_difference]

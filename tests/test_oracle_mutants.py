@@ -57,6 +57,24 @@ MUTANTS = [
     ("decode_drops_new_token",
      "s[i * e + j] = lam * s[i * e + j] + (double)kt[i] * (double)vt[j];",
      "s[i * e + j] = lam * s[i * e + j] + (double)kt[i] * (double)vt[j] * (double)(lam != lam);"),
+    ("feature_map_drops_one",
+     "y[i] = elu + 1.0;",
+     "y[i] = elu;"),
+    ("feature_map_branches_swapped",
+     "double elu = xi > 0.0 ? xi : expm1(xi);",
+     "double elu = xi > 0.0 ? expm1(xi) : xi;"),
+    ("feature_map_exp_not_expm1",
+     "double elu = xi > 0.0 ? xi : expm1(xi);",
+     "double elu = xi > 0.0 ? xi : exp(xi);"),
+    ("feature_map_grad_branches_swapped",
+     "double delu = xi > 0.0 ? 1.0 : exp(xi);",
+     "double delu = xi > 0.0 ? exp(xi) : 1.0;"),
+    ("feature_map_grad_ignores_upstream",
+     "dx[i] = dy[i] * delu;",
+     "dx[i] = delu;"),
+    ("feature_map_grad_is_the_map",
+     "double delu = xi > 0.0 ? 1.0 : exp(xi);",
+     "double delu = xi > 0.0 ? xi + 1.0 : exp(xi);"),
 ]
 
 
