@@ -792,6 +792,104 @@ def run_dlambda(args, world, rank, local):
                     "l2": "inputs 32 MiB (fit in L2); the pass is arithmetic-bound"}, ms, extra)
 
 
+# The feature map's streaming passes per token-head (d = 128, bf16): the map
+# reads q, k and writes phi_q, phi_k (4 x 256 B); its gradient reads q, k,
+# dphi_q, dphi_k and writes dq, dk (6 x 256 B).
+FMAP_BYTES_PER_TH = {"feature_map": 4 * 2 * D, "feature_map_grad": 6 * 2 * D}
+
+
+def hbm_roofline(name, rec, bytes_per_th, th_per_launch, pk, traffic=None):
+    avg = rec["ms"] / rec["launches"]
+    alg = bytes_per_th * th_per_launch
+    ach = alg / (avg / 1e3) / 1e9
+    return {"kernel": name, "bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"],
+            "unit": "GB/s", "frac": round(ach / pk["hbm_gbs"], 4), "traffic": traffic,
+            "alg_bytes_per_launch": alg, "avg_launch_ms": avg,
+            "peak_source": pk["source"] + " (hbm_gbs, STREAM-style copy)"}
+
+
+def run_fmap(args, world, rank, local):
+    """A training step with the feature map phi(x) = elu(x) + 1 on q and k:
+    the map, the attention forward and backward on the mapped inputs, and the
+    map's chain rule, on the B=8, H=32, L=8,192 sweep point (secondary
+    workload)."""
+    import causal_linear_attention_fwd_b200 as la2
+    from causal_linear_attention_fwd_b200 import inputs
+    dev = torch.device("cuda", local)
+    pk = peaks()
+    Bn, L = 8, 8192
+    x = inputs.make_inputs(Bn, H, L, D, E, dtype=torch.bfloat16, device=dev, seed=0)
+    lam = inputs.decay_lambdas(H, dev)
+    buf = {n: torch.empty_like(x[src]) for n, src in
+           (("pq", "q"), ("pk", "k"), ("o", "v"), ("gq", "q"), ("gk", "k"), ("dv", "v"))}
+    ws_n = la2.workspace_size(la2.LA2_OP_BACKWARD, Bn, H, L, D, E, torch.bfloat16)
+    ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device=dev)
+
+    def step():
+        la2.feature_map(x["q"], x["k"], out=(buf["pq"], buf["pk"]))
+        la2.forward(buf["pq"], buf["pk"], x["v"], lam, out=buf["o"], workspace=ws)
+        la2.backward(buf["pq"], buf["pk"], x["v"], lam, x["dO"],
+                     outs=(buf["gq"], buf["gk"], buf["dv"]), workspace=ws,
+                     reuse_forward_states=ws_n > 0)
+        # dq, dk in place over the attention's gradients
+        la2.feature_map_backward(x["q"], x["k"], buf["gq"], buf["gk"], out=(buf["gq"], buf["gk"]))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert la2.last_device_error() == 0
+    clocks = ClockSampler(local)
+    la2.profile_enable(True)
+    la2.profile_report()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    prof = la2.profile_report()
+    la2.profile_enable(False)
+    assert la2.last_device_error() == 0
+    ms = max_over_ranks(a.elapsed_time(b), world)
+    value = world * Bn * L * args.steps / (ms / 1e3)
+    th = Bn * L * H
+    # the dominant kernel, among the attention passes and the map's two
+    name, rec = max(prof.items(), key=lambda kv: kv[1]["ms"])
+    bpt = {**BYTES_PER_TH, **FMAP_BYTES_PER_TH}.get(name)
+    roof = hbm_roofline(name, rec, bpt, th, pk, traffic_for(name, th)) if bpt else None
+    fmap_roof = {n: hbm_roofline(n, prof[n], bpt, th, pk)
+                 for n, bpt in FMAP_BYTES_PER_TH.items() if n in prof}
+    extra = {"dtype": "bf16", "roofline": roof, "roofline_feature_map": fmap_roof,
+             "kernels": prof, "gpu_launches": sum(v["launches"] for v in prof.values()),
+             "clocks": clk}
+    if rank == 0 and not args.no_cpu:
+        import oracle
+        orc = oracle.load()
+        h = {n: t[:1].float().cpu().numpy() for n, t in x.items()}
+        lam_h = lam.double().cpu().numpy()
+        t0 = time.perf_counter()
+        fq, fk = orc.feature_map(h["q"]), orc.feature_map(h["k"])
+        orc.forward(fq, fk, h["v"], lam_h)
+        g = orc.backward(fq, fk, h["v"], lam_h, h["dO"])
+        orc.feature_map_grad(h["q"], g[0])
+        orc.feature_map_grad(h["k"], g[1])
+        dt = time.perf_counter() - t0
+        extra["cpu_baseline"] = {"value": round(L / dt, 1), "unit": "tokens/s",
+                                 "cores": orc.num_threads(), "kind": "oracle",
+                                 "sample": f"one batch row ({H} heads x {L} rows) of the workload"}
+    return _common(world, args.steps, args.warmup, value, "tokens/s",
+                   "fwd+bwd tokens/s with the elu+1 feature map (B=8,H=32,L=8192,d=e=128,bf16)",
+                   {"workload": "training step with the feature map phi(x) = elu(x) + 1 on q "
+                                "and k, B=8, H=32, L=8,192, d=e=128, bf16",
+                    "l2": "inputs 512 MiB per tensor, larger than L2; no flush"}, ms, extra)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -801,9 +899,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--workload", default="sweep",
-                    choices=["sweep", "long", "decode", "varlen", "dlambda"],
+                    choices=["sweep", "long", "decode", "varlen", "dlambda", "fmap"],
                     help="sweep (the metric; default), long (1M-token forward), decode, "
-                         "varlen (packed variable-length fwd+bwd), dlambda (decay gradient)")
+                         "varlen (packed variable-length fwd+bwd), dlambda (decay gradient), "
+                         "fmap (fwd+bwd with the elu+1 feature map)")
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--decode-tokens", type=int, default=1,
                     help="decode workload: tokens per request per call (1 = decode_step)")
@@ -827,7 +926,7 @@ def main():
     world, rank, local = dist_setup(args.gpus)
     try:
         fn = {"sweep": run_la2, "long": run_long, "decode": run_decode,
-              "varlen": run_varlen, "dlambda": run_dlambda}[args.workload]
+              "varlen": run_varlen, "dlambda": run_dlambda, "fmap": run_fmap}[args.workload]
         line = fn(args, world, rank, local)
         if rank == 0:
             print(json.dumps(line), flush=True)

@@ -14,12 +14,13 @@ from ._binding import (  # noqa: F401
     LA2_POOL_CONTINUE, LA2_OP_SHARD_STATE, LA2_OP_DLAMBDA, backward_shard, decode_tokens, forward_pool,
     shard_state, state_prefix, dlambda,
     LA2_OPT_SPLIT, LA2_OPT_TRACE, LA2_OPT_VARIANT, LA2_OPT_VARLEN_ORDER, LA2_OPT_DECODE_BLOCK_TOKENS, trace_read,
-    backward, backward_varlen, decode_step, forward, forward_noalloc, forward_varlen,
+    backward, backward_varlen, decode_step, feature_map, feature_map_backward, forward,
+    forward_noalloc, forward_varlen,
     last_device_error, library, profile_enable, profile_report, set_option, status_string,
     version, workspace_size)
 
 __all__ = ["forward", "forward_noalloc", "backward", "forward_varlen", "backward_varlen",
            "forward_pool", "decode_step", "decode_tokens", "shard_state", "state_prefix",
-           "backward_shard", "dlambda", "workspace_size",
+           "backward_shard", "dlambda", "feature_map", "feature_map_backward", "workspace_size",
            "last_device_error", "set_option", "profile_enable", "profile_report",
            "status_string", "version", "library", "LA2Error"]

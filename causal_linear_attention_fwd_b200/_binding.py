@@ -81,6 +81,10 @@ def library():
         lib.la2_backward_dlambda_ex.restype = I
         lib.la2_decode_step.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
         lib.la2_decode_step.restype = I
+        lib.la2_feature_map.argtypes = [P, P, P, P, I64, I, P]
+        lib.la2_feature_map.restype = I
+        lib.la2_feature_map_backward.argtypes = [P, P, P, P, P, P, I64, I, P]
+        lib.la2_feature_map_backward.restype = I
         lib.la2_last_device_error.argtypes = [P]
         lib.la2_last_device_error.restype = I
         lib.la2_status_string.argtypes = [I]
@@ -463,6 +467,49 @@ def dlambda(q, k, v, lam, dO, kv0=None, *, workspace=None, chunked: bool = True,
                                        _stream(stream))
     _check(code, "la2_backward_dlambda_ex")
     return out
+
+
+def _fmap_args(q, k, extra):
+    _dev(q, "q")
+    if k is not None:
+        _dev(k, "k")
+        if k.shape != q.shape or k.dtype != q.dtype:
+            raise ValueError("q and k must have the same shape and dtype")
+    for name, t in extra:
+        if t is not None:
+            _dev(t, name)
+            if t.shape != q.shape or t.dtype != q.dtype:
+                raise ValueError(f"{name} must match q's shape and dtype")
+
+
+def feature_map(q, k=None, *, out=None, stream=None):
+    """phi(x) = elu(x) + 1 applied to q (and k): returns phi_q (and phi_k).
+    out: (phi_q, phi_k) buffers, which may be q and k themselves (in place)."""
+    lib = library()
+    phi_q, phi_k = out if out is not None else (
+        torch.empty_like(q), None if k is None else torch.empty_like(k))
+    _fmap_args(q, k, (("phi_q", phi_q), ("phi_k", phi_k)))
+    code = lib.la2_feature_map(_ptr(q), _ptr(k), _ptr(phi_q), _ptr(phi_k), q.numel(), _dt(q),
+                               _stream(stream))
+    _check(code, "la2_feature_map")
+    return phi_q if k is None else (phi_q, phi_k)
+
+
+def feature_map_backward(q, k, dphi_q, dphi_k=None, *, out=None, stream=None):
+    """Chain rule through the feature map: dq = dphi_q * phi'(q) (and dk
+    likewise), q, k the unmapped inputs, dphi_* the attention's gradients
+    with respect to phi(q), phi(k).  out may be (dphi_q, dphi_k) (in place).
+    k and dphi_k are both None to map q alone."""
+    lib = library()
+    if (k is None) != (dphi_k is None):
+        raise ValueError("k and dphi_k are both given or both None")
+    dq, dk = out if out is not None else (
+        torch.empty_like(q), None if k is None else torch.empty_like(k))
+    _fmap_args(q, k, (("dphi_q", dphi_q), ("dphi_k", dphi_k), ("dq", dq), ("dk", dk)))
+    code = lib.la2_feature_map_backward(_ptr(q), _ptr(k), _ptr(dphi_q), _ptr(dphi_k), _ptr(dq),
+                                        _ptr(dk), q.numel(), _dt(q), _stream(stream))
+    _check(code, "la2_feature_map_backward")
+    return dq if k is None else (dq, dk)
 
 
 def decode_step(q, k, v, lam, kv, *, out=None, stream=None):

@@ -14,6 +14,7 @@
 #include "../../include/la2.h"
 #include "la2_common.cuh"
 #include "la2_decode.cuh"
+#include "la2_fmap.cuh"
 #include "la2_shard.cuh"
 #include "la2_simt.cuh"
 #include "la2_tc.cuh"
@@ -35,14 +36,14 @@ enum KernelId {
   K_SIMT_FWD_STATE, K_SIMT_FWD_SCAN, K_SIMT_FWD, K_SIMT_DQ, K_SIMT_REV_STATE,
   K_SIMT_REV_SCAN, K_SIMT_DKDV, K_DECODE, K_TC_FWD_STATE, K_TC_FWD, K_TC_DQ,
   K_TC_REV_STATE, K_TC_DV, K_TC_DK, K_SCAN_FWD, K_SCAN_REV, K_SIMT_DLAMBDA,
-  K_SIMT_DLAMBDA_STATE, K_SIMT_DLAMBDA_SCAN, K_TC_DECODE_UNITS, K_COUNT
+  K_SIMT_DLAMBDA_STATE, K_SIMT_DLAMBDA_SCAN, K_TC_DECODE_UNITS, K_FMAP, K_FMAP_GRAD, K_COUNT
 };
 const char *kKernelName[K_COUNT] = {
     "simt_fwd_chunk_state", "simt_scan_fwd", "simt_fwd", "simt_dq",
     "simt_rev_chunk_state", "simt_scan_rev", "simt_dkdv", "decode_step",
     "tc_fwd_chunk_state", "tc_fwd", "tc_dq", "tc_rev_chunk_state", "tc_dv", "tc_dk",
     "scan_fwd", "scan_rev", "simt_dlambda", "simt_dlambda_chunk_state", "simt_dlambda_scan",
-    "tc_decode_units"};
+    "tc_decode_units", "feature_map", "feature_map_grad"};
 
 struct ProfRec {
   int kid;
@@ -459,6 +460,54 @@ cudaError_t prefix(const float *delta, const float *kv0, const float *lam, int R
   return cudaGetLastError();
 }
 
+
+// ------------------------------------------------------------ feature map
+namespace {
+
+// The elementwise calls: tensor t's output may be exactly its own `own`
+// input (in place); every other pair of arguments shares no byte.
+bool fmap_args_ok(const std::vector<Span> &outs, const std::vector<Span> &ins,
+                  const std::vector<const void *> &own) {
+  for (size_t i = 0; i < outs.size(); i++) {
+    if (!outs[i].p) continue;
+    for (size_t j = 0; j < ins.size(); j++)
+      if (overlaps(outs[i], ins[j]) && !(ins[j].p == outs[i].p && ins[j].p == own[i]))
+        return false;
+    for (size_t j = i + 1; j < outs.size(); j++)
+      if (overlaps(outs[i], outs[j])) return false;
+  }
+  return true;
+}
+
+template <bool GRAD>
+la2_status fmap_call(const void *q, const void *k, const void *gq, const void *gk, void *yq,
+                     void *yk, int64_t n, la2_dtype dt, cudaStream_t stream) {
+  if (n < 0) return LA2_ERR_INVALID;
+  if (dt != LA2_F32 && dt != LA2_BF16) return LA2_ERR_UNSUPPORTED;
+  if (n == 0) return LA2_OK;
+  if (!q || !yq || (GRAD && !gq)) return LA2_ERR_INVALID;
+  const bool has_k = k != nullptr;
+  if ((yk != nullptr) != has_k || (GRAD && (gk != nullptr) != has_k)) return LA2_ERR_INVALID;
+  for (const void *p : {q, k, gq, gk, (const void *)yq, (const void *)yk})
+    if (p && !aligned16(p)) return LA2_ERR_INVALID;
+  const size_t bytes = (size_t)n * esize(dt);
+  std::vector<Span> ins = {{q, bytes}, {k, bytes}, {gq, bytes}, {gk, bytes}};
+  std::vector<Span> outs = {{yq, bytes}, {yk, bytes}};
+  // in place: the map over its input, the gradient over its upstream gradient
+  if (!fmap_args_ok(outs, ins, {GRAD ? gq : q, GRAD ? gk : k})) return LA2_ERR_INVALID;
+  const int sms = device_sms();
+  const int grid = dt == LA2_F32 ? la2::fmap::grid_for<float, GRAD>(n, sms)
+                                 : la2::fmap::grid_for<__nv_bfloat16, GRAD>(n, sms);
+  cudaError_t err = timed(GRAD ? K_FMAP_GRAD : K_FMAP, stream, [&] {
+    if (dt == LA2_F32)
+      la2::fmap::enqueue<float, GRAD>(q, gq, yq, k, gk, yk, n, grid, stream);
+    else
+      la2::fmap::enqueue<__nv_bfloat16, GRAD>(q, gq, yq, k, gk, yk, n, grid, stream);
+  });
+  return to_status(err);
+}
+
+}  // namespace
 
 extern "C" {
 
@@ -992,6 +1041,17 @@ la2_status la2_decode_step(const void *q, const void *k, const void *v, const fl
           : LA2_DISPATCH_DE(d, e, decode, __nv_bfloat16, q, k, v, lambda, kv, nullptr, B, o, B, H,
                             1, stream);
   return to_status(err);
+}
+
+la2_status la2_feature_map(const void *q, const void *k, void *phi_q, void *phi_k, int64_t n,
+                           la2_dtype dt, cudaStream_t stream) {
+  return fmap_call<false>(q, k, nullptr, nullptr, phi_q, phi_k, n, dt, stream);
+}
+
+la2_status la2_feature_map_backward(const void *q, const void *k, const void *dphi_q,
+                                    const void *dphi_k, void *dq, void *dk, int64_t n,
+                                    la2_dtype dt, cudaStream_t stream) {
+  return fmap_call<true>(q, k, dphi_q, dphi_k, dq, dk, n, dt, stream);
 }
 
 la2_status la2_decode_tokens(const void *q, const void *k, const void *v, const float *lambda,

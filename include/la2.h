@@ -255,6 +255,44 @@ la2_status la2_backward_dlambda_ex(const void *q, const void *k, const void *v,
                                    cudaStream_t stream);
 
 /*
+ * Feature map phi(x) = elu(x) + 1, applied to q and k before the attention
+ * calls (which take their q and k as already mapped):
+ *     phi(x) = x + 1 for x > 0,  e^x for x <= 0      (elementwise)
+ * The Lightning Attention glossary page (section "主な特徴・仕組み") has
+ * linear attention replace softmax by a kernel feature map so that K^T V can
+ * be aggregated first, but names no map; elu + 1 is the positive map of
+ * "Transformers are RNNs", one of the works the Luna page lists as its basis
+ * next to the ELU paper.  Callers using another map, or none, skip this call.
+ *
+ * la2_feature_map: phi_q = phi(q), phi_k = phi(k); q, k, phi_q, phi_k hold n
+ * values each of type dt (any layout: the map is elementwise; n >= 0, any
+ * value).  k and phi_k may both be NULL (q alone is mapped).  An output may be
+ * the very buffer of its own input (in place: phi_q == q, phi_k == k); any
+ * other shared byte between arguments is LA2_ERR_INVALID.
+ *
+ * la2_feature_map_backward: the chain rule through the map,
+ *     dq = dphi_q * phi'(q),  dk = dphi_k * phi'(k),
+ *     phi'(x) = 1 for x > 0,  e^x for x <= 0,
+ * where dphi_q, dphi_k are the attention's gradients with respect to its
+ * mapped inputs (la2_backward's dq, dk on phi_q, phi_k) and q, k the
+ * unmapped inputs.  k, dphi_k and dk are all NULL or all given.  dq may be
+ * the very buffer of dphi_q (in place), likewise dk of dphi_k.
+ *
+ * Both: one HBM-bound streaming launch over q and k together; arithmetic in
+ * fp32 (e^x: CUDA's expf), results rounded to dt (bf16: to nearest even).
+ * Pointers 16-byte aligned, device memory, caller-owned; asynchronous on
+ * `stream`.  Errors: LA2_ERR_INVALID for n < 0, a NULL required pointer,
+ * misalignment or an overlap other than the in-place ones;
+ * LA2_ERR_UNSUPPORTED for another dt; LA2_ERR_CUDA for a failed launch.
+ * n = 0: nothing is launched.
+ */
+la2_status la2_feature_map(const void *q, const void *k, void *phi_q, void *phi_k, int64_t n,
+                           la2_dtype dt, cudaStream_t stream);
+la2_status la2_feature_map_backward(const void *q, const void *k, const void *dphi_q,
+                                    const void *dphi_k, void *dq, void *dk, int64_t n,
+                                    la2_dtype dt, cudaStream_t stream);
+
+/*
  * State pool for serving: the recurrent states of many requests live in one
  * fp32 array kv_pool [pool_size, H, d, e]; request b of a call uses state
  * slots[b] (device int32 [B], 4-byte aligned).  A negative slot marks an

@@ -269,3 +269,37 @@ def test_product_path_does_not_reference_oracle():
                 for pat in (r"^\s*import\s+oracle", r"^\s*from\s+oracle", r"la2_oracle",
                             r"oracle\.(load|build|Oracle)"):
                     assert not re.search(pat, src, flags=re.M), f"{f} reaches the oracle ({pat})"
+
+
+def test_feature_map_validation(lib):
+    """The elementwise feature-map calls: in-place use is the only overlap
+    allowed (an output over its own input, or over its own upstream
+    gradient); everything else shared, misaligned, missing or negative is
+    rejected before any launch.  Only rejected cases and n = 0 (nothing to
+    launch) are called here."""
+    INV, UNS, OK = B.LA2_ERR_INVALID, B.LA2_ERR_UNSUPPORTED, B.LA2_OK
+    n = 4096
+    f = lambda q=Q, k=K, pq=O, pk=DQ, n=n, dt=B.LA2_BF16: lib.la2_feature_map(
+        q, k, pq, pk, n, dt, None)
+    assert f(n=-1) == INV
+    assert f(dt=7) == UNS
+    assert f(n=0) == OK
+    assert f(q=None) == INV
+    assert f(pq=None) == INV
+    assert f(pk=None) == INV                         # k given, phi_k missing
+    assert f(k=None) == INV                          # phi_k given, k missing
+    assert f(q=Q + 8) == INV
+    assert f(pq=K) == INV                            # phi_q over k
+    assert f(pq=Q + 16) == INV                       # phi_q partly over q
+    assert f(pk=O + 16) == INV                       # outputs share bytes
+    g = lambda q=Q, k=K, gq=DO, gk=DV, dq=DQ, dk=DK, n=n: lib.la2_feature_map_backward(
+        q, k, gq, gk, dq, dk, n, B.LA2_BF16, None)
+    assert g(n=-1) == INV
+    assert g(n=0) == OK
+    assert g(gq=None) == INV
+    assert g(gk=None) == INV                         # k given, dphi_k missing
+    assert g(dk=None) == INV
+    assert g(dq=Q) == INV                            # in place over q: not allowed
+    assert g(dq=DV) == INV                           # dq over dphi_k
+    assert g(dk=DQ) == INV                           # outputs alias
+    assert g(gq=DO + 8) == INV
