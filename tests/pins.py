@@ -394,9 +394,48 @@ def pin_feature_map_finite_difference(orc):
     assert err.max() < 1e-5, f"feature map gradient vs finite differences: {err.max():.3e}"
 
 
+def pin_feature_map_chain(orc):
+    """The chain rule through the map, end to end: for loss(q, k) =
+    sum(forward(phi(q), phi(k), v) * dO) the gradient in the unmapped q is
+    backward(phi(q), phi(k), ...)'s dq times phi'(q) (likewise k), against
+    central differences of the whole loss.  The steps keep q +- h exact in
+    float32; the map's values pass to the attention as float32, which with
+    the O(h^2) truncation bounds the agreement near 1e-5; entries within 2h
+    of the kink at 0 are skipped."""
+    q, k, v, dO, lam, s0 = small_case(B=1, H=2, L=9, d=3, e=4, lams=(0.8, 1.0))
+    q, k = q * 4.0, k * 4.0          # both sides of the map; still exact
+    g = orc.backward(orc.feature_map(q), orc.feature_map(k), v, lam, dO, s0)
+    grads = {"q": orc.feature_map_grad(q, g[0]), "k": orc.feature_map_grad(k, g[1])}
+
+    def loss(qq, kk):
+        o = orc.forward(orc.feature_map(qq), orc.feature_map(kk), v, lam, s0)
+        return float(np.sum(o * dO))
+
+    h = 2.0 ** -8
+    rng = np.random.default_rng(4)
+    for name, arr in (("q", q), ("k", k)):
+        done = 0
+        while done < 6:
+            idx = tuple(int(rng.integers(0, n)) for n in arr.shape)
+            if abs(arr[idx]) < 2 * h:
+                continue
+            plus, minus = arr.copy(), arr.copy()
+            plus[idx] += h
+            minus[idx] -= h
+            if name == "q":
+                fd = (loss(plus, k) - loss(minus, k)) / (2 * h)
+            else:
+                fd = (loss(q, plus) - loss(q, minus)) / (2 * h)
+            want = grads[name][idx]
+            assert abs(fd - want) <= 1e-4 * max(1.0, abs(fd)), \
+                f"feature map chain rule d{name}{idx}: {fd} vs {want}"
+            done += 1
+
+
 ALL_PINS = [pin_bruteforce, pin_prefix_sum, pin_lambda_zero, pin_length_one,
             pin_backward_closed_form, pin_backward_terminal_closed_form, pin_backward_split,
             pin_dlambda_closed_form, pin_dlambda_finite_difference,
             pin_finite_difference, pin_adjoint,
             pin_state_handoff, pin_decode_equals_forward, pin_golden,
-            pin_feature_map_values, pin_feature_map_shape, pin_feature_map_finite_difference]
+            pin_feature_map_values, pin_feature_map_shape, pin_feature_map_finite_difference,
+            pin_feature_map_chain]
