@@ -513,7 +513,7 @@ def run_long(args, world, rank, local):
                 "traffic": traffic_for(name, Hh * L), "alg_bytes_per_launch": alg,
                 "avg_launch_ms": avg}
     extra_cpu = {}
-    if rank == 0 and not args.no_cpu:
+    if rank == 0 and world == 1 and not args.no_cpu:
         # the oracle on 16 heads x the first 65,536 rows (a quarter of the
         # heads, 1/16 of the length): token-heads per second / 64 heads
         import oracle
@@ -591,7 +591,7 @@ def run_varlen(args, world, rank, local):
             "traffic": traffic_for(name + "_packed", Hh * T),
             "alg_bytes_per_launch": alg, "avg_launch_ms": avg}
     extra_cpu = {}
-    if rank == 0 and not args.no_cpu:
+    if rank == 0 and world == 1 and not args.no_cpu:
         # the oracle, fwd+bwd, every head, on the documents in batch order
         # until 8,192 rows (copied to the host before the clock starts)
         import oracle
@@ -698,7 +698,7 @@ def run_decode(args, world, rank, local):
     what = ("one decode step per call" if T == 1 else
             f"{T} tokens per call (la2_decode_tokens)")
     extra = {"dtype": "f32", "roofline": roof, "gpu_launches": calls * args.steps, "clocks": clk}
-    if rank == 0 and not args.no_cpu:
+    if rank == 0 and world == 1 and not args.no_cpu:
         import oracle
         orc = oracle.load()
         st = kv[:4].double().cpu().numpy().copy()
@@ -775,7 +775,7 @@ def run_dlambda(args, world, rank, local):
             "peak_source": f"{sms} SMs x 128 fp32 lanes x 2 flops x {mhz:.0f} MHz (max SM clock)"}
     extra = {"dtype": "f32", "roofline": roof, "kernels": prof,
              "gpu_launches": sum(v["launches"] for v in prof.values()), "clocks": clk}
-    if rank == 0 and not args.no_cpu:
+    if rank == 0 and world == 1 and not args.no_cpu:
         import oracle
         orc = oracle.load()
         h = {n: t[:1].double().cpu().numpy() for n, t in x.items()}
@@ -868,7 +868,7 @@ def run_fmap(args, world, rank, local):
     extra = {"dtype": "bf16", "roofline": roof, "roofline_feature_map": fmap_roof,
              "kernels": prof, "gpu_launches": sum(v["launches"] for v in prof.values()),
              "clocks": clk}
-    if rank == 0 and not args.no_cpu:
+    if rank == 0 and world == 1 and not args.no_cpu:
         import oracle
         orc = oracle.load()
         h = {n: t[:1].float().cpu().numpy() for n, t in x.items()}
