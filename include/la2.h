@@ -42,6 +42,9 @@
  *     values in [0, 1] are the meaningful range (0^0 is taken as 1).
  *   - L, B or H equal to 0 is an empty problem: nothing is computed except
  *     that state outputs are still written (kv_out = kv0 or 0; dkv0 = 0).
+ *   - The elementwise feature-map calls (la2_feature_map,
+ *     la2_feature_map_backward) take a count of values instead of shapes and
+ *     may write in place; their declarations state these exceptions.
  *
  * Errors: LA2_ERR_INVALID for bad arguments (null required pointer, negative
  * size, unaligned pointer, an output overlapping an input, kv_out == kv0,
