@@ -1,4 +1,4 @@
-"""Sequence parallelism's exchange on CPU: two gloo ranks each hold one shard
+"""Sequence parallelism's exchange on CPU: two or three gloo ranks each hold one shard
 of a sequence and run seqpar.forward / seqpar.backward with the library calls
 replaced by plain fp64 stand-ins (the oracle and the definitions of the shard
 summaries); the shards' slices must reassemble the oracle's result for the
@@ -8,6 +8,7 @@ import os
 import socket
 
 import numpy as np
+import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
@@ -94,8 +95,10 @@ def _rank_main(rank, world, port, out):
         dist.destroy_process_group()
 
 
-def test_two_ranks_reassemble_the_whole_sequence(orc):
-    world = 2
+@pytest.mark.parametrize("world", [2, 3])
+def test_ranks_reassemble_the_whole_sequence(orc, world):
+    """Three ranks give the middle rank a predecessor and a successor and the
+    end ranks a summary two shards away, which two ranks cannot show."""
     port = _free_port()
     with mp.Manager() as mgr:
         out = mgr.dict()
