@@ -303,3 +303,16 @@ def test_feature_map_validation(lib):
     assert g(dq=DV) == INV                           # dq over dphi_k
     assert g(dk=DQ) == INV                           # outputs alias
     assert g(gq=DO + 8) == INV
+
+
+def test_feature_map_binding_checks(lib):
+    """The Python binding refuses host tensors and mismatched arguments before
+    calling the library."""
+    import torch
+    q = torch.zeros(4, 8, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        la2.feature_map(q, q.clone())
+    with pytest.raises(ValueError, match="both"):
+        la2.feature_map_backward(q, q.clone(), q.clone(), None)
+    with pytest.raises(ValueError, match="both"):
+        la2.feature_map_backward(q, None, q.clone(), q.clone())
