@@ -162,10 +162,31 @@ def sweep_views(x, Bn, L):
     return {n: t.view(Bn, H, L, t.shape[-1]) for n, t in x.items()}
 
 
-def kernel_source_hash():
+# The sources each kernel family's code comes from: a captured DRAM-traffic
+# figure stays valid while these files are unchanged, whatever else changes.
+SOURCE_GROUPS = {
+    "tc": ("la2_tc.cuh", "la2_sm100.cuh", "la2_common.cuh"),
+    "decode": ("la2_decode.cuh", "la2_common.cuh"),
+    "fmap": ("la2_fmap.cuh", "la2_common.cuh"),
+}
+
+
+def group_of(kernel: str) -> str:
+    if kernel.startswith("tc_"):
+        return "tc"
+    if kernel.startswith("decode"):
+        return "decode"
+    if kernel.startswith("feature_map"):
+        return "fmap"
+    return "other"
+
+
+def kernel_source_hash(group: str = "tc"):
+    """sha256 prefix of the sources of one kernel family."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "causal_linear_attention_fwd_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in SOURCE_GROUPS[group]:
+        h.update(f.encode())
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -173,16 +194,18 @@ def kernel_source_hash():
 
 def traffic_for(kernel: str, units: int):
     """dram bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources; scaled to `units` token-heads."""
+    on the current sources of the kernel's family; scaled to `units`
+    token-heads."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         j = json.load(f)
-    if j.get("source_hash") != kernel_source_hash():
-        return None
     k = j.get("kernels", {}).get(kernel)
-    if not k:
+    group = group_of(kernel)
+    if not k or group not in SOURCE_GROUPS:
+        return None
+    if j.get("source_hashes", {}).get(group) != kernel_source_hash(group):
         return None
     return k["dram_bytes_per_token_head"] * units
 

@@ -135,9 +135,42 @@ def _dev(t: torch.Tensor, name: str):
         raise ValueError(f"{name} must be contiguous")
 
 
-def _stream(stream):
-    s = stream if stream is not None else torch.cuda.current_stream()
+def _devices(*named):
+    """Check (name, tensor) pairs -- None tensors skipped -- as _dev does and
+    that all of them live on one device; return that device.  The library
+    launches on the CURRENT device, so a call with tensors elsewhere would
+    run its kernels and tensor maps over another GPU's memory."""
+    dev = None
+    for name, t in named:
+        if t is None:
+            continue
+        _dev(t, name)
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, other arguments on {dev}")
+    if dev is None:
+        raise ValueError("no tensor arguments")
+    return dev
+
+
+def _stream(stream, device=None):
+    if stream is None:
+        s = torch.cuda.current_stream(device)
+    else:
+        s = stream
+        if device is not None and s.device != device:
+            raise ValueError(f"stream is on {s.device}, the tensors on {device}")
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def _out(t, name, shape, dtype, device):
+    """A caller-provided output buffer: contiguous, on `device`, of this
+    shape and dtype."""
+    _dev(t, name)
+    if t.device != device or tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype} {tuple(shape)} on {device}")
+    return t
 
 
 def set_option(option: int, value: int) -> int:
@@ -163,49 +196,60 @@ def forward(q, k, v, lam, kv0=None, *, want_state: bool = False, out=None,
             workspace=None, stream=None):
     """o = (Q K^T (.) M) V (+ the kv0 term); optionally the final state."""
     lib = library()
-    for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam)):
-        _dev(t, name)
+    dev = _devices(("q", q), ("k", k), ("v", v), ("lam", lam), ("kv0", kv0),
+                   ("workspace", workspace))
     B, H, L, d = q.shape
     e = v.shape[-1]
     if k.shape != q.shape or v.shape[:3] != (B, H, L):
         raise ValueError("shape mismatch among q, k, v")
     if lam.dtype != torch.float32 or lam.numel() != H:
         raise ValueError("lam must be float32 [H]")
-    if kv0 is not None:
-        _dev(kv0, "kv0")
-        if kv0.dtype != torch.float32 or kv0.shape != (B, H, d, e):
-            raise ValueError("kv0 must be float32 [B,H,d,e]")
-    o = out if out is not None else torch.empty((B, H, L, e), dtype=q.dtype, device=q.device)
-    st = torch.empty((B, H, d, e), dtype=torch.float32, device=q.device) if want_state else None
-    ws = workspace
-    if ws is None:
-        ws = _workspace(workspace_size(LA2_OP_FORWARD, B, H, L, d, e, q.dtype), q.device)
-    code = lib.la2_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(o), _ptr(st),
-                           B, H, L, d, e, _dt(q), _ptr(ws), 0 if ws is None else ws.numel(),
-                           _stream(stream))
+    if kv0 is not None and (kv0.dtype != torch.float32 or kv0.shape != (B, H, d, e)):
+        raise ValueError("kv0 must be float32 [B,H,d,e]")
+    with torch.cuda.device(dev):
+        o = (_out(out, "out", (B, H, L, e), q.dtype, dev) if out is not None
+             else torch.empty((B, H, L, e), dtype=q.dtype, device=dev))
+        st = torch.empty((B, H, d, e), dtype=torch.float32, device=dev) if want_state else None
+        ws = workspace
+        if ws is None:
+            ws = _workspace(workspace_size(LA2_OP_FORWARD, B, H, L, d, e, q.dtype), dev)
+        code = lib.la2_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(o),
+                               _ptr(st), B, H, L, d, e, _dt(q), _ptr(ws),
+                               0 if ws is None else ws.numel() * ws.element_size(),
+                               _stream(stream, dev))
     _check(code, "la2_forward")
     return (o, st) if want_state else o
 
 
 def forward_noalloc(q, k, v, lam, kv0=None, *, want_state: bool = False, out=None,
-                    stream=None):
+                    state_out=None, stream=None):
     """forward() for callers that cannot allocate device scratch: the library
     keeps the chunk-boundary states in its own fixed 32 MiB device array
-    (see la2_forward_noalloc in include/la2.h).  Outputs are still allocated
-    here unless `out` (and the caller's own state buffer) are passed."""
+    (see la2_forward_noalloc in include/la2.h).  Outputs are allocated here
+    unless the caller passes them: `out` (o) and, with want_state,
+    `state_out` (the final state)."""
     lib = library()
-    for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam)):
-        _dev(t, name)
+    dev = _devices(("q", q), ("k", k), ("v", v), ("lam", lam), ("kv0", kv0))
     B, H, L, d = q.shape
     e = v.shape[-1]
     if k.shape != q.shape or v.shape[:3] != (B, H, L):
         raise ValueError("shape mismatch among q, k, v")
     if lam.dtype != torch.float32 or lam.numel() != H:
         raise ValueError("lam must be float32 [H]")
-    o = out if out is not None else torch.empty((B, H, L, e), dtype=q.dtype, device=q.device)
-    st = torch.empty((B, H, d, e), dtype=torch.float32, device=q.device) if want_state else None
-    code = lib.la2_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(o),
-                                   _ptr(st), B, H, L, d, e, _dt(q), _stream(stream))
+    if kv0 is not None and (kv0.dtype != torch.float32 or kv0.shape != (B, H, d, e)):
+        raise ValueError("kv0 must be float32 [B,H,d,e]")
+    if state_out is not None and not want_state:
+        raise ValueError("state_out is given but want_state is False")
+    with torch.cuda.device(dev):
+        o = (_out(out, "out", (B, H, L, e), q.dtype, dev) if out is not None
+             else torch.empty((B, H, L, e), dtype=q.dtype, device=dev))
+        st = None
+        if want_state:
+            st = (_out(state_out, "state_out", (B, H, d, e), torch.float32, dev)
+                  if state_out is not None
+                  else torch.empty((B, H, d, e), dtype=torch.float32, device=dev))
+        code = lib.la2_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(o),
+                                       _ptr(st), B, H, L, d, e, _dt(q), _stream(stream, dev))
     _check(code, "la2_forward_noalloc")
     return (o, st) if want_state else o
 
@@ -220,37 +264,40 @@ def backward(q, k, v, lam, dO, kv0=None, *, want_dkv0: bool = False, outs=None,
     if reuse_forward_states and workspace is None:
         raise ValueError("reuse_forward_states needs the forward's workspace")
     lib = library()
-    for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam), ("dO", dO)):
-        _dev(t, name)
+    dev = _devices(("q", q), ("k", k), ("v", v), ("lam", lam), ("dO", dO), ("kv0", kv0),
+                   ("workspace", workspace))
     B, H, L, d = q.shape
     e = v.shape[-1]
     if k.shape != q.shape or v.shape[:3] != (B, H, L) or dO.shape != v.shape:
         raise ValueError("shape mismatch among q, k, v, dO")
     if lam.dtype != torch.float32 or lam.numel() != H:
         raise ValueError("lam must be float32 [H]")
-    if kv0 is not None:
-        _dev(kv0, "kv0")
-    if outs is not None:
-        dq, dk, dv = outs
-    else:
-        dq = torch.empty_like(q)
-        dk = torch.empty_like(k)
-        dv = torch.empty_like(v)
-    dkv0 = torch.empty((B, H, d, e), dtype=torch.float32, device=q.device) if want_dkv0 else None
-    ws = workspace
-    if ws is None:
-        ws = _workspace(workspace_size(LA2_OP_BACKWARD, B, H, L, d, e, q.dtype), q.device)
-    code = lib.la2_backward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(dO),
-                               _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dkv0), B, H, L, d, e, _dt(q),
-                               _ptr(ws), 0 if ws is None else ws.numel(),
-                               1 if reuse_forward_states else 0, _stream(stream))
+    if kv0 is not None and (kv0.dtype != torch.float32 or kv0.shape != (B, H, d, e)):
+        raise ValueError("kv0 must be float32 [B,H,d,e]")
+    with torch.cuda.device(dev):
+        if outs is not None:
+            dq, dk, dv = outs
+            _out(dq, "dq", q.shape, q.dtype, dev)
+            _out(dk, "dk", k.shape, q.dtype, dev)
+            _out(dv, "dv", v.shape, q.dtype, dev)
+        else:
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        dkv0 = torch.empty((B, H, d, e), dtype=torch.float32, device=dev) if want_dkv0 else None
+        ws = workspace
+        if ws is None:
+            ws = _workspace(workspace_size(LA2_OP_BACKWARD, B, H, L, d, e, q.dtype), dev)
+        code = lib.la2_backward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(dO),
+                                   _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dkv0), B, H, L, d, e,
+                                   _dt(q), _ptr(ws),
+                                   0 if ws is None else ws.numel() * ws.element_size(),
+                                   1 if reuse_forward_states else 0, _stream(stream, dev))
     _check(code, "la2_backward")
     return (dq, dk, dv, dkv0) if want_dkv0 else (dq, dk, dv)
 
 
-def _varlen_args(q, k, v, lam, cu_seqlens, kv0):
-    for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam), ("cu_seqlens", cu_seqlens)):
-        _dev(t, name)
+def _varlen_args(q, k, v, lam, cu_seqlens, kv0, *extra):
+    dev = _devices(("q", q), ("k", k), ("v", v), ("lam", lam), ("cu_seqlens", cu_seqlens),
+                   ("kv0", kv0), *extra)
     H, T, d = q.shape
     e = v.shape[-1]
     if k.shape != q.shape or v.shape[:2] != (H, T):
@@ -260,11 +307,9 @@ def _varlen_args(q, k, v, lam, cu_seqlens, kv0):
     if cu_seqlens.dtype != torch.int64 or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
         raise ValueError("cu_seqlens must be int64 [N+1]")
     N = cu_seqlens.numel() - 1
-    if kv0 is not None:
-        _dev(kv0, "kv0")
-        if kv0.dtype != torch.float32 or kv0.shape != (N, H, d, e):
-            raise ValueError("kv0 must be float32 [N,H,d,e]")
-    return N, H, T, d, e
+    if kv0 is not None and (kv0.dtype != torch.float32 or kv0.shape != (N, H, d, e)):
+        raise ValueError("kv0 must be float32 [N,H,d,e]")
+    return dev, N, H, T, d, e
 
 
 def forward_varlen(q, k, v, lam, cu_seqlens, kv0=None, *, want_state: bool = False,
@@ -273,12 +318,14 @@ def forward_varlen(q, k, v, lam, cu_seqlens, kv0=None, *, want_state: bool = Fal
     rows cu_seqlens[n]..cu_seqlens[n+1] of every head; per-sequence states
     [N,H,d,e].  Returns o [H,T,e] (and the final states)."""
     lib = library()
-    N, H, T, d, e = _varlen_args(q, k, v, lam, cu_seqlens, kv0)
-    o = out if out is not None else torch.empty((H, T, e), dtype=q.dtype, device=q.device)
-    st = torch.empty((N, H, d, e), dtype=torch.float32, device=q.device) if want_state else None
-    code = lib.la2_forward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(cu_seqlens),
-                                  _ptr(kv0), _ptr(o), _ptr(st), N, H, T, d, e, _dt(q),
-                                  _stream(stream))
+    dev, N, H, T, d, e = _varlen_args(q, k, v, lam, cu_seqlens, kv0)
+    with torch.cuda.device(dev):
+        o = (_out(out, "out", (H, T, e), q.dtype, dev) if out is not None
+             else torch.empty((H, T, e), dtype=q.dtype, device=dev))
+        st = torch.empty((N, H, d, e), dtype=torch.float32, device=dev) if want_state else None
+        code = lib.la2_forward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(cu_seqlens),
+                                      _ptr(kv0), _ptr(o), _ptr(st), N, H, T, d, e, _dt(q),
+                                      _stream(stream, dev))
     _check(code, "la2_forward_varlen")
     return (o, st) if want_state else o
 
@@ -287,18 +334,21 @@ def backward_varlen(q, k, v, lam, cu_seqlens, dO, kv0=None, *, want_dkv0: bool =
                     outs=None, stream=None):
     """Gradients (dq, dk, dv[, dkv0]) of sum(o * dO) for forward_varlen."""
     lib = library()
-    N, H, T, d, e = _varlen_args(q, k, v, lam, cu_seqlens, kv0)
-    _dev(dO, "dO")
+    dev, N, H, T, d, e = _varlen_args(q, k, v, lam, cu_seqlens, kv0, ("dO", dO))
     if dO.shape != v.shape:
         raise ValueError("dO must match v")
-    if outs is not None:
-        dq, dk, dv = outs
-    else:
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    dkv0 = torch.empty((N, H, d, e), dtype=torch.float32, device=q.device) if want_dkv0 else None
-    code = lib.la2_backward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(cu_seqlens),
-                                   _ptr(kv0), _ptr(dO), _ptr(dq), _ptr(dk), _ptr(dv),
-                                   _ptr(dkv0), N, H, T, d, e, _dt(q), _stream(stream))
+    with torch.cuda.device(dev):
+        if outs is not None:
+            dq, dk, dv = outs
+            _out(dq, "dq", q.shape, q.dtype, dev)
+            _out(dk, "dk", k.shape, q.dtype, dev)
+            _out(dv, "dv", v.shape, q.dtype, dev)
+        else:
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        dkv0 = torch.empty((N, H, d, e), dtype=torch.float32, device=dev) if want_dkv0 else None
+        code = lib.la2_backward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(cu_seqlens),
+                                       _ptr(kv0), _ptr(dO), _ptr(dq), _ptr(dk), _ptr(dv),
+                                       _ptr(dkv0), N, H, T, d, e, _dt(q), _stream(stream, dev))
     _check(code, "la2_backward_varlen")
     return (dq, dk, dv, dkv0) if want_dkv0 else (dq, dk, dv)
 
@@ -309,7 +359,6 @@ LA2_POOL_CONTINUE = 1
 def _slots(slots, B):
     if slots is None:
         return None
-    _dev(slots, "slots")
     if slots.dtype != torch.int32 or slots.shape != (B,):
         raise ValueError("slots must be int32 [B]")
     return slots
@@ -321,8 +370,10 @@ def forward_pool(q, k, v, lam, pool, slots, *, continue_state: bool = False, out
     with continue_state, from pool[slots[b]]) and leaves its final state in
     pool[slots[b]].  Returns o [B,H,L,e]."""
     lib = library()
-    for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam), ("pool", pool)):
-        _dev(t, name)
+    if slots is None:
+        raise ValueError("forward_pool needs a slot table")
+    dev = _devices(("q", q), ("k", k), ("v", v), ("lam", lam), ("pool", pool),
+                   ("slots", slots), ("workspace", workspace))
     B, H, L, d = q.shape
     e = v.shape[-1]
     if k.shape != q.shape or v.shape[:3] != (B, H, L):
@@ -330,17 +381,18 @@ def forward_pool(q, k, v, lam, pool, slots, *, continue_state: bool = False, out
     if pool.dtype != torch.float32 or pool.dim() != 4 or pool.shape[1:] != (H, d, e):
         raise ValueError("pool must be float32 [P,H,d,e]")
     slots = _slots(slots, B)
-    if slots is None:
-        raise ValueError("forward_pool needs a slot table")
-    o = out if out is not None else torch.empty((B, H, L, e), dtype=q.dtype, device=q.device)
-    ws = workspace
-    if ws is None:
-        ws = _workspace(workspace_size(LA2_OP_FORWARD, B, H, L, d, e, q.dtype), q.device)
-    code = lib.la2_forward_pool(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(pool), _ptr(slots),
-                                pool.shape[0], _ptr(o),
-                                LA2_POOL_CONTINUE if continue_state else 0, B, H, L, d, e,
-                                _dt(q), _ptr(ws), 0 if ws is None else ws.numel(),
-                                _stream(stream))
+    with torch.cuda.device(dev):
+        o = (_out(out, "out", (B, H, L, e), q.dtype, dev) if out is not None
+             else torch.empty((B, H, L, e), dtype=q.dtype, device=dev))
+        ws = workspace
+        if ws is None:
+            ws = _workspace(workspace_size(LA2_OP_FORWARD, B, H, L, d, e, q.dtype), dev)
+        code = lib.la2_forward_pool(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(pool),
+                                    _ptr(slots), pool.shape[0], _ptr(o),
+                                    LA2_POOL_CONTINUE if continue_state else 0, B, H, L, d, e,
+                                    _dt(q), _ptr(ws),
+                                    0 if ws is None else ws.numel() * ws.element_size(),
+                                    _stream(stream, dev))
     _check(code, "la2_forward_pool")
     return o
 
@@ -350,8 +402,8 @@ def decode_tokens(q, k, v, lam, pool, slots=None, *, out=None, stream=None):
     of request b is pool[slots[b]] (pool[b] without a slot table), updated
     in place; returns o [B,H,T,e]."""
     lib = library()
-    for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam), ("pool", pool)):
-        _dev(t, name)
+    dev = _devices(("q", q), ("k", k), ("v", v), ("lam", lam), ("pool", pool),
+                   ("slots", slots))
     B, H, T, d = q.shape
     e = v.shape[-1]
     if k.shape != q.shape or v.shape[:3] != (B, H, T):
@@ -359,9 +411,12 @@ def decode_tokens(q, k, v, lam, pool, slots=None, *, out=None, stream=None):
     if pool.dtype != torch.float32 or pool.dim() != 4 or pool.shape[1:] != (H, d, e):
         raise ValueError("pool must be float32 [P,H,d,e]")
     slots = _slots(slots, B)
-    o = out if out is not None else torch.empty((B, H, T, e), dtype=q.dtype, device=q.device)
-    code = lib.la2_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(pool), _ptr(slots),
-                                 pool.shape[0], _ptr(o), B, H, T, d, e, _dt(q), _stream(stream))
+    with torch.cuda.device(dev):
+        o = (_out(out, "out", (B, H, T, e), q.dtype, dev) if out is not None
+             else torch.empty((B, H, T, e), dtype=q.dtype, device=dev))
+        code = lib.la2_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(pool),
+                                     _ptr(slots), pool.shape[0], _ptr(o), B, H, T, d, e, _dt(q),
+                                     _stream(stream, dev))
     _check(code, "la2_decode_tokens")
     return o
 
@@ -371,19 +426,20 @@ def shard_state(a, b, lam, *, reverse: bool = False, workspace=None, stream=None
     lam^(L-1-t) k_t^T v_t, reverse (a = q, b = dO) sum_t lam^t q_t^T dO_t;
     fp32 [B,H,d,e]."""
     lib = library()
-    for name, t in (("a", a), ("b", b), ("lam", lam)):
-        _dev(t, name)
+    dev = _devices(("a", a), ("b", b), ("lam", lam), ("workspace", workspace))
     B, H, L, d = a.shape
     e = b.shape[-1]
     if b.shape[:3] != (B, H, L):
         raise ValueError("shape mismatch between a and b")
-    out = torch.empty((B, H, d, e), dtype=torch.float32, device=a.device)
-    ws = workspace
-    if ws is None:
-        ws = _workspace(workspace_size(LA2_OP_SHARD_STATE, B, H, L, d, e, a.dtype), a.device)
-    code = lib.la2_shard_state(_ptr(a), _ptr(b), _ptr(lam), _ptr(out), B, H, L, d, e, _dt(a),
-                               1 if reverse else 0, _ptr(ws), 0 if ws is None else ws.numel(),
-                               _stream(stream))
+    with torch.cuda.device(dev):
+        out = torch.empty((B, H, d, e), dtype=torch.float32, device=dev)
+        ws = workspace
+        if ws is None:
+            ws = _workspace(workspace_size(LA2_OP_SHARD_STATE, B, H, L, d, e, a.dtype), dev)
+        code = lib.la2_shard_state(_ptr(a), _ptr(b), _ptr(lam), _ptr(out), B, H, L, d, e,
+                                   _dt(a), 1 if reverse else 0, _ptr(ws),
+                                   0 if ws is None else ws.numel() * ws.element_size(),
+                                   _stream(stream, dev))
     _check(code, "la2_shard_state")
     return out
 
@@ -393,16 +449,17 @@ def state_prefix(delta, lam, L_shard: int, kv0=None, *, reverse: bool = False, s
     forward, the state entering shard r (from kv0); reverse, the reverse
     state flowing into shard r from the rows after it."""
     lib = library()
-    for name, t in (("delta", delta), ("lam", lam)):
-        _dev(t, name)
+    dev = _devices(("delta", delta), ("lam", lam), ("kv0", kv0))
     if delta.dtype != torch.float32 or delta.dim() != 5:
         raise ValueError("delta must be float32 [R,B,H,d,e]")
     R, B, H, d, e = delta.shape
-    if kv0 is not None:
-        _dev(kv0, "kv0")
-    out = torch.empty_like(delta)
-    code = lib.la2_state_prefix(_ptr(delta), _ptr(kv0), _ptr(lam), _ptr(out), R, B, H,
-                                int(L_shard), d, e, 1 if reverse else 0, _stream(stream))
+    if kv0 is not None and (kv0.dtype != torch.float32 or kv0.shape != (B, H, d, e)):
+        raise ValueError("kv0 must be float32 [B,H,d,e]")
+    with torch.cuda.device(dev):
+        out = torch.empty_like(delta)
+        code = lib.la2_state_prefix(_ptr(delta), _ptr(kv0), _ptr(lam), _ptr(out), R, B, H,
+                                    int(L_shard), d, e, 1 if reverse else 0,
+                                    _stream(stream, dev))
     _check(code, "la2_state_prefix")
     return out
 
@@ -412,29 +469,32 @@ def backward_shard(q, k, v, lam, dO, kv0=None, dstate_end=None, *, want_dkv0: bo
     """backward() of one shard of a longer sequence: kv0 its entry state,
     dstate_end the reverse state flowing in from the rows after it."""
     lib = library()
-    for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam), ("dO", dO)):
-        _dev(t, name)
+    dev = _devices(("q", q), ("k", k), ("v", v), ("lam", lam), ("dO", dO), ("kv0", kv0),
+                   ("dstate_end", dstate_end), ("workspace", workspace))
     B, H, L, d = q.shape
     e = v.shape[-1]
     if k.shape != q.shape or v.shape[:3] != (B, H, L) or dO.shape != v.shape:
         raise ValueError("shape mismatch among q, k, v, dO")
     for name, t in (("kv0", kv0), ("dstate_end", dstate_end)):
-        if t is not None:
-            _dev(t, name)
-            if t.dtype != torch.float32 or t.shape != (B, H, d, e):
-                raise ValueError(f"{name} must be float32 [B,H,d,e]")
-    if outs is not None:
-        dq, dk, dv = outs
-    else:
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    dkv0 = torch.empty((B, H, d, e), dtype=torch.float32, device=q.device) if want_dkv0 else None
-    ws = workspace
-    if ws is None:
-        ws = _workspace(workspace_size(LA2_OP_BACKWARD, B, H, L, d, e, q.dtype), q.device)
-    code = lib.la2_backward_shard(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(dO),
-                                  _ptr(dstate_end), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dkv0),
-                                  B, H, L, d, e, _dt(q), _ptr(ws),
-                                  0 if ws is None else ws.numel(), 0, _stream(stream))
+        if t is not None and (t.dtype != torch.float32 or t.shape != (B, H, d, e)):
+            raise ValueError(f"{name} must be float32 [B,H,d,e]")
+    with torch.cuda.device(dev):
+        if outs is not None:
+            dq, dk, dv = outs
+            _out(dq, "dq", q.shape, q.dtype, dev)
+            _out(dk, "dk", k.shape, q.dtype, dev)
+            _out(dv, "dv", v.shape, q.dtype, dev)
+        else:
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        dkv0 = torch.empty((B, H, d, e), dtype=torch.float32, device=dev) if want_dkv0 else None
+        ws = workspace
+        if ws is None:
+            ws = _workspace(workspace_size(LA2_OP_BACKWARD, B, H, L, d, e, q.dtype), dev)
+        code = lib.la2_backward_shard(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(dO),
+                                      _ptr(dstate_end), _ptr(dq), _ptr(dk), _ptr(dv),
+                                      _ptr(dkv0), B, H, L, d, e, _dt(q), _ptr(ws),
+                                      0 if ws is None else ws.numel() * ws.element_size(), 0,
+                                      _stream(stream, dev))
     _check(code, "la2_backward_shard")
     return (dq, dk, dv, dkv0) if want_dkv0 else (dq, dk, dv)
 
@@ -445,52 +505,55 @@ def dlambda(q, k, v, lam, dO, kv0=None, *, workspace=None, chunked: bool = True,
     (la2_backward_dlambda_ex with `workspace`, allocated here when None);
     False: one CTA per (b,h), no workspace (la2_backward_dlambda)."""
     lib = library()
-    for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam), ("dO", dO)):
-        _dev(t, name)
+    dev = _devices(("q", q), ("k", k), ("v", v), ("lam", lam), ("dO", dO), ("kv0", kv0),
+                   ("workspace", workspace))
     B, H, L, d = q.shape
     e = v.shape[-1]
     if k.shape != q.shape or v.shape[:3] != (B, H, L) or dO.shape != v.shape:
         raise ValueError("shape mismatch among q, k, v, dO")
-    if kv0 is not None:
-        _dev(kv0, "kv0")
-    out = torch.empty(H, dtype=torch.float32, device=q.device)
-    if not chunked:
-        code = lib.la2_backward_dlambda(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(dO),
-                                        _ptr(out), B, H, L, d, e, _dt(q), _stream(stream))
-        _check(code, "la2_backward_dlambda")
-        return out
-    if workspace is None:
-        workspace = _workspace(workspace_size(LA2_OP_DLAMBDA, B, H, L, d, e, q.dtype), q.device)
-    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    code = lib.la2_backward_dlambda_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0), _ptr(dO),
-                                       _ptr(out), B, H, L, d, e, _dt(q), _ptr(workspace), nbytes,
-                                       _stream(stream))
+    if lam.dtype != torch.float32 or lam.numel() != H:
+        raise ValueError("lam must be float32 [H]")
+    if kv0 is not None and (kv0.dtype != torch.float32 or kv0.shape != (B, H, d, e)):
+        raise ValueError("kv0 must be float32 [B,H,d,e]")
+    with torch.cuda.device(dev):
+        out = torch.empty(H, dtype=torch.float32, device=dev)
+        if not chunked:
+            code = lib.la2_backward_dlambda(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0),
+                                            _ptr(dO), _ptr(out), B, H, L, d, e, _dt(q),
+                                            _stream(stream, dev))
+            _check(code, "la2_backward_dlambda")
+            return out
+        if workspace is None:
+            workspace = _workspace(workspace_size(LA2_OP_DLAMBDA, B, H, L, d, e, q.dtype), dev)
+        nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        code = lib.la2_backward_dlambda_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv0),
+                                           _ptr(dO), _ptr(out), B, H, L, d, e, _dt(q),
+                                           _ptr(workspace), nbytes, _stream(stream, dev))
     _check(code, "la2_backward_dlambda_ex")
     return out
 
 
 def _fmap_args(q, k, extra):
-    _dev(q, "q")
-    if k is not None:
-        _dev(k, "k")
-        if k.shape != q.shape or k.dtype != q.dtype:
-            raise ValueError("q and k must have the same shape and dtype")
+    dev = _devices(("q", q), ("k", k), *extra)
+    if k is not None and (k.shape != q.shape or k.dtype != q.dtype):
+        raise ValueError("q and k must have the same shape and dtype")
     for name, t in extra:
-        if t is not None:
-            _dev(t, name)
-            if t.shape != q.shape or t.dtype != q.dtype:
-                raise ValueError(f"{name} must match q's shape and dtype")
+        if t is not None and (t.shape != q.shape or t.dtype != q.dtype):
+            raise ValueError(f"{name} must match q's shape and dtype")
+    return dev
 
 
 def feature_map(q, k=None, *, out=None, stream=None):
     """phi(x) = elu(x) + 1 applied to q (and k): returns phi_q (and phi_k).
     out: (phi_q, phi_k) buffers, which may be q and k themselves (in place)."""
     lib = library()
-    phi_q, phi_k = out if out is not None else (
-        torch.empty_like(q), None if k is None else torch.empty_like(k))
-    _fmap_args(q, k, (("phi_q", phi_q), ("phi_k", phi_k)))
-    code = lib.la2_feature_map(_ptr(q), _ptr(k), _ptr(phi_q), _ptr(phi_k), q.numel(), _dt(q),
-                               _stream(stream))
+    dev = _fmap_args(q, k, ())
+    with torch.cuda.device(dev):
+        phi_q, phi_k = out if out is not None else (
+            torch.empty_like(q), None if k is None else torch.empty_like(k))
+        _fmap_args(q, k, (("phi_q", phi_q), ("phi_k", phi_k)))
+        code = lib.la2_feature_map(_ptr(q), _ptr(k), _ptr(phi_q), _ptr(phi_k), q.numel(),
+                                   _dt(q), _stream(stream, dev))
     _check(code, "la2_feature_map")
     return phi_q if k is None else (phi_q, phi_k)
 
@@ -503,11 +566,14 @@ def feature_map_backward(q, k, dphi_q, dphi_k=None, *, out=None, stream=None):
     lib = library()
     if (k is None) != (dphi_k is None):
         raise ValueError("k and dphi_k are both given or both None")
-    dq, dk = out if out is not None else (
-        torch.empty_like(q), None if k is None else torch.empty_like(k))
-    _fmap_args(q, k, (("dphi_q", dphi_q), ("dphi_k", dphi_k), ("dq", dq), ("dk", dk)))
-    code = lib.la2_feature_map_backward(_ptr(q), _ptr(k), _ptr(dphi_q), _ptr(dphi_k), _ptr(dq),
-                                        _ptr(dk), q.numel(), _dt(q), _stream(stream))
+    dev = _fmap_args(q, k, (("dphi_q", dphi_q), ("dphi_k", dphi_k)))
+    with torch.cuda.device(dev):
+        dq, dk = out if out is not None else (
+            torch.empty_like(q), None if k is None else torch.empty_like(k))
+        _fmap_args(q, k, (("dphi_q", dphi_q), ("dphi_k", dphi_k), ("dq", dq), ("dk", dk)))
+        code = lib.la2_feature_map_backward(_ptr(q), _ptr(k), _ptr(dphi_q), _ptr(dphi_k),
+                                            _ptr(dq), _ptr(dk), q.numel(), _dt(q),
+                                            _stream(stream, dev))
     _check(code, "la2_feature_map_backward")
     return dq if k is None else (dq, dk)
 
@@ -515,15 +581,16 @@ def feature_map_backward(q, k, dphi_q, dphi_k=None, *, out=None, stream=None):
 def decode_step(q, k, v, lam, kv, *, out=None, stream=None):
     """kv <- lam kv + k^T v (in place); returns o = q kv."""
     lib = library()
-    for name, t in (("q", q), ("k", k), ("v", v), ("lam", lam), ("kv", kv)):
-        _dev(t, name)
+    dev = _devices(("q", q), ("k", k), ("v", v), ("lam", lam), ("kv", kv))
     B, H, d = q.shape
     e = v.shape[-1]
     if kv.dtype != torch.float32 or kv.shape != (B, H, d, e):
         raise ValueError("kv must be float32 [B,H,d,e]")
-    o = out if out is not None else torch.empty((B, H, e), dtype=q.dtype, device=q.device)
-    code = lib.la2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv), _ptr(o),
-                               B, H, d, e, _dt(q), _stream(stream))
+    with torch.cuda.device(dev):
+        o = (_out(out, "out", (B, H, e), q.dtype, dev) if out is not None
+             else torch.empty((B, H, e), dtype=q.dtype, device=dev))
+        code = lib.la2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(kv), _ptr(o),
+                                   B, H, d, e, _dt(q), _stream(stream, dev))
     _check(code, "la2_decode_step")
     return o
 

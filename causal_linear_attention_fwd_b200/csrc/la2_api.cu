@@ -545,10 +545,17 @@ size_t la2_workspace_size(int op, int B, int H, int64_t L, int d, int e, la2_dty
   return ws_bytes(op, g, d, e);
 }
 
-la2_status la2_forward(const void *q, const void *k, const void *v,
-                       const float *lambda, const float *kv0, void *o, float *kv_out,
-                       int B, int H, int64_t L, int d, int e, la2_dtype dt,
-                       void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The argument checks of la2_forward (and of la2_forward_noalloc, which
+// passes no workspace).  LA2_OK with *empty set: B*H == 0, nothing to do.
+la2_status forward_checks(const void *q, const void *k, const void *v, const float *lambda,
+                          const float *kv0, const void *o, const float *kv_out, int B, int H,
+                          int64_t L, int d, int e, la2_dtype dt, const void *workspace,
+                          size_t workspace_bytes, bool *empty) {
+  *empty = false;
   if (B < 0 || H < 0 || L < 0) return LA2_ERR_INVALID;
   if (dt != LA2_F32 && dt != LA2_BF16) return LA2_ERR_UNSUPPORTED;
   if (!shape_supported(d, e, dt)) return LA2_ERR_UNSUPPORTED;
@@ -556,7 +563,10 @@ la2_status la2_forward(const void *q, const void *k, const void *v,
   const size_t es = esize(dt);
   const size_t nq = (size_t)BH * L * d * es, nv = (size_t)BH * L * e * es;
   const size_t ns = (size_t)BH * d * e * sizeof(float);
-  if (BH == 0) return LA2_OK;
+  if (BH == 0) {
+    *empty = true;
+    return LA2_OK;
+  }
   if (!lambda || (L > 0 && (!q || !k || !v || !o))) return LA2_ERR_INVALID;
   for (const void *p : std::initializer_list<const void *>{(const void *)q, (const void *)k, (const void *)v, (const void *)lambda,
                         (const void *)kv0, (const void *)o, (const void *)kv_out, workspace})
@@ -565,6 +575,23 @@ la2_status la2_forward(const void *q, const void *k, const void *v,
   std::vector<Span> ins = {{q, nq}, {k, nq}, {v, nv}, {lambda, (size_t)H * 4}, {kv0, kv0 ? ns : 0}};
   std::vector<Span> outs = {{o, nv}, {kv_out, kv_out ? ns : 0}, {workspace, workspace_bytes}};
   if (any_overlap(outs, ins)) return LA2_ERR_INVALID;
+  return LA2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+la2_status la2_forward(const void *q, const void *k, const void *v,
+                       const float *lambda, const float *kv0, void *o, float *kv_out,
+                       int B, int H, int64_t L, int d, int e, la2_dtype dt,
+                       void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+  bool empty = false;
+  const la2_status chk = forward_checks(q, k, v, lambda, kv0, o, kv_out, B, H, L, d, e, dt,
+                                        workspace, workspace_bytes, &empty);
+  if (chk != LA2_OK || empty) return chk;
+  const int64_t BH = (int64_t)B * H;
+  const size_t ns = (size_t)BH * d * e * sizeof(float);
 
   if (L == 0) {
     if (!kv_out) return LA2_OK;
@@ -1210,13 +1237,18 @@ extern "C" la2_status la2_forward_noalloc(const void *q, const void *k, const vo
                                           const float *lambda, const float *kv0, void *o,
                                           float *kv_out, int B, int H, int64_t L, int d, int e,
                                           la2_dtype dt, cudaStream_t stream) {
+  // la2_forward's argument checks first: a call it would refuse touches
+  // neither the device nor the array.
+  bool empty = false;
+  const la2_status chk = forward_checks(q, k, v, lambda, kv0, o, kv_out, B, H, L, d, e, dt,
+                                        nullptr, 0, &empty);
+  if (chk != LA2_OK || empty) return chk;
   // Same plan as la2_forward; refuse plans whose scratch exceeds the array.
-  if (B > 0 && H > 0 && L > 0 && shape_supported(d, e, dt)) {
+  if (L > 0) {
     const Path p = choose_path(d, e, dt);
-    if (p != PATH_NONE) {
-      const Geo g = plan(B, H, L, block_rows(p), p);
-      if (ws_bytes(LA2_OP_FORWARD, g, d, e) > kNoallocScratchBytes) return LA2_ERR_UNSUPPORTED;
-    }
+    if (p == PATH_NONE) return LA2_ERR_UNSUPPORTED;
+    const Geo g = plan(B, H, L, block_rows(p), p);
+    if (ws_bytes(LA2_OP_FORWARD, g, d, e) > kNoallocScratchBytes) return LA2_ERR_UNSUPPORTED;
   }
   void *scratch = noalloc_scratch_ptr();
   if (!scratch) return LA2_ERR_CUDA;

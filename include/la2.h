@@ -119,9 +119,14 @@ la2_status la2_forward(const void *q, const void *k, const void *v,
  * device array that every GPU loading the library holds until the process
  * exits.  Calls whose plan needs more than 32 MiB of states (B*H*S*d*e*4
  * bytes, S = chunks per sequence) return LA2_ERR_UNSUPPORTED before
- * launching anything.  The first call on a device looks up the array's
- * device address (once per device) and should come before any stream
- * capture.  All calls share the array and it keeps the last call's contents
+ * launching anything.  Arguments are checked exactly as la2_forward checks
+ * them, before the array is touched.  The first valid call on a device looks
+ * up the array's device address (once per device, with that device current)
+ * and should come before any stream capture.  The address is kept for the
+ * life of the process and belongs to the device's current context: after a
+ * cudaDeviceReset() of that device the kept address is stale, so a process
+ * that resets a device must not call this entry point on it again.  All
+ * calls share the array and it keeps the last call's contents
  * (every state it holds is written before it is read, so nothing needs
  * clearing); calls that overlap on the same GPU -- from concurrent streams
  * or host threads -- race on it, so serialise them.  Each GPU has its own

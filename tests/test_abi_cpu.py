@@ -316,3 +316,43 @@ def test_feature_map_binding_checks(lib):
         la2.feature_map_backward(q, q.clone(), q.clone(), None)
     with pytest.raises(ValueError, match="both"):
         la2.feature_map_backward(q, None, q.clone(), q.clone())
+
+
+class _FakeCuda:
+    """A stand-in for a CUDA tensor (no GPU here): only what the binding's
+    device checks read."""
+
+    def __init__(self, device):
+        import torch
+        self.device = torch.device(device)
+        self.is_cuda = True
+
+    def is_contiguous(self):
+        return True
+
+
+def test_binding_rejects_mixed_devices():
+    """Every tensor argument of a call must live on one device: the library
+    launches on the current device, so a tensor on another GPU would be read
+    through the wrong device's tensor maps."""
+    import torch
+    a, b = _FakeCuda("cuda:0"), _FakeCuda("cuda:1")
+    assert B._devices(("q", a), ("k", _FakeCuda("cuda:0")), ("kv0", None)) == torch.device("cuda:0")
+    with pytest.raises(ValueError, match="k is on cuda:1"):
+        B._devices(("q", a), ("k", b))
+    with pytest.raises(ValueError, match="CUDA"):
+        B._devices(("q", a), ("v", torch.zeros(2)))
+    with pytest.raises(ValueError, match="no tensor"):
+        B._devices(("kv0", None))
+
+
+def test_noalloc_binding_checks(lib):
+    """forward_noalloc checks its arguments as forward() does, kv0 included,
+    before anything reaches the library."""
+    import torch
+    q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
+    lam = torch.zeros(2)
+    with pytest.raises(ValueError, match="CUDA"):
+        la2.forward_noalloc(q, q, q, lam)
+    with pytest.raises(ValueError, match="CUDA"):
+        la2.forward(q, q, q, lam)

@@ -40,13 +40,29 @@ def test_traffic_only_for_the_captured_sources(tmp_path, monkeypatch):
                     root / "causal_linear_attention_fwd_b200" / "csrc")
     (root / "profiles").mkdir()
     monkeypatch.setattr(bench, "ROOT", str(root))
-    h = bench.kernel_source_hash()
-    rec = {"source_hash": h, "kernels": {"tc_fwd": {"dram_bytes_per_token_head": 1013.0}}}
+    h = bench.kernel_source_hash("tc")
+    rec = {"source_hashes": {"tc": h},
+           "kernels": {"tc_fwd": {"dram_bytes_per_token_head": 1013.0}}}
     (root / "profiles" / "traffic.json").write_text(json.dumps(rec))
     assert bench.traffic_for("tc_fwd", 1000) == 1013.0 * 1000
     assert bench.traffic_for("tc_dq", 1000) is None                  # not captured
-    # any change to the kernel sources retires the figures
-    f = root / "causal_linear_attention_fwd_b200" / "csrc" / "la2_tc.cuh"
+    csrc = root / "causal_linear_attention_fwd_b200" / "csrc"
+    # a change outside the tensor-core kernels' sources leaves the figures
+    f = csrc / "la2_fmap.cuh"
     f.write_text(f.read_text() + "\n")
-    assert bench.kernel_source_hash() != h
+    assert bench.kernel_source_hash("tc") == h
+    assert bench.traffic_for("tc_fwd", 1000) == 1013.0 * 1000
+    # any change to the tensor-core kernels' sources retires them
+    f = csrc / "la2_tc.cuh"
+    f.write_text(f.read_text() + "\n")
+    assert bench.kernel_source_hash("tc") != h
     assert bench.traffic_for("tc_fwd", 1000) is None
+
+
+def test_source_groups_name_existing_files():
+    csrc = os.path.join(bench.ROOT, "causal_linear_attention_fwd_b200", "csrc")
+    for group, files in bench.SOURCE_GROUPS.items():
+        for f in files:
+            assert os.path.exists(os.path.join(csrc, f)), (group, f)
+    assert bench.group_of("tc_dv") == "tc" and bench.group_of("decode_step") == "decode"
+    assert bench.group_of("feature_map_grad") == "fmap"
