@@ -41,8 +41,9 @@ TOKENS = 65536
 #   kernel reads k,v,dO and writes dq; the dV kernel reads k,q,dO and writes
 #   dv; the dK kernel reads v,dO,q and writes dk (the portable dK/dV kernel
 #   reads q,k,v,dO and writes dk,dv).  The whole fwd+bwd needs at least 2,816 B.
+#   The paired dV/dK launch (tc_dkdv) reads k,q,dO,v once and writes dk,dv.
 BYTES_PER_TH = {"tc_fwd": 1024, "simt_fwd": 1024, "tc_dq": 1024, "simt_dq": 1024,
-                "tc_dv": 1024, "tc_dk": 1024, "simt_dkdv": 1536}
+                "tc_dv": 1024, "tc_dk": 1024, "tc_dkdv": 1536, "simt_dkdv": 1536}
 FWD_BWD_MIN_BYTES = 2816
 # method flops per token-head, intra part over the causal triangle at a
 # fixed C = 64 accounting: fwd (C+1)(d+e) + 4de, bwd (C+1)(3d+2e) + 10de
@@ -913,6 +914,29 @@ def run_fmap(args, world, rank, local):
                     "l2": "inputs 512 MiB per tensor, larger than L2; no flush"}, ms, extra)
 
 
+def run_subrecords(args, world, rank, local):
+    """The two other spec workloads, measured in the same run as the
+    sweep: the long-context forward (B=1, H=64, L=1M) and recurrent decode
+    (batch 256, H=64, 1,024 steps of one token).  Each is the line its own
+    --workload run prints, with --sub-steps timed steps; the sweep's buffers
+    are released first."""
+    import copy
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    sub = copy.copy(args)
+    sub.steps = args.sub_steps
+    sub.warmup = 3
+    out = {}
+    out["long_context"] = run_long(sub, world, rank, local)
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    sub.decode_tokens = 1
+    out["decode"] = run_decode(sub, world, rank, local)
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -929,6 +953,15 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--decode-tokens", type=int, default=1,
                     help="decode workload: tokens per request per call (1 = decode_step)")
+    ap.add_argument("--no-sub", action="store_true",
+                    help="sweep workload: skip the long-context forward and decode "
+                         "sub-records that the default line carries")
+    ap.add_argument("--sub-steps", type=int, default=5,
+                    help="timed steps of each sub-record (decode: graph replays of "
+                         "--decode-steps tokens)")
+    ap.add_argument("--bwd-form", type=int, default=None,
+                    help="profiling aid: LA2_OPT_BWD_FORM for the run (0 paired dV/dK "
+                         "launch, the library's default; 1 two separate passes)")
     ap.add_argument("--only", default=None,
                     help="B:L -- time a single sweep point instead of the whole sweep "
                          "(profiling aid; not the metric)")
@@ -947,10 +980,15 @@ def main():
             print(json.dumps(line), flush=True)
         return
     world, rank, local = dist_setup(args.gpus)
+    if args.bwd_form is not None:
+        import causal_linear_attention_fwd_b200 as la2
+        la2.set_option(la2.LA2_OPT_BWD_FORM, args.bwd_form)
     try:
         fn = {"sweep": run_la2, "long": run_long, "decode": run_decode,
               "varlen": run_varlen, "dlambda": run_dlambda, "fmap": run_fmap}[args.workload]
         line = fn(args, world, rank, local)
+        if args.workload == "sweep" and not args.no_sub and not args.only:
+            line["subrecords"] = run_subrecords(args, world, rank, local)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

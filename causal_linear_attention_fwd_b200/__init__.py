@@ -13,7 +13,8 @@ from ._binding import (  # noqa: F401
     LA2Error, LA2_OP_BACKWARD, LA2_OP_FORWARD, LA2_OPT_INJECT_TIMEOUT, LA2_OPT_PATH,
     LA2_POOL_CONTINUE, LA2_OP_SHARD_STATE, LA2_OP_DLAMBDA, backward_shard, decode_tokens, forward_pool,
     shard_state, state_prefix, dlambda,
-    LA2_OPT_SPLIT, LA2_OPT_TRACE, LA2_OPT_VARIANT, LA2_OPT_VARLEN_ORDER, LA2_OPT_DECODE_BLOCK_TOKENS, trace_read,
+    LA2_OPT_SPLIT, LA2_OPT_TRACE, LA2_OPT_VARIANT, LA2_OPT_VARLEN_ORDER, LA2_OPT_DECODE_BLOCK_TOKENS, LA2_OPT_BWD_FORM,
+    trace_read,
     backward, backward_varlen, decode_step, feature_map, feature_map_backward, forward,
     forward_noalloc, forward_varlen,
     last_device_error, library, profile_enable, profile_report, set_option, status_string,

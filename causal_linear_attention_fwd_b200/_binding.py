@@ -21,7 +21,7 @@ LA2_OK, LA2_ERR_INVALID, LA2_ERR_UNSUPPORTED, LA2_ERR_CUDA, LA2_ERR_TIMEOUT = ra
 LA2_F32, LA2_BF16 = 0, 1
 LA2_OP_FORWARD, LA2_OP_BACKWARD, LA2_OP_SHARD_STATE, LA2_OP_DLAMBDA = 0, 1, 2, 3
 LA2_OPT_SPLIT, LA2_OPT_PATH, LA2_OPT_INJECT_TIMEOUT, LA2_OPT_VARIANT, LA2_OPT_TRACE = 0, 1, 2, 3, 4
-LA2_OPT_VARLEN_ORDER, LA2_OPT_DECODE_BLOCK_TOKENS = 5, 6
+LA2_OPT_VARLEN_ORDER, LA2_OPT_DECODE_BLOCK_TOKENS, LA2_OPT_BWD_FORM = 5, 6, 7
 
 _lock = threading.Lock()
 _lib = None

@@ -9,6 +9,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <type_traits>
 #include <vector>
 
 #include "../../include/la2.h"
@@ -30,20 +31,22 @@ std::atomic<int> g_opt_variant{0};
 std::atomic<int> g_opt_trace{0};
 std::atomic<int> g_opt_varlen_order{0};
 std::atomic<int> g_opt_decode_block{0};
+std::atomic<int> g_opt_bwd_form{0};
 
 // ------------------------------------------------------------ profiling
 enum KernelId {
   K_SIMT_FWD_STATE, K_SIMT_FWD_SCAN, K_SIMT_FWD, K_SIMT_DQ, K_SIMT_REV_STATE,
   K_SIMT_REV_SCAN, K_SIMT_DKDV, K_DECODE, K_TC_FWD_STATE, K_TC_FWD, K_TC_DQ,
   K_TC_REV_STATE, K_TC_DV, K_TC_DK, K_SCAN_FWD, K_SCAN_REV, K_SIMT_DLAMBDA,
-  K_SIMT_DLAMBDA_STATE, K_SIMT_DLAMBDA_SCAN, K_TC_DECODE_UNITS, K_FMAP, K_FMAP_GRAD, K_COUNT
+  K_SIMT_DLAMBDA_STATE, K_SIMT_DLAMBDA_SCAN, K_TC_DECODE_UNITS, K_FMAP, K_FMAP_GRAD, K_TC_DKDV,
+  K_COUNT
 };
 const char *kKernelName[K_COUNT] = {
     "simt_fwd_chunk_state", "simt_scan_fwd", "simt_fwd", "simt_dq",
     "simt_rev_chunk_state", "simt_scan_rev", "simt_dkdv", "decode_step",
     "tc_fwd_chunk_state", "tc_fwd", "tc_dq", "tc_rev_chunk_state", "tc_dv", "tc_dk",
     "scan_fwd", "scan_rev", "simt_dlambda", "simt_dlambda_chunk_state", "simt_dlambda_scan",
-    "tc_decode_units", "feature_map", "feature_map_grad"};
+    "tc_decode_units", "feature_map", "feature_map_grad", "tc_dkdv"};
 
 struct ProfRec {
   int kid;
@@ -68,12 +71,23 @@ cudaEvent_t ev_get() {
 
 // Runs `launch` (which enqueues one kernel on `st`) and, while profiling is
 // on, brackets it with events.  Returns the launch error, if any.
+// Runs a launch callable: one that returns void (the launch's error is
+// then the runtime's last error) or its own cudaError_t.
 template <typename F>
-cudaError_t timed(int kid, cudaStream_t st, F &&launch) {
-  if (!g_prof_on.load(std::memory_order_relaxed)) {
+cudaError_t run_launch(F &&launch) {
+  if constexpr (std::is_same_v<decltype(launch()), cudaError_t>) {
+    const cudaError_t e = launch();
+    const cudaError_t last = cudaGetLastError();
+    return e != cudaSuccess ? e : last;
+  } else {
     launch();
     return cudaGetLastError();
   }
+}
+
+template <typename F>
+cudaError_t timed(int kid, cudaStream_t st, F &&launch) {
+  if (!g_prof_on.load(std::memory_order_relaxed)) return run_launch(launch);
   std::lock_guard<std::mutex> lk(g_prof_mu);
   cudaEvent_t a = nullptr, b = nullptr;
   if (g_prof.size() < kMaxProfRecs) {
@@ -81,8 +95,7 @@ cudaError_t timed(int kid, cudaStream_t st, F &&launch) {
     b = ev_get();
   }
   if (a) cudaEventRecord(a, st);
-  launch();
-  cudaError_t err = cudaGetLastError();
+  cudaError_t err = run_launch(launch);
   if (a && b) {
     cudaEventRecord(b, st);
     g_prof.push_back({kid, a, b});
@@ -150,7 +163,9 @@ Path choose_path(int d, int e, la2_dtype dt) {
 
 // Chunk plan: split each (b,h) sequence into S chunks of Lc rows (Lc a
 // multiple of the block size `blk`) so that B*H*S CTAs fill the GPU.
-Geo plan(int B, int H, int64_t L, int blk, Path path) {
+// slots: how many chunks the GPU runs at once (0: one per SM; the paired
+// reverse pass runs one per two SMs).
+Geo plan(int B, int H, int64_t L, int blk, Path path, int slots = 0) {
   Geo g;
   g.cu = nullptr;
   g.lpt = 0;
@@ -167,7 +182,7 @@ Geo plan(int B, int H, int64_t L, int blk, Path path) {
   if (S <= 0) {
     const int64_t BH = (int64_t)B * H;
     const int sms = device_sms();
-    S = path == PATH_TC ? la2::tc::auto_split(BH, nblk, sms)
+    S = path == PATH_TC ? la2::tc::auto_split(BH, nblk, slots > 0 ? slots : sms)
                         : (BH >= 2 * sms ? 1 : (2 * sms + BH - 1) / BH);
   }
   if (S > nblk) S = nblk;
@@ -210,6 +225,25 @@ Geo plan(int B, int H, int64_t L, int blk, Path path) {
 
 int block_rows(Path p) { return p == PATH_TC ? la2::tc::BLOCK : la2::simt::C; }
 
+// Whether the tensor-core backward runs dV and dK as one paired launch (two
+// CTAs per chunk in clusters of two) rather than as two passes: yes unless
+// LA2_OPT_BWD_FORM = 1 or the phase-serial kernel form is forced.
+bool rev_paired(Path p) {
+  return p == PATH_TC && g_opt_bwd_form.load() != 1 && g_opt_variant.load() != 1;
+}
+
+// Chunk plan of the backward's reverse passes.  Paired, each chunk occupies
+// two SMs, so the automatic split aims at SMs / 2 chunks at a time: fewer
+// chunks per sequence than the forward scan's plan, and so fewer chunk
+// boundaries for the reverse chunk-state pre-pass to cover.  A forced split
+// (LA2_OPT_SPLIT) applies to both plans alike.
+Geo plan_rev(int B, int H, int64_t L, Path p) {
+  if (!rev_paired(p)) return plan(B, H, L, block_rows(p), p);
+  Geo g = plan(B, H, L, block_rows(p), p, device_sms() / 2);
+  g.rev_pair = 1;
+  return g;
+}
+
 // Chunk plan of the decay gradient (fp32-FMA kernel, one CTA per SM): at
 // most one wave, S = floor(SMs / (B*H)) chunks per sequence when B*H is
 // below the SM count (LA2_OPT_SPLIT overrides), Lc a multiple of the block.
@@ -250,6 +284,15 @@ Geo plan_dlambda(int B, int H, int64_t L, bool split_ok) {
   g.wsS = g.nst + 1;
   g.Ssub = g.wsS;
   return g;
+}
+
+// Workspace of a backward: the forward scan's chunk states (plan g) then
+// the reverse scan's (plan gr).
+size_t ws_bwd_bytes(const Geo &g, const Geo &gr, int d, int e) {
+  auto one = [&](const Geo &x) {
+    return x.S > 1 ? (size_t)x.B * x.H * x.wsS * d * e * sizeof(float) : (size_t)0;
+  };
+  return one(g) + one(gr);
 }
 
 size_t ws_bytes(int op, const Geo &g, int d, int e) {
@@ -532,6 +575,7 @@ int la2_set_option(int option, int value) {
   if (option == LA2_OPT_TRACE) return g_opt_trace.exchange(value);
   if (option == LA2_OPT_VARLEN_ORDER) return g_opt_varlen_order.exchange(value);
   if (option == LA2_OPT_DECODE_BLOCK_TOKENS) return g_opt_decode_block.exchange(value);
+  if (option == LA2_OPT_BWD_FORM) return g_opt_bwd_form.exchange(value);
   return -1;
 }
 
@@ -542,6 +586,7 @@ size_t la2_workspace_size(int op, int B, int H, int64_t L, int d, int e, la2_dty
   Path p = choose_path(d, e, dt);
   if (p == PATH_NONE) return 0;
   Geo g = plan(B, H, L, block_rows(p), p);
+  if (op == LA2_OP_BACKWARD) return ws_bwd_bytes(g, plan_rev(B, H, L, p), d, e);
   return ws_bytes(op, g, d, e);
 }
 
@@ -665,16 +710,17 @@ la2_status la2_backward_ex(const void *q, const void *k, const void *v,
   Path p = choose_path(d, e, dt);
   if (p == PATH_NONE) return LA2_ERR_UNSUPPORTED;
   Geo g = plan(B, H, L, block_rows(p), p);
-  const size_t need = ws_bytes(LA2_OP_BACKWARD, g, d, e);
+  const Geo gr = plan_rev(B, H, L, p);
+  const size_t need = ws_bwd_bytes(g, gr, d, e);
   if (need > 0 && (!workspace || workspace_bytes < need)) return LA2_ERR_INVALID;
   float *ws = (float *)workspace;
   cudaError_t err;
   if (p == PATH_TC) {
-    err = la2::tc::backward(q, k, v, lambda, kv0, dO, dq, dk, dv, dkv0, ws, g, reuse, stream,
+    err = la2::tc::backward(q, k, v, lambda, kv0, dO, dq, dk, dv, dkv0, ws, g, gr, reuse, stream,
                             [&](int which, auto &&fn) {
                               static const int ids[] = {K_TC_FWD_STATE, K_SCAN_FWD, K_TC_DQ,
                                                         K_TC_REV_STATE, K_SCAN_REV, K_TC_DV,
-                                                        K_TC_DK};
+                                                        K_TC_DK, K_TC_DKDV};
                               return timed(ids[which], stream, fn);
                             });
   } else if (dt == LA2_F32) {
@@ -790,11 +836,15 @@ la2_status la2_backward_varlen(const void *q, const void *k, const void *v, cons
   Path p = choose_path(d, e, dt);
   if (p == PATH_NONE) return LA2_ERR_UNSUPPORTED;
   Geo g = plan_varlen(N, H, T, cu_seqlens);
+  g.rev_pair = p == PATH_TC && g_opt_bwd_form.load() != 1;
   cudaError_t err;
   if (p == PATH_TC) {
     err = la2::tc::backward_varlen(q, k, v, lambda, kv0, dO, dq, dk, dv, dkv0, g, stream,
                                    [&](int which, auto &&fn) {
-                                     return timed(which == 2 ? K_TC_DQ : which == 5 ? K_TC_DV : K_TC_DK,
+                                     return timed(which == 2   ? K_TC_DQ
+                                                  : which == 5 ? K_TC_DV
+                                                  : which == 6 ? K_TC_DK
+                                                               : K_TC_DKDV,
                                                   stream, fn);
                                    });
   } else if (dt == LA2_F32) {
@@ -965,16 +1015,17 @@ la2_status la2_backward_shard(const void *q, const void *k, const void *v, const
   Path p = choose_path(d, e, dt);
   if (p == PATH_NONE) return LA2_ERR_UNSUPPORTED;
   Geo g = plan(B, H, L, block_rows(p), p);
-  const size_t need = ws_bytes(LA2_OP_BACKWARD, g, d, e);
+  const Geo gr = plan_rev(B, H, L, p);
+  const size_t need = ws_bwd_bytes(g, gr, d, e);
   if (need > 0 && (!workspace || workspace_bytes < need)) return LA2_ERR_INVALID;
   float *ws = (float *)workspace;
   cudaError_t err;
   if (p == PATH_TC) {
-    err = la2::tc::backward(q, k, v, lambda, kv0, dO, dq, dk, dv, dkv0, ws, g, reuse, stream,
+    err = la2::tc::backward(q, k, v, lambda, kv0, dO, dq, dk, dv, dkv0, ws, g, gr, reuse, stream,
                             [&](int which, auto &&fn) {
                               static const int ids[] = {K_TC_FWD_STATE, K_SCAN_FWD, K_TC_DQ,
                                                         K_TC_REV_STATE, K_SCAN_REV, K_TC_DV,
-                                                        K_TC_DK};
+                                                        K_TC_DK, K_TC_DKDV};
                               return timed(ids[which], stream, fn);
                             },
                             dstate_end);

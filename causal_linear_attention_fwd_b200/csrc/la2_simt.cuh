@@ -61,6 +61,7 @@ struct Geo {
                 // completion signal so that its bounded wait runs out
   int variant;  // tensor-core kernel form (0: warp-specialised, 1: phase-serial)
   int trace;    // tensor-core pass whose CTA 0 stamps the trace buffer (-1: none)
+  int rev_pair = 0;  // tensor-core backward: dV and dK as one paired launch
 };
 
 // What one CTA of a pass works on: state slot bh (the (b,h) or (sequence,
@@ -72,13 +73,17 @@ struct Span {
   int h, c;
 };
 // seq >= 0 (packed batch, one CTA per (sequence, head)): the CTA serves that
-// sequence and head blockIdx.x % H instead of its own index's sequence.
-__device__ __forceinline__ Span span_of(const Geo &g, int nch, int c_first, int64_t seq = -1) {
+// sequence and head cta % H instead of its own index's sequence.  cta: the
+// CTA's index in the pass (blockIdx.x unless several CTAs share a work
+// unit, as the two of a cluster in the paired reverse pass do).
+__device__ __forceinline__ Span span_of(const Geo &g, int nch, int c_first, int64_t seq = -1,
+                                        int64_t cta = -1) {
   Span s;
-  const int64_t q = seq >= 0 ? seq * g.H + blockIdx.x % g.H : blockIdx.x / nch;
+  if (cta < 0) cta = blockIdx.x;
+  const int64_t q = seq >= 0 ? seq * g.H + cta % g.H : cta / nch;
   s.bh = q;
   s.h = (int)(q % g.H);
-  s.c = (int)(blockIdx.x % nch) + c_first;
+  s.c = (int)(cta % nch) + c_first;
   if (g.cu) {
     int64_t lo = g.cu[q / g.H], hi = g.cu[q / g.H + 1];
     if (!(0 <= lo && lo <= hi && hi <= g.L)) {

@@ -53,11 +53,15 @@ constexpr uint32_t TILE = 32768; // 128 rows x 128 bf16
 //   RSTATE (-,  Q,  dO) reverse chunk state from zero
 // b_t = lambda^(cb-1-t) (key side, forward), g_s = lambda^s (query side, reverse).
 // The reverse passes use the transposed mask: S^T[t][s] kept for s >= t.
-enum { MODE_FWD = 0, MODE_DQ = 1, MODE_STATE = 2, MODE_DV = 3, MODE_DK = 4, MODE_RSTATE = 5 };
+// RPAIR is DV or DK chosen per CTA at run time (the paired reverse launch):
+// one body serves both, so the two SMs of a pair run the same instructions.
+enum { MODE_FWD = 0, MODE_DQ = 1, MODE_STATE = 2, MODE_DV = 3, MODE_DK = 4, MODE_RSTATE = 5,
+       MODE_RPAIR = 6 };
 
 template <int MODE> struct Traits {
   static constexpr bool OUT = MODE != MODE_STATE && MODE != MODE_RSTATE;
-  static constexpr bool REV = MODE == MODE_DV || MODE == MODE_DK || MODE == MODE_RSTATE;
+  static constexpr bool REV =
+      MODE == MODE_DV || MODE == MODE_DK || MODE == MODE_RSTATE || MODE == MODE_RPAIR;
   static constexpr bool SWAP = MODE == MODE_DQ || MODE == MODE_DK;  // state A/B from (B2, B1)
   static constexpr bool X_MN = MODE == MODE_FWD || MODE == MODE_DV; // X's B operand MN-major
 };
@@ -585,21 +589,31 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 // pool, so one CTA per SM walks ~B*H/SMs units back to back (a range spans
 // at most two heads: two decay tables).
 constexpr int KIND_PLAIN = 0, KIND_VARLEN = 1, KIND_UNITS = 2;
+// The body of one pass for one CTA.  cta / ncta: the CTA's index among the
+// pass's CTAs and their number (blockIdx.x / gridDim.x, except in the paired
+// reverse pass, where the two CTAs of a cluster serve the same chunk);
+// trace_me: this CTA's pass is the traced one (TRACE instantiations only);
+// is_dk: MODE_RPAIR only, the CTA computes dK (else dV).
 template <int MODE, bool TRACE, int KIND>
-__global__ void __launch_bounds__(NT2, 1)
-chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
-              const __grid_constant__ CUtensorMap tm2, const __grid_constant__ CUtensorMap tmo,
-              const float *__restrict__ lambda, const float *__restrict__ kv0,
-              float *__restrict__ ws, float *__restrict__ kv_out, __nv_bfloat16 *__restrict__ outp,
-              Geo g) {
+__device__ __forceinline__ void
+chunk_body(const CUtensorMap *tm0, const CUtensorMap *tm1, const CUtensorMap *tm2,
+           const CUtensorMap *tmo, const float *__restrict__ lambda, const float *__restrict__ kv0,
+           float *__restrict__ ws, float *__restrict__ kv_out, __nv_bfloat16 *__restrict__ outp,
+           const Geo &g, const int64_t cta, const int64_t ncta, const bool trace_me,
+           const bool is_dk = false) {
   using LY = Layout2<MODE>;
   using TR = Traits<MODE>;
   constexpr bool VARLEN = KIND == KIND_VARLEN, UNITS = KIND == KIND_UNITS;
   constexpr bool OUT = LY::OUT;
   constexpr bool REV = TR::REV;
   constexpr int NS = LY::NSTAGE;
+  // the state term's B operand layout and the state update's operand order
+  // (fixed per mode; chosen per CTA in the paired reverse launch)
+  const bool X_MN = MODE == MODE_RPAIR ? !is_dk : TR::X_MN;
+  const bool SWAP = MODE == MODE_RPAIR ? is_dk : TR::SWAP;
   constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
-  constexpr uint32_t IDESC_X = idesc_bf16(128, 128, false, TR::X_MN);
+  const uint32_t IDESC_X =
+      X_MN ? idesc_bf16(128, 128, false, true) : idesc_bf16(128, 128, false, false);
   constexpr uint32_t IDESC_Y = idesc_bf16(128, 128, false, true);
   constexpr uint32_t IDESC_D = idesc_bf16(128, 128, true, true);
   constexpr int BAR_EPI = 2;
@@ -636,8 +650,8 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   int64_t u0 = 0;  // decode-unit form: the CTA's units [u0, u0 + nblk)
   if constexpr (UNITS) {
     const int64_t U = (int64_t)g.B * g.H;
-    u0 = (int64_t)blockIdx.x * U / gridDim.x;
-    const int64_t u1 = ((int64_t)blockIdx.x + 1) * U / gridDim.x;
+    u0 = cta * U / ncta;
+    const int64_t u1 = (cta + 1) * U / ncta;
     bh = slab = 0;
     c = 0;
     h = (int)(u0 / g.B);  // the range's first head
@@ -647,17 +661,17 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
     int64_t seq = -1;
     if (g.lpt) {  // longest sequences first
       if (warp == 0) {
-        const int n = lpt_sequence(g.cu, g.B, (int)(blockIdx.x / g.H));
+        const int n = lpt_sequence(g.cu, g.B, (int)(cta / g.H));
         if (lane == 0) tmem_slot[2] = (uint32_t)n;
       }
       __syncthreads();
       seq = tmem_slot[2];
     }
-    const Span sp = span_of(g, 1, 0, seq);
+    const Span sp = span_of(g, 1, 0, seq, cta);
     bh = sp.bh, a = sp.a, b = sp.b, slab = sp.slab, c = sp.c, h = sp.h;
   } else {
-    bh = blockIdx.x / nch;
-    c = blockIdx.x % nch + (OUT ? 0 : g.c0);
+    bh = cta / nch;
+    c = (int)(cta % nch) + (OUT ? 0 : g.c0);
     h = (int)(bh % g.H);
     a = (int64_t)c * g.Lc;
     b = g.L < a + g.Lc ? g.L : a + g.Lc;
@@ -692,7 +706,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
   // start, 4 mask done, 5 epilogue start, 6 state handed back, 7 store read
   // done, 8 kernel entry, 9 set-up done, 12 S issue begins, 13 products
   // issue begin, 14 row decays done, 15 output tile staged
-  const bool tracing = TRACE && blockIdx.x == 0;
+  const bool tracing = TRACE && trace_me && cta == 0;
   const bool tracing_all = TRACE;  // per-CTA entry / exit (events 10, 11)
   if (tid == 0) LA2_TRACE(8, 0);
   if (tid == 0 && tracing_all && blockIdx.x < kTraceBlocks)
@@ -722,10 +736,10 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
     mbar_init(b_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    if (OUT) tma_prefetch_desc(&tm0);
-    tma_prefetch_desc(&tm1);
-    tma_prefetch_desc(&tm2);
-    if (OUT) tma_prefetch_desc(&tmo);
+    if (OUT) tma_prefetch_desc(tm0);
+    tma_prefetch_desc(tm1);
+    tma_prefetch_desc(tm2);
+    if (OUT) tma_prefetch_desc(tmo);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), LY::TMEM_COLS);
@@ -750,19 +764,19 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
         if (j >= NS && !mbar_wait(b_eab + 8 * st, ph, abort_flag)) break;
         mbar_expect_tx(b_fab + 8 * st, LY::AB_BYTES);
         if (OUT) {
-          tma_load_3d(dst, &tm0, b_fab + 8 * st, 0, y, z);
-          tma_load_3d(dst + BOX, &tm0, b_fab + 8 * st, 64, y, z);
+          tma_load_3d(dst, tm0, b_fab + 8 * st, 0, y, z);
+          tma_load_3d(dst + BOX, tm0, b_fab + 8 * st, 64, y, z);
           dst += TILE;
         }
-        tma_load_3d(dst, &tm1, b_fab + 8 * st, 0, y, z);
-        tma_load_3d(dst + BOX, &tm1, b_fab + 8 * st, 64, y, z);
+        tma_load_3d(dst, tm1, b_fab + 8 * st, 0, y, z);
+        tma_load_3d(dst + BOX, tm1, b_fab + 8 * st, 64, y, z);
         nab++;
         // B2: its slot free once block j-NS's output has left it
         if (j >= NS && !mbar_wait(b_ec + 8 * st, ph, abort_flag)) break;
         dst = sbase + st * LY::STAGE + LY::C_OFF;
         mbar_expect_tx(b_fc + 8 * st, TILE);
-        tma_load_3d(dst, &tm2, b_fc + 8 * st, 0, y, z);
-        tma_load_3d(dst + BOX, &tm2, b_fc + 8 * st, 64, y, z);
+        tma_load_3d(dst, tm2, b_fc + 8 * st, 0, y, z);
+        tma_load_3d(dst + BOX, tm2, b_fc + 8 * st, 64, y, z);
         nc++;
         LA2_TRACE(0, j);
       }
@@ -803,13 +817,13 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
 #pragma unroll
           for (int k = 0; k < 8; k++) {
             const uint32_t koff = (k >> 2) * BOX + (k & 3) * 32;
-            const uint64_t bd = TR::X_MN ? sdesc_sw128(sKV + k * 2048, BOX, 1024)
-                                         : sdesc_sw128(sKV + koff, 16, 1024);
+            const uint64_t bd = X_MN ? sdesc_sw128(sKV + k * 2048, BOX, 1024)
+                                     : sdesc_sw128(sKV + koff, 16, 1024);
             mma_ss(tmem + LY::COL_O, sdesc_sw128(sA0 + koff, 16, 1024), bd, IDESC_X, 1);
           }
         }
-        const uint32_t sA = TR::SWAP ? sB2 : sB1;
-        const uint32_t sB = TR::SWAP ? sB1 : sB2;
+        const uint32_t sA = SWAP ? sB2 : sB1;
+        const uint32_t sB = SWAP ? sB1 : sB2;
 #pragma unroll
         for (int k = 0; k < 8; k++)
           mma_ss(tmem + LY::COL_KV, sdesc_sw128(sA + k * 2048, BOX, 1024),
@@ -1003,7 +1017,7 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
           const int64_t so = state_slot(g, bh);
           init = (kv0 && so >= 0) ? kv0 + so * 128 * 128 : nullptr;
         }
-      } else if (MODE == MODE_DV || MODE == MODE_DK) {
+      } else if (MODE == MODE_DV || MODE == MODE_DK || MODE == MODE_RPAIR) {
         // the last chunk starts from the reverse state past the sequence end
         // (kv0 carries it in the reverse passes; NULL: zero)
         if (c != g.S - 1) init = ws + (bh * g.wsS + (int64_t)(c + 1) * g.M - 1) * (int64_t)128 * 128;
@@ -1024,8 +1038,8 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
     }
     if (MODE == MODE_STATE) dst = ws + (bh * g.wsS + c + 1) * (int64_t)128 * 128;
     if (MODE == MODE_RSTATE) dst = ws + (bh * g.wsS + c - 1) * (int64_t)128 * 128;
-    if (MODE == MODE_DV && c == 0 && kv_out) {  // dkv0 = lambda * D(0)
-      dst = kv_out + bh * 128 * 128;
+    if ((MODE == MODE_DV || (MODE == MODE_RPAIR && !is_dk)) && c == 0 && kv_out) {
+      dst = kv_out + bh * 128 * 128;  // dkv0 = lambda * D(0)
       dscale = lambda[h];
     }
     for (int i = 0; i < nblk; i++) {
@@ -1116,8 +1130,8 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
         if (OUT && !tail_rows && (!UNITS || unit_state(kv_out, i))) {
           const uint32_t sst = sbase + st * LY::STAGE + LY::C_OFF;
           const int y = (int)p_of(i), z = (int)slab_of(i);
-          tma_store_3d(&tmo, sst, 0, y, z);
-          tma_store_3d(&tmo, sst + BOX, 64, y, z);
+          tma_store_3d(tmo, sst, 0, y, z);
+          tma_store_3d(tmo, sst + BOX, 64, y, z);
           tma_store_commit();
           tma_store_wait_read0();
         }
@@ -1169,6 +1183,41 @@ chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ C
     tc_fence_after();
     tmem_dealloc(tmem, LY::TMEM_COLS);
   }
+}
+
+template <int MODE, bool TRACE, int KIND>
+__global__ void __launch_bounds__(NT2, 1)
+chunk_kernel2(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
+              const __grid_constant__ CUtensorMap tm2, const __grid_constant__ CUtensorMap tmo,
+              const float *__restrict__ lambda, const float *__restrict__ kv0,
+              float *__restrict__ ws, float *__restrict__ kv_out, __nv_bfloat16 *__restrict__ outp,
+              Geo g) {
+  chunk_body<MODE, TRACE, KIND>(&tm0, &tm1, &tm2, &tmo, lambda, kv0, ws, kv_out, outp, g,
+                                blockIdx.x, gridDim.x, true);
+}
+
+// The reverse scan's two output passes in one launch: clusters of two CTAs,
+// both on the same chunk, the even one writing dV (tiles K, Q, dO) and the
+// odd one dK (tiles V, dO, Q).  Each carries its own copy of the reverse
+// state D and neither waits for the other, but a cluster's CTAs start
+// together and walk the same blocks at the same pace, so the Q and dO tiles
+// one of them loads are still in L2 when the other asks for them: per block
+// the pair reads K, Q, dO, V from HBM once and writes dK and dV, where two
+// separate passes read Q and dO twice.  dkv0 comes from the dV member.
+template <bool TRACE, int KIND>
+__global__ void __launch_bounds__(NT2, 1)
+rev_pair_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tq,
+                const __grid_constant__ CUtensorMap tg, const __grid_constant__ CUtensorMap tv,
+                const __grid_constant__ CUtensorMap tdv, const __grid_constant__ CUtensorMap tdk,
+                const float *__restrict__ lambda, const float *__restrict__ dend,
+                float *__restrict__ ws, float *__restrict__ dkv0, __nv_bfloat16 *__restrict__ outp_dv,
+                __nv_bfloat16 *__restrict__ outp_dk, Geo g) {
+  const int64_t cta = blockIdx.x >> 1, ncta = gridDim.x >> 1;
+  const bool dk = blockIdx.x & 1;
+  chunk_body<MODE_RPAIR, TRACE, KIND>(dk ? &tv : &tk, dk ? &tg : &tq, dk ? &tq : &tg,
+                                      dk ? &tdk : &tdv, lambda, dend, ws, dk ? nullptr : dkv0,
+                                      dk ? outp_dk : outp_dv, g, cta, ncta,
+                                      g.trace == (dk ? MODE_DK : MODE_DV), dk);
 }
 
 // ------------------------------------------------------------------ host
@@ -1232,6 +1281,37 @@ cudaError_t launch_chunk(const CUtensorMap &m0, const CUtensorMap &m1, const CUt
   return cudaGetLastError();
 }
 
+// The paired reverse pass (rev_pair_kernel): 2 CTAs per chunk, launched as
+// clusters of two so that both members of a pair run at the same time.
+template <int KIND>
+cudaError_t launch_pair(const CUtensorMap &mk, const CUtensorMap &mq, const CUtensorMap &mg,
+                        const CUtensorMap &mv, const CUtensorMap &mdv, const CUtensorMap &mdk,
+                        const float *lam, const float *dend, float *ws, float *dkv0, void *outp_dv,
+                        void *outp_dk, const Geo &g, cudaStream_t st) {
+  using LY = Layout2<MODE_DV>;
+  static_assert(Layout2<MODE_DV>::SMEM == Layout2<MODE_RPAIR>::SMEM, "the pair's layout");
+  const int64_t units = (int64_t)g.B * g.H * g.S;
+  const bool trace = g.trace == MODE_DV || g.trace == MODE_DK;
+  auto k = trace ? rev_pair_kernel<true, KIND> : rev_pair_kernel<false, KIND>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::SMEM);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * units));
+  cfg.blockDim = dim3(NT2);
+  cfg.dynamicSmemBytes = LY::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, mk, mq, mg, mv, mdv, mdk, lam, dend, ws, dkv0,
+                            static_cast<__nv_bfloat16 *>(outp_dv),
+                            static_cast<__nv_bfloat16 *>(outp_dk), g);
+}
+
 inline bool geometry_ok(const Geo &g) {
   return g.L < (int64_t(1) << 31) && (int64_t)g.B * g.H < (int64_t(1) << 31);
 }
@@ -1258,18 +1338,22 @@ cudaError_t forward(const void *q, const void *k, const void *v, const float *la
     });
     if (err) return err;
   }
-  return timed(2, [&] { launch_chunk<MODE_FWD>(mq, mk, mv, mo, lam, kv0, ws, kv_out, g, st); });
+  return timed(2, [&] { launch_chunk<MODE_FWD>(mq, mk, mv, mo, lam, kv0, ws, kv_out, g, st, o); });
 }
 
 // Backward: dQ by a forward scan (chunk states of K, V + scan), then dV and
 // dK by reverse scans (chunk states of Q, dO + reverse scan); dkv0 comes
-// out of the dV pass's first chunk.
+// out of the dV pass's first chunk.  gr is the reverse passes' chunk plan:
+// with gr.rev_pair the dV and dK passes run as one paired launch, two CTAs
+// per chunk, so gr splits each sequence for half as many chunks as g (the
+// reverse pre-pass then covers fewer chunk boundaries).  The reverse states
+// follow the forward ones in the workspace.
 template <typename Timed>
 cudaError_t backward(const void *q, const void *k, const void *v, const float *lam,
                      const float *kv0, const void *dO, void *dq, void *dk, void *dv, float *dkv0,
-                     float *ws, const Geo &g, bool reuse_fwd, cudaStream_t st, Timed &&timed,
-                     const float *dend = nullptr) {
-  if (!geometry_ok(g)) return cudaErrorInvalidValue;
+                     float *ws, const Geo &g, const Geo &gr, bool reuse_fwd, cudaStream_t st,
+                     Timed &&timed, const float *dend = nullptr) {
+  if (!geometry_ok(g) || !geometry_ok(gr)) return cudaErrorInvalidValue;
   const int64_t BH = (int64_t)g.B * g.H;
   CUtensorMap mq, mk, mv, mg, mdq, mdk, mdv;
   if (!make_map(&mq, q, BH, g.L) || !make_map(&mk, k, BH, g.L) || !make_map(&mv, v, BH, g.L) ||
@@ -1277,9 +1361,9 @@ cudaError_t backward(const void *q, const void *k, const void *v, const float *l
       !make_map(&mdk, dk, BH, g.L) || !make_map(&mdv, dv, BH, g.L))
     return cudaErrorInvalidValue;
   float *wsf = ws;
-  float *wsr = ws ? ws + (size_t)BH * g.wsS * 128 * 128 : nullptr;
+  float *wsr = ws ? ws + (g.S > 1 ? (size_t)BH * g.wsS * 128 * 128 : 0) : nullptr;
   const dim3 sgrid(128 * 128 / la2::simt::NT, (unsigned)BH);
-  const Geo gf = state_geo(g, false), gr = state_geo(g, true);
+  const Geo gf = state_geo(g, false), grs = state_geo(gr, true);
   cudaError_t err = cudaSuccess;
   // the forward pass leaves the same chunk entry states in the same place
   if (g.S > 1 && !reuse_fwd) {
@@ -1290,19 +1374,24 @@ cudaError_t backward(const void *q, const void *k, const void *v, const float *l
     });
     if (err) return err;
   }
-  err = timed(2, [&] { launch_chunk<MODE_DQ>(mg, mv, mk, mdq, lam, kv0, wsf, nullptr, g, st); });
+  err = timed(2, [&] { launch_chunk<MODE_DQ>(mg, mv, mk, mdq, lam, kv0, wsf, nullptr, g, st, dq); });
   if (err) return err;
-  if (g.S > 1) {
-    err = timed(3, [&] { launch_chunk<MODE_RSTATE>(mq, mq, mg, mq, lam, nullptr, wsr, nullptr, gr, st); });
+  if (gr.S > 1) {
+    err = timed(3, [&] { launch_chunk<MODE_RSTATE>(mq, mq, mg, mq, lam, nullptr, wsr, nullptr, grs, st); });
     if (err) return err;
     err = timed(4, [&] {
-      la2::simt::scan_rev_kernel<128, 128><<<sgrid, la2::simt::NT, 0, st>>>(wsr, lam, dend, gr);
+      la2::simt::scan_rev_kernel<128, 128><<<sgrid, la2::simt::NT, 0, st>>>(wsr, lam, dend, grs);
     });
     if (err) return err;
   }
-  err = timed(5, [&] { launch_chunk<MODE_DV>(mk, mq, mg, mdv, lam, dend, wsr, dkv0, g, st); });
+  if (gr.rev_pair)
+    return timed(7, [&] {
+      return launch_pair<KIND_PLAIN>(mk, mq, mg, mv, mdv, mdk, lam, dend, wsr, dkv0, nullptr, nullptr,
+                                     gr, st);
+    });
+  err = timed(5, [&] { launch_chunk<MODE_DV>(mk, mq, mg, mdv, lam, dend, wsr, dkv0, gr, st, dv); });
   if (err) return err;
-  return timed(6, [&] { launch_chunk<MODE_DK>(mv, mg, mq, mdk, lam, dend, wsr, nullptr, g, st); });
+  return timed(6, [&] { launch_chunk<MODE_DK>(mv, mg, mq, mdk, lam, dend, wsr, nullptr, gr, st, dk); });
 }
 
 // Decode units: T <= 128 new tokens for each of B requests x H heads, [B,H,T,.]
@@ -1377,6 +1466,11 @@ cudaError_t backward_varlen(const void *q, const void *k, const void *v, const f
     launch_chunk<MODE_DQ>(mg, mv, mk, mdq, lam, kv0, nullptr, nullptr, g, st, dq);
   });
   if (err) return err;
+  if (g.rev_pair)
+    return timed(7, [&] {
+      return launch_pair<KIND_VARLEN>(mk, mq, mg, mv, mdv, mdk, lam, nullptr, nullptr, dkv0, dv, dk,
+                                      g, st);
+    });
   err = timed(5, [&] { launch_chunk<MODE_DV>(mk, mq, mg, mdv, lam, nullptr, nullptr, dkv0, g, st, dv); });
   if (err) return err;
   return timed(6, [&] { launch_chunk<MODE_DK>(mv, mg, mq, mdk, lam, nullptr, nullptr, nullptr, g, st, dk); });

@@ -432,11 +432,21 @@ const char *la2_status_string(la2_status s);
  * LA2_OPT_DECODE_BLOCK_TOKENS: 0 (default) = la2_decode_tokens runs the
  * tensor-core block form from the library's crossover number of tokens per
  * request on, the token-by-token kernel below it; n > 0 = from n tokens on.
+ * LA2_OPT_BWD_FORM: 0 (default) = the tensor-core backward computes dV and
+ * dK in one paired launch (two CTAs per chunk, clusters of two, the pair
+ * reading Q and dO from HBM once); 1 = two separate passes (for comparison).
+ * Under the same chunk split the results are bitwise the same; under the
+ * automatic split the paired form may cut a long sequence into fewer chunks
+ * (each chunk occupies two SMs), which changes only the rounding.  The
+ * workspace size of a backward
+ * depends on this option, so query la2_workspace_size with the option that
+ * the call will run under.
  * Returns the previous value, or -1 for an unknown option.
  */
 enum {
     LA2_OPT_SPLIT = 0, LA2_OPT_PATH = 1, LA2_OPT_INJECT_TIMEOUT = 2, LA2_OPT_VARIANT = 3,
-    LA2_OPT_TRACE = 4, LA2_OPT_VARLEN_ORDER = 5, LA2_OPT_DECODE_BLOCK_TOKENS = 6
+    LA2_OPT_TRACE = 4, LA2_OPT_VARLEN_ORDER = 5, LA2_OPT_DECODE_BLOCK_TOKENS = 6,
+    LA2_OPT_BWD_FORM = 7
 };
 
 /*

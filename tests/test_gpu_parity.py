@@ -233,11 +233,33 @@ def sweep_buffers():
     return x, n
 
 
+def sweep_picks(Bn, H=32, n=8):
+    """n distinct (b, h) sequences of a [Bn, H] sweep point: the first and
+    the last, middle heads of the middle batch row, and others spread over
+    the rows and heads."""
+    cand = [(0, 0), (Bn - 1, H - 1), (Bn // 2, H // 2), (Bn // 2, 0), (0, H - 1),
+            ((Bn - 1) // 3, 21 % H), ((2 * Bn) // 3, 10 % H), (Bn - 1, 0),
+            (Bn // 2, 5), (Bn // 2, 26), (0, 13), (Bn - 1, 18)]
+    out = []
+    for p in cand:
+        if p not in out:
+            out.append(p)
+    return out[:n]
+
+
+def test_sweep_picks_are_spread():
+    for Bn, _ in SWEEP:
+        p = sweep_picks(Bn)
+        assert len(p) == 8 and len(set(p)) == 8
+        assert (0, 0) in p and (Bn - 1, 31) in p and (Bn // 2, 16) in p
+
+
 @pytest.mark.parametrize("BL", SWEEP, ids=[f"B{b}_L{l}" for b, l in SWEEP])
 def test_sweep_sampled_heads(orc, sweep_buffers, BL):
     """Full-size sweep point in the bench's launch configuration; the oracle
-    recomputes two whole heads (first and last (b,h)); adjoint identities
-    hold over every head."""
+    recomputes eight whole (b,h) sequences (first, last, middle heads of the
+    middle batch row, and others spread over rows and heads); adjoint
+    identities hold over every head."""
     Bn, L = BL
     xs, _ = sweep_buffers
     x = {n: t.view(Bn, 32, L, 128) for n, t in xs.items()}
@@ -247,8 +269,8 @@ def test_sweep_sampled_heads(orc, sweep_buffers, BL):
     torch.cuda.synchronize()
     assert la2.last_device_error() == 0
     lam_h = lam.double().cpu().numpy()
-    picks = ((0, 0), (Bn - 1, 31))
-    # the two sampled heads go to the oracle as one [1, 2, L, .] problem
+    picks = sweep_picks(Bn)
+    # the sampled sequences go to the oracle as one [1, n, L, .] problem
     sub = {n: np.concatenate([host(t[b:b + 1, h:h + 1]) for b, h in picks], axis=1)
            for n, t in x.items()}
     lh = np.array([lam_h[h] for _, h in picks])
@@ -271,7 +293,7 @@ def test_sweep_sampled_heads(orc, sweep_buffers, BL):
 # ------------------------------------------ workload: long context (forward)
 def test_long_context_1m_sampled(orc):
     """B=1, H=64, L=1,048,576, forward only (8K+ blocks of on-chip carry);
-    the oracle recomputes heads 0 and 63 over the full length."""
+    the oracle recomputes heads 0, 21, 42 and 63 over the full length."""
     B, H, L = 1, 64, 1 << 20
     free, _ = torch.cuda.mem_get_info()
     if free < 80 * (1 << 30):
@@ -283,7 +305,7 @@ def test_long_context_1m_sampled(orc):
     torch.cuda.synchronize()
     assert la2.last_device_error() == 0
     lam_h = lam.double().cpu().numpy()
-    heads = [0, 63]
+    heads = [0, 21, 42, 63]
     sub = {n: np.concatenate([host(t[:, h:h + 1]) for h in heads], axis=1) for n, t in x.items()}
     o_r, st_r = orc.forward(sub["q"], sub["k"], sub["v"], lam_h[heads], want_state=True)
     for i, h in enumerate(heads):
@@ -472,3 +494,62 @@ def test_random_shapes_match_oracle(orc, case):
         got = run_fwd_bwd(x, lam, x["kv0"])
     compare(got, oracle_all(orc, x, lam, x["kv0"]), torch.bfloat16,
             f"B={B} H={H} L={L} split={split}")
+
+
+# ------------------------------------------- paired dV/dK reverse launch
+@contextlib.contextmanager
+def bwd_form(form):
+    old = la2.set_option(la2.LA2_OPT_BWD_FORM, form)
+    try:
+        yield
+    finally:
+        la2.set_option(la2.LA2_OPT_BWD_FORM, old)
+
+
+@pytest.mark.parametrize("split", [1, 2, 5])
+@pytest.mark.parametrize("L", [127, 1000, 2048])
+def test_paired_reverse_matches_two_passes(orc, L, split):
+    """dV and dK from the paired launch (two CTAs per chunk, clusters of
+    two) are bitwise those of the two separate passes under the same split,
+    and the oracle's, dkv0 included."""
+    B, H = 2, 3
+    x = inputs.make_inputs(B, H, L, 128, 128, dtype=torch.bfloat16, device=DEV, seed=L + split,
+                           with_kv0=True)
+    lam = inputs.fixed_lambdas((1.0, 0.95, 0.0), DEV)
+    res = {}
+    for form in (0, 1):
+        with bwd_form(form), options(path="tc", split=split):
+            res[form] = run_fwd_bwd(x, lam, x["kv0"])
+    for name, a, b in zip(NAMES, res[0], res[1]):
+        assert torch.equal(a, b), name
+    compare(res[0], oracle_all(orc, x, lam, x["kv0"]), torch.bfloat16,
+            f"paired L={L} S={split}")
+
+
+@pytest.mark.parametrize("BL", [(1, 32768), (1, 65536), (2, 20000)])
+def test_paired_reverse_automatic_split(orc, BL):
+    """Under the automatic split the paired form plans its own (coarser)
+    reverse chunks; few (b,h) sequences so that the reverse pre-pass runs:
+    every gradient of two sampled heads against the oracle, and the
+    workspace the binding sizes is the one the call needs."""
+    Bn, L = BL
+    H = 4
+    x = inputs.make_inputs(Bn, H, L, 128, 128, dtype=torch.bfloat16, device=DEV, seed=L,
+                           with_kv0=True)
+    lam = inputs.decay_lambdas(H, DEV)
+    n_pair = la2.workspace_size(la2.LA2_OP_BACKWARD, Bn, H, L, 128, 128, torch.bfloat16)
+    with bwd_form(1):
+        n_two = la2.workspace_size(la2.LA2_OP_BACKWARD, Bn, H, L, 128, 128, torch.bfloat16)
+    assert 0 < n_pair <= n_two
+    got = run_fwd_bwd(x, lam, x["kv0"])
+    picks = [(0, 0), (Bn - 1, H - 1)]
+    lam_h = lam.double().cpu().numpy()
+    sub = {n: np.concatenate([host(t[b:b + 1, h:h + 1]) for b, h in picks], axis=1)
+           for n, t in x.items()}
+    lh = np.array([lam_h[h] for _, h in picks])
+    ref = (orc.forward(sub["q"], sub["k"], sub["v"], lh, sub["kv0"], want_state=True)
+           + tuple(orc.backward(sub["q"], sub["k"], sub["v"], lh, sub["dO"], sub["kv0"])))
+    for i, (b, h) in enumerate(picks):
+        for name, a, r in zip(NAMES, got, ref):
+            check(f"auto split B{Bn} L{L} (b={b},h={h}) {name}", a[b:b + 1, h:h + 1],
+                  r[:, i:i + 1], torch.bfloat16)

@@ -226,3 +226,22 @@ def test_varlen_random_batches_agree_with_per_document_calls(case):
                            ("dk", got[3][:, a:b], dk[0]), ("dv", got[4][:, a:b], dv[0]),
                            ("kv_out", got[1][n], st[0]), ("dkv0", got[5][n], dkv0[0])):
             check(f"{tag} {name}", u, host(r), torch.bfloat16)
+
+
+@pytest.mark.parametrize("order", [0, 1])
+def test_varlen_paired_reverse_matches_two_passes(order):
+    """The packed backward's dV and dK from the paired launch equal the two
+    separate passes' bitwise (both CTA orders; an empty, a one-row and a
+    ragged sequence included)."""
+    lens = [300, 0, 1, 1000, 129, 2000, 7]
+    x, kv0, cu = packed_inputs(lens, 4, 128, 128, torch.bfloat16, seed=17)
+    lam = inputs.decay_lambdas(4, DEV)
+    res = {}
+    for form in (0, 1):
+        old = la2.set_option(la2.LA2_OPT_BWD_FORM, form)
+        try:
+            res[form] = _varlen_all(x, kv0, cu, lam, order)
+        finally:
+            la2.set_option(la2.LA2_OPT_BWD_FORM, old)
+    for a, b in zip(res[0], res[1]):
+        assert torch.equal(a, b)
