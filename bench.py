@@ -783,21 +783,38 @@ def run_dlambda(args, world, rank, local):
     value = world * Bn * L * args.steps / (ms / 1e3)
     name, rec = max(prof.items(), key=lambda kv: kv[1]["ms"])
     avg = rec["ms"] / rec["launches"]
-    # fp32 FMA work of the block schedule per token-head (C = 32 rows): the
-    # state terms q KV and q W, the updates of KV and W (2 d e flops each),
-    # and the block's own pairs, (C-1)/2 of them per row at 2 (d + e) flops
-    fl_th = 8 * D * E + (32 - 1) * (D + E)
-    alg = fl_th * Bn * Hh * L
-    ach = alg / (avg / 1e3) / 1e12
-    with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-        mhz = float(json.load(f).get("sm_max_mhz", 1965.0))
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    peak = sms * 128 * 2 * mhz * 1e6 / 1e12  # fp32 lanes x FMA x max SM clock
-    roof = {"kernel": name, "bound": "alu", "achieved": round(ach, 2), "peak": round(peak, 1),
-            "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
-            "alg_flops_per_launch": alg, "avg_launch_ms": avg,
-            "peak_source": f"{sms} SMs x 128 fp32 lanes x 2 flops x {mhz:.0f} MHz (max SM clock)"}
-    extra = {"dtype": "f32", "roofline": roof, "kernels": prof,
+    pk = peaks()
+    tensor = name.startswith("tc_")
+    if tensor:
+        # tensor-core form (C = 128 rows, two CTAs per chunk, one per half
+        # of e): the MMA flops it executes per token-head -- S = Q K^T by
+        # both CTAs (2 x 2 C d), G = dO V^T in halves (2 C e), Q KV and Q W
+        # and the KV and W updates each as a bf16 pair of products (4 x 4 d e)
+        fl_th = 4 * 128 * D + 2 * 128 * E + 16 * D * E
+        alg = fl_th * Bn * Hh * L
+        ach = alg / (avg / 1e3) / 1e12
+        roof = {"kernel": name, "bound": "tensor", "achieved": round(ach, 2),
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(ach / pk["bf16_tflops"], 4), "traffic": None,
+                "alg_flops_per_launch": alg, "avg_launch_ms": avg,
+                "peak_source": pk["source"] + " (bf16_tflops, burst: a kernel timed alone)",
+                "note": "executed MMA flops of the tensor-core form (operand pairs counted twice)"}
+    else:
+        # fp32 FMA work of the block schedule per token-head (C = 32 rows): the
+        # state terms q KV and q W, the updates of KV and W (2 d e flops each),
+        # and the block's own pairs, (C-1)/2 of them per row at 2 (d + e) flops
+        fl_th = 8 * D * E + (32 - 1) * (D + E)
+        alg = fl_th * Bn * Hh * L
+        ach = alg / (avg / 1e3) / 1e12
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            mhz = float(json.load(f).get("sm_max_mhz", 1965.0))
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        peak = sms * 128 * 2 * mhz * 1e6 / 1e12  # fp32 lanes x FMA x max SM clock
+        roof = {"kernel": name, "bound": "alu", "achieved": round(ach, 2), "peak": round(peak, 1),
+                "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
+                "alg_flops_per_launch": alg, "avg_launch_ms": avg,
+                "peak_source": f"{sms} SMs x 128 fp32 lanes x 2 flops x {mhz:.0f} MHz (max SM clock)"}
+    extra = {"dtype": "bf16" if tensor else "f32", "roofline": roof, "kernels": prof,
              "gpu_launches": sum(v["launches"] for v in prof.values()), "clocks": clk}
     if rank == 0 and world == 1 and not args.no_cpu:
         import oracle
@@ -810,7 +827,7 @@ def run_dlambda(args, world, rank, local):
                                  "cores": orc.num_threads(), "kind": "oracle",
                                  "sample": f"one batch row (16 heads x {L} rows) of the workload"}
     return _common(world, args.steps, args.warmup, value, "tokens/s",
-                   "dlambda tokens/s (B=4,H=16,L=2048,d=e=128, bf16 inputs, fp32 FMA)",
+                   "dlambda tokens/s (B=4,H=16,L=2048,d=e=128, bf16 inputs)",
                    {"workload": "gradient w.r.t. the decay, B=4, H=16, L=2,048, d=e=128, bf16 "
                                 "inputs",
                     "l2": "inputs 32 MiB (fit in L2); the pass is arithmetic-bound"}, ms, extra)

@@ -15,6 +15,7 @@
 #include "../../include/la2.h"
 #include "la2_common.cuh"
 #include "la2_decode.cuh"
+#include "la2_dlam_tc.cuh"
 #include "la2_fmap.cuh"
 #include "la2_shard.cuh"
 #include "la2_simt.cuh"
@@ -39,14 +40,15 @@ enum KernelId {
   K_SIMT_REV_SCAN, K_SIMT_DKDV, K_DECODE, K_TC_FWD_STATE, K_TC_FWD, K_TC_DQ,
   K_TC_REV_STATE, K_TC_DV, K_TC_DK, K_SCAN_FWD, K_SCAN_REV, K_SIMT_DLAMBDA,
   K_SIMT_DLAMBDA_STATE, K_SIMT_DLAMBDA_SCAN, K_TC_DECODE_UNITS, K_FMAP, K_FMAP_GRAD, K_TC_DKDV,
-  K_COUNT
+  K_TC_DLAMBDA, K_TC_DLAMBDA_STATE, K_COUNT
 };
 const char *kKernelName[K_COUNT] = {
     "simt_fwd_chunk_state", "simt_scan_fwd", "simt_fwd", "simt_dq",
     "simt_rev_chunk_state", "simt_scan_rev", "simt_dkdv", "decode_step",
     "tc_fwd_chunk_state", "tc_fwd", "tc_dq", "tc_rev_chunk_state", "tc_dv", "tc_dk",
     "scan_fwd", "scan_rev", "simt_dlambda", "simt_dlambda_chunk_state", "simt_dlambda_scan",
-    "tc_decode_units", "feature_map", "feature_map_grad", "tc_dkdv"};
+    "tc_decode_units", "feature_map", "feature_map_grad", "tc_dkdv", "tc_dlambda",
+    "tc_dlambda_chunk_state"};
 
 struct ProfRec {
   int kid;
@@ -244,15 +246,16 @@ Geo plan_rev(int B, int H, int64_t L, Path p) {
   return g;
 }
 
-// Chunk plan of the decay gradient (fp32-FMA kernel, one CTA per SM): at
-// most one wave, S = floor(SMs / (B*H)) chunks per sequence when B*H is
-// below the SM count (LA2_OPT_SPLIT overrides), Lc a multiple of the block.
+// Chunk plan of the decay gradient (one CTA per SM; blocks of blk rows: 32
+// for the fp32-FMA kernel, 128 for the tensor-core one): at most one wave,
+// S = floor(SMs / (B*H)) chunks per sequence when B*H is below the SM count
+// (LA2_OPT_SPLIT overrides), Lc a multiple of the block.
 // The chunk-state pre-pass covers chunks 0..S-2 only, so it runs on M
 // sub-chunks of Ls rows per chunk (Lc = M Ls), M filling the SMs (at most
 // 8); the workspace holds (S-1) M + 1 (KV, W) pairs per (b,h).
-Geo plan_dlambda(int B, int H, int64_t L, bool split_ok) {
-  Geo g = plan(B, H, L, la2::simt::C, PATH_SIMT);
-  const int64_t blk = la2::simt::C, nblk = (L + blk - 1) / blk;
+Geo plan_dlambda(int B, int H, int64_t L, bool split_ok, int blk_rows) {
+  Geo g = plan(B, H, L, blk_rows, PATH_SIMT);
+  const int64_t blk = blk_rows, nblk = (L + blk - 1) / blk;
   const int64_t BH = (int64_t)B * H;
   const int sms = device_sms();
   int64_t S = g_opt_split.load();
@@ -581,7 +584,11 @@ int la2_set_option(int option, int value) {
 
 size_t la2_workspace_size(int op, int B, int H, int64_t L, int d, int e, la2_dtype dt) {
   if (B <= 0 || H <= 0 || L <= 0 || !shape_supported(d, e, dt)) return 0;
-  if (op == LA2_OP_DLAMBDA) return ws_bytes(op, plan_dlambda(B, H, L, true), d, e);
+  if (op == LA2_OP_DLAMBDA) {
+    const Path p = choose_path(d, e, dt);
+    if (p == PATH_NONE) return 0;
+    return ws_bytes(op, plan_dlambda(B, H, L, true, block_rows(p)), d, e);
+  }
   if (op != LA2_OP_FORWARD && op != LA2_OP_BACKWARD && op != LA2_OP_SHARD_STATE) return 0;
   Path p = choose_path(d, e, dt);
   if (p == PATH_NONE) return 0;
@@ -1065,10 +1072,20 @@ la2_status dlambda_call(const void *q, const void *k, const void *v, const float
   if (BH == 0 || L == 0) {  // no token depends on lambda
     return to_status(cudaMemsetAsync(dlambda, 0, (size_t)H * sizeof(float), stream));
   }
-  const Geo g = plan_dlambda(B, H, L, split);
+  const Path p = choose_path(d, e, dt);
+  if (p == PATH_NONE) return LA2_ERR_UNSUPPORTED;
+  const Geo g = plan_dlambda(B, H, L, split, block_rows(p));
   const size_t need = ws_bytes(LA2_OP_DLAMBDA, g, d, e);
   if (need > 0 && (!workspace || workspace_bytes < need)) return LA2_ERR_INVALID;
   float *ws = (float *)workspace;
+  if (p == PATH_TC)
+    return to_status(la2::tcd::dlambda(q, k, v, dO, lambda, kv0, dlambda, ws, g, stream,
+                                       [&](int which, auto &&fn) {
+                                         static const int ids[] = {K_TC_DLAMBDA_STATE,
+                                                                   K_SIMT_DLAMBDA_SCAN,
+                                                                   K_TC_DLAMBDA};
+                                         return timed(ids[which], stream, fn);
+                                       }));
   cudaError_t err =
       dt == LA2_F32
           ? LA2_DISPATCH_DE(d, e, simt_dlambda, float, q, k, v, dO, lambda, kv0, dlambda, ws, g,

@@ -553,3 +553,42 @@ def test_paired_reverse_automatic_split(orc, BL):
         for name, a, r in zip(NAMES, got, ref):
             check(f"auto split B{Bn} L{L} (b={b},h={h}) {name}", a[b:b + 1, h:h + 1],
                   r[:, i:i + 1], torch.bfloat16)
+
+
+# ------------------------------------------ decay gradient on the tensor cores
+@pytest.mark.parametrize("split", [0, 1, 3])
+@pytest.mark.parametrize("L", [1, 127, 129, 1000])
+def test_dlambda_tc_decay_range(orc, L, split):
+    """The tensor-core decay gradient (bf16, d = e = 128; blocks of 128 rows,
+    bf16 copies of the carried KV and W as MMA operands) over decays from 0
+    to 1, an initial state, ragged blocks and forced splits, every head
+    against the oracle at the 1e-3 bar."""
+    x = inputs.make_inputs(2, 6, L, 128, 128, dtype=torch.bfloat16, device=DEV, seed=L + 7 * split,
+                           with_kv0=True)
+    lam = inputs.fixed_lambdas((0.0, 0.3, 0.9, 0.99, 0.999, 1.0), DEV)
+    old = la2.set_option(la2.LA2_OPT_SPLIT, split)
+    try:
+        got = la2.dlambda(x["q"], x["k"], x["v"], lam, x["dO"], x["kv0"])
+        torch.cuda.synchronize()
+    finally:
+        la2.set_option(la2.LA2_OPT_SPLIT, old)
+    assert la2.last_device_error() == 0
+    h = {n: host(t) for n, t in x.items()}
+    ref = orc.dlambda(h["q"], h["k"], h["v"], lam.double().cpu().numpy(), h["dO"], h["kv0"])
+    err = np.max(np.abs(got.double().cpu().numpy() - ref))
+    assert err <= 1e-3 * max(float(np.max(np.abs(ref))), 1e-6), (got, ref)
+
+
+def test_dlambda_tc_matches_fp32_form():
+    """The tensor-core and fp32-FMA forms of the decay gradient agree on the
+    bench's shape (two independent kernels, one chunk plan each)."""
+    B, H, L = 4, 16, 2048
+    x = inputs.make_inputs(B, H, L, 128, 128, dtype=torch.bfloat16, device=DEV, seed=3)
+    lam = inputs.decay_lambdas(H, DEV)
+    tc = la2.dlambda(x["q"], x["k"], x["v"], lam, x["dO"])
+    with options(path="simt"):
+        ref = la2.dlambda(x["q"], x["k"], x["v"], lam, x["dO"])
+    torch.cuda.synchronize()
+    assert la2.last_device_error() == 0
+    err = float((tc.double() - ref.double()).abs().max())
+    assert err <= 1e-3 * float(ref.double().abs().max()), (tc, ref)
