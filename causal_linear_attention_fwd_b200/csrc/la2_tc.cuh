@@ -72,7 +72,9 @@ template <int MODE> struct Layout {
   static constexpr uint32_t STAGE = OUT ? 3 * TILE : 2 * TILE;
   static constexpr uint32_t KVBF = NSTAGE * STAGE;
   static constexpr uint32_t MISC = KVBF + (OUT ? TILE : 0);
-  static constexpr uint32_t MISC_BYTES = 8 * (NSTAGE + 1) + 16 + 4 * (BLOCK + 1);
+  // full[NS], mma, done (abort path), then the TMEM slot, the abort flag
+  // and the decay table
+  static constexpr uint32_t MISC_BYTES = 8 * (NSTAGE + 2) + 16 + 4 * (BLOCK + 1);
   static constexpr uint32_t SMEM = MISC + MISC_BYTES + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = OUT ? 512 : 128;
   static constexpr uint32_t COL_S = 0, COL_X = 128, COL_Y = 256;
@@ -151,11 +153,12 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + LY::MISC);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NS + 1);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NS + 2);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   float *pw = reinterpret_cast<float *>(tmem_slot + 4);
   const uint32_t bar_full0 = smem_u32(bars);
   const uint32_t bar_mma = smem_u32(bars + NS);
+  const uint32_t bar_done = smem_u32(bars + NS + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quarter = warp & 3, half = warp >> 2;
@@ -172,6 +175,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
   if (tid == 0) {
     for (int s = 0; s < NS; s++) mbar_init(bar_full0 + 8 * s, 1);
     mbar_init(bar_mma, 1);
+    mbar_init(bar_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
     if (OUT) tma_prefetch_desc(&tm0);
@@ -442,11 +446,14 @@ chunk_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CU
       }
     }
   } else if (tid == 0) {
-    // drain the loads still in flight before the shared memory is released
-    for (int j = i; j < issued; j++) {
-      volatile int dummy = 0;
+    // drain the loads still in flight before the shared memory is released,
+    // and the MMAs issued (a wait that gave up may have left some running)
+    // before TMEM is
+    volatile int dummy = 0;
+    for (int j = i; j < issued; j++)
       mbar_wait(bar_full0 + 8 * (j % NS), (uint32_t)((j / NS) & 1), &dummy);
-    }
+    mma_commit(bar_done);
+    mbar_wait(bar_done, 0, &dummy);
   }
   if (OUT && tid == 0) tma_store_wait0();
   tc_fence_before();

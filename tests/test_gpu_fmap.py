@@ -15,8 +15,10 @@ pytestmark = pytest.mark.gpu
 
 DEV = "cuda:0"
 # the kernel's arithmetic is fp32 with CUDA's expf (2 ulp), its result
-# rounded to the I/O type: half a bf16 ulp (2^-9) plus the fp32 error for
-# bf16, a few fp32 ulp for fp32
+# rounded to the I/O type.  For bf16 one rounding errs by at most half an ulp,
+# which relative to the value is below 2^-8 (2^-9 at the top of a binade, up
+# to just under 2^-8 at its bottom); the fp32 error (~2^-22) fits in the gap
+# below 2^-8.  For fp32, a few fp32 ulp.
 REL = {torch.bfloat16: 2.0 ** -8, torch.float32: 5e-7}
 SPECIAL = [0.0, -0.0, 1.0, -1.0, 50.0, -30.0, -87.0, -100.0, 1e-3, -1e-3]
 
