@@ -40,7 +40,7 @@ enum KernelId {
   K_SIMT_REV_SCAN, K_SIMT_DKDV, K_DECODE, K_TC_FWD_STATE, K_TC_FWD, K_TC_DQ,
   K_TC_REV_STATE, K_TC_DV, K_TC_DK, K_SCAN_FWD, K_SCAN_REV, K_SIMT_DLAMBDA,
   K_SIMT_DLAMBDA_STATE, K_SIMT_DLAMBDA_SCAN, K_TC_DECODE_UNITS, K_FMAP, K_FMAP_GRAD, K_TC_DKDV,
-  K_TC_DLAMBDA, K_TC_DLAMBDA_STATE, K_COUNT
+  K_TC_DLAMBDA, K_TC_DLAMBDA_STATE, K_STATE_PAD, K_COUNT
 };
 const char *kKernelName[K_COUNT] = {
     "simt_fwd_chunk_state", "simt_scan_fwd", "simt_fwd", "simt_dq",
@@ -48,7 +48,7 @@ const char *kKernelName[K_COUNT] = {
     "tc_fwd_chunk_state", "tc_fwd", "tc_dq", "tc_rev_chunk_state", "tc_dv", "tc_dk",
     "scan_fwd", "scan_rev", "simt_dlambda", "simt_dlambda_chunk_state", "simt_dlambda_scan",
     "tc_decode_units", "feature_map", "feature_map_grad", "tc_dkdv", "tc_dlambda",
-    "tc_dlambda_chunk_state"};
+    "tc_dlambda_chunk_state", "state_pad"};
 
 struct ProfRec {
   int kid;
@@ -153,11 +153,16 @@ bool shape_supported(int d, int e, la2_dtype dt) {
 
 size_t esize(la2_dtype dt) { return dt == LA2_F32 ? 4 : 2; }
 
-// Which kernel family serves a call.
+// Which kernel family serves a call.  any_head: the entry point runs the
+// tensor-core passes for head sizes 64 too (its 64-column tensors read with
+// zero columns beyond their width, its states padded to 128 x 128 in
+// workspace scratch); else bf16 with d = e = 128 only.
 enum Path { PATH_SIMT = 0, PATH_TC = 1, PATH_NONE = 2 };
-Path choose_path(int d, int e, la2_dtype dt) {
+Path choose_path(int d, int e, la2_dtype dt, bool any_head = false) {
   const int opt = g_opt_path.load();
-  const bool tc_ok = la2::tc::supports(d, e, dt == LA2_BF16) && device_cc() == 100;
+  const bool shape_ok = la2::tc::supports(d, e, dt == LA2_BF16) ||
+                        (any_head && dt == LA2_BF16 && shape_supported(d, e, dt));
+  const bool tc_ok = shape_ok && device_cc() == 100;
   if (opt == 1) return PATH_SIMT;
   if (opt == 2) return tc_ok ? PATH_TC : PATH_NONE;
   return tc_ok ? PATH_TC : PATH_SIMT;
@@ -297,6 +302,12 @@ size_t ws_bwd_bytes(const Geo &g, const Geo &gr, int d, int e) {
   };
   return one(g) + one(gr);
 }
+
+// A tensor-core call with a 64-column head size keeps its initial and final
+// states padded to 128 x 128 fp32 in scratch after the chunk states: n
+// states per (b,h).
+bool padded(Path p, int d, int e) { return p == PATH_TC && (d != 128 || e != 128); }
+size_t pad_bytes(const Geo &g, int n) { return (size_t)g.B * g.H * 128 * 128 * sizeof(float) * n; }
 
 size_t ws_bytes(int op, const Geo &g, int d, int e) {
   if (op == LA2_OP_DLAMBDA)  // (KV, W) per sub-chunk boundary
@@ -590,10 +601,13 @@ size_t la2_workspace_size(int op, int B, int H, int64_t L, int d, int e, la2_dty
     return ws_bytes(op, plan_dlambda(B, H, L, true, block_rows(p)), d, e);
   }
   if (op != LA2_OP_FORWARD && op != LA2_OP_BACKWARD && op != LA2_OP_SHARD_STATE) return 0;
-  Path p = choose_path(d, e, dt);
+  Path p = choose_path(d, e, dt, op != LA2_OP_SHARD_STATE);
   if (p == PATH_NONE) return 0;
   Geo g = plan(B, H, L, block_rows(p), p);
-  if (op == LA2_OP_BACKWARD) return ws_bwd_bytes(g, plan_rev(B, H, L, p), d, e);
+  const int sd = p == PATH_TC ? 128 : d, se = p == PATH_TC ? 128 : e;  // state slot shape
+  if (op == LA2_OP_BACKWARD)
+    return ws_bwd_bytes(g, plan_rev(B, H, L, p), sd, se) + (padded(p, d, e) ? pad_bytes(g, 2) : 0);
+  if (op == LA2_OP_FORWARD) return ws_bytes(op, g, sd, se) + (padded(p, d, e) ? pad_bytes(g, 2) : 0);
   return ws_bytes(op, g, d, e);
 }
 
@@ -651,20 +665,40 @@ la2_status la2_forward(const void *q, const void *k, const void *v,
                           : cudaMemsetAsync(kv_out, 0, ns, stream);
     return to_status(err);
   }
-  Path p = choose_path(d, e, dt);
+  Path p = choose_path(d, e, dt, true);
   if (p == PATH_NONE) return LA2_ERR_UNSUPPORTED;
   Geo g = plan(B, H, L, block_rows(p), p);
-  const size_t need = ws_bytes(LA2_OP_FORWARD, g, d, e);
+  const bool pad = padded(p, d, e);
+  const size_t states = ws_bytes(LA2_OP_FORWARD, g, p == PATH_TC ? 128 : d, p == PATH_TC ? 128 : e);
+  const size_t need = states + (pad ? pad_bytes(g, 2) : 0);
   if (need > 0 && (!workspace || workspace_bytes < need)) return LA2_ERR_INVALID;
   float *ws = (float *)workspace;
   cudaError_t err;
   if (p == PATH_TC) {
     g.inject = g_opt_inject.exchange(0);
-    err = la2::tc::forward(q, k, v, lambda, kv0, o, kv_out, ws, g, stream,
+    g.d = d;
+    g.e = e;
+    // 64-column heads: the states in and out padded to 128 x 128
+    float *scratch = pad ? reinterpret_cast<float *>(reinterpret_cast<char *>(workspace) + states)
+                         : nullptr;
+    const float *kv0_t = kv0;
+    float *kv_out_t = kv_out;
+    if (pad) {
+      kv0_t = kv0 ? scratch : nullptr;
+      kv_out_t = kv_out ? scratch + (size_t)BH * 128 * 128 : nullptr;
+      if (kv0) {
+        err = timed(K_STATE_PAD, stream, [&] { la2::tc::pad_states(kv0, scratch, BH, d, e, stream); });
+        if (err != cudaSuccess) return to_status(err);
+      }
+    }
+    err = la2::tc::forward(q, k, v, lambda, kv0_t, o, kv_out_t, ws, g, stream,
                            [&](int which, auto &&fn) {
                              return timed(which == 0 ? K_TC_FWD_STATE : which == 1 ? K_SCAN_FWD : K_TC_FWD,
                                           stream, fn);
                            });
+    if (err == cudaSuccess && pad && kv_out)
+      err = timed(K_STATE_PAD, stream,
+                  [&] { la2::tc::unpad_states(kv_out_t, kv_out, BH, d, e, stream); });
   } else if (dt == LA2_F32) {
     err = LA2_DISPATCH_DE(d, e, simt_forward, float, q, k, v, lambda, kv0, o, kv_out, ws, g, stream);
   } else {
@@ -714,22 +748,43 @@ la2_status la2_backward_ex(const void *q, const void *k, const void *v,
     if (!dkv0) return LA2_OK;
     return to_status(cudaMemsetAsync(dkv0, 0, ns, stream));
   }
-  Path p = choose_path(d, e, dt);
+  Path p = choose_path(d, e, dt, true);
   if (p == PATH_NONE) return LA2_ERR_UNSUPPORTED;
   Geo g = plan(B, H, L, block_rows(p), p);
-  const Geo gr = plan_rev(B, H, L, p);
-  const size_t need = ws_bwd_bytes(g, gr, d, e);
+  Geo gr = plan_rev(B, H, L, p);
+  const bool pad = padded(p, d, e);
+  const size_t states =
+      ws_bwd_bytes(g, gr, p == PATH_TC ? 128 : d, p == PATH_TC ? 128 : e);
+  const size_t need = states + (pad ? pad_bytes(g, 2) : 0);
   if (need > 0 && (!workspace || workspace_bytes < need)) return LA2_ERR_INVALID;
   float *ws = (float *)workspace;
   cudaError_t err;
   if (p == PATH_TC) {
-    err = la2::tc::backward(q, k, v, lambda, kv0, dO, dq, dk, dv, dkv0, ws, g, gr, reuse, stream,
+    g.d = gr.d = d;
+    g.e = gr.e = e;
+    // 64-column heads: kv0 in and dkv0 out padded to 128 x 128
+    float *scratch = pad ? reinterpret_cast<float *>(reinterpret_cast<char *>(workspace) + states)
+                         : nullptr;
+    const float *kv0_t = kv0;
+    float *dkv0_t = dkv0;
+    if (pad) {
+      kv0_t = kv0 ? scratch : nullptr;
+      dkv0_t = dkv0 ? scratch + (size_t)BH * 128 * 128 : nullptr;
+      if (kv0) {
+        err = timed(K_STATE_PAD, stream, [&] { la2::tc::pad_states(kv0, scratch, BH, d, e, stream); });
+        if (err != cudaSuccess) return to_status(err);
+      }
+    }
+    err = la2::tc::backward(q, k, v, lambda, kv0_t, dO, dq, dk, dv, dkv0_t, ws, g, gr, reuse, stream,
                             [&](int which, auto &&fn) {
                               static const int ids[] = {K_TC_FWD_STATE, K_SCAN_FWD, K_TC_DQ,
                                                         K_TC_REV_STATE, K_SCAN_REV, K_TC_DV,
                                                         K_TC_DK, K_TC_DKDV};
                               return timed(ids[which], stream, fn);
                             });
+    if (err == cudaSuccess && pad && dkv0)
+      err = timed(K_STATE_PAD, stream,
+                  [&] { la2::tc::unpad_states(dkv0_t, dkv0, BH, d, e, stream); });
   } else if (dt == LA2_F32) {
     err = LA2_DISPATCH_DE(d, e, simt_backward, float, q, k, v, lambda, kv0, dO, dq, dk, dv, dkv0,
                           ws, g, reuse, stream);
@@ -1312,12 +1367,8 @@ extern "C" la2_status la2_forward_noalloc(const void *q, const void *k, const vo
                                         nullptr, 0, &empty);
   if (chk != LA2_OK || empty) return chk;
   // Same plan as la2_forward; refuse plans whose scratch exceeds the array.
-  if (L > 0) {
-    const Path p = choose_path(d, e, dt);
-    if (p == PATH_NONE) return LA2_ERR_UNSUPPORTED;
-    const Geo g = plan(B, H, L, block_rows(p), p);
-    if (ws_bytes(LA2_OP_FORWARD, g, d, e) > kNoallocScratchBytes) return LA2_ERR_UNSUPPORTED;
-  }
+  if (L > 0 && la2_workspace_size(LA2_OP_FORWARD, B, H, L, d, e, dt) > kNoallocScratchBytes)
+    return LA2_ERR_UNSUPPORTED;
   void *scratch = noalloc_scratch_ptr();
   if (!scratch) return LA2_ERR_CUDA;
   return la2_forward(q, k, v, lambda, kv0, o, kv_out, B, H, L, d, e, dt, scratch,

@@ -62,6 +62,10 @@ struct Geo {
   int variant;  // tensor-core kernel form (0: warp-specialised, 1: phase-serial)
   int trace;    // tensor-core pass whose CTA 0 stamps the trace buffer (-1: none)
   int rev_pair = 0;  // tensor-core backward: dV and dK as one paired launch
+  // tensor-core passes: the head sizes of the tensors (64 or 128; the
+  // kernels work on 128 columns, a 64-column tensor read with zeros beyond
+  // its width and its states padded to 128 x 128 by the caller)
+  int d = 128, e = 128;
 };
 
 // What one CTA of a pass works on: state slot bh (the (b,h) or (sequence,

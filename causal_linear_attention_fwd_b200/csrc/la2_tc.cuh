@@ -618,6 +618,11 @@ chunk_body(const CUtensorMap *tm0, const CUtensorMap *tm1, const CUtensorMap *tm
   // (fixed per mode; chosen per CTA in the paired reverse launch)
   const bool X_MN = MODE == MODE_RPAIR ? !is_dk : TR::X_MN;
   const bool SWAP = MODE == MODE_RPAIR ? is_dk : TR::SWAP;
+  // the output tensor has 64 columns (the second box is not stored): O and
+  // dV have e columns, dQ and dK have d
+  const bool out_is_e =
+      MODE == MODE_FWD || MODE == MODE_DV || (MODE == MODE_RPAIR && !is_dk);
+  const bool out64 = (out_is_e ? g.e : g.d) == 64;
   constexpr uint32_t IDESC_S = idesc_bf16(128, 128, false, false);
   const uint32_t IDESC_X =
       X_MN ? idesc_bf16(128, 128, false, true) : idesc_bf16(128, 128, false, false);
@@ -1138,7 +1143,7 @@ chunk_body(const CUtensorMap *tm0, const CUtensorMap *tm1, const CUtensorMap *tm
           const uint32_t sst = sbase + st * LY::STAGE + LY::C_OFF;
           const int y = (int)p_of(i), z = (int)slab_of(i);
           tma_store_3d(tmo, sst, 0, y, z);
-          tma_store_3d(tmo, sst + BOX, 64, y, z);
+          if (!out64) tma_store_3d(tmo, sst + BOX, 64, y, z);
           tma_store_commit();
           tma_store_wait_read0();
         }
@@ -1248,13 +1253,16 @@ inline EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [BH, L, 128] bf16, boxes of 128 rows x 64 columns, 128-byte swizzle; rows
-// outside [0, L) read as zero and are not written.
-inline bool make_map(CUtensorMap *m, const void *ptr, int64_t BH, int64_t L) {
+// [BH, L, W] bf16 (W = 128 or 64), boxes of 128 rows x 64 columns, 128-byte
+// swizzle; rows outside [0, L) read as zero and are not written.  With W =
+// 64 the kernels' second box (columns 64..127) lies wholly outside the
+// tensor: it loads as zeros (the head size padded to 128 with zero columns,
+// which every product carries through exactly) and is not stored.
+inline bool make_map(CUtensorMap *m, const void *ptr, int64_t BH, int64_t L, int W = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[3] = {128, (cuuint64_t)L, (cuuint64_t)BH};
-  cuuint64_t strides[2] = {128 * 2, (cuuint64_t)L * 128 * 2};
+  cuuint64_t dims[3] = {(cuuint64_t)W, (cuuint64_t)L, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)W * 2, (cuuint64_t)L * W * 2};
   cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box,
@@ -1319,6 +1327,30 @@ cudaError_t launch_pair(const CUtensorMap &mk, const CUtensorMap &mq, const CUte
                             static_cast<__nv_bfloat16 *>(outp_dk), g);
 }
 
+// States [BH, d, e] fp32 <-> [BH, 128, 128] fp32 with zeros outside d x e
+// (the tensor-core passes' state shape for 64-column heads).
+__global__ void pad_state_kernel(const float *__restrict__ src, float *__restrict__ dst, int d,
+                                 int e) {
+  const int64_t bh = blockIdx.y;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;  // < 128 * 128
+  const int r = idx >> 7, c = idx & 127;
+  dst[bh * 16384 + idx] = (r < d && c < e) ? src[(bh * d + r) * e + c] : 0.f;
+}
+__global__ void unpad_state_kernel(const float *__restrict__ src, float *__restrict__ dst, int d,
+                                   int e) {
+  const int64_t bh = blockIdx.y;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;  // < d * e
+  if (idx >= d * e) return;
+  const int r = idx / e, c = idx % e;
+  dst[bh * d * e + idx] = src[bh * 16384 + r * 128 + c];
+}
+inline void pad_states(const float *src, float *dst, int64_t BH, int d, int e, cudaStream_t st) {
+  pad_state_kernel<<<dim3(16384 / 256, (unsigned)BH), 256, 0, st>>>(src, dst, d, e);
+}
+inline void unpad_states(const float *src, float *dst, int64_t BH, int d, int e, cudaStream_t st) {
+  unpad_state_kernel<<<dim3((d * e + 255) / 256, (unsigned)BH), 256, 0, st>>>(src, dst, d, e);
+}
+
 inline bool geometry_ok(const Geo &g) {
   return g.L < (int64_t(1) << 31) && (int64_t)g.B * g.H < (int64_t(1) << 31);
 }
@@ -1331,8 +1363,8 @@ cudaError_t forward(const void *q, const void *k, const void *v, const float *la
   if (!geometry_ok(g)) return cudaErrorInvalidValue;
   const int64_t BH = (int64_t)g.B * g.H;
   CUtensorMap mq, mk, mv, mo;
-  if (!make_map(&mq, q, BH, g.L) || !make_map(&mk, k, BH, g.L) || !make_map(&mv, v, BH, g.L) ||
-      !make_map(&mo, o, BH, g.L))
+  if (!make_map(&mq, q, BH, g.L, g.d) || !make_map(&mk, k, BH, g.L, g.d) ||
+      !make_map(&mv, v, BH, g.L, g.e) || !make_map(&mo, o, BH, g.L, g.e))
     return cudaErrorInvalidValue;
   cudaError_t err = cudaSuccess;
   if (g.S > 1) {
@@ -1363,9 +1395,10 @@ cudaError_t backward(const void *q, const void *k, const void *v, const float *l
   if (!geometry_ok(g) || !geometry_ok(gr)) return cudaErrorInvalidValue;
   const int64_t BH = (int64_t)g.B * g.H;
   CUtensorMap mq, mk, mv, mg, mdq, mdk, mdv;
-  if (!make_map(&mq, q, BH, g.L) || !make_map(&mk, k, BH, g.L) || !make_map(&mv, v, BH, g.L) ||
-      !make_map(&mg, dO, BH, g.L) || !make_map(&mdq, dq, BH, g.L) ||
-      !make_map(&mdk, dk, BH, g.L) || !make_map(&mdv, dv, BH, g.L))
+  if (!make_map(&mq, q, BH, g.L, g.d) || !make_map(&mk, k, BH, g.L, g.d) ||
+      !make_map(&mv, v, BH, g.L, g.e) || !make_map(&mg, dO, BH, g.L, g.e) ||
+      !make_map(&mdq, dq, BH, g.L, g.d) || !make_map(&mdk, dk, BH, g.L, g.d) ||
+      !make_map(&mdv, dv, BH, g.L, g.e))
     return cudaErrorInvalidValue;
   float *wsf = ws;
   float *wsr = ws ? ws + (g.S > 1 ? (size_t)BH * g.wsS * 128 * 128 : 0) : nullptr;

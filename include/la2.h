@@ -29,7 +29,12 @@
  *     `dt` (LA2_F32 or LA2_BF16) is the element type of q, k, v, o, dO, dq,
  *     dk, dv.  Arithmetic is fp32 (bf16 tensor-core products with fp32
  *     accumulation for LA2_BF16; fp32 FMA for LA2_F32).
- *   - Supported head sizes: d, e in {64, 128}.
+ *   - Supported head sizes: d, e in {64, 128}.  With LA2_BF16, la2_forward
+ *     and la2_backward run every size on the tensor cores (a 64-column
+ *     tensor is read with zero columns up to 128, its states padded to
+ *     128 x 128 in workspace scratch, which la2_workspace_size includes);
+ *     the other entry points do so for d = e = 128 and use fp32 FMA
+ *     kernels for 64.
  *   - Every pointer must be 16-byte aligned.
  *   - The caller owns all memory.  The library allocates nothing on the
  *     device: scratch memory comes from the caller as `workspace`, sized by
