@@ -979,14 +979,20 @@ def main():
     ap.add_argument("--bwd-form", type=int, default=None,
                     help="profiling aid: LA2_OPT_BWD_FORM for the run (0 paired dV/dK "
                          "launch, the library's default; 1 two separate passes)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="profiling aid: tokens per sweep batch (default 65,536; with --only, "
+                         "B*L must equal it); smaller batches keep ncu captures small")
     ap.add_argument("--only", default=None,
                     help="B:L -- time a single sweep point instead of the whole sweep "
                          "(profiling aid; not the metric)")
     args = ap.parse_args()
+    global SWEEP, TOKENS
+    if args.tokens:
+        assert args.only, "--tokens is a profiling aid: give the point with --only B:L"
+        TOKENS = args.tokens
     if args.only:
-        global SWEEP
         b_, l_ = (int(x) for x in args.only.split(":"))
-        assert b_ * l_ == TOKENS, "--only must keep 65,536 tokens per batch"
+        assert b_ * l_ == TOKENS, "--only must keep the batch's tokens (65,536 unless --tokens)"
         SWEEP = [(b_, l_)]
     args.warmup = max(args.warmup, 3) if args.impl == "la2" else args.warmup
     if args.impl == "reference":
