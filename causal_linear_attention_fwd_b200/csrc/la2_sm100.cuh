@@ -1,6 +1,6 @@
 // la2_sm100.cuh -- thin wrappers over the sm_100a instructions the
 // tensor-core kernels use: mbarriers with bounded waits, TMA (tiled bulk
-// tensor copies, no multicast), tcgen05 MMA / TMEM load-store / commit /
+// tensor copies into the issuing CTA's own shared memory), tcgen05 MMA / TMEM load-store / commit /
 // alloc, and the shared-memory matrix descriptors.  Written from the PTX ISA
 // description of these instructions.
 #pragma once

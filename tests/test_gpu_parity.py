@@ -147,17 +147,21 @@ def test_tc_phase_serial_variant(orc, L, split):
     compare(got, oracle_all(orc, x, lam, x["kv0"]), torch.bfloat16, f"v1 L={L} S={split}")
 
 
+@pytest.mark.parametrize("de", [(128, 128), (64, 128), (64, 64)])
 @pytest.mark.parametrize("path", ["simt", "tc"])
-def test_backward_reuses_forward_states(orc, path):
+def test_backward_reuses_forward_states(orc, path, de):
     """A training step that hands the forward's workspace to the backward
     (LA2_BWD_REUSE_FORWARD_STATES) gives the same gradients as a backward
-    that recomputes the chunk states, and the oracle's."""
+    that recomputes the chunk states, and the oracle's (with 64-column heads
+    the tensor-core workspace also holds the padded states after the chunk
+    states)."""
     B, H, L = 1, 3, 1000
-    x = inputs.make_inputs(B, H, L, 128, 128, dtype=torch.bfloat16, device=DEV, seed=13,
+    d, e = de
+    x = inputs.make_inputs(B, H, L, d, e, dtype=torch.bfloat16, device=DEV, seed=13,
                            with_kv0=True)
     lam = inputs.fixed_lambdas((1.0, 0.95, 0.5), DEV)
     with options(path=path, split=4):
-        n = la2.workspace_size(la2.LA2_OP_BACKWARD, B, H, L, 128, 128, torch.bfloat16)
+        n = la2.workspace_size(la2.LA2_OP_BACKWARD, B, H, L, d, e, torch.bfloat16)
         assert n > 0
         ws = torch.empty(n, dtype=torch.uint8, device=DEV)
         o = la2.forward(x["q"], x["k"], x["v"], lam, x["kv0"], workspace=ws)

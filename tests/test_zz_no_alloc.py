@@ -60,11 +60,14 @@ def test_noalloc_forward_matches_oracle_and_workspace_forward(orc):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("de", [(128, 128), (64, 64)])
 @pytest.mark.parametrize("with_kv0", [True, False])
-def test_noalloc_python_wrapper(orc, with_kv0):
+def test_noalloc_python_wrapper(orc, with_kv0, de):
     """la2.forward_noalloc (the binding) against la2.forward and the oracle,
-    with and without an initial state, outputs allocated by the caller."""
-    B, H, L, d, e = 2, 3, 1000, 128, 128
+    with and without an initial state, outputs allocated by the caller (with
+    64-column heads the array also holds the padded states)."""
+    B, H, L = 2, 3, 1000
+    d, e = de
     x = inputs.make_inputs(B, H, L, d, e, dtype=torch.bfloat16, device=DEV, seed=7,
                            with_dO=False, with_kv0=True)
     kv0 = x["kv0"] if with_kv0 else None
