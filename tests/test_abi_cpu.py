@@ -48,6 +48,11 @@ def test_status_strings(lib):
 def test_set_option_roundtrip(lib):
     old = la2.set_option(la2.LA2_OPT_SPLIT, 5)
     assert la2.set_option(la2.LA2_OPT_SPLIT, old) == 5
+    for opt in (la2.LA2_OPT_PATH, la2.LA2_OPT_VARIANT, la2.LA2_OPT_VARLEN_ORDER,
+                la2.LA2_OPT_DECODE_BLOCK_TOKENS, la2.LA2_OPT_BWD_FORM):
+        old = la2.set_option(opt, 1)
+        assert old >= 0
+        assert la2.set_option(opt, old) == 1
     assert la2.set_option(99, 1) == -1
 
 
