@@ -251,29 +251,33 @@ Geo plan_rev(int B, int H, int64_t L, Path p) {
   return g;
 }
 
-// Chunk plan of the decay gradient (one CTA per SM; blocks of blk rows: 32
-// for the fp32-FMA kernel, 128 for the tensor-core one): at most one wave,
-// S = floor(SMs / (B*H)) chunks per sequence when B*H is below the SM count
-// (LA2_OPT_SPLIT overrides), Lc a multiple of the block.
+// Chunk plan of the decay gradient (blocks of blk rows: 32 for the fp32-FMA
+// kernel, one CTA per chunk; 128 for the tensor-core one, two CTAs per chunk,
+// one per half of the e columns): at most one wave, S = floor(slots / (B*H))
+// chunks per sequence when B*H is below the slots -- the SMs, or half of them
+// for the tensor-core kernel (LA2_OPT_SPLIT overrides) -- Lc a multiple of
+// the block.  (Counting a tensor-core chunk as one slot would split B*H = 64
+// sequences in two on 148 SMs: 256 CTAs, two waves as long as the one wave of
+// 128 unsplit, plus the pre-pass and the scan.)
 // The chunk-state pre-pass covers chunks 0..S-2 only, so it runs on M
-// sub-chunks of Ls rows per chunk (Lc = M Ls), M filling the SMs (at most
+// sub-chunks of Ls rows per chunk (Lc = M Ls), M filling the slots (at most
 // 8); the workspace holds (S-1) M + 1 (KV, W) pairs per (b,h).
 Geo plan_dlambda(int B, int H, int64_t L, bool split_ok, int blk_rows) {
   Geo g = plan(B, H, L, blk_rows, PATH_SIMT);
   const int64_t blk = blk_rows, nblk = (L + blk - 1) / blk;
   const int64_t BH = (int64_t)B * H;
-  const int sms = device_sms();
+  const int slots = blk_rows == la2::tc::BLOCK ? device_sms() / 2 : device_sms();
   int64_t S = g_opt_split.load();
-  if (S <= 0) S = BH >= sms ? 1 : sms / BH;
+  if (S <= 0) S = BH >= slots ? 1 : slots / BH;
   if (!split_ok || S > nblk) S = split_ok ? nblk : 1;
   if (S < 1) S = 1;
   int64_t per = (nblk + S - 1) / S;  // blocks per chunk
   S = (nblk + per - 1) / per;
   int64_t M = 1;
   if (S > 1) {
-    // the largest M <= min(8, SMs / (B*H*(S-1))) whose whole sub-chunks
+    // the largest M <= min(8, slots / (B*H*(S-1))) whose whole sub-chunks
     // keep S chunks
-    int64_t want = sms / (BH * (S - 1));
+    int64_t want = slots / (BH * (S - 1));
     if (want > 8) want = 8;
     for (int64_t m = want; m > 1; m--) {
       const int64_t p = ((per + m - 1) / m) * m;
