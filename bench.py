@@ -859,6 +859,8 @@ def run_fmap(args, world, rank, local):
     dev = torch.device("cuda", local)
     pk = peaks()
     Bn, L = 8, 8192
+    if args.tokens:  # profiling aid: fewer batch rows of the same length
+        Bn = max(1, args.tokens // L)
     x = inputs.make_inputs(Bn, H, L, D, E, dtype=torch.bfloat16, device=dev, seed=0)
     lam = inputs.decay_lambdas(H, dev)
     buf = {n: torch.empty_like(x[src]) for n, src in
@@ -925,10 +927,11 @@ def run_fmap(args, world, rank, local):
                                  "cores": orc.num_threads(), "kind": "oracle",
                                  "sample": f"one batch row ({H} heads x {L} rows) of the workload"}
     return _common(world, args.steps, args.warmup, value, "tokens/s",
-                   "fwd+bwd tokens/s with the elu+1 feature map (B=8,H=32,L=8192,d=e=128,bf16)",
+                   f"fwd+bwd tokens/s with the elu+1 feature map (B={Bn},H={H},L={L},d=e=128,bf16)",
                    {"workload": "training step with the feature map phi(x) = elu(x) + 1 on q "
-                                "and k, B=8, H=32, L=8,192, d=e=128, bf16",
-                    "l2": "inputs 512 MiB per tensor, larger than L2; no flush"}, ms, extra)
+                                f"and k, B={Bn}, H={H}, L={L:,}, d=e=128, bf16",
+                    "l2": f"inputs {Bn * H * L * D * 2 >> 20} MiB per tensor, larger than L2; "
+                          "no flush"}, ms, extra)
 
 
 def run_subrecords(args, world, rank, local):
@@ -981,13 +984,14 @@ def main():
                          "launch, the library's default; 1 two separate passes)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="profiling aid: tokens per sweep batch (default 65,536; with --only, "
-                         "B*L must equal it); smaller batches keep ncu captures small")
+                         "B*L must equal it), or per batch of --workload fmap (rows of 8,192); "
+                         "smaller batches keep ncu captures small")
     ap.add_argument("--only", default=None,
                     help="B:L -- time a single sweep point instead of the whole sweep "
                          "(profiling aid; not the metric)")
     args = ap.parse_args()
     global SWEEP, TOKENS
-    if args.tokens:
+    if args.tokens and args.workload == "sweep":
         assert args.only, "--tokens is a profiling aid: give the point with --only B:L"
         TOKENS = args.tokens
     if args.only:
