@@ -418,7 +418,7 @@ template <typename T, int D, int E>
 cudaError_t decode(const void *q, const void *k, const void *v, const float *lam,
                    float *pool, const int *slots, int pool_size, void *o, int B, int H,
                    int ntok, cudaStream_t st) {
-  auto kern = ntok == 1 ? la2::dec::decode_kernel<T, D, E, 1> : la2::dec::decode_kernel<T, D, E, 4>;
+  auto kern = ntok == 1 ? la2::dec::decode_kernel<T, D, E, 1> : la2::dec::tokens_kernel<T, D, E, 4>;
   return timed(K_DECODE, st, [&] {
     kern<<<(unsigned)((int64_t)B * H), la2::dec::NT, 0, st>>>(
         (const T *)q, (const T *)k, (const T *)v, lam, pool, slots, pool_size, (T *)o, H, ntok);

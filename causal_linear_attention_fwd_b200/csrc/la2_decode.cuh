@@ -138,5 +138,97 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
   }
 }
 
+// Several tokens per call (T = ntok >= 2): decode_kernel's state update
+// with the tokens' q, k, v staged in shared memory up to TS = 8 at a time (one
+// load of all of them, in flight together with the state's), and the
+// per-group cross-warp sums double-buffered, so each group of G tokens costs
+// one block barrier and no exposed global-load latency.
+template <typename T, int D, int E, int G>
+__global__ void __launch_bounds__(NT)
+tokens_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+              const float *__restrict__ lambda, float *__restrict__ pool,
+              const int *__restrict__ slots, int pool_size, T *__restrict__ o, int H, int ntok) {
+  constexpr int ROWS = D / NW;
+  constexpr int VEC = E / 32;
+  constexpr int TS = 8;  // tokens staged at once (static shared memory: 44 KB at d = e = 128)
+  using V = vec_t<VEC>;
+  __shared__ float qs[TS][D], ks[TS][D], vs[TS][E];
+  __shared__ float red[2][NW][G][E];
+
+  const int64_t bh = blockIdx.x;
+  const int64_t b = bh / H;
+  const int h = (int)(bh % H);
+  const int tid = threadIdx.x, w = tid / 32, l = tid % 32;
+  int64_t slot = b;
+  if (slots) {
+    slot = slots[b];
+    if (slot < 0) return;  // inactive request
+    if (slot >= pool_size) {
+      if (tid == 0) raise_error(ERR_BOUNDS);
+      return;
+    }
+  }
+  const float lam = lambda[h];
+  float *base = pool + (slot * H + h) * (int64_t)D * E + (int64_t)(w * ROWS) * E + l * VEC;
+  typename V::type x[ROWS];
+#pragma unroll
+  for (int r = 0; r < ROWS; r++) x[r] = V::ld(base + (int64_t)r * E);
+
+  int gi = 0;  // groups done (the parity picks the sums buffer)
+  for (int c0 = 0; c0 < ntok; c0 += TS) {
+    const int nc = ntok - c0 < TS ? ntok - c0 : TS;
+    const int64_t tokc = bh * ntok + c0;
+    // (the previous chunk's q, k, v were last read before the barrier of
+    // its last group, which every thread has passed)
+    for (int idx = tid; idx < nc * D; idx += NT) {
+      qs[idx / D][idx % D] = io<T>::ld(q + tokc * D + idx);
+      ks[idx / D][idx % D] = io<T>::ld(k + tokc * D + idx);
+    }
+    for (int idx = tid; idx < nc * E; idx += NT) vs[idx / E][idx % E] = io<T>::ld(v + tokc * E + idx);
+    __syncthreads();  // the chunk's q, k, v in
+    for (int t0 = 0; t0 < nc; t0 += G) {
+      const int ng = nc - t0 < G ? nc - t0 : G;
+      // sums buffer of this group: the group before last read it before the
+      // last group's barrier
+      float(*rb)[G][E] = red[gi & 1];
+      gi++;
+#pragma unroll
+      for (int g = 0; g < G; g++) {
+        if (g >= ng) break;
+        const int tt = t0 + g;
+        float vv[VEC], acc[VEC];
+#pragma unroll
+        for (int c = 0; c < VEC; c++) {
+          vv[c] = vs[tt][l * VEC + c];
+          acc[c] = 0.f;
+        }
+#pragma unroll
+        for (int r = 0; r < ROWS; r++) {
+          const int i = w * ROWS + r;
+          const float ki = ks[tt][i], qi = qs[tt][i];
+#pragma unroll
+          for (int c = 0; c < VEC; c++) {
+            float sv = fmaf(lam, V::at(x[r], c), ki * vv[c]);
+            V::at(x[r], c) = sv;
+            acc[c] = fmaf(qi, sv, acc[c]);
+          }
+          // the last token's row goes out as soon as it is final
+          if (c0 + tt == ntok - 1) V::st(base + (int64_t)r * E, x[r]);
+        }
+#pragma unroll
+        for (int c = 0; c < VEC; c++) rb[w][g][l * VEC + c] = acc[c];
+      }
+      __syncthreads();  // every warp's partial sums of the group in
+      for (int idx = tid; idx < ng * E; idx += NT) {
+        const int g = idx / E, j = idx % E;
+        float sum = 0.f;
+#pragma unroll
+        for (int ww = 0; ww < NW; ww++) sum += rb[ww][g][j];
+        io<T>::st(o + (tokc + t0 + g) * E + j, sum);
+      }
+    }
+  }
+}
+
 }  // namespace dec
 }  // namespace la2
