@@ -418,9 +418,16 @@ template <typename T, int D, int E>
 cudaError_t decode(const void *q, const void *k, const void *v, const float *lam,
                    float *pool, const int *slots, int pool_size, void *o, int B, int H,
                    int ntok, cudaStream_t st) {
-  auto kern = ntok == 1 ? la2::dec::decode_kernel<T, D, E, 1> : la2::dec::tokens_kernel<T, D, E, 4>;
+  if (ntok == 1)
+    return timed(K_DECODE, st, [&] {
+      la2::dec::decode_kernel<T, D, E, 1><<<(unsigned)((int64_t)B * H), la2::dec::NT, 0, st>>>(
+          (const T *)q, (const T *)k, (const T *)v, lam, pool, slots, pool_size, (T *)o, H, ntok);
+    });
+  auto kern = la2::dec::tokens_kernel<T, D, E, 4>;
+  constexpr size_t smem = la2::dec::tokens_smem<E, 4>();
+  if (cudaError_t e = opt_in_smem(kern, smem)) return e;
   return timed(K_DECODE, st, [&] {
-    kern<<<(unsigned)((int64_t)B * H), la2::dec::NT, 0, st>>>(
+    kern<<<(unsigned)((int64_t)B * H), la2::dec::NTT, smem, st>>>(
         (const T *)q, (const T *)k, (const T *)v, lam, pool, slots, pool_size, (T *)o, H, ntok);
   });
 }
@@ -440,8 +447,8 @@ la2_status to_status(cudaError_t e) { return e == cudaSuccess ? LA2_OK : LA2_ERR
 // token-by-token register update.  Measured on B200 at batch 256 x 64 heads:
 // the decode-unit kernel takes ~0.93 ms per call for any T <= 128 (148 CTAs,
 // ~110 units each, set by each unit's state round trip), the token kernel
-// 0.41 ms at T = 4, 0.62 at 8, 0.96 at 16 and 1.77 at 32.
-constexpr int kDecodeBlockTokens = 16;
+// 0.40 ms at T = 4, 0.50 at 8, 0.89 at 16 and 1.18 at 24 (~0.05 ms a token).
+constexpr int kDecodeBlockTokens = 17;
 
 // ------------------------------------------------------- d lambda helper
 // dlam = 0; split: chunk-state pre-pass over the sub-chunks of chunks

@@ -56,8 +56,8 @@ template <> struct vec_t<2> {
 // b); a negative slot marks an inactive request (nothing read or written), a
 // slot >= pool_size is recorded as a bounds error and skipped.  q, k
 // [B,H,T,D], v, o [B,H,T,E]; T = 1 is the single decode step.
-// G: tokens per group (1 for single-token calls, which then compile to the
-// plain one-token loop; 4 for multi-token calls).
+// G: tokens per group; the library runs it for single-token calls (G = 1,
+// the plain one-token loop) and tokens_kernel for several tokens per call.
 template <typename T, int D, int E, int G>
 __global__ void __launch_bounds__(NT)
 decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
@@ -143,17 +143,23 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
 // load of all of them, in flight together with the state's), and the
 // per-group cross-warp sums double-buffered, so each group of G tokens costs
 // one block barrier and no exposed global-load latency.
+constexpr int NTT = 512;           // threads per state (tokens_kernel)
+constexpr int NWT = NTT / 32;
+template <int E, int G> constexpr size_t tokens_smem() { return sizeof(float) * 2 * NWT * G * E; }
+
 template <typename T, int D, int E, int G>
-__global__ void __launch_bounds__(NT)
+__global__ void __launch_bounds__(NTT)
 tokens_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
               const float *__restrict__ lambda, float *__restrict__ pool,
               const int *__restrict__ slots, int pool_size, T *__restrict__ o, int H, int ntok) {
+  constexpr int NT = NTT, NW = NWT;  // (this kernel's CTA: 16 warps of D / 16 rows)
   constexpr int ROWS = D / NW;
   constexpr int VEC = E / 32;
-  constexpr int TS = 8;  // tokens staged at once (static shared memory: 44 KB at d = e = 128)
+  constexpr int TS = 8;  // tokens staged at once
   using V = vec_t<VEC>;
   __shared__ float qs[TS][D], ks[TS][D], vs[TS][E];
-  __shared__ float red[2][NW][G][E];
+  extern __shared__ float red_raw[];  // [2][NW][G][E] cross-warp sums, double-buffered
+  auto red = reinterpret_cast<float(*)[NW][G][E]>(red_raw);
 
   const int64_t bh = blockIdx.x;
   const int64_t b = bh / H;

@@ -329,7 +329,7 @@ la2_status la2_feature_map_backward(const void *q, const void *k, const void *dp
  * v, o [B,H,T,e]: for t = 0..T-1, kv <- lambda kv + k_t^T v_t, o_t = q_t kv
  * (the la2_decode_step recurrence applied T times), reading and writing the
  * slot's state once per call instead of once per token.  slots may be NULL:
- * request b then uses state b (pool_size >= B).  From 16 tokens per request
+ * request b then uses state b (pool_size >= B).  From 17 tokens per request
  * on (bf16, d = e = 128; LA2_OPT_DECODE_BLOCK_TOKENS overrides) the call runs
  * each request's tokens as one block of the chunk schedule on the tensor
  * cores: up to 128 tokens, one CTA per SM walks a contiguous range of the

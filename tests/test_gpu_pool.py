@@ -134,8 +134,8 @@ def test_pool_slot_past_end_reported():
 def test_decode_tokens_bench_batch_sampled(orc, T):
     """Multi-token decode on the batch the bench times (256 requests x H 64,
     d = e = 128, bf16 tokens, fp32 state of 1 GiB): two calls of T tokens,
-    token by token below 32 per call and through the tensor-core block path
-    from 32; sampled requests against the oracle's decode steps."""
+    token by token at T = 4 and through the tensor-core block path at T = 64;
+    sampled requests against the oracle's decode steps."""
     B, H, d, e = 256, 64, 128, 128
     kv = inputs.decode_state0(B, H, d, e, device=DEV, seed=0)
     kv0 = kv[[0, 77, 255]].double().cpu().numpy()
