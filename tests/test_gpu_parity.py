@@ -295,6 +295,35 @@ def test_sweep_sampled_heads(orc, sweep_buffers, BL):
 
 
 # ------------------------------------------ workload: long context (forward)
+@pytest.mark.parametrize("de", [(128, 128), (64, 64), (64, 128)], ids=["d128e128", "d64e64", "d64e128"])
+def test_split_point_with_state_sampled(orc, de):
+    """The L = 32K sweep shape (B = 2, H = 32: each sequence split across
+    CTAs, the initial state entering through the chunk-state scan) with an
+    initial state kv0 and, for 64-column heads, the zero-padded tensors and
+    128 x 128 padded states of the tensor-core path: forward (o, final
+    state) and backward (dq, dk, dv, dkv0) of four (b, h) sequences against
+    the oracle."""
+    d, e = de
+    Bn, H, L = 2, 32, 32768
+    x = inputs.make_inputs(Bn, H, L, d, e, dtype=torch.bfloat16, device=DEV, seed=d + e + 7,
+                           with_kv0=True)
+    lam = inputs.decay_lambdas(H, DEV)
+    with options(path="tc"):
+        got = run_fwd_bwd(x, lam, x["kv0"])
+    assert got is not None
+    lam_h = lam.double().cpu().numpy()
+    picks = [(0, 0), (1, 31), (1, 16), (0, 9)]
+    sub = {n: np.concatenate([host(t[b:b + 1, h:h + 1]) for b, h in picks], axis=1)
+           for n, t in x.items()}
+    lh = np.array([lam_h[h] for _, h in picks])
+    ref = oracle_all(orc, {n: torch.from_numpy(v) for n, v in sub.items()},
+                     torch.from_numpy(lh), torch.from_numpy(sub["kv0"]))
+    for i, (b, h) in enumerate(picks):
+        for name, a, r in zip(NAMES, got, ref):
+            check(f"L32K d{d} e{e} kv0 (b={b},h={h}) {name}", a[b:b + 1, h:h + 1],
+                  r[:, i:i + 1], torch.bfloat16)
+
+
 def test_long_context_1m_sampled(orc):
     """B=1, H=64, L=1,048,576, forward only (8K+ blocks of on-chip carry);
     the oracle recomputes heads 0, 21, 42 and 63 over the full length."""
