@@ -25,13 +25,14 @@ def tokens(B, H, T, d, e, dtype, seed):
 
 
 @pytest.mark.parametrize("block_from", [0, 1, 100000])
-@pytest.mark.parametrize("T", [1, 3, 8, 40, 128, 129])
+@pytest.mark.parametrize("T", [1, 3, 8, 9, 16, 17, 40, 128, 129])
 @pytest.mark.parametrize("dtype,de", [(torch.bfloat16, (128, 128)), (torch.float32, (64, 64))])
 def test_decode_tokens_matches_oracle(orc, T, dtype, de, block_from):
-    """block_from: 0 = the library's crossover, 1 = the tensor-core block form
-    for every T (up to 128 tokens the decode-unit kernel, beyond it one
-    chunk-schedule CTA per request; bf16 128 x 128 only), 100000 = the
-    token-by-token kernel for every T (groups of 4 tokens and a ragged last
+    """block_from: 0 = the library's crossover (token by token up to 16 tokens,
+    the decode-unit kernel from 17), 1 = the tensor-core block form for every
+    T (up to 128 tokens the decode-unit kernel, beyond it one chunk-schedule
+    CTA per request; bf16 128 x 128 only), 100000 = the token-by-token kernel
+    for every T (tokens staged 8 at a time, groups of 4 and a ragged last
     group)."""
     d, e = de
     B, H, P = 6, 3, 10
