@@ -142,7 +142,12 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
 // with the tokens' q, k, v staged in shared memory up to TS = 8 at a time (one
 // load of all of them, in flight together with the state's), and the
 // per-group cross-warp sums double-buffered, so each group of G tokens costs
-// one block barrier and no exposed global-load latency.
+// one block barrier and no exposed global-load latency.  512 threads per
+// state (16 warps of D / 16 rows): from T ~ 8 the per-state token work, not
+// the state's traffic, sets the time, and this spreads it over twice
+// decode_kernel's threads while two states still fit an SM (measured on
+// B200: 0.50 against 0.58 ms per call at T = 8 for batch 256 x 64 heads;
+// 1,024 threads, one state per SM, 0.71 ms).
 constexpr int NTT = 512;           // threads per state (tokens_kernel)
 constexpr int NWT = NTT / 32;
 template <int E, int G> constexpr size_t tokens_smem() { return sizeof(float) * 2 * NWT * G * E; }
